@@ -1,0 +1,276 @@
+// api.cpp - the launch entry points of libtide.so: host-side validation,
+// pointer-table upload and dispatch to the kernels or the copy engines.
+//
+// Every check runs before anything is enqueued, so an error status means the
+// stream is untouched.  Checks: plan usable on the current device, enum
+// values, null pointers (a NULL buffer is accepted only where it would hold
+// zero elements), element alignment, buffer sizes against the plan, and
+// overlap between any written buffer and any other buffer of the call.
+#include <algorithm>
+#include <cstring>
+#include <vector>
+
+#include "tide_internal.h"
+
+namespace {
+
+struct Span {
+    uintptr_t lo, hi;
+    bool write;
+};
+
+// True if a written span overlaps any other span (read spans may overlap each other).
+bool overlaps(std::vector<Span>& spans) {
+    std::sort(spans.begin(), spans.end(), [](const Span& a, const Span& b) { return a.lo < b.lo; });
+    uintptr_t max_hi = 0, max_hi_write = 0;
+    for (const Span& s : spans) {
+        if (s.lo == s.hi) continue;
+        if (s.lo < max_hi_write) return true;
+        if (s.write && s.lo < max_hi) return true;
+        max_hi = std::max(max_hi, s.hi);
+        if (s.write) max_hi_write = std::max(max_hi_write, s.hi);
+    }
+    return false;
+}
+
+void add_span(std::vector<Span>& v, const void* p, int64_t bytes, bool write) {
+    if (p == nullptr || bytes <= 0) return;
+    const uintptr_t lo = reinterpret_cast<uintptr_t>(p);
+    v.push_back({lo, lo + (uintptr_t)bytes, write});
+}
+
+// A host-only plan passes here (so that argument validation can run without a
+// GPU) and is refused by `launchable` once the arguments have been checked.
+tide_status_t check_plan(const tide_plan* p) {
+    if (p == nullptr) return TIDE_ERR_INVALID_ARG;
+    if (p->flags & TIDE_PLAN_HOST_ONLY) return TIDE_OK;
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return TIDE_ERR_CUDA;
+    if (cur != p->device) return TIDE_ERR_DEVICE;
+    return TIDE_OK;
+}
+
+tide_status_t launchable(const tide_plan* p) {
+    return (p->flags & TIDE_PLAN_HOST_ONLY) ? TIDE_ERR_DEVICE : TIDE_OK;
+}
+
+// A device buffer of `need` elements of size `esize` at `ptr` with `have` elements.
+tide_status_t check_buf(const void* ptr, int64_t have, int64_t need, int esize) {
+    if (need == 0) return TIDE_OK;
+    if (ptr == nullptr) return TIDE_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(ptr) % (uintptr_t)esize != 0) return TIDE_ERR_ALIGNMENT;
+    if (have < need) return TIDE_ERR_SIZE;
+    return TIDE_OK;
+}
+
+tide_status_t check_grads(const tide_plan* p, const void* const* grads, const int64_t* grad_numel,
+                          std::vector<Span>& spans) {
+    const int64_t W = p->world, P = p->n_params;
+    if (W * P > 0 && (grads == nullptr || grad_numel == nullptr)) return TIDE_ERR_INVALID_ARG;
+    for (int64_t k = 0; k < W; ++k)
+        for (int64_t i = 0; i < P; ++i) {
+            const int64_t j = k * P + i;
+            tide_status_t st = check_buf(grads[j], grad_numel[j], p->numel[i], 2);
+            if (st != TIDE_OK) return st;
+            add_span(spans, grads[j], 2 * p->numel[i], false);
+        }
+    return TIDE_OK;
+}
+
+tide_status_t check_slots(const tide_plan* p, void* const* slots, int64_t slot_numel,
+                          std::vector<Span>& spans) {
+    const int64_t W = p->world, need = W * p->shard_numel;
+    if (slots == nullptr) return TIDE_ERR_INVALID_ARG;
+    for (int64_t k = 0; k < W; ++k) {
+        tide_status_t st = check_buf(slots[k], slot_numel, need, 2);
+        if (st != TIDE_OK) return st;
+        add_span(spans, slots[k], 2 * need, true);
+    }
+    return TIDE_OK;
+}
+
+tide_status_t check_enums(int32_t engine, int32_t max_ctas) {
+    if (engine != TIDE_ENGINE_SM && engine != TIDE_ENGINE_CE) return TIDE_ERR_INVALID_ARG;
+    if (max_ctas < 0) return TIDE_ERR_INVALID_ARG;
+    return TIDE_OK;
+}
+
+tide_status_t check_reduce_modes(int32_t scale_mode, int32_t order) {
+    if (scale_mode != TIDE_SCALE_NONE && scale_mode != TIDE_SCALE_INV_WORLD) return TIDE_ERR_INVALID_ARG;
+    if (order != TIDE_ORDER_RANK && order != TIDE_ORDER_TREE) return TIDE_ERR_INVALID_ARG;
+    return TIDE_OK;
+}
+
+// Upload a pointer table unless the device copy already holds these pointers.
+tide_status_t sync_table(PtrTable& t, const void* const* ptrs, int64_t n, cudaStream_t stream) {
+    if (n == 0) return TIDE_OK;
+    if (n > t.capacity || t.dev == nullptr) return TIDE_ERR_INVALID_ARG;
+    if (t.valid && (int64_t)t.host.size() == n &&
+        std::memcmp(t.host.data(), ptrs, sizeof(void*) * (size_t)n) == 0)
+        return TIDE_OK;
+    t.host.assign(ptrs, ptrs + n);
+    // Pageable source: the runtime stages it before returning, so the host
+    // mirror may change afterwards; the device copy is stream-ordered.
+    cudaError_t e = cudaMemcpyAsync(t.dev, t.host.data(), sizeof(void*) * (size_t)n,
+                                    cudaMemcpyHostToDevice, stream);
+    t.valid = (e == cudaSuccess);
+    return e == cudaSuccess ? TIDE_OK : TIDE_ERR_CUDA;
+}
+
+int grid_for(const tide_plan* p, int kernel, int32_t max_ctas) {
+    int32_t g = 0;
+    tide_launch_ctas(p, kernel, max_ctas, &g);
+    return g;
+}
+
+float inv_world(int32_t world) { return 1.0f / (float)world; }
+
+tide_status_t stage_impl(tide_plan* p, const void* const* grads, void* const* slots,
+                         int64_t slot_numel, int32_t engine, int32_t max_ctas, cudaStream_t s) {
+    if (p->tiles.empty()) return TIDE_OK;
+    cudaError_t e;
+    if (engine == TIDE_ENGINE_CE) {
+        e = tide::ce_slot_stage(p, grads, slots, s);
+    } else {
+        tide_status_t st = sync_table(p->grad_tab, grads, (int64_t)p->world * p->n_params, s);
+        if (st == TIDE_OK)
+            st = sync_table(p->slot_tab, const_cast<const void* const*>(slots), p->world, s);
+        if (st != TIDE_OK) return st;
+        e = tide::launch_slot_stage(p, p->grad_tab.dev, p->slot_tab.dev, slot_numel,
+                                    grid_for(p, K_STAGE, max_ctas), s);
+    }
+    return e == cudaSuccess ? TIDE_OK : TIDE_ERR_CUDA;
+}
+
+tide_status_t reduce_slots_impl(tide_plan* p, void* const* slots, int64_t slot_numel, float* out,
+                                int64_t out_numel, int32_t scale_mode, int32_t order,
+                                int32_t max_ctas, cudaStream_t s) {
+    if (p->tiles.empty()) return TIDE_OK;
+    tide_status_t st = sync_table(p->slot_tab, const_cast<const void* const*>(slots), p->world, s);
+    if (st != TIDE_OK) return st;
+    cudaError_t e = tide::launch_rs_reduce(p, p->slot_tab.dev, true, slot_numel, out, out_numel,
+                                           inv_world(p->world), scale_mode == TIDE_SCALE_INV_WORLD,
+                                           order, grid_for(p, K_SLOT_RS, max_ctas), s);
+    return e == cudaSuccess ? TIDE_OK : TIDE_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" tide_status_t tide_ag_place(const tide_plan_t* cplan, const void* ag_buf,
+                                       int64_t ag_numel, void* const* param_storage,
+                                       const int64_t* param_numel, int32_t engine,
+                                       int32_t max_ctas, void* stream) {
+    tide_plan* p = const_cast<tide_plan*>(cplan);
+    tide_status_t st = check_plan(p);
+    if (st != TIDE_OK) return st;
+    if ((st = check_enums(engine, max_ctas)) != TIDE_OK) return st;
+    const int64_t W = p->world, P = p->n_params;
+    std::vector<Span> spans;
+    if ((st = check_buf(ag_buf, ag_numel, W * p->shard_numel, 2)) != TIDE_OK) return st;
+    add_span(spans, ag_buf, 2 * W * p->shard_numel, false);
+    if (P > 0 && (param_storage == nullptr || param_numel == nullptr)) return TIDE_ERR_INVALID_ARG;
+    for (int64_t i = 0; i < P; ++i) {
+        if ((st = check_buf(param_storage[i], param_numel[i], W * p->chunk[i], 2)) != TIDE_OK) return st;
+        add_span(spans, param_storage[i], 2 * W * p->chunk[i], true);
+    }
+    if (overlaps(spans)) return TIDE_ERR_INVALID_ARG;
+    if ((st = launchable(p)) != TIDE_OK) return st;
+    if (p->tiles.empty()) return TIDE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (engine == TIDE_ENGINE_CE) {
+        e = tide::ce_ag_place(p, static_cast<const uint16_t*>(ag_buf), param_storage, s);
+    } else {
+        if ((st = sync_table(p->param_tab, const_cast<const void* const*>(param_storage), P, s)) != TIDE_OK)
+            return st;
+        e = tide::launch_ag_place(p, static_cast<const uint16_t*>(ag_buf), ag_numel, p->param_tab.dev,
+                                  grid_for(p, K_AG, max_ctas), s);
+    }
+    return e == cudaSuccess ? TIDE_OK : TIDE_ERR_CUDA;
+}
+
+extern "C" tide_status_t tide_rs_reduce(const tide_plan_t* cplan, const void* const* grads,
+                                        const int64_t* grad_numel, float* out, int64_t out_numel,
+                                        int32_t scale_mode, int32_t order, void* const* slots,
+                                        int64_t slot_numel, int32_t engine, int32_t max_ctas,
+                                        void* stream) {
+    tide_plan* p = const_cast<tide_plan*>(cplan);
+    tide_status_t st = check_plan(p);
+    if (st != TIDE_OK) return st;
+    if ((st = check_enums(engine, max_ctas)) != TIDE_OK) return st;
+    if ((st = check_reduce_modes(scale_mode, order)) != TIDE_OK) return st;
+    const int64_t W = p->world, P = p->n_params, n_out = W * p->shard_numel;
+    std::vector<Span> spans;
+    if ((st = check_grads(p, grads, grad_numel, spans)) != TIDE_OK) return st;
+    if ((st = check_buf(out, out_numel, n_out, 4)) != TIDE_OK) return st;
+    add_span(spans, out, 4 * n_out, true);
+    if (slots != nullptr && (st = check_slots(p, slots, slot_numel, spans)) != TIDE_OK) return st;
+    if (overlaps(spans)) return TIDE_ERR_INVALID_ARG;
+    if ((st = launchable(p)) != TIDE_OK) return st;
+    if (p->tiles.empty()) return TIDE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (slots != nullptr) {
+        st = stage_impl(p, grads, slots, slot_numel, engine, max_ctas, s);
+        if (st != TIDE_OK) return st;
+        return reduce_slots_impl(p, slots, slot_numel, out, out_numel, scale_mode, order, max_ctas, s);
+    }
+    if ((st = sync_table(p->grad_tab, grads, W * P, s)) != TIDE_OK) return st;
+    cudaError_t e = tide::launch_rs_reduce(p, p->grad_tab.dev, false, 0, out, out_numel,
+                                           inv_world(p->world), scale_mode == TIDE_SCALE_INV_WORLD,
+                                           order, grid_for(p, K_RS, max_ctas), s);
+    return e == cudaSuccess ? TIDE_OK : TIDE_ERR_CUDA;
+}
+
+extern "C" tide_status_t tide_rs_stage(const tide_plan_t* cplan, const void* const* grads,
+                                       const int64_t* grad_numel, void* const* slots,
+                                       int64_t slot_numel, int32_t engine, int32_t max_ctas,
+                                       void* stream) {
+    tide_plan* p = const_cast<tide_plan*>(cplan);
+    tide_status_t st = check_plan(p);
+    if (st != TIDE_OK) return st;
+    if ((st = check_enums(engine, max_ctas)) != TIDE_OK) return st;
+    std::vector<Span> spans;
+    if ((st = check_grads(p, grads, grad_numel, spans)) != TIDE_OK) return st;
+    if ((st = check_slots(p, slots, slot_numel, spans)) != TIDE_OK) return st;
+    if (overlaps(spans)) return TIDE_ERR_INVALID_ARG;
+    if ((st = launchable(p)) != TIDE_OK) return st;
+    return stage_impl(p, grads, slots, slot_numel, engine, max_ctas, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" tide_status_t tide_rs_reduce_slots(const tide_plan_t* cplan, const void* const* slots,
+                                              int64_t slot_numel, float* out, int64_t out_numel,
+                                              int32_t scale_mode, int32_t order, int32_t max_ctas,
+                                              void* stream) {
+    tide_plan* p = const_cast<tide_plan*>(cplan);
+    tide_status_t st = check_plan(p);
+    if (st != TIDE_OK) return st;
+    if ((st = check_enums(TIDE_ENGINE_SM, max_ctas)) != TIDE_OK) return st;
+    if ((st = check_reduce_modes(scale_mode, order)) != TIDE_OK) return st;
+    const int64_t n_out = (int64_t)p->world * p->shard_numel;
+    std::vector<Span> spans;
+    if ((st = check_slots(p, const_cast<void* const*>(slots), slot_numel, spans)) != TIDE_OK) return st;
+    // slots are only read in this phase: re-tag them as read spans
+    for (Span& sp : spans) sp.write = false;
+    if ((st = check_buf(out, out_numel, n_out, 4)) != TIDE_OK) return st;
+    add_span(spans, out, 4 * n_out, true);
+    if (overlaps(spans)) return TIDE_ERR_INVALID_ARG;
+    if ((st = launchable(p)) != TIDE_OK) return st;
+    return reduce_slots_impl(p, const_cast<void* const*>(slots), slot_numel, out, out_numel, scale_mode,
+                             order, max_ctas, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" tide_status_t tide_plan_check(tide_plan_t* p, void* stream) {
+    tide_status_t st = check_plan(p);
+    if (st != TIDE_OK) return st;
+    if ((st = launchable(p)) != TIDE_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int32_t h = 0;
+    if (cudaMemcpyAsync(&h, p->d_err, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return TIDE_ERR_CUDA;
+    if (h == 0) return TIDE_OK;
+    if (cudaMemsetAsync(p->d_err, 0, sizeof(int32_t), s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return TIDE_ERR_CUDA;
+    return TIDE_ERR_KERNEL_CHECK;
+}

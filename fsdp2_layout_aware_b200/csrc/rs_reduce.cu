@@ -1,0 +1,266 @@
+// rs_reduce.cu - TIDE-RS reduction kernel for sm_100a.
+//
+// Method: "The Endgame of FSDP Communication" (weekinpapers.com, Abstract,
+// TIDE-RS): per-parameter bf16 gradients are consumed where they lie and
+// reduced into fp32 shards, with no fp32 packing buffer in between.  Here the
+// W ranks are W sets of buffers on this GPU; one launch produces every rank's
+// fp32 shard:
+//   out[r*Ns + off_i + e] = s * fl32(sum_{k=0..W-1} fp32(g_{k,i}[r*c_i + e]))
+// and +0.0 at pad positions.  In Slot-Reuse mode the sources are the W staged
+// slots in the all-gather layout, read at the output position itself.
+//
+// Design (HBM-bound: W*2 bytes read and 4 bytes written per output element,
+// ~(W-1)/(2W+4) flop/byte, so no tensor cores):
+//   - a persistent grid, at most max_ctas CTAs, walks the plan's tile list
+//     round-robin; a tile is a piece of one (param, rank) chunk of up to
+//     TIDE_TILE_ELEMS elements, so tiny MoE chunks and huge dense chunks mix;
+//   - per tile the W source addresses are staged in shared memory once;
+//   - each thread owns 8 consecutive outputs per step: W independent 16-byte
+//     streaming loads (in groups of G ranks to bound registers), an fp32 sum
+//     with __fadd_rn (no contraction), the optional __fmul_rn scale, two 16-byte
+//     streaming stores;
+//   - tiles whose addresses are not all 16-byte aligned (possible only when
+//     the group's sizes break alignment) fall back to coalesced scalar loads;
+//   - ragged tile ends and pad rows are finished element by element.
+// Rank order (ORDER_RANK) adds g_0 + g_1 + ... exactly as the stock
+// pack-then-reduce does, so the result is bit-identical to it.  Tree order
+// adds adjacent ranks pairwise inside each group of G and merges group sums
+// with a binary counter (a pairwise tree over groups).
+#include "device_common.cuh"
+#include "tide_internal.h"
+
+namespace tide {
+namespace {
+
+struct RsParams {
+    const tide_tile_t* tiles;
+    int64_t n_tiles;
+    const void* const* src_tab;  // plain: [W*P] grads, index k*P + i; slot mode: [W] slots
+    const int64_t* numel;        // [P] unpadded numel (plain-mode source bound)
+    int64_t slot_numel;          // slot-mode source bound
+    float* out;
+    int64_t out_numel;
+    int32_t world;
+    int32_t n_params;
+    float scale;
+    int32_t do_scale;
+    int32_t* err;
+};
+
+constexpr int kMaxTreeLevels = 6;  // binary counter over ceil(W/G) <= 63 groups
+
+// Lane l (0..7) of a 16-byte vector of 8 bf16, or the single bf16 of a scalar,
+// as fp32 (exact).  l is a compile-time constant after unrolling.
+__device__ __forceinline__ float lane(const uint4& x, int l) {
+    const uint32_t w = l < 2 ? x.x : l < 4 ? x.y : l < 6 ? x.z : x.w;
+    return (l & 1) ? bf16_hi(w) : bf16_lo(w);
+}
+__device__ __forceinline__ float lane(uint32_t x, int) { return __uint_as_float(x << 16); }
+
+// Reduce W ranks for L lanes (L = 8: one 16-byte vector per rank; L = 1: one
+// element).  load(k) returns rank k's raw bf16 bits; loads are issued G ranks
+// at a time, before any add, and converted to fp32 inside the adds.
+//   Rank order: acc = g_0, then acc = acc + g_k for k = 1..W-1, one add per
+//   rank in order (grouping only batches the loads, never the adds).
+//   Tree: within a group, adjacent ranks are added pairwise level by level (an
+//   unpaired last one is carried); group sums are merged pairwise through a
+//   binary counter, which is a balanced tree when the group count is a power
+//   of two.
+template <int G, int L, bool TREE, class Raw, class Load>
+__device__ __forceinline__ void reduce_ranks(int W, Load load, float (&acc)[L]) {
+    float stack[TREE ? kMaxTreeLevels : 1][L];
+    int gidx = 0;
+    for (int k0 = 0; k0 < W; k0 += G, ++gidx) {
+        Raw x[G];
+        const int n_in = min(G, W - k0);
+#pragma unroll
+        for (int j = 0; j < G; ++j) {
+            if (j < n_in) x[j] = load(k0 + j);
+        }
+        if (!TREE) {
+#pragma unroll
+            for (int j = 0; j < G; ++j) {
+                if (j < n_in) {
+                    if (k0 + j == 0) {
+#pragma unroll
+                        for (int l = 0; l < L; ++l) acc[l] = lane(x[0], l);
+                    } else {
+#pragma unroll
+                        for (int l = 0; l < L; ++l) acc[l] = __fadd_rn(acc[l], lane(x[j], l));
+                    }
+                }
+            }
+        } else {
+            // level 1 straight from the raw values, then in place
+            constexpr int H = (G + 1) / 2;
+            float f[H][L];
+#pragma unroll
+            for (int j = 0; j < G; j += 2) {
+#pragma unroll
+                for (int l = 0; l < L; ++l) {
+                    if (j + 1 < n_in) f[j / 2][l] = __fadd_rn(lane(x[j], l), lane(x[j + 1], l));
+                    else if (j < n_in) f[j / 2][l] = lane(x[j], l);
+                }
+            }
+            const int n_half = (n_in + 1) / 2;
+#pragma unroll
+            for (int step = 1; step < H; step <<= 1) {
+#pragma unroll
+                for (int j = 0; j + step < H; j += 2 * step) {
+                    if (j + step < n_half) {
+#pragma unroll
+                        for (int l = 0; l < L; ++l) f[j][l] = __fadd_rn(f[j][l], f[j + step][l]);
+                    }
+                }
+            }
+            // push the group sum as a level-0 node; merge while the counter carries
+#pragma unroll
+            for (int lvl = 0; lvl < kMaxTreeLevels; ++lvl) {
+                if ((gidx >> lvl) & 1) {
+#pragma unroll
+                    for (int l = 0; l < L; ++l) f[0][l] = __fadd_rn(stack[lvl][l], f[0][l]);
+                } else {
+#pragma unroll
+                    for (int l = 0; l < L; ++l) stack[lvl][l] = f[0][l];
+                    break;
+                }
+            }
+        }
+    }
+    if (TREE) {
+        // gidx is now the group count; occupied levels are its set bits
+        bool have = false;
+#pragma unroll
+        for (int lvl = 0; lvl < kMaxTreeLevels; ++lvl) {
+            if ((gidx >> lvl) & 1) {
+#pragma unroll
+                for (int l = 0; l < L; ++l)
+                    acc[l] = have ? __fadd_rn(stack[lvl][l], acc[l]) : stack[lvl][l];
+                have = true;
+            }
+        }
+    }
+}
+
+template <int G, int U, bool SLOT, bool TREE>
+__global__ void __launch_bounds__(kThreads) rs_reduce_kernel(const RsParams a) {
+    __shared__ const uint16_t* s_src[TIDE_MAX_WORLD];
+    __shared__ tide_tile_t s_tile;
+    const int tid = threadIdx.x;
+    const int W = a.world;
+
+    for (int64_t t = blockIdx.x; t < a.n_tiles; t += gridDim.x) {
+        __syncthreads();  // the previous tile is done with s_tile and s_src
+        if (tid == 0) s_tile = a.tiles[t];
+        __syncthreads();
+        const tide_tile_t tl = s_tile;
+
+        // Range check of the descriptor against the buffers the host validated.
+        const bool param_ok = tl.param >= 0 && tl.param < a.n_params;
+        const int64_t src_off = SLOT ? tl.dst_off : tl.src_off;
+        const int64_t src_lim = SLOT ? a.slot_numel : (param_ok ? a.numel[tl.param] : -1);
+        const bool ok = param_ok && tl.n_valid >= 0 && tl.n_valid <= tl.n_total &&
+                        tl.dst_off >= 0 && tl.dst_off + tl.n_total <= a.out_numel &&
+                        src_off >= 0 && src_off + tl.n_valid <= src_lim;
+        if (!ok) {
+            if (tid == 0) atomicOr(a.err, TIDE_KCHECK_TILE);
+            continue;
+        }
+
+        bool misaligned = false;
+        for (int k = tid; k < W; k += kThreads) {
+            const void* base = a.src_tab[SLOT ? k : (int64_t)k * a.n_params + tl.param];
+            const uint16_t* p = static_cast<const uint16_t*>(base) + src_off;
+            s_src[k] = p;
+            misaligned |= (reinterpret_cast<uintptr_t>(p) & 15) != 0;
+        }
+        float* __restrict__ dst = a.out + tl.dst_off;
+        misaligned |= (reinterpret_cast<uintptr_t>(dst) & 15) != 0;
+        const bool scalar_only = __syncthreads_or(misaligned);
+
+        // Vector body: 8 outputs per thread per unit, U units per step.
+        const int nv = scalar_only ? 0 : (tl.n_valid >> 3);
+        for (int v0 = 0; v0 < nv; v0 += kThreads * U) {
+            float acc[U][8];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int v = v0 + u * kThreads + tid;
+                if (v < nv) {
+                    auto load = [&](int k) { return ld_stream_v4(s_src[k] + 8 * (int64_t)v); };
+                    reduce_ranks<G, 8, TREE, uint4>(W, load, acc[u]);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int v = v0 + u * kThreads + tid;
+                if (v < nv) {
+                    if (a.do_scale) {
+#pragma unroll
+                        for (int l = 0; l < 8; ++l) acc[u][l] = __fmul_rn(acc[u][l], a.scale);
+                    }
+                    float* o = dst + 8 * (int64_t)v;
+                    st_stream_f4(o, acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
+                    st_stream_f4(o + 4, acc[u][4], acc[u][5], acc[u][6], acc[u][7]);
+                }
+            }
+        }
+        // Remaining valid elements one by one (ragged end, or a misaligned tile).
+        for (int e = 8 * nv + tid; e < tl.n_valid; e += kThreads) {
+            float acc[1];
+            auto load = [&](int k) { return (uint32_t)ld_stream_u16(s_src[k] + e); };
+            reduce_ranks<G, 1, TREE, uint32_t>(W, load, acc);
+            if (a.do_scale) acc[0] = __fmul_rn(acc[0], a.scale);
+            dst[e] = acc[0];
+        }
+        // Pad positions are +0.0.
+        for (int e = tl.n_valid + tid; e < tl.n_total; e += kThreads) dst[e] = 0.0f;
+    }
+}
+
+using KernelFn = void (*)(const RsParams);
+
+template <bool SLOT, bool TREE>
+KernelFn pick(int world) {
+    if (world <= 2) return rs_reduce_kernel<2, 4, SLOT, TREE>;
+    if (world <= 4) return rs_reduce_kernel<4, 2, SLOT, TREE>;
+    return rs_reduce_kernel<8, 1, SLOT, TREE>;
+}
+
+KernelFn select(int world, bool slot, int order) {
+    const bool tree = order == TIDE_ORDER_TREE;
+    if (slot) return tree ? pick<true, true>(world) : pick<true, false>(world);
+    return tree ? pick<false, true>(world) : pick<false, false>(world);
+}
+
+}  // namespace
+
+int rs_blocks_per_sm(int world, bool slot, int order) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, select(world, slot, order), kThreads, 0) !=
+        cudaSuccess)
+        return 0;
+    return n;
+}
+
+cudaError_t launch_rs_reduce(const tide_plan* p, const void* const* d_src_tab, bool slot,
+                             int64_t src_bound, float* out, int64_t out_numel, float scale,
+                             bool do_scale, int order, int grid, cudaStream_t stream) {
+    if (p->tiles.empty() || grid <= 0) return cudaSuccess;
+    RsParams a;
+    a.tiles = p->d_tiles;
+    a.n_tiles = (int64_t)p->tiles.size();
+    a.src_tab = d_src_tab;
+    a.numel = p->d_numel;
+    a.slot_numel = src_bound;
+    a.out = out;
+    a.out_numel = out_numel;
+    a.world = p->world;
+    a.n_params = p->n_params;
+    a.scale = scale;
+    a.do_scale = do_scale ? 1 : 0;
+    a.err = p->d_err;
+    select(p->world, slot, order)<<<grid, kThreads, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace tide

@@ -1,0 +1,73 @@
+// tide_internal.h - plan object and kernel launchers shared by the libtide.so
+// translation units (not part of the public ABI; see include/tide.h).
+#pragma once
+
+#include <cstdint>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "tide.h"
+
+// Bits of the device error word.
+enum : int32_t {
+    TIDE_KCHECK_TILE = 1,   // a tile descriptor pointed outside its buffers
+};
+
+// Kernel ids (match tide_launch_ctas).
+enum : int32_t { K_RS = 0, K_AG = 1, K_STAGE = 2, K_SLOT_RS = 3, K_COUNT = 4 };
+
+// A device pointer table with a host mirror: re-uploaded only when it changes.
+struct PtrTable {
+    const void** dev = nullptr;          // device array of `capacity` pointers
+    std::vector<const void*> host;       // last uploaded contents
+    int64_t capacity = 0;
+    bool valid = false;                  // host mirror matches the device copy
+};
+
+struct tide_plan {
+    int32_t device = -1;
+    int32_t world = 0;
+    int32_t n_params = 0;
+    uint32_t flags = 0;
+    int64_t shard_numel = 0;             // Ns
+    std::vector<int64_t> dim0, inner, numel, rows, chunk, offset;   // per param: d0, inner, d0*inner, S, c, off
+    std::vector<tide_tile_t> tiles;
+
+    // device tables (absent for TIDE_PLAN_HOST_ONLY)
+    tide_tile_t* d_tiles = nullptr;
+    int64_t* d_numel = nullptr;
+    int32_t* d_err = nullptr;
+    PtrTable grad_tab, param_tab, slot_tab;
+    int64_t workspace_bytes = 0;
+
+    int32_t sm_count = 0;
+    int32_t blocks_per_sm[K_COUNT] = {0, 0, 0, 0};
+};
+
+namespace tide {
+
+constexpr int kThreads = 256;
+
+// Occupancy (resident CTAs per SM) of each kernel at kThreads threads.
+int rs_blocks_per_sm(int world, bool slot, int order);
+int ag_blocks_per_sm();
+int stage_blocks_per_sm();
+
+// Kernel launches; return the launch's cudaError_t.
+cudaError_t launch_rs_reduce(const tide_plan* p, const void* const* d_src_tab, bool slot,
+                             int64_t src_bound, float* out, int64_t out_numel, float scale,
+                             bool do_scale, int order, int grid, cudaStream_t stream);
+cudaError_t launch_ag_place(const tide_plan* p, const uint16_t* ag, int64_t ag_numel,
+                            const void* const* d_param_tab, int grid, cudaStream_t stream);
+cudaError_t launch_slot_stage(const tide_plan* p, const void* const* d_grad_tab,
+                              const void* const* d_slot_tab, int64_t slot_numel, int grid,
+                              cudaStream_t stream);
+
+// Copy-engine variants (no kernels).
+cudaError_t ce_ag_place(const tide_plan* p, const uint16_t* ag, void* const* params,
+                        cudaStream_t stream);
+cudaError_t ce_slot_stage(const tide_plan* p, const void* const* grads, void* const* slots,
+                          cudaStream_t stream);
+
+}  // namespace tide

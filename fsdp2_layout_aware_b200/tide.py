@@ -1,0 +1,307 @@
+"""ctypes binding of libtide.so (include/tide.h): argument marshalling only.
+
+Each ``tide_*`` function here has the C entry point's name and arguments, with
+Python ints for pointers and sizes; every step of the work runs in the
+library's CUDA kernels or copy-engine calls.  If the library has not been
+built the import fails loudly: there is no fallback path.
+
+``Plan`` is a thin convenience wrapper that takes torch tensors (device memory
+and the current CUDA stream come from PyTorch) and forwards their pointers.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtide.so")
+
+TIDE_OK = 0
+TIDE_ERR_INVALID_ARG = -1
+TIDE_ERR_ALIGNMENT = -2
+TIDE_ERR_SIZE = -3
+TIDE_ERR_CUDA = -4
+TIDE_ERR_NOMEM = -5
+TIDE_ERR_DEVICE = -6
+TIDE_ERR_KERNEL_CHECK = -7
+
+TIDE_ENGINE_SM = 0
+TIDE_ENGINE_CE = 1
+TIDE_ORDER_RANK = 0
+TIDE_ORDER_TREE = 1
+TIDE_SCALE_NONE = 0
+TIDE_SCALE_INV_WORLD = 1
+TIDE_PLAN_HOST_ONLY = 1
+TIDE_MAX_WORLD = 256
+TIDE_TILE_ELEMS = 8192
+
+K_RS, K_AG, K_STAGE, K_SLOT_RS = 0, 1, 2, 3
+
+
+class tide_param_t(ctypes.Structure):
+    _fields_ = [("dim0", ctypes.c_int64), ("inner", ctypes.c_int64)]
+
+
+class tide_tile_t(ctypes.Structure):
+    _fields_ = [("src_off", ctypes.c_int64), ("dst_off", ctypes.c_int64),
+                ("param", ctypes.c_int32), ("rank", ctypes.c_int32),
+                ("n_valid", ctypes.c_int32), ("n_total", ctypes.c_int32)]
+
+
+class TideError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {tide_status_string(status)} ({status})")
+
+
+_lib = None
+
+_i32, _i64, _u32, _vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_void_p
+_P = ctypes.POINTER
+
+_SIGNATURES = {
+    "tide_plan_group": (_i32, [_P(tide_param_t), _i32, _i32, _i32, _u32, _P(_vp)]),
+    "tide_plan_destroy": (None, [_vp]),
+    "tide_plan_info": (_i32, [_vp, _P(_i32), _P(_i32), _P(_i64), _P(_i64), _P(_i64)]),
+    "tide_plan_query": (_i32, [_vp, _i32, _P(_i64), _P(_i64), _P(_i64), _P(_i64)]),
+    "tide_plan_tiles": (_i32, [_vp, _P(tide_tile_t), _i64, _P(_i64)]),
+    "tide_ag_place": (_i32, [_vp, _vp, _i64, _P(_vp), _P(_i64), _i32, _i32, _vp]),
+    "tide_rs_reduce": (_i32, [_vp, _P(_vp), _P(_i64), _vp, _i64, _i32, _i32, _P(_vp), _i64,
+                              _i32, _i32, _vp]),
+    "tide_rs_stage": (_i32, [_vp, _P(_vp), _P(_i64), _P(_vp), _i64, _i32, _i32, _vp]),
+    "tide_rs_reduce_slots": (_i32, [_vp, _P(_vp), _i64, _vp, _i64, _i32, _i32, _i32, _vp]),
+    "tide_plan_check": (_i32, [_vp, _vp]),
+    "tide_launch_ctas": (_i32, [_vp, _i32, _i32, _P(_i32)]),
+    "tide_status_string": (ctypes.c_char_p, [_i32]),
+    "tide_abi_version": (_i32, []),
+}
+
+
+def lib():
+    """The loaded libtide.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libtide.so is not built ({LIB_PATH}); run "
+                               "`python -m fsdp2_layout_aware_b200.build` (there is no CPU fallback)")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _ptr_array(ptrs):
+    arr = (_vp * max(1, len(ptrs)))()
+    for j, p in enumerate(ptrs):
+        arr[j] = p
+    return arr
+
+
+def _i64_array(vals):
+    arr = (_i64 * max(1, len(vals)))()
+    for j, v in enumerate(vals):
+        arr[j] = int(v)
+    return arr
+
+
+def _check(status: int, where: str) -> None:
+    if status != TIDE_OK:
+        raise TideError(status, where)
+
+
+# --------------------------------------------------------------------------- C-ABI mirrors
+
+
+def tide_status_string(status: int) -> str:
+    return lib().tide_status_string(status).decode()
+
+
+def tide_abi_version() -> int:
+    return lib().tide_abi_version()
+
+
+def tide_plan_group(params, world: int, device: int, flags: int = 0):
+    """params: sequence of (dim0, inner).  Returns (status, plan handle or None)."""
+    arr = (tide_param_t * max(1, len(params)))()
+    for j, (d0, inner) in enumerate(params):
+        arr[j].dim0, arr[j].inner = int(d0), int(inner)
+    out = _vp()
+    st = lib().tide_plan_group(arr, len(params), world, device, flags, ctypes.byref(out))
+    return st, (out.value if st == TIDE_OK else None)
+
+
+def tide_plan_destroy(plan) -> None:
+    lib().tide_plan_destroy(plan)
+
+
+def tide_plan_info(plan):
+    w, p = _i32(), _i32()
+    ns, nt, ws = _i64(), _i64(), _i64()
+    st = lib().tide_plan_info(plan, ctypes.byref(w), ctypes.byref(p), ctypes.byref(ns),
+                              ctypes.byref(nt), ctypes.byref(ws))
+    return st, dict(world=w.value, n_params=p.value, shard_numel=ns.value, n_tiles=nt.value,
+                    workspace_bytes=ws.value)
+
+
+def tide_plan_query(plan, param: int):
+    a, b, c, d = _i64(), _i64(), _i64(), _i64()
+    st = lib().tide_plan_query(plan, param, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c),
+                               ctypes.byref(d))
+    return st, dict(shard_rows=a.value, shard_offset=b.value, padded_numel=c.value,
+                    chunk_numel=d.value)
+
+
+def tide_plan_tiles(plan, capacity: int):
+    arr = (tide_tile_t * max(1, capacity))()
+    n = _i64()
+    st = lib().tide_plan_tiles(plan, arr, capacity, ctypes.byref(n))
+    return st, arr[: n.value]
+
+
+def tide_ag_place(plan, ag_buf: int, ag_numel: int, param_storage, param_numel, engine: int,
+                  max_ctas: int, stream: int) -> int:
+    return lib().tide_ag_place(plan, ag_buf, ag_numel, _ptr_array(param_storage),
+                               _i64_array(param_numel), engine, max_ctas, stream)
+
+
+def tide_rs_reduce(plan, grads, grad_numel, out: int, out_numel: int, scale_mode: int, order: int,
+                   slots, slot_numel: int, engine: int, max_ctas: int, stream: int) -> int:
+    slot_arr = _ptr_array(slots) if slots is not None else None
+    return lib().tide_rs_reduce(plan, _ptr_array(grads), _i64_array(grad_numel), out, out_numel,
+                                scale_mode, order, slot_arr, slot_numel, engine, max_ctas, stream)
+
+
+def tide_rs_stage(plan, grads, grad_numel, slots, slot_numel: int, engine: int, max_ctas: int,
+                  stream: int) -> int:
+    slot_arr = _ptr_array(slots) if slots is not None else None
+    return lib().tide_rs_stage(plan, _ptr_array(grads), _i64_array(grad_numel), slot_arr,
+                               slot_numel, engine, max_ctas, stream)
+
+
+def tide_rs_reduce_slots(plan, slots, slot_numel: int, out: int, out_numel: int, scale_mode: int,
+                         order: int, max_ctas: int, stream: int) -> int:
+    slot_arr = _ptr_array(slots) if slots is not None else None
+    return lib().tide_rs_reduce_slots(plan, slot_arr, slot_numel, out, out_numel, scale_mode,
+                                      order, max_ctas, stream)
+
+
+def tide_plan_check(plan, stream: int) -> int:
+    return lib().tide_plan_check(plan, stream)
+
+
+def tide_launch_ctas(plan, kernel: int, max_ctas: int):
+    n = _i32()
+    st = lib().tide_launch_ctas(plan, kernel, max_ctas, ctypes.byref(n))
+    return st, n.value
+
+
+# --------------------------------------------------------------------------- torch convenience
+
+
+def _stream_handle(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+class Plan:
+    """A parameter group over `world` simulated ranks, planned on one device.
+
+    shapes: parameter shapes (dim 0 first).  Tensors passed to the methods are
+    only read for their data pointers and sizes.
+    """
+
+    def __init__(self, shapes, world: int, device=None, host_only: bool = False):
+        self.shapes = [tuple(int(d) for d in s) for s in shapes]
+        self.world = int(world)
+        if host_only:
+            dev = 0
+        else:
+            import torch
+            dev = torch.cuda.current_device() if device is None else torch.device(device).index
+            dev = 0 if dev is None else dev
+        params = [(s[0], _prod(s[1:])) for s in self.shapes]
+        st, handle = tide_plan_group(params, self.world, dev,
+                                     TIDE_PLAN_HOST_ONLY if host_only else 0)
+        _check(st, "tide_plan_group")
+        self.handle = handle
+        self.device_index = dev
+        st, info = tide_plan_info(handle)
+        _check(st, "tide_plan_info")
+        self.shard_numel = info["shard_numel"]
+        self.n_tiles = info["n_tiles"]
+        self.workspace_bytes = info["workspace_bytes"]
+        self.n_params = info["n_params"]
+
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            tide_plan_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def query(self, param: int) -> dict:
+        st, q = tide_plan_query(self.handle, param)
+        _check(st, "tide_plan_query")
+        return q
+
+    def tiles(self):
+        st, t = tide_plan_tiles(self.handle, self.n_tiles)
+        _check(st, "tide_plan_tiles")
+        return t
+
+    def launch_ctas(self, kernel: int, max_ctas: int = 0) -> int:
+        st, n = tide_launch_ctas(self.handle, kernel, max_ctas)
+        _check(st, "tide_launch_ctas")
+        return n
+
+    def ag_place(self, ag, params, engine: int = TIDE_ENGINE_SM, max_ctas: int = 0,
+                 stream=None) -> None:
+        st = tide_ag_place(self.handle, ag.data_ptr(), ag.numel(), [p.data_ptr() for p in params],
+                           [p.numel() for p in params], engine, max_ctas, _stream_handle(stream))
+        _check(st, "tide_ag_place")
+
+    def rs_reduce(self, grads, out, scale_mode: int = TIDE_SCALE_INV_WORLD,
+                  order: int = TIDE_ORDER_RANK, slots=None, engine: int = TIDE_ENGINE_SM,
+                  max_ctas: int = 0, stream=None) -> None:
+        """grads[k][i]: rank k's gradient of param i; out: fp32 [W*Ns]."""
+        flat = [g for row in grads for g in row]
+        st = tide_rs_reduce(self.handle, [g.data_ptr() for g in flat], [g.numel() for g in flat],
+                            out.data_ptr(), out.numel(), scale_mode, order,
+                            None if slots is None else [s.data_ptr() for s in slots],
+                            0 if slots is None else min(s.numel() for s in slots),
+                            engine, max_ctas, _stream_handle(stream))
+        _check(st, "tide_rs_reduce")
+
+    def rs_stage(self, grads, slots, engine: int = TIDE_ENGINE_SM, max_ctas: int = 0,
+                 stream=None) -> None:
+        flat = [g for row in grads for g in row]
+        st = tide_rs_stage(self.handle, [g.data_ptr() for g in flat], [g.numel() for g in flat],
+                           [s.data_ptr() for s in slots], min(s.numel() for s in slots), engine,
+                           max_ctas, _stream_handle(stream))
+        _check(st, "tide_rs_stage")
+
+    def rs_reduce_slots(self, slots, out, scale_mode: int = TIDE_SCALE_INV_WORLD,
+                        order: int = TIDE_ORDER_RANK, max_ctas: int = 0, stream=None) -> None:
+        st = tide_rs_reduce_slots(self.handle, [s.data_ptr() for s in slots],
+                                  min(s.numel() for s in slots), out.data_ptr(), out.numel(),
+                                  scale_mode, order, max_ctas, _stream_handle(stream))
+        _check(st, "tide_rs_reduce_slots")
+
+    def check(self, stream=None) -> None:
+        _check(tide_plan_check(self.handle, _stream_handle(stream)), "tide_plan_check")
+
+
+def _prod(dims) -> int:
+    n = 1
+    for d in dims:
+        n *= int(d)
+    return n

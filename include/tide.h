@@ -1,0 +1,209 @@
+/*
+ * tide.h - C ABI of libtide.so: layout-aware reduce-scatter and all-gather
+ * placement for FSDP2-style per-parameter storage, on one GPU.
+ *
+ * Source of the method: "The Endgame of FSDP Communication: Layout-Aware
+ * Collectives on Copy Engines, RDMA, and NVSwitch" (weekinpapers.com, Abstract)
+ * and the kongchang.com article "The Endgame of FSDP Communication: TIDE
+ * Zero-Copy Collective Communication Optimization" (sections "The Root of FSDP2
+ * Communication Overhead" and "TIDE's Design Approach").  TIDE computes the
+ * final address of every shard element inside the collective itself: the
+ * all-gather result lands directly in per-parameter storage (TIDE-AG) and the
+ * reduce-scatter reads per-parameter bf16 gradients where they are and writes
+ * fp32 shards (TIDE-RS), so neither a copy-out nor a packed fp32 staging
+ * buffer exists.  This library implements the per-rank arithmetic and
+ * addressing of those two collectives with the network taken out: the W
+ * data-parallel ranks are W sets of buffers on the calling GPU.
+ *
+ * Layout (the pages leave it open; this is the reading every call follows):
+ *   param i has shape (d0_i, ...) with inner_i = product of the trailing dims;
+ *   S_i = ceil(d0_i / W) rows per shard, c_i = S_i * inner_i elements per chunk;
+ *   rank r owns rows [r*S_i, min((r+1)*S_i, d0_i)); rows d0_i .. W*S_i-1 are pad;
+ *   inside a rank's shard, params follow the group order with no gaps:
+ *   off_i = sum_{j<i} c_j, Ns = sum_i c_i; a rank-major buffer is [W][Ns].
+ *
+ * Conventions for every call:
+ *   - The caller owns every data buffer.  All pointers to data are device
+ *     pointers of the plan's device; pointer ARRAYS (grads, params, slots) and
+ *     numel arrays are host arrays that are only read during the call.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and never synchronize the device, except tide_plan_group,
+ *     tide_plan_destroy and tide_plan_check where stated.
+ *   - All arguments are validated on the host before anything is enqueued; on
+ *     any error status nothing has been enqueued.
+ *   - A plan keeps small device tables (tile list, pointer tables, an error
+ *     word).  A pointer table is re-uploaded, stream-ordered, only when its
+ *     contents change.  One plan must be used from one stream at a time (or the
+ *     caller orders the streams).
+ *   - bf16 buffers must be 2-byte aligned and fp32 buffers 4-byte aligned; any
+ *     such alignment is accepted (16-byte alignment gives the fast path).
+ *   - No call allocates device memory except tide_plan_group.
+ */
+#ifndef TIDE_H
+#define TIDE_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TIDE_API __attribute__((visibility("default")))
+#else
+#define TIDE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TIDE_OK = 0,
+    TIDE_ERR_INVALID_ARG = -1,  /* null pointer, bad enum, bad shape, aliasing */
+    TIDE_ERR_ALIGNMENT = -2,    /* buffer not aligned to its element size */
+    TIDE_ERR_SIZE = -3,         /* a buffer is smaller than the plan needs */
+    TIDE_ERR_CUDA = -4,         /* a CUDA runtime call or launch failed */
+    TIDE_ERR_NOMEM = -5,        /* host or device allocation failed */
+    TIDE_ERR_DEVICE = -6,       /* wrong current device, or a host-only plan */
+    TIDE_ERR_KERNEL_CHECK = -7  /* a kernel's own range check rejected a tile */
+} tide_status_t;
+
+enum { TIDE_ENGINE_SM = 0, TIDE_ENGINE_CE = 1 };
+enum { TIDE_ORDER_RANK = 0, TIDE_ORDER_TREE = 1 };
+enum { TIDE_SCALE_NONE = 0, TIDE_SCALE_INV_WORLD = 1 };
+enum { TIDE_PLAN_HOST_ONLY = 1 }; /* flag: build the tables on the host only (no CUDA calls) */
+
+#define TIDE_MAX_WORLD 256
+#define TIDE_TILE_ELEMS 8192
+
+/* One parameter: dim 0 and the product of the remaining dims (1 for a 1-D param). */
+typedef struct {
+    int64_t dim0;
+    int64_t inner;
+} tide_param_t;
+
+/*
+ * One unit of kernel work: elements [e0, e0 + n_total) of the chunk of param
+ * `param` that rank `rank` owns, with e0 a multiple of TIDE_TILE_ELEMS.
+ *   src_off = rank*c_i + e0        offset into the param's own tensor
+ *   dst_off = rank*Ns + off_i + e0 offset into a rank-major [W][Ns] buffer
+ *   the first n_valid elements hold data; the remaining ones are padding.
+ */
+typedef struct {
+    int64_t src_off;
+    int64_t dst_off;
+    int32_t param;
+    int32_t rank;
+    int32_t n_valid;
+    int32_t n_total;
+} tide_tile_t;
+
+typedef struct tide_plan tide_plan_t;
+
+/*
+ * Build the address tables of a parameter group for W = `world` ranks: per
+ * param S_i, c_i, off_i; per (param, rank) chunk the valid and pad lengths; the
+ * tile list the kernels walk.  These tables are where the per-parameter layout
+ * enters the collective's address computation (weekinpapers.com Abstract),
+ * built once per group.  1 <= world <= TIDE_MAX_WORLD, 0 <= n_params, dims >= 0.
+ * Unless flags has TIDE_PLAN_HOST_ONLY, the tables are uploaded to `device`
+ * (cudaMalloc + synchronous copies; the current device is restored).
+ * On success *out_plan owns the tables; free it with tide_plan_destroy.
+ */
+TIDE_API tide_status_t tide_plan_group(const tide_param_t* params, int32_t n_params, int32_t world,
+                              int32_t device, uint32_t flags, tide_plan_t** out_plan);
+
+/* Free a plan (NULL is accepted).  Synchronizes the plan's device first, so
+ * that no enqueued call can still read the tables. */
+TIDE_API void tide_plan_destroy(tide_plan_t* plan);
+
+/* Group-level sizes.  Any output pointer may be NULL.  workspace_bytes counts
+ * every byte of device memory the plan holds (tables only: no staging). */
+TIDE_API tide_status_t tide_plan_info(const tide_plan_t* plan, int32_t* world, int32_t* n_params,
+                             int64_t* shard_numel, int64_t* n_tiles, int64_t* workspace_bytes);
+
+/* Per-param layout: S_i, off_i, padded numel W*c_i, and c_i.  Any output may be NULL. */
+TIDE_API tide_status_t tide_plan_query(const tide_plan_t* plan, int32_t param, int64_t* shard_rows,
+                              int64_t* shard_offset, int64_t* padded_numel, int64_t* chunk_numel);
+
+/* Copy up to `capacity` tiles into out (host array); *n_written gets the count. */
+TIDE_API tide_status_t tide_plan_tiles(const tide_plan_t* plan, tide_tile_t* out, int64_t capacity,
+                              int64_t* n_written);
+
+/*
+ * TIDE-AG placement (weekinpapers.com Abstract, TIDE-AG; kongchang.com
+ * "TIDE's Design Approach"): the rank-major all-gather buffer ag_buf (bf16
+ * [W][Ns], ag_numel >= W*Ns) is written straight into per-parameter padded
+ * storage: param_storage[i] (bf16, param_numel[i] >= W*c_i) receives
+ *   param_i[r*c_i + e] = ag[r*Ns + off_i + e]  for r*c_i + e < d0_i*inner_i,
+ *   param_i[r*c_i + e] = +0                    for the pad rows.
+ * Pad positions of ag_buf are never read.  engine: TIDE_ENGINE_SM (one kernel
+ * launch, at most max_ctas CTAs, 0 = as many as fit) or TIDE_ENGINE_CE (copy
+ * engine memcpys and memsets only; max_ctas is ignored).  ag_buf must not
+ * overlap any param storage.
+ */
+TIDE_API tide_status_t tide_ag_place(const tide_plan_t* plan, const void* ag_buf, int64_t ag_numel,
+                            void* const* param_storage, const int64_t* param_numel,
+                            int32_t engine, int32_t max_ctas, void* stream);
+
+/*
+ * TIDE-RS (weekinpapers.com Abstract, TIDE-RS and the two-phase pipeline;
+ * kongchang.com "TIDE's Design Approach"): per-parameter bf16 gradients are
+ * reduced straight into fp32 rank-major shards with no packed fp32 buffer.
+ * grads is a host array of W*P device pointers, grads[k*P + i] = rank k's
+ * unpadded gradient of param i (grad_numel[k*P+i] >= d0_i*inner_i).  out is
+ * fp32 [W][Ns] (out_numel >= W*Ns); rank r's shard is out[r*Ns, (r+1)*Ns):
+ *   out[r*Ns + off_i + e] = s * fl32(sum_{k=0..W-1} fp32(g_{k,i}[r*c_i + e]))
+ * for r*c_i + e < d0_i*inner_i, and +0.0 at pad positions.  scale_mode
+ * TIDE_SCALE_INV_WORLD multiplies once by fl32(1/W) after the sum; NONE skips it.
+ * order TIDE_ORDER_RANK adds in rank order 0..W-1 (bit-exact against the stock
+ * pack-then-reduce result); TIDE_ORDER_TREE adds pairwise (within
+ * |err| <= 1e-6 * sum|terms| of the exact sum).
+ * slots == NULL: one kernel launch.  slots != NULL: Slot-Reuse, the two phases
+ * of tide_rs_stage (with `engine`) and tide_rs_reduce_slots run back to back;
+ * slots is a host array of W device pointers to bf16 [W][Ns] buffers
+ * (slot_numel elements each, >= W*Ns) whose contents are overwritten.
+ * out must not overlap grads or slots; slots must not overlap grads.
+ */
+TIDE_API tide_status_t tide_rs_reduce(const tide_plan_t* plan, const void* const* grads,
+                             const int64_t* grad_numel, float* out, int64_t out_numel,
+                             int32_t scale_mode, int32_t order, void* const* slots,
+                             int64_t slot_numel, int32_t engine, int32_t max_ctas, void* stream);
+
+/*
+ * Slot-Reuse phase 1 (weekinpapers.com Abstract: gradients staged in vacated
+ * all-gather slots; gradient reads are the pipeline's first phase): rank k's
+ * gradients are copied, still bf16, into slot k in the all-gather layout,
+ *   slot_k[r*Ns + off_i + e] = g_{k,i}[r*c_i + e]  for valid positions;
+ * pad positions of the slots are not written.  engine SM (one launch) or CE.
+ */
+TIDE_API tide_status_t tide_rs_stage(const tide_plan_t* plan, const void* const* grads,
+                            const int64_t* grad_numel, void* const* slots, int64_t slot_numel,
+                            int32_t engine, int32_t max_ctas, void* stream);
+
+/*
+ * Slot-Reuse phase 2: out[r*Ns + j] = s * fl32(sum_k fp32(slot_k[r*Ns + j])) at
+ * valid positions (from the plan), +0.0 at pad positions.  One kernel launch.
+ */
+TIDE_API tide_status_t tide_rs_reduce_slots(const tide_plan_t* plan, const void* const* slots,
+                                   int64_t slot_numel, float* out, int64_t out_numel,
+                                   int32_t scale_mode, int32_t order, int32_t max_ctas,
+                                   void* stream);
+
+/*
+ * Read and clear the plan's device error word: synchronizes `stream`, then
+ * returns TIDE_ERR_KERNEL_CHECK if a kernel enqueued before it rejected a tile
+ * (the tile is skipped, nothing outside the buffers is touched), else TIDE_OK.
+ */
+TIDE_API tide_status_t tide_plan_check(tide_plan_t* plan, void* stream);
+
+/* The number of CTAs a kernel call with this max_ctas would launch.
+ * kernel: 0 = RS reduce, 1 = AG place, 2 = Slot-Reuse stage, 3 = slot reduce. */
+TIDE_API tide_status_t tide_launch_ctas(const tide_plan_t* plan, int32_t kernel, int32_t max_ctas,
+                               int32_t* ctas);
+
+TIDE_API const char* tide_status_string(tide_status_t status);
+TIDE_API int32_t tide_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TIDE_H */

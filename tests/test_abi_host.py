@@ -1,0 +1,261 @@
+"""The C-ABI library on the host (no GPU): exports, plan tables, argument validation.
+
+Plans are built with TIDE_PLAN_HOST_ONLY, which makes every entry point run its
+full argument validation and then refuse to launch (TIDE_ERR_DEVICE); data
+pointers are fake addresses that validation never dereferences.
+"""
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from fsdp2_layout_aware_b200 import tide as T
+from synth import configs
+
+from _groups import degenerate, mini_sweep, mini_wan, random_group
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"^TIDE_API\s+[\w\s\*]+?\b(tide_\w+)\s*\(", text, flags=re.M)
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    names = declared_symbols()
+    assert len(names) >= 13
+    lib = T.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert T.tide_abi_version() == 1
+
+
+def test_status_strings():
+    for code in range(0, -8, -1):
+        assert T.tide_status_string(code) not in ("", "unknown status")
+    assert T.tide_status_string(-99) == "unknown status"
+
+
+def host_plan(group):
+    return T.Plan(group.shapes, group.world, host_only=True)
+
+
+@pytest.mark.parametrize("name", ["tiny", "llama70b", "qwen3moe", "wan14b", "sweep_w2", "sweep_w64"])
+def test_plan_layout_matches_oracle(name):
+    g = configs.by_name(name)
+    plan = host_plan(g)
+    L = oracle.layout(g.world, g.shapes)
+    assert plan.shard_numel == L.Ns
+    for i in range(g.n_params):
+        q = plan.query(i)
+        assert q["shard_rows"] == L.S[i]
+        assert q["shard_offset"] == L.off[i]
+        assert q["chunk_numel"] == L.c[i]
+        assert q["padded_numel"] == g.world * L.c[i]
+    assert plan.workspace_bytes == 0          # host-only: no device tables
+
+
+def check_tiles(group):
+    plan = host_plan(group)
+    L = oracle.layout(group.world, group.shapes)
+    tiles = plan.tiles()
+    assert len(tiles) == plan.n_tiles
+    W, Ns = group.world, L.Ns
+    cover = np.zeros(W * Ns, dtype=np.int32)
+    last = -1
+    for t in tiles:
+        i, r = t.param, t.rank
+        assert 0 <= i < group.n_params and 0 <= r < W
+        assert 0 < t.n_total <= T.TIDE_TILE_ELEMS and 0 <= t.n_valid <= t.n_total
+        e0 = t.src_off - r * L.c[i]
+        assert e0 % T.TIDE_TILE_ELEMS == 0 and 0 <= e0 < L.c[i]
+        assert t.dst_off == r * Ns + L.off[i] + e0
+        assert t.dst_off > last                      # sorted by output position
+        last = t.dst_off
+        assert t.n_valid == min(t.n_total, max(0, group.numel(i) - t.src_off))
+        cover[t.dst_off: t.dst_off + t.n_total] += 1
+        # validity agrees with the oracle's per-position locate, at both ends
+        for e in {0, t.n_total - 1, t.n_valid - 1, t.n_valid}:
+            if 0 <= e < t.n_total:
+                st, p, src = oracle.locate(W, group.shapes, r, t.dst_off - r * Ns + e)
+                assert p == i and src == t.src_off + e and st == (1 if e < t.n_valid else 0)
+    assert np.all(cover == 1)                        # every output position exactly once
+
+
+@pytest.mark.parametrize("group", [configs.tiny(), degenerate(), mini_wan(), mini_sweep(64),
+                                   configs.qwen3moe(4), configs.Group("big_chunk", 3, ((40000, 3),))],
+                         ids=lambda g: g.name)
+def test_tiles_cover_output_exactly_once(group):
+    check_tiles(group)
+
+
+def test_tiles_random_groups():
+    rng = np.random.default_rng(99)
+    for w in (1, 2, 3, 7, 16, 64, 256):
+        check_tiles(random_group(rng, w, int(rng.integers(1, 9)), max_rows=2000))
+
+
+def test_full_config_tile_counts():
+    for name in ("llama70b", "qwen3moe", "wan14b"):
+        g = configs.by_name(name)
+        plan = host_plan(g)
+        L = oracle.layout(g.world, g.shapes)
+        expect = sum(g.world * -(-c // T.TIDE_TILE_ELEMS) for c in L.c)
+        assert plan.n_tiles == expect
+
+
+@pytest.mark.parametrize("world,params,status", [
+    (0, [(4, 4)], T.TIDE_ERR_INVALID_ARG),
+    (T.TIDE_MAX_WORLD + 1, [(4, 4)], T.TIDE_ERR_INVALID_ARG),
+    (4, [(-1, 4)], T.TIDE_ERR_INVALID_ARG),
+    (4, [(4, -2)], T.TIDE_ERR_INVALID_ARG),
+    (4, [(2 ** 40, 2 ** 40)], T.TIDE_ERR_INVALID_ARG),
+])
+def test_plan_group_rejects(world, params, status):
+    st, h = T.tide_plan_group(params, world, 0, T.TIDE_PLAN_HOST_ONLY)
+    assert st == status and h is None
+
+
+def test_plan_group_rejects_unknown_flag_and_empty_group_ok():
+    st, _ = T.tide_plan_group([(4, 4)], 2, 0, 0x80)
+    assert st == T.TIDE_ERR_INVALID_ARG
+    st, h = T.tide_plan_group([], 4, 0, T.TIDE_PLAN_HOST_ONLY)
+    assert st == T.TIDE_OK
+    st, info = T.tide_plan_info(h)
+    assert info["shard_numel"] == 0 and info["n_tiles"] == 0
+    T.tide_plan_destroy(h)
+    T.tide_plan_destroy(None)
+
+
+# --------------------------------------------------------------------------- argument validation
+
+BASE = 0x7F0000000000   # fake, 256-byte aligned device addresses; never dereferenced
+
+
+class Fake:
+    """Non-overlapping fake buffers laid out for one call."""
+
+    def __init__(self):
+        self.next = BASE
+
+    def buf(self, nbytes):
+        p = self.next
+        self.next += ((nbytes + 4095) // 4096 + 1) * 4096
+        return p
+
+
+def fake_args(group):
+    W, P = group.world, group.n_params
+    L = oracle.layout(W, group.shapes)
+    f = Fake()
+    grads = [f.buf(2 * group.numel(i)) for _ in range(W) for i in range(P)]
+    gnum = [group.numel(i) for _ in range(W) for i in range(P)]
+    out = f.buf(4 * W * L.Ns)
+    ag = f.buf(2 * W * L.Ns)
+    params = [f.buf(2 * W * L.c[i]) for i in range(P)]
+    pnum = [W * L.c[i] for i in range(P)]
+    slots = [f.buf(2 * W * L.Ns) for _ in range(W)]
+    return dict(grads=grads, gnum=gnum, out=out, n_out=W * L.Ns, ag=ag, n_ag=W * L.Ns,
+                params=params, pnum=pnum, slots=slots, n_slot=W * L.Ns)
+
+
+def rs(plan, a, **kw):
+    args = dict(a)
+    args.update(kw)
+    return T.tide_rs_reduce(plan.handle, args["grads"], args["gnum"], args["out"], args["n_out"],
+                            args.get("scale", 1), args.get("order", 0), args.get("use_slots"),
+                            args["n_slot"], args.get("engine", 0), args.get("max_ctas", 0), 0)
+
+
+def ag(plan, a, **kw):
+    args = dict(a)
+    args.update(kw)
+    return T.tide_ag_place(plan.handle, args["ag"], args["n_ag"], args["params"], args["pnum"],
+                           args.get("engine", 0), args.get("max_ctas", 0), 0)
+
+
+@pytest.fixture(scope="module")
+def tiny_plan():
+    return host_plan(configs.tiny())
+
+
+@pytest.fixture
+def args():
+    return fake_args(configs.tiny())
+
+
+def test_valid_arguments_reach_the_device_check(tiny_plan, args):
+    assert rs(tiny_plan, args) == T.TIDE_ERR_DEVICE
+    assert rs(tiny_plan, args, use_slots=args["slots"]) == T.TIDE_ERR_DEVICE
+    assert ag(tiny_plan, args) == T.TIDE_ERR_DEVICE
+    assert ag(tiny_plan, args, engine=1) == T.TIDE_ERR_DEVICE
+    h = tiny_plan.handle
+    assert T.tide_rs_stage(h, args["grads"], args["gnum"], args["slots"], args["n_slot"], 0, 0, 0) \
+        == T.TIDE_ERR_DEVICE
+    assert T.tide_rs_reduce_slots(h, args["slots"], args["n_slot"], args["out"], args["n_out"], 1, 0,
+                                  0, 0) == T.TIDE_ERR_DEVICE
+    assert T.tide_plan_check(h, 0) == T.TIDE_ERR_DEVICE
+    assert T.tide_launch_ctas(h, 0, 0)[0] == T.TIDE_ERR_DEVICE
+
+
+def test_rs_validation(tiny_plan, args):
+    E = T
+    g = list(args["grads"])
+    assert rs(tiny_plan, args, scale=2) == E.TIDE_ERR_INVALID_ARG
+    assert rs(tiny_plan, args, order=5) == E.TIDE_ERR_INVALID_ARG
+    assert rs(tiny_plan, args, engine=7) == E.TIDE_ERR_INVALID_ARG
+    assert rs(tiny_plan, args, max_ctas=-1) == E.TIDE_ERR_INVALID_ARG
+    g0 = list(g); g0[3] = 0
+    assert rs(tiny_plan, args, grads=g0) == E.TIDE_ERR_INVALID_ARG           # null grad
+    g1 = list(g); g1[2] += 1
+    assert rs(tiny_plan, args, grads=g1) == E.TIDE_ERR_ALIGNMENT             # odd bf16 address
+    n1 = list(args["gnum"]); n1[4] -= 1
+    assert rs(tiny_plan, args, gnum=n1) == E.TIDE_ERR_SIZE                  # undersized grad
+    assert rs(tiny_plan, args, out=0) == E.TIDE_ERR_INVALID_ARG
+    assert rs(tiny_plan, args, out=args["out"] + 2) == E.TIDE_ERR_ALIGNMENT  # fp32 needs 4 bytes
+    assert rs(tiny_plan, args, n_out=args["n_out"] - 1) == E.TIDE_ERR_SIZE
+    assert rs(tiny_plan, args, out=g[5]) == E.TIDE_ERR_INVALID_ARG           # out aliases a grad
+    s = list(args["slots"]); s[1] = s[0] + 64
+    assert rs(tiny_plan, args, use_slots=s) == E.TIDE_ERR_INVALID_ARG       # slots overlap
+    s = list(args["slots"]); s[2] = g[0]
+    assert rs(tiny_plan, args, use_slots=s) == E.TIDE_ERR_INVALID_ARG       # slot aliases a grad
+    assert rs(tiny_plan, args, use_slots=args["slots"], n_slot=args["n_slot"] - 8) == E.TIDE_ERR_SIZE
+    # grads may alias each other (read only)
+    g2 = list(g); g2[1 * 5 + 0] = g[0]
+    assert rs(tiny_plan, args, grads=g2) == E.TIDE_ERR_DEVICE
+
+
+def test_ag_validation(tiny_plan, args):
+    E = T
+    assert ag(tiny_plan, args, ag=0) == E.TIDE_ERR_INVALID_ARG
+    assert ag(tiny_plan, args, ag=args["ag"] + 1) == E.TIDE_ERR_ALIGNMENT
+    assert ag(tiny_plan, args, n_ag=args["n_ag"] - 1) == E.TIDE_ERR_SIZE
+    p = list(args["params"]); p[2] = 0
+    assert ag(tiny_plan, args, params=p) == E.TIDE_ERR_INVALID_ARG
+    n = list(args["pnum"]); n[4] -= 1
+    assert ag(tiny_plan, args, pnum=n) == E.TIDE_ERR_SIZE
+    p = list(args["params"]); p[1] = args["ag"] + 2
+    assert ag(tiny_plan, args, params=p) == E.TIDE_ERR_INVALID_ARG          # param aliases ag
+    p = list(args["params"]); p[3] = p[0] + 2
+    assert ag(tiny_plan, args, params=p) == E.TIDE_ERR_INVALID_ARG          # params overlap
+    assert ag(tiny_plan, args, engine=3) == E.TIDE_ERR_INVALID_ARG
+
+
+def test_null_allowed_only_for_empty_buffers():
+    g = degenerate()
+    plan = host_plan(g)
+    a = fake_args(g)
+    empty = [i for i in range(g.n_params) if g.numel(i) == 0]
+    assert empty
+    grads = list(a["grads"])
+    for k in range(g.world):
+        for i in empty:
+            grads[k * g.n_params + i] = 0
+    assert rs(plan, a, grads=grads) == T.TIDE_ERR_DEVICE

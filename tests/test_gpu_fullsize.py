@@ -1,0 +1,165 @@
+"""GPU parity at the full workload sizes, in the launch configuration the benchmark times.
+
+Inputs are generated on the device by the generator's CUDA twin; the oracle
+side regenerates only the values it needs on the host.  Checked outputs: a
+seeded random sample plus the first and last element of every chunk of every
+rank (pad boundaries included) for RS, and the same for AG placement, each
+compared bit for bit with the oracle's per-element answer.  This also checks
+that the device generator reproduces the host generator.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from fsdp2_layout_aware_b200 import tide as T
+from synth import configs
+
+from _gpu_helpers import bits_of
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+SEED = 1
+
+
+def sample_positions(group, L, n_random, rng):
+    """(rank, j) output positions: random ones plus both ends of every chunk and its valid part."""
+    W, Ns = group.world, L.Ns
+    pos = set()
+    if Ns == 0:
+        return []
+    for r in range(W):
+        for i in range(group.n_params):
+            c = L.c[i]
+            if c == 0:
+                continue
+            valid = max(0, min(c, group.numel(i) - r * c))
+            for e in {0, c - 1, valid - 1, valid, c // 2}:
+                if 0 <= e < c:
+                    pos.add((r, L.off[i] + e))
+    flat = rng.integers(0, W * Ns, size=n_random)
+    pos.update((int(f // Ns), int(f % Ns)) for f in flat)
+    return sorted(pos)
+
+
+def expected_rs(group, L, positions, scale):
+    """Oracle value at each sampled output position, from host-regenerated inputs."""
+    W = group.world
+    zero = [synth.zero_grad_params(group, SEED, k) for k in range(W)]
+    located = [oracle.locate(W, group.shapes, r, j) for r, j in positions]
+    need = {}
+    for n, (st, i, src) in enumerate(located):
+        if st == 1:
+            need.setdefault(i, []).append((n, src))
+    vals = np.zeros((len(positions), W), dtype=np.uint16)
+    for i, lst in need.items():
+        idx = np.array([s for _, s in lst], dtype=np.int64)
+        rows = np.array([n for n, _ in lst])
+        for k in range(W):
+            if i in zero[k]:
+                continue
+            vals[rows, k] = synth.gather_bf16(idx, SEED, synth.STREAM_GRAD, k, i, group.grad_sigma)
+    out = np.zeros(len(positions), dtype=np.float32)
+    for n, (st, _, _) in enumerate(located):
+        out[n] = oracle.sum_ranks(vals[n], scale) if st == 1 else np.float32(0.0)
+    return out
+
+
+def check_rs(group, out, L, scale, rng, n_random=20000):
+    pos = sample_positions(group, L, n_random, rng)
+    flat = torch.tensor([r * L.Ns + j for r, j in pos], dtype=torch.int64, device=out.device)
+    got = out[flat].cpu().numpy()
+    exp = expected_rs(group, L, pos, scale)
+    bad = np.nonzero(got.view(np.uint32) != exp.view(np.uint32))[0]
+    assert bad.size == 0, f"{bad.size} mismatches, first at {pos[bad[0]]}: {got[bad[0]]} vs {exp[bad[0]]}"
+
+
+def check_ag(group, params, L, rng, n_random=4000):
+    W, Ns = group.world, L.Ns
+    for i in range(group.n_params):
+        c = L.c[i]
+        if c == 0:
+            continue
+        qs = set(rng.integers(0, W * c, size=max(1, n_random // group.n_params)).tolist())
+        for r in range(W):
+            valid = max(0, min(c, group.numel(i) - r * c))
+            for e in {0, c - 1, valid - 1, valid}:
+                if 0 <= e < c:
+                    qs.add(r * c + e)
+        qs = sorted(qs)
+        got = bits_of(params[i][torch.tensor(qs, dtype=torch.int64, device=params[i].device)])
+        exp = np.zeros(len(qs), dtype=np.uint16)
+        by_rank = {}
+        for n, q in enumerate(qs):
+            st, a = oracle.ag_source(W, group.shapes, i, q)
+            if st == 1:
+                by_rank.setdefault(a // Ns, []).append((n, a % Ns))
+        for r, lst in by_rank.items():
+            idx = np.array([j for _, j in lst], dtype=np.int64)
+            exp[[n for n, _ in lst]] = synth.gather_bf16(idx, SEED, synth.STREAM_AG, r, 0,
+                                                         group.param_sigma)
+        assert np.array_equal(got, exp), f"param {i}"
+
+
+FULL = ["llama70b", "qwen3moe", "wan14b"] + [f"sweep_w{w}" for w in configs.SWEEP_WORLDS]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_rs_and_ag(name):
+    group = configs.by_name(name)
+    rng = np.random.default_rng(7)
+    torch.cuda.empty_cache()
+    plan = T.Plan(group.shapes, group.world)
+    L = oracle.layout(group.world, group.shapes)
+    assert plan.shard_numel == L.Ns
+    grads = synth.dev_grads(group, SEED)
+    out = torch.full((group.world * L.Ns,), float("nan"), device="cuda")
+    plan.rs_reduce(grads, out, scale_mode=T.TIDE_SCALE_INV_WORLD)     # the benchmark's call
+    torch.cuda.synchronize()
+    plan.check()
+    check_rs(group, out, L, 1, rng)
+    if name == "wan14b":
+        # Slot-Reuse: stage into vacated all-gather slots, then reduce: must equal plain mode
+        ref = out.clone()
+        slots = [torch.empty(group.world * L.Ns, dtype=torch.bfloat16, device="cuda")
+                 for _ in range(group.world)]
+        for engine in (T.TIDE_ENGINE_SM, T.TIDE_ENGINE_CE):
+            out.fill_(float("nan"))
+            plan.rs_reduce(grads, out, scale_mode=T.TIDE_SCALE_INV_WORLD, slots=slots, engine=engine)
+            torch.cuda.synchronize()
+            assert torch.equal(out.view(torch.int32), ref.view(torch.int32))
+        del slots, ref
+    del grads, out
+    torch.cuda.empty_cache()
+    ag = synth.dev_ag(group, L.Ns, SEED)
+    params = [torch.full((group.world * L.c[i],), 0x7777, dtype=torch.int16, device="cuda")
+              .view(torch.bfloat16) for i in range(group.n_params)]
+    for engine in (T.TIDE_ENGINE_SM, T.TIDE_ENGINE_CE):
+        plan.ag_place(ag, params, engine=engine)
+        torch.cuda.synchronize()
+        plan.check()
+        check_ag(group, params, L, rng)
+        for p in params:
+            p.view(torch.int16).fill_(0x7777)
+    del ag, params
+    torch.cuda.empty_cache()
+
+
+def test_device_generator_matches_host():
+    g = configs.tiny()
+    dev = synth.dev_grads(g, 5)
+    host = synth.grads_host(g, 5)
+    for k in range(g.world):
+        for i in range(g.n_params):
+            assert np.array_equal(bits_of(dev[k][i]), host[k][i])
+    q = configs.qwen3moe(20)                      # one unrouted expert per rank
+    assert q.n_zero_experts == 1
+    devq = synth.dev_grads(q, 3)
+    for k in range(q.world):
+        zero = synth.zero_grad_params(q, 3, k)
+        assert len(zero) == 3
+        for i in sorted(zero | {0, 4, 7, q.n_params - 1}):
+            h = synth.grad_host(q, 3, k, i)
+            assert np.array_equal(bits_of(devq[k][i]), h)
+            assert (i in zero) == (not h.any())

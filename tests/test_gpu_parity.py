@@ -1,0 +1,303 @@
+"""GPU parity: the CUDA path through the C-ABI against the CPU oracle, element by element.
+
+Bars: AG placement, Slot-Reuse staging and rank-order RS bit-exact; tree-order
+RS within 1e-6 * sum|terms| of the exact fp64 sum.  Sizes are small enough for
+the oracle to finish in seconds but span many tiles, ragged tile ends,
+misaligned chunk offsets, pad rows and all-pad chunks.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from fsdp2_layout_aware_b200 import tide as T
+from synth import configs
+
+from _gpu_helpers import bits_of, f32_bits, grads_to_dev, padded_params, poison_pads, to_dev
+from _groups import degenerate, mini_sweep, mini_wan, random_group
+
+pytestmark = pytest.mark.gpu
+
+
+def parity_groups():
+    rng = np.random.default_rng(2024)
+    out = [configs.tiny(), degenerate(), mini_wan(), mini_sweep(2), mini_sweep(64),
+           configs.qwen3moe(4), configs.Group("long_chunk", 3, ((30011, 7), (5,), (40000,)))]
+    for w in (1, 2, 3, 5, 8, 16, 64):
+        out.append(random_group(rng, w, int(rng.integers(1, 8)), max_rows=1500, name=f"rand_w{w}"))
+    return out
+
+
+GROUPS = parity_groups()
+IDS = [f"{g.name}_w{g.world}" for g in GROUPS]
+
+
+def run_rs(group, grads_host, scale=1, order=0, max_ctas=0, slots=False, engine=0):
+    plan = T.Plan(group.shapes, group.world)
+    grads = grads_to_dev(group, grads_host)
+    out = torch.full((group.world * plan.shard_numel,), float("nan"), device="cuda")
+    slot_bufs = None
+    if slots:
+        slot_bufs = [torch.full((group.world * plan.shard_numel,), -1, dtype=torch.int16,
+                                device="cuda").view(torch.bfloat16) for _ in range(group.world)]
+    plan.rs_reduce(grads, out, scale_mode=scale, order=order, slots=slot_bufs, engine=engine,
+                   max_ctas=max_ctas)
+    torch.cuda.synchronize()
+    plan.check()
+    return out, slot_bufs, plan
+
+
+@pytest.mark.parametrize("group", GROUPS, ids=IDS)
+@pytest.mark.parametrize("scale", [0, 1])
+def test_rs_rank_order_bit_exact(group, scale):
+    grads = synth.grads_host(group, seed=31)
+    out, _, _ = run_rs(group, grads, scale=scale)
+    ref = oracle.rs_reduce(group.world, group.shapes, grads, scale)
+    assert np.array_equal(f32_bits(out), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("seed", range(1, 17))
+def test_rs_tiny_all_seeds(seed):
+    g = configs.tiny()
+    grads = synth.grads_host(g, seed=seed)
+    out, _, _ = run_rs(g, grads, scale=1)
+    assert np.array_equal(f32_bits(out), oracle.rs_reduce(g.world, g.shapes, grads, 1).view(np.uint32))
+
+
+@pytest.mark.parametrize("group", GROUPS, ids=IDS)
+def test_rs_tree_order_within_tolerance(group):
+    grads = synth.grads_host(group, seed=32)
+    out, _, _ = run_rs(group, grads, scale=0, order=1)
+    E, A = oracle.exact_f64(group.world, group.shapes, grads)
+    got = out.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - E) <= 1e-6 * A)
+    L = oracle.layout(group.world, group.shapes)
+    pad = np.ones(group.world * L.Ns, dtype=bool)
+    ref = oracle.rs_reduce(group.world, group.shapes, grads, 0)
+    pad[np.nonzero(A)[0]] = False
+    assert np.all(f32_bits(out)[A == 0] == ref.view(np.uint32)[A == 0])   # zeros / pads agree bitwise
+
+
+@pytest.mark.parametrize("W", [2, 4, 8, 16, 64, 256])
+def test_rs_identical_ranks_closed_form(W):
+    """All ranks equal: unscaled sum is W*g exactly (any order), scaled is g."""
+    g = configs.Group("ident", W, ((3 * W + 5, 17), (W // 2 + 1,)))
+    one = synth.grads_host(configs.Group("src", 1, g.shapes), seed=5)[0]
+    grads = [one for _ in range(W)]
+    ref = oracle.pack_f32(W, g.shapes, one).astype(np.float64)
+    for order in (0, 1):
+        out, _, _ = run_rs(g, grads, scale=0, order=order)
+        assert np.array_equal(out.cpu().numpy().astype(np.float64), W * ref)
+        out, _, _ = run_rs(g, grads, scale=1, order=order)
+        assert np.array_equal(out.cpu().numpy().astype(np.float64), ref)
+
+
+def test_rs_rank_order_pin_on_gpu():
+    # (1 + 2^-24) + 2^-24 = 1 in fp32 while 2^-24 + 2^-24 + 1 = 1 + 2^-23
+    shapes = ((64,),)
+    g = configs.Group("order", 3, shapes)
+    def grads_of(vals):
+        return [[np.full(64, np.array([v], np.float32).view(np.uint32)[0] >> 16, np.uint16)]
+                for v in vals]
+    for order, vals, exp in ((0, [1.0, 2.0 ** -24, 2.0 ** -24], 1.0),
+                             (0, [2.0 ** -24, 2.0 ** -24, 1.0], 1.0 + 2.0 ** -23)):
+        out, _, _ = run_rs(g, grads_of(vals), scale=0, order=order)
+        L = oracle.layout(3, shapes)
+        valid = out.cpu().numpy()[: L.c[0]]
+        assert np.all(valid == np.float32(exp))
+
+
+@pytest.mark.parametrize("group", GROUPS, ids=IDS)
+@pytest.mark.parametrize("engine", [T.TIDE_ENGINE_SM, T.TIDE_ENGINE_CE])
+def test_ag_place_bit_exact(group, engine):
+    plan = T.Plan(group.shapes, group.world)
+    L = oracle.layout(group.world, group.shapes)
+    ag_bits = poison_pads(synth.ag_host(group, L.Ns, seed=41).reshape(-1), group, L)
+    ag = to_dev(ag_bits)
+    params = padded_params(plan, group)
+    plan.ag_place(ag, params, engine=engine)
+    torch.cuda.synchronize()
+    plan.check()
+    ref = oracle.ag_copyout(group.world, group.shapes, ag_bits)
+    for p, r in zip(params, ref):
+        assert np.array_equal(bits_of(p), r)
+
+
+@pytest.mark.parametrize("group", [configs.tiny(), degenerate(), mini_wan(), configs.qwen3moe(4),
+                                   GROUPS[-3]], ids=lambda g: f"{g.name}_w{g.world}")
+@pytest.mark.parametrize("engine", [T.TIDE_ENGINE_SM, T.TIDE_ENGINE_CE])
+def test_slot_reuse_equals_plain_and_oracle(group, engine):
+    grads = synth.grads_host(group, seed=51)
+    out, slots, plan = run_rs(group, grads, scale=1, slots=True, engine=engine)
+    ref = oracle.rs_reduce(group.world, group.shapes, grads, 1)
+    assert np.array_equal(f32_bits(out), ref.view(np.uint32))
+    L = oracle.layout(group.world, group.shapes)
+    for k in range(group.world):
+        exp = np.full(group.world * L.Ns, 0xFFFF, dtype=np.uint16)   # slots started as -1 (0xFFFF)
+        oracle.slot_stage(group.world, group.shapes, grads[k], exp)
+        assert np.array_equal(bits_of(slots[k]), exp)
+
+
+def test_slot_phases_separately():
+    group = mini_wan()
+    grads = synth.grads_host(group, seed=52)
+    plan = T.Plan(group.shapes, group.world)
+    dev = grads_to_dev(group, grads)
+    n = group.world * plan.shard_numel
+    slots = [torch.zeros(n, dtype=torch.bfloat16, device="cuda") for _ in range(group.world)]
+    plan.rs_stage(dev, slots, engine=T.TIDE_ENGINE_SM)
+    out = torch.empty(n, device="cuda")
+    for order in (0, 1):
+        plan.rs_reduce_slots(slots, out, scale_mode=0, order=order)
+        torch.cuda.synchronize()
+        if order == 0:
+            assert np.array_equal(f32_bits(out),
+                                  oracle.rs_reduce(group.world, group.shapes, grads, 0).view(np.uint32))
+        else:
+            E, A = oracle.exact_f64(group.world, group.shapes, grads)
+            assert np.all(np.abs(out.cpu().numpy() - E) <= 1e-6 * A)
+
+
+@pytest.mark.parametrize("group", [configs.tiny(), mini_sweep(8), configs.qwen3moe(4)],
+                         ids=lambda g: g.name)
+def test_max_ctas_does_not_change_bits(group):
+    grads = synth.grads_host(group, seed=61)
+    L = oracle.layout(group.world, group.shapes)
+    ag_bits = synth.ag_host(group, L.Ns, seed=62).reshape(-1)
+    ref_rs, ref_ag = None, None
+    for ctas in (1, 8, 16, 32, 0):
+        out, _, plan = run_rs(group, grads, scale=1, max_ctas=ctas)
+        params = padded_params(plan, group)
+        plan.ag_place(to_dev(ag_bits), params, max_ctas=ctas)
+        torch.cuda.synchronize()
+        rs_bits = f32_bits(out)
+        ag_b = [bits_of(p) for p in params]
+        if ref_rs is None:
+            ref_rs, ref_ag = rs_bits, ag_b
+        assert np.array_equal(rs_bits, ref_rs)
+        for a, b in zip(ag_b, ref_ag):
+            assert np.array_equal(a, b)
+        if ctas:
+            assert plan.launch_ctas(T.K_RS, ctas) == min(ctas, plan.n_tiles)
+
+
+@pytest.mark.parametrize("shift", [1, 3, 8])
+def test_misaligned_buffers_and_guard_bands(shift):
+    """Buffers at 2-byte (not 16-byte) offsets take the scalar path; guards stay intact."""
+    group = configs.Group("mis", 4, ((37, 16), (1000,), (129, 64)))
+    grads = synth.grads_host(group, seed=71)
+    plan = T.Plan(group.shapes, group.world)
+    W, P, Ns = group.world, group.n_params, plan.shard_numel
+    guard = 64
+    pool = []
+    dev = []
+    for k in range(W):
+        row = []
+        for i in range(P):
+            n = group.numel(i)
+            buf = torch.full((n + shift + guard,), -3, dtype=torch.int16, device="cuda")
+            buf[shift: shift + n] = to_dev(grads[k][i]).view(torch.int16)
+            pool.append(buf)
+            row.append(buf[shift: shift + n].view(torch.bfloat16))
+        dev.append(row)
+    out_buf = torch.full((W * Ns + 2 * guard + shift,), 12345.0, device="cuda")
+    out = out_buf[guard + shift: guard + shift + W * Ns]
+    plan.rs_reduce(dev, out, scale_mode=1)
+    torch.cuda.synchronize()
+    ref = oracle.rs_reduce(W, group.shapes, grads, 1)
+    assert np.array_equal(f32_bits(out), ref.view(np.uint32))
+    ob = out_buf.cpu().numpy()
+    assert np.all(ob[: guard + shift] == 12345.0) and np.all(ob[guard + shift + W * Ns:] == 12345.0)
+    for buf in pool:          # inputs untouched
+        assert torch.all(buf[:shift] == -3) and torch.all(buf[-guard:] == -3)
+    # AG into misaligned parameter storage with guards
+    L = oracle.layout(W, group.shapes)
+    ag_bits = synth.ag_host(group, L.Ns, seed=72).reshape(-1)
+    ag_buf = torch.zeros(W * Ns + shift, dtype=torch.int16, device="cuda")
+    ag_buf[shift:] = to_dev(ag_bits).view(torch.int16)
+    bufs, params = [], []
+    for i in range(P):
+        n = W * L.c[i]
+        b = torch.full((n + shift + guard,), 0x5555, dtype=torch.int16, device="cuda")
+        bufs.append(b)
+        params.append(b[shift: shift + n].view(torch.bfloat16))
+    for engine in (T.TIDE_ENGINE_SM, T.TIDE_ENGINE_CE):
+        plan.ag_place(ag_buf[shift:].view(torch.bfloat16), params, engine=engine)
+        torch.cuda.synchronize()
+        refp = oracle.ag_copyout(W, group.shapes, ag_bits)
+        for b, p, r in zip(bufs, params, refp):
+            assert np.array_equal(bits_of(p), r)
+            assert torch.all(b[:shift] == 0x5555) and torch.all(b[-guard:] == 0x5555)
+
+
+def test_guard_bands_aligned_fast_path():
+    group = mini_sweep(8)
+    grads = synth.grads_host(group, seed=73)
+    plan = T.Plan(group.shapes, group.world)
+    n = group.world * plan.shard_numel
+    guard = 4096
+    out_buf = torch.full((n + 2 * guard,), -7.0, device="cuda")
+    out = out_buf[guard: guard + n]
+    plan.rs_reduce(grads_to_dev(group, grads), out, scale_mode=1)
+    torch.cuda.synchronize()
+    assert np.array_equal(f32_bits(out), oracle.rs_reduce(8, group.shapes, grads, 1).view(np.uint32))
+    assert torch.all(out_buf[:guard] == -7.0) and torch.all(out_buf[guard + n:] == -7.0)
+
+
+def test_pointer_table_changes_between_calls():
+    group = configs.tiny()
+    plan = T.Plan(group.shapes, group.world)
+    n = group.world * plan.shard_numel
+    outs = []
+    seeds = (81, 82, 81)
+    keep = []
+    for s in seeds:
+        g = synth.grads_host(group, seed=s)
+        dev = grads_to_dev(group, g)
+        keep.append(dev)                       # distinct buffers each call
+        out = torch.empty(n, device="cuda")
+        plan.rs_reduce(dev, out, scale_mode=1)
+        outs.append((out, g))
+    torch.cuda.synchronize()
+    for out, g in outs:
+        assert np.array_equal(f32_bits(out), oracle.rs_reduce(4, group.shapes, g, 1).view(np.uint32))
+
+
+def test_side_stream_and_empty_groups():
+    group = configs.tiny()
+    grads = synth.grads_host(group, seed=91)
+    plan = T.Plan(group.shapes, group.world)
+    s = torch.cuda.Stream()
+    dev = grads_to_dev(group, grads)
+    torch.cuda.synchronize()
+    out = torch.empty(group.world * plan.shard_numel, device="cuda")
+    with torch.cuda.stream(s):
+        plan.rs_reduce(dev, out, scale_mode=1, stream=s)
+    s.synchronize()
+    assert np.array_equal(f32_bits(out), oracle.rs_reduce(4, group.shapes, grads, 1).view(np.uint32))
+    # a group with no elements: every call is a no-op that succeeds
+    empty = configs.Group("empty", 4, ((0,), (0, 9), (7, 0)))
+    ep = T.Plan(empty.shapes, 4)
+    z = torch.empty(0, dtype=torch.bfloat16, device="cuda")
+    ep.rs_reduce([[z, z, z] for _ in range(4)], torch.empty(0, device="cuda"))
+    ep.ag_place(z, [z, z, z])
+    ep.ag_place(z, [z, z, z], engine=T.TIDE_ENGINE_CE)
+    torch.cuda.synchronize()
+    ep.check()
+
+
+def test_wrong_device_index_rejected():
+    group = configs.tiny()
+    st, h = T.tide_plan_group([(s[0], int(np.prod(s[1:]))) for s in group.shapes], 4,
+                              torch.cuda.device_count(), 0)
+    assert st in (T.TIDE_ERR_DEVICE, T.TIDE_ERR_CUDA) and h is None
+
+
+def test_workspace_is_tables_only():
+    for name in ("tiny", "wan14b"):
+        g = configs.by_name(name)
+        plan = T.Plan(g.shapes, g.world)
+        W, P = g.world, g.n_params
+        expect = plan.n_tiles * 32 + 2 * P * 8 + 4 + W * P * 8 + P * 8 + W * 8
+        assert plan.workspace_bytes == expect
