@@ -1,0 +1,575 @@
+#!/usr/bin/env python
+"""Benchmark of the TIDE hot path on B200: RS reduce + AG placement, HBM GB/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama70b]
+    python bench.py --impl reference ...          # the CPU oracle, timed on host cores
+    python bench.py --suite                       # every workload, one JSON line each
+
+A step is one pass of the hot path over one synthetic parameter group:
+tide_ag_place (SM engine) places the rank-major bf16 all-gather buffer into
+padded per-parameter storage, then tide_rs_reduce (rank order, x fl32(1/W))
+reduces the W simulated ranks' bf16 gradients into fp32 rank-major shards.
+The metric is algorithmic HBM bytes moved per second (bytes each element must
+cross HBM once: RS 2W B read per valid element + 4 B written per shard
+element; AG 2 B read per valid element + 2 B written per padded element).
+
+Timing: W untimed steps, then K steps between a barrier + synchronize on each
+side, CUDA events on the launching stream; multi-GPU runs are independent
+replicas (no collective on the data path) and report the max over ranks.
+Inputs are generated on the device by the seeded generator and exceed L2.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "RS/AG-place achieved HBM GB/s and % of B200 peak (70B layer, W=8)"
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 2 ** 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama70b")
+    ap.add_argument("--seed", type=int, default=1)
+    ap.add_argument("--max-ctas", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-budget-s", type=float, default=10.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-variants", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--interference", action="store_true",
+                    help="also run the concurrent-GEMM interference sweep")
+    ap.add_argument("--suite", action="store_true", help="one JSON line per workload")
+    ap.add_argument("--profile-small", action="store_true",
+                    help="a short run of the sweep_w8 workload, sized for an ncu capture")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------- helpers
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest(*rel):
+    h = hashlib.sha256()
+    for r in rel:
+        with open(os.path.join(ROOT, r), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+RS_SOURCES = ("fsdp2_layout_aware_b200/csrc/rs_reduce.cu", "fsdp2_layout_aware_b200/csrc/device_common.cuh")
+AG_SOURCES = ("fsdp2_layout_aware_b200/csrc/ag_place.cu", "fsdp2_layout_aware_b200/csrc/device_common.cuh")
+
+
+def ncu_traffic(kernel: str, workload: str, sources):
+    """Per-launch DRAM bytes from profiles/ncu_traffic.txt, if taken on the current source."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    digest = source_digest(*sources)
+    for line in open(path):
+        parts = line.split()
+        if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel and parts[1] == workload:
+            return float(parts[3]) if parts[2] == digest else None
+    return None
+
+
+class ClockSampler:
+    """Polls NVML for SM clock and clock-event reasons while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons = [], 0
+        self.period = period_s
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML absent: report it rather than guess
+            self.err = repr(e)
+
+    def _reasons(self):
+        nv = self.nv
+        fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        return fn(self.h)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self._reasons())
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "err", "")}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+def alg_bytes(group, L):
+    W = group.world
+    N = sum(group.numel(i) for i in range(group.n_params))
+    Npad = W * L.Ns
+    return {"rs": 2 * W * N + 4 * Npad, "ag": 2 * N + 2 * Npad, "stage": 4 * W * N,
+            "slot_rs": 2 * W * N + 4 * Npad, "N": N, "Npad": Npad}
+
+
+# --------------------------------------------------------------------------- our arm
+
+
+class Workload:
+    """Device buffers of one parameter group, plus the plan."""
+
+    def __init__(self, group, seed, device):
+        import torch
+        import synth
+        from fsdp2_layout_aware_b200 import tide as T
+        self.group = group
+        self.plan = T.Plan(group.shapes, group.world, device=device)
+        self.Ns = self.plan.shard_numel
+        W = group.world
+        self.grads = synth.dev_grads(group, seed, device=device)
+        self.ag = synth.dev_ag(group, self.Ns, seed, device=device)
+        self.out = torch.empty(W * self.Ns, dtype=torch.float32, device=device)
+        self.params = [torch.empty(self.plan.query(i)["padded_numel"], dtype=torch.bfloat16,
+                                   device=device) for i in range(group.n_params)]
+        self.slots = None
+
+    def ensure_slots(self):
+        import torch
+        if self.slots is None:
+            n = self.group.world * self.Ns
+            self.slots = [torch.empty(n, dtype=torch.bfloat16, device=self.out.device)
+                          for _ in range(self.group.world)]
+        return self.slots
+
+    def drop_slots(self):
+        self.slots = None
+
+
+def timed_calls(fn, K, stream, flush=None):
+    """Mean device time of fn() over K calls, each bracketed by events on `stream`."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    torch.cuda.synchronize()
+    for a, b in evs:
+        if flush is not None:
+            flush()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+
+def make_flush(device, nbytes):
+    import torch
+    buf = torch.empty(nbytes // 4, dtype=torch.float32, device=device)
+    return lambda: buf.zero_()
+
+
+def run_variants(wl, K, stream, peak, flush):
+    """The other hot-path modes on the same workload, each timed on its own."""
+    from fsdp2_layout_aware_b200 import tide as T
+    B = alg_bytes(wl.group, oracle_free_layout(wl))
+    out = {}
+
+    def rec(name, ms, nbytes, launches):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_of_peak": round(gbs / peak, 4),
+                     "alg_bytes": nbytes, "kernel_launches": launches}
+
+    rec("ag_place_ce", timed_calls(lambda: wl.plan.ag_place(wl.ag, wl.params, engine=T.TIDE_ENGINE_CE),
+                                   K, stream, flush), B["ag"], 0)
+    rec("rs_reduce_tree", timed_calls(lambda: wl.plan.rs_reduce(wl.grads, wl.out, order=T.TIDE_ORDER_TREE),
+                                      K, stream, flush), B["rs"], 1)
+    slots = wl.ensure_slots()
+    for eng, name in ((T.TIDE_ENGINE_SM, "sm"), (T.TIDE_ENGINE_CE, "ce")):
+        rec(f"slot_stage_{name}", timed_calls(lambda: wl.plan.rs_stage(wl.grads, slots, engine=eng),
+                                              K, stream, flush), B["stage"], 1 if eng == 0 else 0)
+    rec("slot_reduce", timed_calls(lambda: wl.plan.rs_reduce_slots(slots, wl.out), K, stream, flush),
+        B["slot_rs"], 1)
+    wl.drop_slots()
+    return out
+
+
+def oracle_free_layout(wl):
+    """Layout sizes from the plan (the product side never calls the oracle)."""
+    class L:
+        pass
+    L.Ns = wl.Ns
+    return L
+
+
+def run_e2e(wl, K, stream):
+    """Same step through the C-ABI with host buffers: H2D inputs, AG + RS, D2H results."""
+    import torch
+    g_host = [[t.cpu().pin_memory() for t in row] for row in wl.grads]
+    ag_host = wl.ag.cpu().pin_memory()
+    out_host = torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory()
+    par_host = [torch.empty(p.shape, dtype=p.dtype).pin_memory() for p in wl.params]
+    h2d = sum(t.numel() * t.element_size() for row in g_host for t in row) + ag_host.numel() * 2
+    d2h = out_host.numel() * 4 + sum(p.numel() * 2 for p in par_host)
+
+    def step():
+        for row_d, row_h in zip(wl.grads, g_host):
+            for d, h in zip(row_d, row_h):
+                d.copy_(h, non_blocking=True)
+        wl.ag.copy_(ag_host, non_blocking=True)
+        wl.plan.ag_place(wl.ag, wl.params)
+        wl.plan.rs_reduce(wl.grads, wl.out)
+        out_host.copy_(wl.out, non_blocking=True)
+        for d, h in zip(wl.params, par_host):
+            h.copy_(d, non_blocking=True)
+
+    step()
+    ms = timed_calls(step, K, stream)
+    del g_host, ag_host, out_host, par_host
+    return ms, h2d, d2h
+
+
+def cpu_baseline(group, seed, budget_s):
+    """The oracle as it stands (single thread) on a bounded prefix of the group's params.
+
+    Each sampled param is run as a one-param group over the same W (same
+    per-element work: W bf16 reads, W-1 fp32 adds, scale, one fp32 write; and
+    the copy-out), in group order until `budget_s` of oracle time is spent.
+    """
+    import numpy as np
+    import oracle
+    import synth
+    from synth import configs
+    W = group.world
+    spent, nbytes, names = 0.0, 0, []
+    for i in range(group.n_params):
+        sub = configs.Group("sample", W, (group.shapes[i],))
+        grads = [[synth.grad_host(group, seed, k, i)] for k in range(W)]
+        L = oracle.layout(W, sub.shapes)
+        ag = synth.fill_bf16(W * L.Ns, seed, synth.STREAM_AG, 0, i, group.param_sigma)
+        t0 = time.perf_counter()
+        oracle.rs_reduce(W, sub.shapes, grads, 1)
+        oracle.ag_copyout(W, sub.shapes, ag)
+        spent += time.perf_counter() - t0
+        n = sub.numel(0)
+        nbytes += (2 * W * n + 4 * W * L.Ns) + (2 * n + 2 * W * L.Ns)
+        names.append(group.names[i] if group.names else str(i))
+        del grads, ag
+        if spent >= budget_s:
+            break
+    cores = 1
+    return {"value": round(nbytes / spent / 1e9, 3), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{group.name}: params {names} (each as a one-param group, W={W}), "
+                      f"RS x fl32(1/W) + AG copy-out, {nbytes / 1e9:.2f} GB algorithmic, "
+                      f"{spent:.1f} s single-thread C oracle, generation excluded",
+            "seconds": round(spent, 2)}
+
+
+def run_interference(device, stream_main, seed, peak):
+    """Slowdown of a concurrent bf16 8192^3 GEMM vs the RS kernel's CTA count (sweep_w8 group)."""
+    import torch
+    from synth import configs
+    from fsdp2_layout_aware_b200 import tide as T
+    wl = Workload(configs.sweep(8), seed, device)
+    B = alg_bytes(wl.group, oracle_free_layout(wl))
+    a = torch.randn(8192, 8192, dtype=torch.bfloat16, device=device)
+    b = torch.randn(8192, 8192, dtype=torch.bfloat16, device=device)
+    c = torch.empty(8192, 8192, dtype=torch.bfloat16, device=device)
+    s_gemm = torch.cuda.Stream(device)
+    s_rs = torch.cuda.Stream(device)
+    n_gemm = 20
+
+    def gemm_batch():
+        for _ in range(n_gemm):
+            torch.matmul(a, b, out=c)
+
+    for _ in range(3):
+        gemm_batch()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s_gemm):
+        e0.record(s_gemm); gemm_batch(); e1.record(s_gemm)
+    torch.cuda.synchronize()
+    alone = e0.elapsed_time(e1) / n_gemm
+    res = {"gemm": "bf16 8192x8192x8192 torch.matmul (cuBLAS)", "gemm_ms_alone": round(alone, 4),
+           "rs_workload": "sweep_w8 (16 x 512x4096 params, W=8)", "points": []}
+    for ctas in (8, 16, 32, 0):
+        n_ctas = wl.plan.launch_ctas(T.K_RS, ctas)
+        rs_ms = timed_calls(lambda: wl.plan.rs_reduce(wl.grads, wl.out, max_ctas=ctas, stream=s_rs), 5, s_rs)
+        reps = int((alone * n_gemm * 1.3) / max(rs_ms, 1e-3)) + 2
+        torch.cuda.synchronize()
+        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(s_rs):
+            r0.record(s_rs)
+            for _ in range(reps):
+                wl.plan.rs_reduce(wl.grads, wl.out, max_ctas=ctas, stream=s_rs)
+            r1.record(s_rs)
+        with torch.cuda.stream(s_gemm):
+            e0.record(s_gemm); gemm_batch(); e1.record(s_gemm)
+        torch.cuda.synchronize()
+        conc = e0.elapsed_time(e1) / n_gemm
+        rs_conc = r0.elapsed_time(r1) / reps
+        res["points"].append({
+            "max_ctas": ctas, "ctas": n_ctas, "rs_ms_alone": round(rs_ms, 4),
+            "rs_GBps_alone": round(B["rs"] / (rs_ms * 1e-3) / 1e9, 1),
+            "rs_ms_concurrent": round(rs_conc, 4), "gemm_ms_concurrent": round(conc, 4),
+            "gemm_slowdown": round(conc / alone - 1.0, 4),
+            "rs_sm_ms_per_call": round(n_ctas * rs_ms, 2)})
+    del wl, a, b, c
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_workload(args, group, rank, world, device, dist_on):
+    import torch
+    from fsdp2_layout_aware_b200 import tide as T
+    peak, peak_src = load_peaks()
+    wl = Workload(group, args.seed, device)
+    B = alg_bytes(group, oracle_free_layout(wl))
+    stream = torch.cuda.current_stream(device)
+    in_bytes = 2 * B["N"] * group.world
+    flush = None if in_bytes > 4 * L2_BYTES else make_flush(device, 2 * L2_BYTES)
+
+    def step():
+        wl.plan.ag_place(wl.ag, wl.params, max_ctas=args.max_ctas)
+        wl.plan.rs_reduce(wl.grads, wl.out, max_ctas=args.max_ctas)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    wl.plan.check()
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(device.index) as clk:
+        start.record(stream)
+        for e in evs:
+            if flush is not None:
+                flush()
+            e[0].record(stream)
+            wl.plan.ag_place(wl.ag, wl.params, max_ctas=args.max_ctas)
+            e[1].record(stream)
+            wl.plan.rs_reduce(wl.grads, wl.out, max_ctas=args.max_ctas)
+            e[2].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    wl.plan.check()
+    total_ms = start.elapsed_time(end)
+    ag_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    rs_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    step_ms = ag_ms + rs_ms if flush is not None else total_ms / K
+    if dist_on:
+        t = torch.tensor([step_ms, ag_ms, rs_ms], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        step_ms, ag_ms, rs_ms = (float(x) for x in t.tolist())
+
+    step_bytes = B["ag"] + B["rs"]
+    value = world * step_bytes / (step_ms * 1e-3) / 1e9
+    rs_gbs = B["rs"] / (rs_ms * 1e-3) / 1e9
+    ag_gbs = B["ag"] / (ag_ms * 1e-3) / 1e9
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(step_ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16/f32", "data": "synthetic",
+        "config": {
+            "workload": f"{group.name} layer group, W={group.world} simulated ranks, "
+                        f"{group.n_params} params, {B['N']} elements",
+            "step": "tide_ag_place(SM) + tide_rs_reduce(rank order, x fl32(1/W))",
+            "alg_bytes_per_step": step_bytes, "max_ctas": args.max_ctas,
+            "l2": ("inputs larger than L2, no flush" if flush is None else
+                   "L2 flushed (256 MB write) before every timed step"),
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "roofline": {"bound": "hbm", "achieved": round(rs_gbs, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(rs_gbs / peak, 4), "peak_source": f"{peak_src} hbm_gbs",
+                     "kernel": "rs_reduce_kernel", "alg_bytes_per_launch": B["rs"],
+                     "avg_launch_ms": round(rs_ms, 4),
+                     "traffic": ncu_traffic("rs_reduce_kernel", group.name, RS_SOURCES)},
+        "kernels": {
+            "rs_reduce_kernel": {"ms": round(rs_ms, 4), "GB/s": round(rs_gbs, 1),
+                                 "frac_of_peak": round(rs_gbs / peak, 4), "alg_bytes": B["rs"],
+                                 "ctas": wl.plan.launch_ctas(T.K_RS, args.max_ctas)},
+            "ag_place_kernel": {"ms": round(ag_ms, 4), "GB/s": round(ag_gbs, 1),
+                                "frac_of_peak": round(ag_gbs / peak, 4), "alg_bytes": B["ag"],
+                                "ctas": wl.plan.launch_ctas(T.K_AG, args.max_ctas),
+                                "traffic": ncu_traffic("ag_place_kernel", group.name, AG_SOURCES)}},
+        "gpu_launches": 2 * K,
+        "clocks": clk.summary(),
+        "workspace_bytes": wl.plan.workspace_bytes,
+    }
+    if not args.no_variants:
+        res["variants"] = run_variants(wl, max(3, min(K, 20)), stream, peak, flush)
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = run_e2e(wl, max(1, args.e2e_steps), stream)
+        if dist_on:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        res["e2e"] = {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                      "ms_per_step": round(e2e_ms, 3), "steps": max(1, args.e2e_steps),
+                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    del wl
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_ours(args):
+    import torch
+    from synth import configs
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    try:
+        if args.suite:
+            names = configs.ALL
+        elif args.profile_small:
+            names = ("sweep_w8",)
+        else:
+            names = (args.workload,)
+        for name in names:
+            res = bench_workload(args, configs.by_name(name), rank, world, device, dist_on)
+            if rank == 0 and world == 1 and not args.no_cpu and not args.profile_small:
+                res["cpu_baseline"] = cpu_baseline(configs.by_name(name), args.seed, args.cpu_budget_s)
+            if args.interference and name == names[0]:
+                res["interference"] = run_interference(device, torch.cuda.current_stream(), args.seed,
+                                                       load_peaks()[0])
+            if rank == 0:
+                print(json.dumps(res), flush=True)
+    finally:
+        if dist_on:
+            torch.distributed.destroy_process_group()
+
+
+# --------------------------------------------------------------------------- reference arm
+
+
+def run_reference(args):
+    """The CPU oracle as it stands, on host cores, on a bounded sample of the workload."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    import synth
+    from synth import configs
+    group = configs.by_name(args.workload)
+    W = group.world
+    # per step: the largest param of the group that is at most 1/8 of the group, as a one-param group
+    total = sum(group.numel(i) for i in range(group.n_params))
+    cand = [i for i in range(group.n_params) if group.numel(i) <= total / 8] or [0]
+    i = max(cand, key=group.numel)
+    sub = configs.Group("sample", W, (group.shapes[i],))
+    grads = [[synth.grad_host(group, args.seed, k, i)] for k in range(W)]
+    L = oracle.layout(W, sub.shapes)
+    ag = synth.fill_bf16(W * L.Ns, args.seed, synth.STREAM_AG, 0, i, group.param_sigma)
+    n = sub.numel(0)
+    step_bytes = (2 * W * n + 4 * W * L.Ns) + (2 * n + 2 * W * L.Ns)
+
+    def step():
+        oracle.ag_copyout(W, sub.shapes, ag)
+        oracle.rs_reduce(W, sub.shapes, grads, 1)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = step_bytes / dt / 1e9
+    name = group.names[i] if group.names else str(i)
+    sample = (f"{group.name}: param {name} {group.shapes[i]} as a one-param group over W={W}; "
+              f"AG copy-out + RS x fl32(1/W), {step_bytes / 1e9:.3f} GB algorithmic per step")
+    res = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s",
+           "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "bf16/f32", "data": "synthetic",
+           "config": {"workload": f"{group.name} layer group, W={W} simulated ranks, "
+                                  f"{group.n_params} params, {total} elements",
+                      "sample": sample},
+           "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

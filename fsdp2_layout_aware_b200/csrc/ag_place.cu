@@ -79,9 +79,11 @@ __global__ void __launch_bounds__(kThreads) slot_stage_kernel(const StageParams 
         __syncthreads();
         const tide_tile_t tl = s_tile;
         const bool param_ok = tl.param >= 0 && tl.param < a.n_params;
+        // (an all-pad tile copies nothing; its gradient offset may lie past the tensor)
         const bool ok = param_ok && tl.n_valid >= 0 && tl.n_valid <= tl.n_total &&
-                        tl.src_off >= 0 && tl.src_off + tl.n_valid <= a.numel[tl.param] &&
-                        tl.dst_off >= 0 && tl.dst_off + tl.n_valid <= a.slot_numel;
+                        (tl.n_valid == 0 ||
+                         (tl.src_off >= 0 && tl.src_off + tl.n_valid <= a.numel[tl.param] &&
+                          tl.dst_off >= 0 && tl.dst_off + tl.n_valid <= a.slot_numel));
         if (!ok) {
             if (threadIdx.x == 0) atomicOr(a.err, TIDE_KCHECK_TILE);
             continue;

@@ -159,9 +159,10 @@ __global__ void __launch_bounds__(kThreads) rs_reduce_kernel(const RsParams a) {
         const bool param_ok = tl.param >= 0 && tl.param < a.n_params;
         const int64_t src_off = SLOT ? tl.dst_off : tl.src_off;
         const int64_t src_lim = SLOT ? a.slot_numel : (param_ok ? a.numel[tl.param] : -1);
+        // (an all-pad tile reads nothing, so its source offset may lie past the tensor)
         const bool ok = param_ok && tl.n_valid >= 0 && tl.n_valid <= tl.n_total &&
                         tl.dst_off >= 0 && tl.dst_off + tl.n_total <= a.out_numel &&
-                        src_off >= 0 && src_off + tl.n_valid <= src_lim;
+                        (tl.n_valid == 0 || (src_off >= 0 && src_off + tl.n_valid <= src_lim));
         if (!ok) {
             if (tid == 0) atomicOr(a.err, TIDE_KCHECK_TILE);
             continue;
