@@ -124,6 +124,7 @@ cudaError_t launch_ag_place(const tide_plan* p, const uint16_t* ag, int64_t ag_n
     a.numel = p->d_numel;
     a.n_params = p->n_params;
     a.err = p->d_err;
+    (void)cudaGetLastError();  // drop an error left by an earlier failed runtime call
     ag_place_kernel<<<grid, kThreads, 0, stream>>>(a);
     return cudaGetLastError();
 }
@@ -142,6 +143,7 @@ cudaError_t launch_slot_stage(const tide_plan* p, const void* const* d_grad_tab,
     a.world = p->world;
     a.n_params = p->n_params;
     a.err = p->d_err;
+    (void)cudaGetLastError();  // drop an error left by an earlier failed runtime call
     slot_stage_kernel<<<grid, kThreads, 0, stream>>>(a);
     return cudaGetLastError();
 }

@@ -45,8 +45,14 @@ void free_device(tide_plan* p) {
 
 tide_status_t upload(tide_plan* p) {
     int prev = -1;
-    if (cudaGetDevice(&prev) != cudaSuccess) return TIDE_ERR_CUDA;
-    if (cudaSetDevice(p->device) != cudaSuccess) return TIDE_ERR_DEVICE;
+    if (cudaGetDevice(&prev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return TIDE_ERR_CUDA;
+    }
+    if (cudaSetDevice(p->device) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return TIDE_ERR_DEVICE;
+    }
     tide_status_t st = TIDE_OK;
     int64_t total = 0;
     const int64_t W = p->world, P = p->n_params, T = (int64_t)p->tiles.size();
@@ -88,6 +94,7 @@ tide_status_t upload(tide_plan* p) {
     p->workspace_bytes = total;
     if (st != TIDE_OK) free_device(p);
     cudaSetDevice(prev);
+    if (st != TIDE_OK) (void)cudaGetLastError();  // leave no stale error for later launches
     return st;
 }
 

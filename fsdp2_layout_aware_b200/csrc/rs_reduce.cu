@@ -260,6 +260,7 @@ cudaError_t launch_rs_reduce(const tide_plan* p, const void* const* d_src_tab, b
     a.scale = scale;
     a.do_scale = do_scale ? 1 : 0;
     a.err = p->d_err;
+    (void)cudaGetLastError();  // drop an error left by an earlier failed runtime call
     select(p->world, slot, order)<<<grid, kThreads, 0, stream>>>(a);
     return cudaGetLastError();
 }

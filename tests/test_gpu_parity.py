@@ -292,6 +292,10 @@ def test_wrong_device_index_rejected():
     st, h = T.tide_plan_group([(s[0], int(np.prod(s[1:]))) for s in group.shapes], 4,
                               torch.cuda.device_count(), 0)
     assert st in (T.TIDE_ERR_DEVICE, T.TIDE_ERR_CUDA) and h is None
+    # the failed call leaves no stale runtime error behind: the next launch succeeds
+    grads = synth.grads_host(group, seed=92)
+    out, _, _ = run_rs(group, grads, scale=1)
+    assert np.array_equal(f32_bits(out), oracle.rs_reduce(4, group.shapes, grads, 1).view(np.uint32))
 
 
 def test_workspace_is_tables_only():
