@@ -19,7 +19,7 @@ BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libtide.so")
 INCLUDE = os.path.join(ROOT, "include")
 
-SOURCES = ["plan.cpp", "api.cpp", "ce.cpp", "rs_reduce.cu", "ag_place.cu"]
+SOURCES = ["plan.cpp", "api.cpp", "ce.cpp", "rs_reduce.cu", "ag_place.cu", "rs_reduce_noalloc.cu"]
 HEADERS = ["tide_internal.h", "device_common.cuh"]
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",

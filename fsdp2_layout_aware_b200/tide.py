@@ -34,6 +34,7 @@ TIDE_SCALE_INV_WORLD = 1
 TIDE_PLAN_HOST_ONLY = 1
 TIDE_MAX_WORLD = 256
 TIDE_TILE_ELEMS = 8192
+TIDE_NOALLOC_SCRATCH_BYTES = 1 << 20
 
 K_RS, K_AG, K_STAGE, K_SLOT_RS = 0, 1, 2, 3
 
@@ -70,6 +71,8 @@ _SIGNATURES = {
                               _i32, _i32, _vp]),
     "tide_rs_stage": (_i32, [_vp, _P(_vp), _P(_i64), _P(_vp), _i64, _i32, _i32, _vp]),
     "tide_rs_reduce_slots": (_i32, [_vp, _P(_vp), _i64, _vp, _i64, _i32, _i32, _i32, _vp]),
+    "tide_rs_reduce_noalloc": (_i32, [_P(tide_param_t), _i32, _i32, _P(_vp), _P(_i64), _vp, _i64,
+                                      _i32, _i32, _vp]),
     "tide_plan_check": (_i32, [_vp, _vp]),
     "tide_launch_ctas": (_i32, [_vp, _i32, _i32, _P(_i32)]),
     "tide_status_string": (ctypes.c_char_p, [_i32]),
@@ -186,6 +189,17 @@ def tide_rs_reduce_slots(plan, slots, slot_numel: int, out: int, out_numel: int,
     slot_arr = _ptr_array(slots) if slots is not None else None
     return lib().tide_rs_reduce_slots(plan, slot_arr, slot_numel, out, out_numel, scale_mode,
                                       order, max_ctas, stream)
+
+
+def tide_rs_reduce_noalloc(params, world: int, grads, grad_numel, out: int, out_numel: int,
+                           scale_mode: int, max_ctas: int, stream: int) -> int:
+    """params: sequence of (dim0, inner); grads: W*P device pointers, index k*P + i."""
+    arr = (tide_param_t * max(1, len(params)))()
+    for j, (d0, inner) in enumerate(params):
+        arr[j].dim0, arr[j].inner = int(d0), int(inner)
+    return lib().tide_rs_reduce_noalloc(arr, len(params), world, _ptr_array(grads),
+                                        _i64_array(grad_numel), out, out_numel, scale_mode,
+                                        max_ctas, stream)
 
 
 def tide_plan_check(plan, stream: int) -> int:

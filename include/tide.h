@@ -72,6 +72,7 @@ enum { TIDE_PLAN_HOST_ONLY = 1 }; /* flag: build the tables on the host only (no
 
 #define TIDE_MAX_WORLD 256
 #define TIDE_TILE_ELEMS 8192
+#define TIDE_NOALLOC_SCRATCH_BYTES (1 << 20)
 
 /* One parameter: dim 0 and the product of the remaining dims (1 for a 1-D param). */
 typedef struct {
@@ -193,6 +194,34 @@ TIDE_API tide_status_t tide_rs_reduce_slots(const tide_plan_t* plan, const void*
  * (the tile is skipped, nothing outside the buffers is touched), else TIDE_OK.
  */
 TIDE_API tide_status_t tide_plan_check(tide_plan_t* plan, void* stream);
+
+/*
+ * Allocation-free rank-order reduction.  The paper has no counterpart: this
+ * entry point exists for callers that cannot allocate device memory, which
+ * tide_plan_group does.  Examples: a training runtime whose caching allocator
+ * has already reserved the GPU's memory for its own arena (a foreign
+ * cudaMalloc then fails or fragments it), or a hot loop that cannot afford the
+ * device-wide synchronisation cudaMalloc/cudaFree may cause.
+ * Computes exactly what tide_rs_reduce computes with slots == NULL and
+ * TIDE_ORDER_RANK (same bits), for the group given directly by params /
+ * n_params / world instead of a plan; grads, grad_numel, out, out_numel,
+ * scale_mode, max_ctas and stream mean what they mean there.
+ * It calls no cudaMalloc, cudaFree or other allocating routine.  Its tables
+ * (32*P + 8*W*P bytes) live in one file-scope device array of
+ * TIDE_NOALLOC_SCRATCH_BYTES (1 MiB) that every GPU loading this library
+ * holds until the process exits; a larger group is rejected with
+ * TIDE_ERR_SIZE before anything is enqueued.  The first call on each device
+ * looks up that device's address of the array; make that first call before
+ * any stream capture.  Every call rewrites the tables its kernel reads, so no
+ * state carries over, but all calls share the one array: calls that may
+ * overlap on the GPU (on streams the caller does not order) race and must not
+ * be issued.
+ */
+TIDE_API tide_status_t tide_rs_reduce_noalloc(const tide_param_t* params, int32_t n_params,
+                                              int32_t world, const void* const* grads,
+                                              const int64_t* grad_numel, float* out,
+                                              int64_t out_numel, int32_t scale_mode,
+                                              int32_t max_ctas, void* stream);
 
 /* The number of CTAs a kernel call with this max_ctas would launch.
  * kernel: 0 = RS reduce, 1 = AG place, 2 = Slot-Reuse stage, 3 = slot reduce. */
