@@ -243,6 +243,11 @@ def run_variants(wl, K, stream, peak, flush):
                                    K, stream, flush), B["ag"], 0)
     rec("rs_reduce_tree", timed_calls(lambda: wl.plan.rs_reduce(wl.grads, wl.out, order=T.TIDE_ORDER_TREE),
                                       K, stream, flush), B["rs"], 1)
+    tma_plan = T.Plan(wl.group.shapes, wl.group.world, device=wl.out.device, tma=True)
+    rec("rs_reduce_tma", timed_calls(lambda: tma_plan.rs_reduce(wl.grads, wl.out), K, stream, flush),
+        B["rs"], 1)
+    out["rs_reduce_tma"]["kernel"] = ["lsu", "ag", "stage", "slot_lsu", "tma", "slot_tma"][tma_plan.last_launch()[0]]
+    tma_plan.close()
     slots = wl.ensure_slots()
     for eng, name in ((T.TIDE_ENGINE_SM, "sm"), (T.TIDE_ENGINE_CE, "ce")):
         rec(f"slot_stage_{name}", timed_calls(lambda: wl.plan.rs_stage(wl.grads, slots, engine=eng),
@@ -324,56 +329,75 @@ def cpu_baseline(group, seed, budget_s):
             "seconds": round(spent, 2)}
 
 
-def run_interference(device, stream_main, seed, peak):
-    """Slowdown of a concurrent bf16 8192^3 GEMM vs the RS kernel's CTA count (sweep_w8 group)."""
+def run_interference(device, seed):
+    """Slowdown of a concurrent bf16 8192^3 GEMM vs the RS kernel's CTA count (sweep_w8 group).
+
+    Per point: the GEMM batch alone, then concurrently with back-to-back RS
+    launches on a second stream (started first, enough of them to outlast the
+    GEMMs), then alone again; slowdown = concurrent / mean(alone) - 1.  Done
+    for the load/store RS kernel and for the bulk-copy (TMA) one.
+    """
     import torch
     from synth import configs
     from fsdp2_layout_aware_b200 import tide as T
-    wl = Workload(configs.sweep(8), seed, device)
-    B = alg_bytes(wl.group, oracle_free_layout(wl))
+    group = configs.sweep(8)
+    wl = Workload(group, seed, device)
+    plans = {"lsu": wl.plan, "tma": T.Plan(group.shapes, group.world, device=device, tma=True)}
+    B = alg_bytes(group, oracle_free_layout(wl))
     a = torch.randn(8192, 8192, dtype=torch.bfloat16, device=device)
     b = torch.randn(8192, 8192, dtype=torch.bfloat16, device=device)
     c = torch.empty(8192, 8192, dtype=torch.bfloat16, device=device)
     s_gemm = torch.cuda.Stream(device)
     s_rs = torch.cuda.Stream(device)
-    n_gemm = 20
+    n_gemm = 40
 
     def gemm_batch():
         for _ in range(n_gemm):
             torch.matmul(a, b, out=c)
 
-    for _ in range(3):
-        gemm_batch()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(s_gemm):
-        e0.record(s_gemm); gemm_batch(); e1.record(s_gemm)
-    torch.cuda.synchronize()
-    alone = e0.elapsed_time(e1) / n_gemm
-    res = {"gemm": "bf16 8192x8192x8192 torch.matmul (cuBLAS)", "gemm_ms_alone": round(alone, 4),
-           "rs_workload": "sweep_w8 (16 x 512x4096 params, W=8)", "points": []}
-    for ctas in (8, 16, 32, 0):
-        n_ctas = wl.plan.launch_ctas(T.K_RS, ctas)
-        rs_ms = timed_calls(lambda: wl.plan.rs_reduce(wl.grads, wl.out, max_ctas=ctas, stream=s_rs), 5, s_rs)
-        reps = int((alone * n_gemm * 1.3) / max(rs_ms, 1e-3)) + 2
+    def gemm_alone():
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
-        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(s_rs):
-            r0.record(s_rs)
-            for _ in range(reps):
-                wl.plan.rs_reduce(wl.grads, wl.out, max_ctas=ctas, stream=s_rs)
-            r1.record(s_rs)
         with torch.cuda.stream(s_gemm):
             e0.record(s_gemm); gemm_batch(); e1.record(s_gemm)
         torch.cuda.synchronize()
-        conc = e0.elapsed_time(e1) / n_gemm
-        rs_conc = r0.elapsed_time(r1) / reps
-        res["points"].append({
-            "max_ctas": ctas, "ctas": n_ctas, "rs_ms_alone": round(rs_ms, 4),
-            "rs_GBps_alone": round(B["rs"] / (rs_ms * 1e-3) / 1e9, 1),
-            "rs_ms_concurrent": round(rs_conc, 4), "gemm_ms_concurrent": round(conc, 4),
-            "gemm_slowdown": round(conc / alone - 1.0, 4),
-            "rs_sm_ms_per_call": round(n_ctas * rs_ms, 2)})
+        return e0.elapsed_time(e1) / n_gemm
+
+    for _ in range(5):
+        gemm_alone()
+    res = {"gemm": "bf16 8192x8192x8192 torch.matmul (cuBLAS), 40 per batch",
+           "rs_workload": "sweep_w8 (16 x 512x4096 params, W=8), rank order, x fl32(1/W)",
+           "points": []}
+    for kind, plan in plans.items():
+        for ctas in (8, 16, 32, 0):
+            rs_ms = timed_calls(lambda: plan.rs_reduce(wl.grads, wl.out, max_ctas=ctas, stream=s_rs), 5, s_rs)
+            kernel, n_ctas = plan.last_launch()
+            before = gemm_alone()
+            reps = int((before * n_gemm * 1.2) / max(rs_ms, 1e-3)) + 2
+            torch.cuda.synchronize()
+            r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with ClockSampler(device.index) as clk:
+                with torch.cuda.stream(s_rs):
+                    r0.record(s_rs)
+                    for _ in range(reps):
+                        plan.rs_reduce(wl.grads, wl.out, max_ctas=ctas, stream=s_rs)
+                    r1.record(s_rs)
+                with torch.cuda.stream(s_gemm):
+                    e0.record(s_gemm); gemm_batch(); e1.record(s_gemm)
+                torch.cuda.synchronize()
+            conc = e0.elapsed_time(e1) / n_gemm
+            after = gemm_alone()
+            alone = 0.5 * (before + after)
+            res["points"].append({
+                "rs_kernel": kind, "max_ctas": ctas, "ctas": n_ctas, "rs_ms_alone": round(rs_ms, 4),
+                "rs_GBps_alone": round(B["rs"] / (rs_ms * 1e-3) / 1e9, 1),
+                "rs_ms_concurrent": round(r0.elapsed_time(r1) / reps, 4),
+                "gemm_ms_alone": round(alone, 4), "gemm_ms_concurrent": round(conc, 4),
+                "gemm_slowdown": round(conc / alone - 1.0, 4),
+                "rs_cta_ms_per_call": round(n_ctas * rs_ms, 2),
+                "sm_mhz_concurrent": clk.summary().get("sm_mhz")})
+    plans["tma"].close()
     del wl, a, b, c
     torch.cuda.empty_cache()
     return res
@@ -419,6 +443,7 @@ def bench_workload(args, group, rank, world, device, dist_on):
     if dist_on:
         torch.distributed.barrier()
     wl.plan.check()
+    rs_kernel, rs_ctas = wl.plan.last_launch()
     total_ms = start.elapsed_time(end)
     ag_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     rs_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
@@ -452,7 +477,7 @@ def bench_workload(args, group, rank, world, device, dist_on):
         "kernels": {
             "rs_reduce_kernel": {"ms": round(rs_ms, 4), "GB/s": round(rs_gbs, 1),
                                  "frac_of_peak": round(rs_gbs / peak, 4), "alg_bytes": B["rs"],
-                                 "ctas": wl.plan.launch_ctas(T.K_RS, args.max_ctas)},
+                                 "ctas": rs_ctas, "kernel_id": rs_kernel},
             "ag_place_kernel": {"ms": round(ag_ms, 4), "GB/s": round(ag_gbs, 1),
                                 "frac_of_peak": round(ag_gbs / peak, 4), "alg_bytes": B["ag"],
                                 "ctas": wl.plan.launch_ctas(T.K_AG, args.max_ctas),
@@ -502,8 +527,7 @@ def run_ours(args):
             if rank == 0 and world == 1 and not args.no_cpu and not args.profile_small:
                 res["cpu_baseline"] = cpu_baseline(configs.by_name(name), args.seed, args.cpu_budget_s)
             if args.interference and name == names[0]:
-                res["interference"] = run_interference(device, torch.cuda.current_stream(), args.seed,
-                                                       load_peaks()[0])
+                res["interference"] = run_interference(device, args.seed)
             if rank == 0:
                 print(json.dumps(res), flush=True)
     finally:

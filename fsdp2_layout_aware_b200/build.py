@@ -19,8 +19,9 @@ BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libtide.so")
 INCLUDE = os.path.join(ROOT, "include")
 
-SOURCES = ["plan.cpp", "api.cpp", "ce.cpp", "rs_reduce.cu", "ag_place.cu", "rs_reduce_noalloc.cu"]
-HEADERS = ["tide_internal.h", "device_common.cuh"]
+SOURCES = ["plan.cpp", "api.cpp", "ce.cpp", "rs_reduce.cu", "rs_reduce_tma.cu", "ag_place.cu",
+           "rs_reduce_noalloc.cu"]
+HEADERS = ["tide_internal.h", "device_common.cuh", "reduce_ranks.cuh", "tma.cuh"]
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
               "--fmad=false", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall", "-Xcompiler", "-fvisibility=hidden",
@@ -34,29 +35,31 @@ def _stale(target: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(verbose: bool = False, ptxas_verbose: bool = False, force: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(verbose: bool = False, ptxas_verbose: bool = False, force: bool = False,
+          defines=(), build_dir: str = BUILD, lib_path: str = LIB) -> str:
+    """Compile (incrementally) and link; `defines` are extra -D tuning macros."""
+    os.makedirs(build_dir, exist_ok=True)
     headers = [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(INCLUDE, "tide.h")]
     objs = []
     for src in SOURCES:
         path = os.path.join(CSRC, src)
-        obj = os.path.join(BUILD, src + ".o")
+        obj = os.path.join(build_dir, src + ".o")
         objs.append(obj)
         if not force and not _stale(obj, [path] + headers + [__file__]):
             continue
-        cmd = ["nvcc", *NVCC_FLAGS, "-c", path, "-o", obj]
+        cmd = ["nvcc", *NVCC_FLAGS, *[f"-D{d}" for d in defines], "-c", path, "-o", obj]
         if ptxas_verbose and src.endswith(".cu"):
             cmd[1:1] = ["-Xptxas", "-v"]
         if verbose:
             print(" ".join(cmd), flush=True)
         subprocess.run(cmd, check=True)
-    if force or _stale(LIB, objs):
+    if force or _stale(lib_path, objs):
         cmd = ["nvcc", "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-cudart", "static",
-               "-o", LIB, *objs]
+               "-o", lib_path, *objs]
         if verbose:
             print(" ".join(cmd), flush=True)
         subprocess.run(cmd, check=True)
-    return LIB
+    return lib_path
 
 
 if __name__ == "__main__":

@@ -109,6 +109,9 @@ tide_status_t sync_table(PtrTable& t, const void* const* ptrs, int64_t n, cudaSt
         std::memcmp(t.host.data(), ptrs, sizeof(void*) * (size_t)n) == 0)
         return TIDE_OK;
     t.host.assign(ptrs, ptrs + n);
+    t.aligned16 = true;
+    for (int64_t j = 0; j < n; ++j)
+        if ((reinterpret_cast<uintptr_t>(ptrs[j]) & 15) != 0) t.aligned16 = false;
     // Pageable source: the runtime stages it before returning, so the host
     // mirror may change afterwards; the device copy is stream-ordered.
     cudaError_t e = cudaMemcpyAsync(t.dev, t.host.data(), sizeof(void*) * (size_t)n,
@@ -125,19 +128,48 @@ int grid_for(const tide_plan* p, int kernel, int32_t max_ctas) {
 
 float inv_world(int32_t world) { return 1.0f / (float)world; }
 
+// The bulk-copy (TMA) reduction runs when the plan asks for it and every tile
+// starts on an 8-element boundary with 16-byte aligned sources and output;
+// otherwise the load/store kernel runs.
+bool use_tma(const tide_plan* p, const PtrTable& src, const float* out, int kernel) {
+    return (p->flags & TIDE_PLAN_TMA) && p->tiles_aligned8 && p->blocks_per_sm[kernel] > 0 &&
+           src.aligned16 && (reinterpret_cast<uintptr_t>(out) & 15) == 0;
+}
+
+// Launch the reduction over `tab` on the chosen kernel and record it in the plan.
+cudaError_t launch_reduce(tide_plan* p, PtrTable& tab, bool slot, int64_t bound, float* out,
+                          int64_t out_numel, int32_t scale_mode, int32_t order, int32_t max_ctas,
+                          cudaStream_t s) {
+    const int k_tma = slot ? K_SLOT_RS_TMA : K_RS_TMA, k_lsu = slot ? K_SLOT_RS : K_RS;
+    const bool tma = use_tma(p, tab, out, k_tma);
+    const int kernel = tma ? k_tma : k_lsu;
+    const int grid = grid_for(p, kernel, max_ctas);
+    p->last_kernel = kernel;
+    p->last_ctas = grid;
+    const float scale = inv_world(p->world);
+    const bool do_scale = scale_mode == TIDE_SCALE_INV_WORLD;
+    return tma ? tide::launch_rs_reduce_tma(p, tab.dev, slot, bound, out, out_numel, scale, do_scale,
+                                            order, grid, s)
+               : tide::launch_rs_reduce(p, tab.dev, slot, bound, out, out_numel, scale, do_scale,
+                                        order, grid, s);
+}
+
 tide_status_t stage_impl(tide_plan* p, const void* const* grads, void* const* slots,
                          int64_t slot_numel, int32_t engine, int32_t max_ctas, cudaStream_t s) {
     if (p->tiles.empty()) return TIDE_OK;
     cudaError_t e;
     if (engine == TIDE_ENGINE_CE) {
+        p->last_kernel = -1;
+        p->last_ctas = 0;
         e = tide::ce_slot_stage(p, grads, slots, s);
     } else {
         tide_status_t st = sync_table(p->grad_tab, grads, (int64_t)p->world * p->n_params, s);
         if (st == TIDE_OK)
             st = sync_table(p->slot_tab, const_cast<const void* const*>(slots), p->world, s);
         if (st != TIDE_OK) return st;
-        e = tide::launch_slot_stage(p, p->grad_tab.dev, p->slot_tab.dev, slot_numel,
-                                    grid_for(p, K_STAGE, max_ctas), s);
+        p->last_kernel = K_STAGE;
+        p->last_ctas = grid_for(p, K_STAGE, max_ctas);
+        e = tide::launch_slot_stage(p, p->grad_tab.dev, p->slot_tab.dev, slot_numel, p->last_ctas, s);
     }
     return e == cudaSuccess ? TIDE_OK : TIDE_ERR_CUDA;
 }
@@ -148,9 +180,8 @@ tide_status_t reduce_slots_impl(tide_plan* p, void* const* slots, int64_t slot_n
     if (p->tiles.empty()) return TIDE_OK;
     tide_status_t st = sync_table(p->slot_tab, const_cast<const void* const*>(slots), p->world, s);
     if (st != TIDE_OK) return st;
-    cudaError_t e = tide::launch_rs_reduce(p, p->slot_tab.dev, true, slot_numel, out, out_numel,
-                                           inv_world(p->world), scale_mode == TIDE_SCALE_INV_WORLD,
-                                           order, grid_for(p, K_SLOT_RS, max_ctas), s);
+    cudaError_t e = launch_reduce(p, p->slot_tab, true, slot_numel, out, out_numel, scale_mode, order,
+                                  max_ctas, s);
     return e == cudaSuccess ? TIDE_OK : TIDE_ERR_CUDA;
 }
 
@@ -179,12 +210,16 @@ extern "C" tide_status_t tide_ag_place(const tide_plan_t* cplan, const void* ag_
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e;
     if (engine == TIDE_ENGINE_CE) {
+        p->last_kernel = -1;
+        p->last_ctas = 0;
         e = tide::ce_ag_place(p, static_cast<const uint16_t*>(ag_buf), param_storage, s);
     } else {
         if ((st = sync_table(p->param_tab, const_cast<const void* const*>(param_storage), P, s)) != TIDE_OK)
             return st;
+        p->last_kernel = K_AG;
+        p->last_ctas = grid_for(p, K_AG, max_ctas);
         e = tide::launch_ag_place(p, static_cast<const uint16_t*>(ag_buf), ag_numel, p->param_tab.dev,
-                                  grid_for(p, K_AG, max_ctas), s);
+                                  p->last_ctas, s);
     }
     return e == cudaSuccess ? TIDE_OK : TIDE_ERR_CUDA;
 }
@@ -215,9 +250,7 @@ extern "C" tide_status_t tide_rs_reduce(const tide_plan_t* cplan, const void* co
         return reduce_slots_impl(p, slots, slot_numel, out, out_numel, scale_mode, order, max_ctas, s);
     }
     if ((st = sync_table(p->grad_tab, grads, W * P, s)) != TIDE_OK) return st;
-    cudaError_t e = tide::launch_rs_reduce(p, p->grad_tab.dev, false, 0, out, out_numel,
-                                           inv_world(p->world), scale_mode == TIDE_SCALE_INV_WORLD,
-                                           order, grid_for(p, K_RS, max_ctas), s);
+    cudaError_t e = launch_reduce(p, p->grad_tab, false, 0, out, out_numel, scale_mode, order, max_ctas, s);
     return e == cudaSuccess ? TIDE_OK : TIDE_ERR_CUDA;
 }
 

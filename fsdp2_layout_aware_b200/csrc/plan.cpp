@@ -88,8 +88,11 @@ tide_status_t upload(tide_plan* p) {
         p->blocks_per_sm[K_SLOT_RS] = tide::rs_blocks_per_sm(p->world, true, TIDE_ORDER_RANK);
         p->blocks_per_sm[K_AG] = tide::ag_blocks_per_sm();
         p->blocks_per_sm[K_STAGE] = tide::stage_blocks_per_sm();
-        for (int k = 0; k < K_COUNT; ++k)
+        for (int k = 0; k < K_RS_TMA; ++k)
             if (p->blocks_per_sm[k] <= 0) st = TIDE_ERR_CUDA;
+        // 0 here (not enough shared memory) only disables the bulk-copy path
+        p->blocks_per_sm[K_RS_TMA] = p->blocks_per_sm[K_SLOT_RS_TMA] = tide::rs_tma_blocks_per_sm(p->world);
+        (void)cudaGetLastError();
     }
     p->workspace_bytes = total;
     if (st != TIDE_OK) free_device(p);
@@ -107,7 +110,7 @@ extern "C" tide_status_t tide_plan_group(const tide_param_t* params, int32_t n_p
     *out_plan = nullptr;
     if (n_params < 0 || (n_params > 0 && params == nullptr)) return TIDE_ERR_INVALID_ARG;
     if (world < 1 || world > TIDE_MAX_WORLD) return TIDE_ERR_INVALID_ARG;
-    if ((flags & ~(uint32_t)TIDE_PLAN_HOST_ONLY) != 0) return TIDE_ERR_INVALID_ARG;
+    if ((flags & ~(uint32_t)(TIDE_PLAN_HOST_ONLY | TIDE_PLAN_TMA)) != 0) return TIDE_ERR_INVALID_ARG;
     if (!(flags & TIDE_PLAN_HOST_ONLY) && device < 0) return TIDE_ERR_DEVICE;
 
     tide_plan* p = new (std::nothrow) tide_plan;
@@ -154,6 +157,7 @@ extern "C" tide_status_t tide_plan_group(const tide_param_t* params, int32_t n_p
                     t.rank = (int32_t)r;
                     t.n_total = (int32_t)std::min<int64_t>(TIDE_TILE_ELEMS, c - e0);
                     t.n_valid = (int32_t)std::min<int64_t>(t.n_total, std::max<int64_t>(0, valid - e0));
+                    if ((t.src_off & 7) != 0 || (t.dst_off & 7) != 0) p->tiles_aligned8 = false;
                     p->tiles.push_back(t);
                 }
             }
@@ -227,10 +231,22 @@ extern "C" tide_status_t tide_launch_ctas(const tide_plan_t* plan, int32_t kerne
     if (plan->flags & TIDE_PLAN_HOST_ONLY) return TIDE_ERR_DEVICE;
     int64_t units = (int64_t)plan->tiles.size();
     if (kernel == K_STAGE) units *= plan->world;
+    if ((kernel == K_RS_TMA || kernel == K_SLOT_RS_TMA) && plan->blocks_per_sm[kernel] <= 0) {
+        *ctas = 0;
+        return TIDE_OK;
+    }
     int64_t grid = (int64_t)plan->blocks_per_sm[kernel] * plan->sm_count;
     if (max_ctas > 0) grid = std::min<int64_t>(grid, max_ctas);
     grid = std::min(grid, units);
     *ctas = (int32_t)std::max<int64_t>(grid, 0);
+    return TIDE_OK;
+}
+
+extern "C" tide_status_t tide_plan_last_launch(const tide_plan_t* plan, int32_t* kernel,
+                                               int32_t* ctas) {
+    if (plan == nullptr || kernel == nullptr || ctas == nullptr) return TIDE_ERR_INVALID_ARG;
+    *kernel = plan->last_kernel;
+    *ctas = plan->last_ctas;
     return TIDE_OK;
 }
 

@@ -27,7 +27,15 @@
 // adds adjacent ranks pairwise inside each group of G and merges group sums
 // with a binary counter (a pairwise tree over groups).
 #include "device_common.cuh"
+#include "reduce_ranks.cuh"
 #include "tide_internal.h"
+
+#ifndef TIDE_RS_U8
+#define TIDE_RS_U8 1        // 16-byte vectors per thread per step when W > 4
+#endif
+#ifndef TIDE_RS_PREFETCH
+#define TIDE_RS_PREFETCH 0  // prefetch the tile this many grid strides ahead into L2 (0 = off)
+#endif
 
 namespace tide {
 namespace {
@@ -46,101 +54,6 @@ struct RsParams {
     int32_t do_scale;
     int32_t* err;
 };
-
-constexpr int kMaxTreeLevels = 6;  // binary counter over ceil(W/G) <= 63 groups
-
-// Lane l (0..7) of a 16-byte vector of 8 bf16, or the single bf16 of a scalar,
-// as fp32 (exact).  l is a compile-time constant after unrolling.
-__device__ __forceinline__ float lane(const uint4& x, int l) {
-    const uint32_t w = l < 2 ? x.x : l < 4 ? x.y : l < 6 ? x.z : x.w;
-    return (l & 1) ? bf16_hi(w) : bf16_lo(w);
-}
-__device__ __forceinline__ float lane(uint32_t x, int) { return __uint_as_float(x << 16); }
-
-// Reduce W ranks for L lanes (L = 8: one 16-byte vector per rank; L = 1: one
-// element).  load(k) returns rank k's raw bf16 bits; loads are issued G ranks
-// at a time, before any add, and converted to fp32 inside the adds.
-//   Rank order: acc = g_0, then acc = acc + g_k for k = 1..W-1, one add per
-//   rank in order (grouping only batches the loads, never the adds).
-//   Tree: within a group, adjacent ranks are added pairwise level by level (an
-//   unpaired last one is carried); group sums are merged pairwise through a
-//   binary counter, which is a balanced tree when the group count is a power
-//   of two.
-template <int G, int L, bool TREE, class Raw, class Load>
-__device__ __forceinline__ void reduce_ranks(int W, Load load, float (&acc)[L]) {
-    float stack[TREE ? kMaxTreeLevels : 1][L];
-    int gidx = 0;
-    for (int k0 = 0; k0 < W; k0 += G, ++gidx) {
-        Raw x[G];
-        const int n_in = min(G, W - k0);
-#pragma unroll
-        for (int j = 0; j < G; ++j) {
-            if (j < n_in) x[j] = load(k0 + j);
-        }
-        if (!TREE) {
-#pragma unroll
-            for (int j = 0; j < G; ++j) {
-                if (j < n_in) {
-                    if (k0 + j == 0) {
-#pragma unroll
-                        for (int l = 0; l < L; ++l) acc[l] = lane(x[0], l);
-                    } else {
-#pragma unroll
-                        for (int l = 0; l < L; ++l) acc[l] = __fadd_rn(acc[l], lane(x[j], l));
-                    }
-                }
-            }
-        } else {
-            // level 1 straight from the raw values, then in place
-            constexpr int H = (G + 1) / 2;
-            float f[H][L];
-#pragma unroll
-            for (int j = 0; j < G; j += 2) {
-#pragma unroll
-                for (int l = 0; l < L; ++l) {
-                    if (j + 1 < n_in) f[j / 2][l] = __fadd_rn(lane(x[j], l), lane(x[j + 1], l));
-                    else if (j < n_in) f[j / 2][l] = lane(x[j], l);
-                }
-            }
-            const int n_half = (n_in + 1) / 2;
-#pragma unroll
-            for (int step = 1; step < H; step <<= 1) {
-#pragma unroll
-                for (int j = 0; j + step < H; j += 2 * step) {
-                    if (j + step < n_half) {
-#pragma unroll
-                        for (int l = 0; l < L; ++l) f[j][l] = __fadd_rn(f[j][l], f[j + step][l]);
-                    }
-                }
-            }
-            // push the group sum as a level-0 node; merge while the counter carries
-#pragma unroll
-            for (int lvl = 0; lvl < kMaxTreeLevels; ++lvl) {
-                if ((gidx >> lvl) & 1) {
-#pragma unroll
-                    for (int l = 0; l < L; ++l) f[0][l] = __fadd_rn(stack[lvl][l], f[0][l]);
-                } else {
-#pragma unroll
-                    for (int l = 0; l < L; ++l) stack[lvl][l] = f[0][l];
-                    break;
-                }
-            }
-        }
-    }
-    if (TREE) {
-        // gidx is now the group count; occupied levels are its set bits
-        bool have = false;
-#pragma unroll
-        for (int lvl = 0; lvl < kMaxTreeLevels; ++lvl) {
-            if ((gidx >> lvl) & 1) {
-#pragma unroll
-                for (int l = 0; l < L; ++l)
-                    acc[l] = have ? __fadd_rn(stack[lvl][l], acc[l]) : stack[lvl][l];
-                have = true;
-            }
-        }
-    }
-}
 
 template <int G, int U, bool SLOT, bool TREE>
 __global__ void __launch_bounds__(kThreads) rs_reduce_kernel(const RsParams a) {
@@ -177,6 +90,23 @@ __global__ void __launch_bounds__(kThreads) rs_reduce_kernel(const RsParams a) {
         }
         float* __restrict__ dst = a.out + tl.dst_off;
         misaligned |= (reinterpret_cast<uintptr_t>(dst) & 15) != 0;
+#if TIDE_RS_PREFETCH
+        // thread k asks L2 for rank k's source range of a later tile of this CTA
+        if (tid < W) {
+            const int64_t tn = t + (int64_t)TIDE_RS_PREFETCH * gridDim.x;
+            if (tn < a.n_tiles) {
+                const tide_tile_t nt = a.tiles[tn];
+                if (nt.param >= 0 && nt.param < a.n_params && nt.n_valid >= 8) {
+                    const int64_t noff = SLOT ? nt.dst_off : nt.src_off;
+                    const int64_t lim = SLOT ? a.slot_numel : a.numel[nt.param];
+                    const void* base = a.src_tab[SLOT ? tid : (int64_t)tid * a.n_params + nt.param];
+                    const uint16_t* p = static_cast<const uint16_t*>(base) + noff;
+                    if (noff >= 0 && noff + nt.n_valid <= lim && (reinterpret_cast<uintptr_t>(p) & 15) == 0)
+                        prefetch_l2_bulk(p, (uint32_t)(2 * nt.n_valid) & ~15u);
+                }
+            }
+        }
+#endif
         const bool scalar_only = __syncthreads_or(misaligned);
 
         // Vector body: 8 outputs per thread per unit, U units per step.
@@ -224,7 +154,7 @@ template <bool SLOT, bool TREE>
 KernelFn pick(int world) {
     if (world <= 2) return rs_reduce_kernel<2, 4, SLOT, TREE>;
     if (world <= 4) return rs_reduce_kernel<4, 2, SLOT, TREE>;
-    return rs_reduce_kernel<8, 1, SLOT, TREE>;
+    return rs_reduce_kernel<8, TIDE_RS_U8, SLOT, TREE>;
 }
 
 KernelFn select(int world, bool slot, int order) {

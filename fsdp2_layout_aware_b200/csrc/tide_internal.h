@@ -11,11 +11,14 @@
 
 // Bits of the device error word.
 enum : int32_t {
-    TIDE_KCHECK_TILE = 1,   // a tile descriptor pointed outside its buffers
+    TIDE_KCHECK_TILE = 1,     // a tile descriptor pointed outside its buffers
+    TIDE_KCHECK_TIMEOUT = 2,  // a bounded mbarrier wait gave up
 };
 
-// Kernel ids (match tide_launch_ctas).
-enum : int32_t { K_RS = 0, K_AG = 1, K_STAGE = 2, K_SLOT_RS = 3, K_COUNT = 4 };
+// Kernel ids (match tide_launch_ctas and tide_plan_last_launch).
+enum : int32_t {
+    K_RS = 0, K_AG = 1, K_STAGE = 2, K_SLOT_RS = 3, K_RS_TMA = 4, K_SLOT_RS_TMA = 5, K_COUNT = 6
+};
 
 // A device pointer table with a host mirror: re-uploaded only when it changes.
 struct PtrTable {
@@ -23,6 +26,7 @@ struct PtrTable {
     std::vector<const void*> host;       // last uploaded contents
     int64_t capacity = 0;
     bool valid = false;                  // host mirror matches the device copy
+    bool aligned16 = false;              // every pointer in it is 16-byte aligned
 };
 
 struct tide_plan {
@@ -33,6 +37,7 @@ struct tide_plan {
     int64_t shard_numel = 0;             // Ns
     std::vector<int64_t> dim0, inner, numel, rows, chunk, offset;   // per param: d0, inner, d0*inner, S, c, off
     std::vector<tide_tile_t> tiles;
+    bool tiles_aligned8 = true;          // every tile starts on 8-element boundaries (src and dst)
 
     // device tables (absent for TIDE_PLAN_HOST_ONLY)
     tide_tile_t* d_tiles = nullptr;
@@ -42,7 +47,9 @@ struct tide_plan {
     int64_t workspace_bytes = 0;
 
     int32_t sm_count = 0;
-    int32_t blocks_per_sm[K_COUNT] = {0, 0, 0, 0};
+    int32_t blocks_per_sm[K_COUNT] = {0, 0, 0, 0, 0, 0};
+    int32_t last_kernel = -1;            // kernel id of the last launch (-1: none or copy engines)
+    int32_t last_ctas = 0;
 };
 
 namespace tide {
@@ -51,6 +58,7 @@ constexpr int kThreads = 256;
 
 // Occupancy (resident CTAs per SM) of each kernel at kThreads threads.
 int rs_blocks_per_sm(int world, bool slot, int order);
+int rs_tma_blocks_per_sm(int world);  // also opts the TMA kernels in to their shared memory
 int ag_blocks_per_sm();
 int stage_blocks_per_sm();
 
@@ -58,6 +66,9 @@ int stage_blocks_per_sm();
 cudaError_t launch_rs_reduce(const tide_plan* p, const void* const* d_src_tab, bool slot,
                              int64_t src_bound, float* out, int64_t out_numel, float scale,
                              bool do_scale, int order, int grid, cudaStream_t stream);
+cudaError_t launch_rs_reduce_tma(const tide_plan* p, const void* const* d_src_tab, bool slot,
+                                 int64_t src_bound, float* out, int64_t out_numel, float scale,
+                                 bool do_scale, int order, int grid, cudaStream_t stream);
 cudaError_t launch_ag_place(const tide_plan* p, const uint16_t* ag, int64_t ag_numel,
                             const void* const* d_param_tab, int grid, cudaStream_t stream);
 cudaError_t launch_slot_stage(const tide_plan* p, const void* const* d_grad_tab,

@@ -32,11 +32,12 @@ TIDE_ORDER_TREE = 1
 TIDE_SCALE_NONE = 0
 TIDE_SCALE_INV_WORLD = 1
 TIDE_PLAN_HOST_ONLY = 1
+TIDE_PLAN_TMA = 2
 TIDE_MAX_WORLD = 256
 TIDE_TILE_ELEMS = 8192
 TIDE_NOALLOC_SCRATCH_BYTES = 1 << 20
 
-K_RS, K_AG, K_STAGE, K_SLOT_RS = 0, 1, 2, 3
+K_RS, K_AG, K_STAGE, K_SLOT_RS, K_RS_TMA, K_SLOT_RS_TMA = 0, 1, 2, 3, 4, 5
 
 
 class tide_param_t(ctypes.Structure):
@@ -75,6 +76,7 @@ _SIGNATURES = {
                                       _i32, _i32, _vp]),
     "tide_plan_check": (_i32, [_vp, _vp]),
     "tide_launch_ctas": (_i32, [_vp, _i32, _i32, _P(_i32)]),
+    "tide_plan_last_launch": (_i32, [_vp, _P(_i32), _P(_i32)]),
     "tide_status_string": (ctypes.c_char_p, [_i32]),
     "tide_abi_version": (_i32, []),
 }
@@ -206,6 +208,12 @@ def tide_plan_check(plan, stream: int) -> int:
     return lib().tide_plan_check(plan, stream)
 
 
+def tide_plan_last_launch(plan):
+    k, n = _i32(), _i32()
+    st = lib().tide_plan_last_launch(plan, ctypes.byref(k), ctypes.byref(n))
+    return st, k.value, n.value
+
+
 def tide_launch_ctas(plan, kernel: int, max_ctas: int):
     n = _i32()
     st = lib().tide_launch_ctas(plan, kernel, max_ctas, ctypes.byref(n))
@@ -229,7 +237,8 @@ class Plan:
     only read for their data pointers and sizes.
     """
 
-    def __init__(self, shapes, world: int, device=None, host_only: bool = False):
+    def __init__(self, shapes, world: int, device=None, host_only: bool = False,
+                 tma: bool = False):
         self.shapes = [tuple(int(d) for d in s) for s in shapes]
         self.world = int(world)
         if host_only:
@@ -239,8 +248,8 @@ class Plan:
             dev = torch.cuda.current_device() if device is None else torch.device(device).index
             dev = 0 if dev is None else dev
         params = [(s[0], _prod(s[1:])) for s in self.shapes]
-        st, handle = tide_plan_group(params, self.world, dev,
-                                     TIDE_PLAN_HOST_ONLY if host_only else 0)
+        flags = (TIDE_PLAN_HOST_ONLY if host_only else 0) | (TIDE_PLAN_TMA if tma else 0)
+        st, handle = tide_plan_group(params, self.world, dev, flags)
         _check(st, "tide_plan_group")
         self.handle = handle
         self.device_index = dev
@@ -276,6 +285,12 @@ class Plan:
         st, n = tide_launch_ctas(self.handle, kernel, max_ctas)
         _check(st, "tide_launch_ctas")
         return n
+
+    def last_launch(self):
+        """(kernel id, CTAs) of the most recent kernel launch on this plan."""
+        st, k, n = tide_plan_last_launch(self.handle)
+        _check(st, "tide_plan_last_launch")
+        return k, n
 
     def ag_place(self, ag, params, engine: int = TIDE_ENGINE_SM, max_ctas: int = 0,
                  stream=None) -> None:

@@ -68,7 +68,10 @@ typedef enum {
 enum { TIDE_ENGINE_SM = 0, TIDE_ENGINE_CE = 1 };
 enum { TIDE_ORDER_RANK = 0, TIDE_ORDER_TREE = 1 };
 enum { TIDE_SCALE_NONE = 0, TIDE_SCALE_INV_WORLD = 1 };
-enum { TIDE_PLAN_HOST_ONLY = 1 }; /* flag: build the tables on the host only (no CUDA calls) */
+enum {
+    TIDE_PLAN_HOST_ONLY = 1, /* flag: build the tables on the host only (no CUDA calls) */
+    TIDE_PLAN_TMA = 2        /* flag: reduce with the bulk-copy (TMA) kernel where it applies */
+};
 
 #define TIDE_MAX_WORLD 256
 #define TIDE_TILE_ELEMS 8192
@@ -223,10 +226,23 @@ TIDE_API tide_status_t tide_rs_reduce_noalloc(const tide_param_t* params, int32_
                                               int64_t out_numel, int32_t scale_mode,
                                               int32_t max_ctas, void* stream);
 
-/* The number of CTAs a kernel call with this max_ctas would launch.
- * kernel: 0 = RS reduce, 1 = AG place, 2 = Slot-Reuse stage, 3 = slot reduce. */
+/* The number of CTAs a kernel call with this max_ctas would launch (0 if that
+ * kernel cannot run on this plan).  kernel: 0 = RS reduce (load/store kernel),
+ * 1 = AG place, 2 = Slot-Reuse stage, 3 = slot reduce (load/store), 4 = RS
+ * reduce with bulk-copy staging, 5 = slot reduce with bulk-copy staging.
+ * The reductions use kernels 4/5 (one CTA per SM, TMA loads into shared memory)
+ * when the plan was built with TIDE_PLAN_TMA, every tile starts on an
+ * 8-element boundary and every source and the output are 16-byte aligned;
+ * otherwise kernels 0/3.  Both give the same bits.  With the whole grid the
+ * load/store kernels are the faster ones on B200; the bulk-copy kernels move
+ * more bytes per CTA, which matters when max_ctas is small. */
 TIDE_API tide_status_t tide_launch_ctas(const tide_plan_t* plan, int32_t kernel, int32_t max_ctas,
                                int32_t* ctas);
+
+/* The kernel id (as in tide_launch_ctas; -1 for copy-engine calls or none yet)
+ * and CTA count of the plan's most recent kernel launch. */
+TIDE_API tide_status_t tide_plan_last_launch(const tide_plan_t* plan, int32_t* kernel,
+                                             int32_t* ctas);
 
 TIDE_API const char* tide_status_string(tide_status_t status);
 TIDE_API int32_t tide_abi_version(void);

@@ -33,8 +33,8 @@ GROUPS = parity_groups()
 IDS = [f"{g.name}_w{g.world}" for g in GROUPS]
 
 
-def run_rs(group, grads_host, scale=1, order=0, max_ctas=0, slots=False, engine=0):
-    plan = T.Plan(group.shapes, group.world)
+def run_rs(group, grads_host, scale=1, order=0, max_ctas=0, slots=False, engine=0, tma=False):
+    plan = T.Plan(group.shapes, group.world, tma=tma)
     grads = grads_to_dev(group, grads_host)
     out = torch.full((group.world * plan.shard_numel,), float("nan"), device="cuda")
     slot_bufs = None
@@ -50,11 +50,48 @@ def run_rs(group, grads_host, scale=1, order=0, max_ctas=0, slots=False, engine=
 
 @pytest.mark.parametrize("group", GROUPS, ids=IDS)
 @pytest.mark.parametrize("scale", [0, 1])
-def test_rs_rank_order_bit_exact(group, scale):
+@pytest.mark.parametrize("tma", [False, True], ids=["lsu", "tma"])
+def test_rs_rank_order_bit_exact(group, scale, tma):
     grads = synth.grads_host(group, seed=31)
-    out, _, _ = run_rs(group, grads, scale=scale)
+    out, _, plan = run_rs(group, grads, scale=scale, tma=tma)
     ref = oracle.rs_reduce(group.world, group.shapes, grads, scale)
     assert np.array_equal(f32_bits(out), ref.view(np.uint32))
+    kernel, ctas = plan.last_launch()
+    if plan.n_tiles:
+        assert kernel in ((T.K_RS, T.K_RS_TMA) if tma else (T.K_RS,)) and ctas > 0
+
+
+def aligned_group(world, seed):
+    """Shapes whose chunks all start on 8-element boundaries (the bulk-copy path)."""
+    rng = np.random.default_rng(seed)
+    shapes = []
+    for _ in range(int(rng.integers(2, 7))):
+        d0 = int(rng.integers(1, 3000))
+        shapes.append((d0, 8 * int(rng.integers(1, 40))))
+    shapes.append((world * 8 * int(rng.integers(1, 50)),))
+    return configs.Group(f"aligned_w{world}", world, tuple(shapes))
+
+
+TMA_GROUPS = [aligned_group(w, w) for w in (1, 2, 3, 8, 16, 64, 256)] + [mini_sweep(8), configs.qwen3moe(4)]
+
+
+@pytest.mark.parametrize("group", TMA_GROUPS, ids=[f"{g.name}_w{g.world}" for g in TMA_GROUPS])
+def test_rs_bulk_copy_path(group):
+    """The TMA reduction (opt-in): taken for aligned groups, bit-exact, any CTA count, both orders."""
+    grads = synth.grads_host(group, seed=33)
+    ref = oracle.rs_reduce(group.world, group.shapes, grads, 1)
+    E, A = oracle.exact_f64(group.world, group.shapes, grads)
+    for ctas in (1, 7, 0):
+        out, _, plan = run_rs(group, grads, scale=1, max_ctas=ctas, tma=True)
+        assert plan.last_launch()[0] == T.K_RS_TMA
+        assert np.array_equal(f32_bits(out), ref.view(np.uint32)), f"max_ctas={ctas}"
+    out, _, plan = run_rs(group, grads, scale=0, order=1, tma=True)
+    assert plan.last_launch()[0] == T.K_RS_TMA
+    assert np.all(np.abs(out.cpu().numpy().astype(np.float64) - E) <= 1e-6 * A)
+    for engine in (T.TIDE_ENGINE_SM, T.TIDE_ENGINE_CE):
+        out, _, plan = run_rs(group, grads, scale=1, slots=True, engine=engine, tma=True)
+        assert plan.last_launch()[0] == T.K_SLOT_RS_TMA
+        assert np.array_equal(f32_bits(out), ref.view(np.uint32))
 
 
 @pytest.mark.parametrize("seed", range(1, 17))
