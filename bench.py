@@ -88,7 +88,8 @@ def source_digest(*rel):
     return h.hexdigest()[:16]
 
 
-RS_SOURCES = ("fsdp2_layout_aware_b200/csrc/rs_reduce.cu", "fsdp2_layout_aware_b200/csrc/device_common.cuh")
+RS_SOURCES = ("fsdp2_layout_aware_b200/csrc/rs_reduce.cu", "fsdp2_layout_aware_b200/csrc/reduce_ranks.cuh",
+              "fsdp2_layout_aware_b200/csrc/device_common.cuh")
 AG_SOURCES = ("fsdp2_layout_aware_b200/csrc/ag_place.cu", "fsdp2_layout_aware_b200/csrc/device_common.cuh")
 
 
@@ -164,6 +165,22 @@ class ClockSampler:
         names = [n for bit, n in self.REASONS.items() if self.reasons & bit]
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
                 "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+def max_over_ranks(values, device):
+    """Element-wise max of a list of floats over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def replica_throughput(n_ranks: int, bytes_per_rank_step: int, max_step_ms: float) -> float:
+    """Whole-job GB/s of independent replicas: all ranks' bytes over the slowest rank's time."""
+    return n_ranks * bytes_per_rank_step / (max_step_ms * 1e-3) / 1e9
 
 
 def alg_bytes(group, L):
@@ -330,12 +347,14 @@ def cpu_baseline(group, seed, budget_s):
 
 
 def run_interference(device, seed):
-    """Slowdown of a concurrent bf16 8192^3 GEMM vs the RS kernel's CTA count (sweep_w8 group).
+    """Slowdown of a concurrent bf16 GEMM vs the RS kernel's CTA count (sweep_w8 group).
 
-    Per point: the GEMM batch alone, then concurrently with back-to-back RS
-    launches on a second stream (started first, enough of them to outlast the
-    GEMMs), then alone again; slowdown = concurrent / mean(alone) - 1.  Done
-    for the load/store RS kernel and for the bulk-copy (TMA) one.
+    GEMMs: the configured 8192x8192x8192 (cuBLAS picks a 1024-CTA kernel on
+    B200, i.e. not single-wave) and 3072x3072x16384, whose kernel fits in one
+    wave.  Per point, three trials of: the GEMM batch alone, then concurrently
+    with back-to-back RS launches on a second stream (started first, enough of
+    them to outlast the GEMMs); slowdown = median(concurrent) / median(alone)
+    - 1.  Done for the load/store RS kernel and for the bulk-copy (TMA) one.
     """
     import torch
     from synth import configs
@@ -344,61 +363,64 @@ def run_interference(device, seed):
     wl = Workload(group, seed, device)
     plans = {"lsu": wl.plan, "tma": T.Plan(group.shapes, group.world, device=device, tma=True)}
     B = alg_bytes(group, oracle_free_layout(wl))
-    a = torch.randn(8192, 8192, dtype=torch.bfloat16, device=device)
-    b = torch.randn(8192, 8192, dtype=torch.bfloat16, device=device)
-    c = torch.empty(8192, 8192, dtype=torch.bfloat16, device=device)
     s_gemm = torch.cuda.Stream(device)
     s_rs = torch.cuda.Stream(device)
-    n_gemm = 40
+    res = {"rs_workload": "sweep_w8 (16 x 512x4096 params, W=8), rank order, x fl32(1/W)",
+           "trials": 3, "gemms": []}
+    for (m, n, k, n_gemm) in ((8192, 8192, 8192, 40), (3072, 3072, 16384, 120)):
+        a = torch.randn(m, k, dtype=torch.bfloat16, device=device)
+        b = torch.randn(k, n, dtype=torch.bfloat16, device=device)
+        c = torch.empty(m, n, dtype=torch.bfloat16, device=device)
 
-    def gemm_batch():
-        for _ in range(n_gemm):
-            torch.matmul(a, b, out=c)
+        def gemm_batch():
+            for _ in range(n_gemm):
+                torch.matmul(a, b, out=c)
 
-    def gemm_alone():
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        with torch.cuda.stream(s_gemm):
-            e0.record(s_gemm); gemm_batch(); e1.record(s_gemm)
-        torch.cuda.synchronize()
-        return e0.elapsed_time(e1) / n_gemm
-
-    for _ in range(5):
-        gemm_alone()
-    res = {"gemm": "bf16 8192x8192x8192 torch.matmul (cuBLAS), 40 per batch",
-           "rs_workload": "sweep_w8 (16 x 512x4096 params, W=8), rank order, x fl32(1/W)",
-           "points": []}
-    for kind, plan in plans.items():
-        for ctas in (8, 16, 32, 0):
-            rs_ms = timed_calls(lambda: plan.rs_reduce(wl.grads, wl.out, max_ctas=ctas, stream=s_rs), 5, s_rs)
-            kernel, n_ctas = plan.last_launch()
-            before = gemm_alone()
-            reps = int((before * n_gemm * 1.2) / max(rs_ms, 1e-3)) + 2
-            torch.cuda.synchronize()
-            r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        def gemm_alone():
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            with ClockSampler(device.index) as clk:
-                with torch.cuda.stream(s_rs):
-                    r0.record(s_rs)
-                    for _ in range(reps):
-                        plan.rs_reduce(wl.grads, wl.out, max_ctas=ctas, stream=s_rs)
-                    r1.record(s_rs)
-                with torch.cuda.stream(s_gemm):
-                    e0.record(s_gemm); gemm_batch(); e1.record(s_gemm)
-                torch.cuda.synchronize()
-            conc = e0.elapsed_time(e1) / n_gemm
-            after = gemm_alone()
-            alone = 0.5 * (before + after)
-            res["points"].append({
-                "rs_kernel": kind, "max_ctas": ctas, "ctas": n_ctas, "rs_ms_alone": round(rs_ms, 4),
-                "rs_GBps_alone": round(B["rs"] / (rs_ms * 1e-3) / 1e9, 1),
-                "rs_ms_concurrent": round(r0.elapsed_time(r1) / reps, 4),
-                "gemm_ms_alone": round(alone, 4), "gemm_ms_concurrent": round(conc, 4),
-                "gemm_slowdown": round(conc / alone - 1.0, 4),
-                "rs_cta_ms_per_call": round(n_ctas * rs_ms, 2),
-                "sm_mhz_concurrent": clk.summary().get("sm_mhz")})
+            torch.cuda.synchronize()
+            with torch.cuda.stream(s_gemm):
+                e0.record(s_gemm); gemm_batch(); e1.record(s_gemm)
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) / n_gemm
+
+        for _ in range(5):
+            gemm_alone()
+        g = {"gemm": f"bf16 {m}x{n}x{k} torch.matmul (cuBLAS), {n_gemm} per batch", "points": []}
+        for kind, plan in plans.items():
+            for ctas in (8, 16, 32, 0):
+                rs_ms = timed_calls(lambda: plan.rs_reduce(wl.grads, wl.out, max_ctas=ctas, stream=s_rs),
+                                    5, s_rs)
+                _, n_ctas = plan.last_launch()
+                alone, conc, rs_conc = [], [], []
+                for _ in range(3):
+                    alone.append(gemm_alone())
+                    reps = int((alone[-1] * n_gemm * 1.2) / max(rs_ms, 1e-3)) + 2
+                    torch.cuda.synchronize()
+                    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    with torch.cuda.stream(s_rs):
+                        r0.record(s_rs)
+                        for _ in range(reps):
+                            plan.rs_reduce(wl.grads, wl.out, max_ctas=ctas, stream=s_rs)
+                        r1.record(s_rs)
+                    with torch.cuda.stream(s_gemm):
+                        e0.record(s_gemm); gemm_batch(); e1.record(s_gemm)
+                    torch.cuda.synchronize()
+                    conc.append(e0.elapsed_time(e1) / n_gemm)
+                    rs_conc.append(r0.elapsed_time(r1) / reps)
+                ga, gc = statistics.median(alone), statistics.median(conc)
+                g["points"].append({
+                    "rs_kernel": kind, "max_ctas": ctas, "ctas": n_ctas, "rs_ms_alone": round(rs_ms, 4),
+                    "rs_GBps_alone": round(B["rs"] / (rs_ms * 1e-3) / 1e9, 1),
+                    "rs_ms_concurrent": round(statistics.median(rs_conc), 4),
+                    "gemm_ms_alone": round(ga, 4), "gemm_ms_concurrent": round(gc, 4),
+                    "gemm_slowdown": round(gc / ga - 1.0, 4),
+                    "rs_cta_ms_per_call": round(n_ctas * rs_ms, 2)})
+        res["gemms"].append(g)
+        del a, b, c
     plans["tma"].close()
-    del wl, a, b, c
+    del wl
     torch.cuda.empty_cache()
     return res
 
@@ -448,13 +470,10 @@ def bench_workload(args, group, rank, world, device, dist_on):
     ag_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     rs_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     step_ms = ag_ms + rs_ms if flush is not None else total_ms / K
-    if dist_on:
-        t = torch.tensor([step_ms, ag_ms, rs_ms], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        step_ms, ag_ms, rs_ms = (float(x) for x in t.tolist())
+    step_ms, ag_ms, rs_ms = max_over_ranks([step_ms, ag_ms, rs_ms], device)
 
     step_bytes = B["ag"] + B["rs"]
-    value = world * step_bytes / (step_ms * 1e-3) / 1e9
+    value = replica_throughput(world, step_bytes, step_ms)
     rs_gbs = B["rs"] / (rs_ms * 1e-3) / 1e9
     ag_gbs = B["ag"] / (ag_ms * 1e-3) / 1e9
     res = {
@@ -490,11 +509,8 @@ def bench_workload(args, group, rank, world, device, dist_on):
         res["variants"] = run_variants(wl, max(3, min(K, 20)), stream, peak, flush)
     if not args.no_e2e:
         e2e_ms, h2d, d2h = run_e2e(wl, max(1, args.e2e_steps), stream)
-        if dist_on:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        res["e2e"] = {"value": round(world * step_bytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+        e2e_ms = max_over_ranks([e2e_ms], device)[0]
+        res["e2e"] = {"value": round(replica_throughput(world, step_bytes, e2e_ms), 2), "unit": "GB/s",
                       "ms_per_step": round(e2e_ms, 3), "steps": max(1, args.e2e_steps),
                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     del wl

@@ -36,18 +36,22 @@ def _stale(target: str, deps) -> bool:
 
 
 def build(verbose: bool = False, ptxas_verbose: bool = False, force: bool = False,
-          defines=(), build_dir: str = BUILD, lib_path: str = LIB) -> str:
+          defines=(), build_dir: str = BUILD, lib_path: str = LIB, src_dir: str = CSRC,
+          include_dir: str = INCLUDE) -> str:
     """Compile (incrementally) and link; `defines` are extra -D tuning macros."""
     os.makedirs(build_dir, exist_ok=True)
-    headers = [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(INCLUDE, "tide.h")]
+    headers = [os.path.join(src_dir, h) for h in HEADERS] + [os.path.join(include_dir, "tide.h")]
+    flags = [f for f in NVCC_FLAGS]
+    flags[flags.index(INCLUDE)] = include_dir
+    flags[flags.index(CSRC)] = src_dir
     objs = []
     for src in SOURCES:
-        path = os.path.join(CSRC, src)
+        path = os.path.join(src_dir, src)
         obj = os.path.join(build_dir, src + ".o")
         objs.append(obj)
         if not force and not _stale(obj, [path] + headers + [__file__]):
             continue
-        cmd = ["nvcc", *NVCC_FLAGS, *[f"-D{d}" for d in defines], "-c", path, "-o", obj]
+        cmd = ["nvcc", *flags, *[f"-D{d}" for d in defines], "-c", path, "-o", obj]
         if ptxas_verbose and src.endswith(".cu"):
             cmd[1:1] = ["-Xptxas", "-v"]
         if verbose:

@@ -15,13 +15,12 @@
 //
 // Both are pure copies (2 bytes read + 2 written per element): HBM-bound.
 // Each CTA walks the plan's tiles round-robin and moves a tile with 16-byte
-// streaming loads/stores, U vectors in flight per thread.
+// streaming loads/stores, U vectors in flight per thread.  (Measured
+// alternatives that were slower on B200: a bulk L2 prefetch of the next tile,
+// every thread loading the descriptor itself with no barrier, and thread 0
+// prefetching the next descriptor into a double-buffered slot.)
 #include "device_common.cuh"
 #include "tide_internal.h"
-
-#ifndef TIDE_AG_PREFETCH
-#define TIDE_AG_PREFETCH 0  // prefetch the tile this many grid strides ahead into L2 (0 = off)
-#endif
 
 namespace tide {
 namespace {
@@ -55,18 +54,6 @@ __global__ void __launch_bounds__(kThreads) ag_place_kernel(const AgParams a) {
             continue;
         }
         uint16_t* dst = static_cast<uint16_t*>(const_cast<void*>(a.param_tab[tl.param])) + tl.src_off;
-#if TIDE_AG_PREFETCH
-        if (threadIdx.x == 0) {
-            const int64_t tn = t + (int64_t)TIDE_AG_PREFETCH * gridDim.x;
-            if (tn < a.n_tiles) {
-                const tide_tile_t nt = a.tiles[tn];
-                const uint16_t* p = a.ag + nt.dst_off;
-                if (nt.n_valid >= 8 && nt.dst_off >= 0 && nt.dst_off + nt.n_valid <= a.ag_numel &&
-                    (reinterpret_cast<uintptr_t>(p) & 15) == 0)
-                    prefetch_l2_bulk(p, (uint32_t)(2 * nt.n_valid) & ~15u);
-            }
-        }
-#endif
         block_copy_bf16<kCopyU, kThreads>(a.ag + tl.dst_off, dst, tl.n_valid);
         if (tl.n_total > tl.n_valid) block_zero_bf16<kThreads>(dst + tl.n_valid, tl.n_total - tl.n_valid);
     }

@@ -42,13 +42,6 @@ __device__ __forceinline__ void st_stream_f4(float* p, float a, float b, float c
                  : "memory");
 }
 
-// Bulk prefetch of [p, p + bytes) into L2 (p 16-byte aligned, bytes a multiple
-// of 16, the whole range inside one live buffer).  Lets DRAM stream the next
-// tile while the current one is being reduced; the loads then hit L2.
-__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" : : "l"(p), "r"(bytes) : "memory");
-}
-
 // bf16 -> fp32 is exact: the bf16 bits are the top half of the fp32 bits.
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }

@@ -14,7 +14,8 @@
 //   - a persistent grid, at most max_ctas CTAs, walks the plan's tile list
 //     round-robin; a tile is a piece of one (param, rank) chunk of up to
 //     TIDE_TILE_ELEMS elements, so tiny MoE chunks and huge dense chunks mix;
-//   - per tile the W source addresses are staged in shared memory once;
+//   - per tile the W source addresses are staged in shared memory once (one
+//     barrier per tile; the next tile's descriptor is already in registers);
 //   - each thread owns 8 consecutive outputs per step: W independent 16-byte
 //     streaming loads (in groups of G ranks to bound registers), an fp32 sum
 //     with __fadd_rn (no contraction), the optional __fmul_rn scale, two 16-byte
@@ -32,9 +33,6 @@
 
 #ifndef TIDE_RS_U8
 #define TIDE_RS_U8 1        // 16-byte vectors per thread per step when W > 4
-#endif
-#ifndef TIDE_RS_PREFETCH
-#define TIDE_RS_PREFETCH 0  // prefetch the tile this many grid strides ahead into L2 (0 = off)
 #endif
 
 namespace tide {
@@ -57,16 +55,19 @@ struct RsParams {
 
 template <int G, int U, bool SLOT, bool TREE>
 __global__ void __launch_bounds__(kThreads) rs_reduce_kernel(const RsParams a) {
-    __shared__ const uint16_t* s_src[TIDE_MAX_WORLD];
-    __shared__ tide_tile_t s_tile;
+    // s_src is double-buffered: tile i writes buffer i&1 while no thread can
+    // still be reading the same buffer from tile i-2 (a barrier lies between).
+    __shared__ const uint16_t* s_src[2][TIDE_MAX_WORLD];
     const int tid = threadIdx.x;
     const int W = a.world;
 
-    for (int64_t t = blockIdx.x; t < a.n_tiles; t += gridDim.x) {
-        __syncthreads();  // the previous tile is done with s_tile and s_src
-        if (tid == 0) s_tile = a.tiles[t];
-        __syncthreads();
-        const tide_tile_t tl = s_tile;
+    // Every thread keeps the next tile's descriptor in registers: its load is
+    // in flight while the current tile is reduced, so no tile waits on it.
+    int64_t t = blockIdx.x;
+    tide_tile_t next = t < a.n_tiles ? a.tiles[t] : tide_tile_t{};
+    for (int buf = 0; t < a.n_tiles; t += gridDim.x, buf ^= 1) {
+        const tide_tile_t tl = next;
+        if (t + gridDim.x < a.n_tiles) next = a.tiles[t + gridDim.x];
 
         // Range check of the descriptor against the buffers the host validated.
         const bool param_ok = tl.param >= 0 && tl.param < a.n_params;
@@ -76,38 +77,20 @@ __global__ void __launch_bounds__(kThreads) rs_reduce_kernel(const RsParams a) {
         const bool ok = param_ok && tl.n_valid >= 0 && tl.n_valid <= tl.n_total &&
                         tl.dst_off >= 0 && tl.dst_off + tl.n_total <= a.out_numel &&
                         (tl.n_valid == 0 || (src_off >= 0 && src_off + tl.n_valid <= src_lim));
-        if (!ok) {
-            if (tid == 0) atomicOr(a.err, TIDE_KCHECK_TILE);
-            continue;
-        }
+        if (!ok && tid == 0) atomicOr(a.err, TIDE_KCHECK_TILE);
 
+        const uint16_t** srcs = s_src[buf];
         bool misaligned = false;
-        for (int k = tid; k < W; k += kThreads) {
+        for (int k = tid; ok && k < W; k += kThreads) {
             const void* base = a.src_tab[SLOT ? k : (int64_t)k * a.n_params + tl.param];
             const uint16_t* p = static_cast<const uint16_t*>(base) + src_off;
-            s_src[k] = p;
+            srcs[k] = p;
             misaligned |= (reinterpret_cast<uintptr_t>(p) & 15) != 0;
         }
         float* __restrict__ dst = a.out + tl.dst_off;
         misaligned |= (reinterpret_cast<uintptr_t>(dst) & 15) != 0;
-#if TIDE_RS_PREFETCH
-        // thread k asks L2 for rank k's source range of a later tile of this CTA
-        if (tid < W) {
-            const int64_t tn = t + (int64_t)TIDE_RS_PREFETCH * gridDim.x;
-            if (tn < a.n_tiles) {
-                const tide_tile_t nt = a.tiles[tn];
-                if (nt.param >= 0 && nt.param < a.n_params && nt.n_valid >= 8) {
-                    const int64_t noff = SLOT ? nt.dst_off : nt.src_off;
-                    const int64_t lim = SLOT ? a.slot_numel : a.numel[nt.param];
-                    const void* base = a.src_tab[SLOT ? tid : (int64_t)tid * a.n_params + nt.param];
-                    const uint16_t* p = static_cast<const uint16_t*>(base) + noff;
-                    if (noff >= 0 && noff + nt.n_valid <= lim && (reinterpret_cast<uintptr_t>(p) & 15) == 0)
-                        prefetch_l2_bulk(p, (uint32_t)(2 * nt.n_valid) & ~15u);
-                }
-            }
-        }
-#endif
         const bool scalar_only = __syncthreads_or(misaligned);
+        if (!ok) continue;  // skipped after the barrier, so every tile keeps exactly one
 
         // Vector body: 8 outputs per thread per unit, U units per step.
         const int nv = scalar_only ? 0 : (tl.n_valid >> 3);
@@ -117,7 +100,7 @@ __global__ void __launch_bounds__(kThreads) rs_reduce_kernel(const RsParams a) {
             for (int u = 0; u < U; ++u) {
                 const int v = v0 + u * kThreads + tid;
                 if (v < nv) {
-                    auto load = [&](int k) { return ld_stream_v4(s_src[k] + 8 * (int64_t)v); };
+                    auto load = [&](int k) { return ld_stream_v4(srcs[k] + 8 * (int64_t)v); };
                     reduce_ranks<G, 8, TREE, uint4>(W, load, acc[u]);
                 }
             }
@@ -138,7 +121,7 @@ __global__ void __launch_bounds__(kThreads) rs_reduce_kernel(const RsParams a) {
         // Remaining valid elements one by one (ragged end, or a misaligned tile).
         for (int e = 8 * nv + tid; e < tl.n_valid; e += kThreads) {
             float acc[1];
-            auto load = [&](int k) { return (uint32_t)ld_stream_u16(s_src[k] + e); };
+            auto load = [&](int k) { return (uint32_t)ld_stream_u16(srcs[k] + e); };
             reduce_ranks<G, 1, TREE, uint32_t>(W, load, acc);
             if (a.do_scale) acc[0] = __fmul_rn(acc[0], a.scale);
             dst[e] = acc[0];

@@ -1,0 +1,76 @@
+"""Host-side pieces of bench.py: byte accounting, replica aggregation over ranks, the reference arm."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+import oracle
+from synth import configs
+
+from _dist_helpers import free_port
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_algorithmic_bytes_llama70b():
+    g = configs.llama70b()
+    B = bench.alg_bytes(g, oracle.layout(g.world, g.shapes))
+    assert B["rs"] == 13_690_470_400 + 3_422_617_600 == 17_113_088_000
+    assert B["ag"] == 2 * 855_654_400 + 2 * 855_654_400
+    assert B["stage"] == 2 * 8 * 855_654_400 * 2
+
+
+def test_algorithmic_bytes_count_pads_on_the_write_side():
+    g = configs.wan14b()
+    L = oracle.layout(g.world, g.shapes)
+    B = bench.alg_bytes(g, L)
+    N = sum(g.numel(i) for i in range(g.n_params))
+    assert B["N"] == N and B["Npad"] == g.world * L.Ns > N      # modulation rows 6..15 are pad
+    assert B["rs"] == 2 * g.world * N + 4 * g.world * L.Ns
+
+
+def _agg_worker(rank, world, port, out_dir):
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        got = bench.max_over_ranks([1.0 + rank, 5.0 - rank, 0.25 * rank], "cpu")
+        with open(os.path.join(out_dir, f"agg_{rank}.json"), "w") as f:
+            json.dump(got, f)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_replica_aggregation_takes_the_slowest_rank(tmp_path):
+    mp.spawn(_agg_worker, args=(2, free_port(), str(tmp_path)), nprocs=2, join=True)
+    for r in range(2):
+        assert json.load(open(tmp_path / f"agg_{r}.json")) == [2.0, 5.0, 0.25]
+    # whole-job throughput: both replicas' bytes over the slowest rank's step time
+    assert bench.replica_throughput(2, 10**9, 2.0) == pytest.approx(1000.0)
+    assert bench.max_over_ranks([3.0], "cpu") == [3.0]          # no process group: identity
+
+
+def _run_reference(rank):
+    env = dict(os.environ, RANK=str(rank), WORLD_SIZE="2", LOCAL_RANK=str(rank))
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                           "--workload", "tiny", "--steps", "2", "--warmup", "1", "--gpus", "2"],
+                          capture_output=True, text=True, env=env, timeout=300)
+
+
+def test_reference_arm_rank0_prints_one_line_other_ranks_exit_quietly():
+    r1 = _run_reference(1)
+    assert r1.returncode == 0 and r1.stdout.strip() == ""
+    r0 = _run_reference(0)
+    assert r0.returncode == 0, r0.stderr
+    lines = [ln for ln in r0.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "GB/s"
+    assert d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["higher_is_better"] is True
