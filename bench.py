@@ -504,6 +504,8 @@ def bench_workload(args, group, rank, world, device, dist_on):
         "gpu_launches": 2 * K,
         "clocks": clk.summary(),
         "workspace_bytes": wl.plan.workspace_bytes,
+        # what the stock path would hold instead: one full-group fp32 rank-major buffer per rank
+        "stock_fp32_buffer_bytes": 4 * group.world * wl.Ns,
     }
     if not args.no_variants:
         res["variants"] = run_variants(wl, max(3, min(K, 20)), stream, peak, flush)
