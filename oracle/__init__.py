@@ -41,9 +41,14 @@ def build(verbose: bool = False) -> None:
 def _load():
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
-            build()
-        lib = ctypes.CDLL(LIB)
+        # TIDE_ORACLE_LIB points the pins at a deliberately broken build of this
+        # oracle (tests/test_oracle_mutants.py) to show that they catch it.
+        path = os.environ.get("TIDE_ORACLE_LIB")
+        if path is None:
+            if not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
+                build()
+            path = LIB
+        lib = ctypes.CDLL(path)
         i64, i32, vp = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p
         p64 = ctypes.POINTER(ctypes.c_int64)
         lib.orc_layout.argtypes = [i64, i64, vp, vp, vp, vp, vp, p64]

@@ -1,0 +1,50 @@
+"""The oracle's pins are strong enough to catch plausible mistakes.
+
+Each case plants one mistake in a copy of oracle/tide_oracle.c (on the CPU,
+in a temporary directory), builds it, points the pin tests at it through
+TIDE_ORACLE_LIB and checks that at least one pin fails.  Every mutation keeps
+all memory accesses inside their buffers.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "tide_oracle.c")
+
+MUTANTS = {
+    "drops_last_rank": ("    for (int64_t k = 0; k < W; ++k) {\n        if (k == 0) {",
+                        "    for (int64_t k = 0; k < W - 1; ++k) {\n        if (k == 0) {"),
+    "subtracts_instead_of_adds": ("out[j] = out[j] + packed[j];", "out[j] = out[j] - packed[j];"),
+    "rows_per_shard_off_by_one": ("S[i] = (d0[i] + W - 1) / W;", "S[i] = d0[i] / W + 1;"),
+    "pack_uses_local_row": ("bf16_to_f32(g[i][row * inner[i] + t])", "bf16_to_f32(g[i][s * inner[i] + t])"),
+    "scales_by_W_not_inverse": ("        float s = 1.0f / (float)W;\n        for (int64_t j = 0; j < n; ++j) out[j] = out[j] * s;",
+                                "        float s = (float)W;\n        for (int64_t j = 0; j < n; ++j) out[j] = out[j] * s;"),
+    "sum_starts_from_plus_zero": ("        if (k == 0) {\n            pack_f32(W, P, d0, inner, S, off, Ns, grads, out);\n        } else {",
+                                  "        if (k == 0) for (int64_t j = 0; j < n; ++j) out[j] = 0.0f;\n        {"),
+    "ag_pad_rows_not_zeroed": ("for (int64_t t = 0; t < inner[i]; ++t) dst[t] = 0;", ";"),
+    "ag_source_stride_dropped": ("const uint16_t* src = ag + r * Ns + off[i] + s * inner[i];",
+                                 "const uint16_t* src = ag + r * Ns + off[i] + s;"),
+    "ranks_added_in_reverse": ("pack_f32(W, P, d0, inner, S, off, Ns, grads + k * P, packed);",
+                               "pack_f32(W, P, d0, inner, S, off, Ns, grads + (W - k) * P, packed);"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, tmp_path):
+    old, new = MUTANTS[name]
+    text = open(SRC).read()
+    assert text.count(old) == 1, f"mutation anchor for {name} not unique"
+    mutant_c = tmp_path / "mutant.c"
+    mutant_c.write_text(text.replace(old, new))
+    lib = tmp_path / "libmutant.so"
+    subprocess.run(["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared", "-o",
+                    str(lib), str(mutant_c)], check=True)
+    env = dict(os.environ, TIDE_ORACLE_LIB=str(lib))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        "-k", "not gloo", os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"no pin caught mutant {name}:\n{r.stdout[-2000:]}"
+    assert "failed" in r.stdout or "Error" in r.stdout
