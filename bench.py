@@ -271,6 +271,55 @@ def run_variants(wl, K, stream, peak, flush):
                                               K, stream, flush), B["stage"], 1 if eng == 0 else 0)
     rec("slot_reduce", timed_calls(lambda: wl.plan.rs_reduce_slots(slots, wl.out), K, stream, flush),
         B["slot_rs"], 1)
+    # both phases: one after the other (CE staging, then the reduce kernel) ...
+    rec("slot_reuse_serial_ce",
+        timed_calls(lambda: wl.plan.rs_reduce(wl.grads, wl.out, slots=slots, engine=T.TIDE_ENGINE_CE),
+                    K, stream, flush), B["stage"] + B["slot_rs"], 1)
+    # ... and overlapped: the copy engines stage group s+1 while the SMs reduce group s
+    import torch
+    cs = torch.cuda.Stream(wl.out.device)
+    W = wl.group.world
+    for nseg in sorted({1, min(4, W), W}):
+        rec(f"slot_reuse_pipelined_seg{nseg}",
+            timed_calls(lambda: wl.plan.rs_reduce_pipelined(wl.grads, wl.out, slots, nseg, cs),
+                        K, stream, flush), B["stage"] + B["slot_rs"], nseg)
+    wl.drop_slots()
+    del slots
+    # Context: the stock FSDP2 layout conversion with torch's own kernels on the same GPU
+    # (gradients packed by torch._chunk_cat into a fp32 rank-major buffer per rank, summed in
+    # rank order, scaled; all-gather copy-out by torch.split_with_sizes_copy).  Same bits as
+    # ours; rated against the same algorithmic bytes so the GB/s compare directly.
+    Ns = wl.Ns
+    chunks = [wl.plan.query(i)["chunk_numel"] for i in range(wl.group.n_params)]
+    pack = torch.empty(W, Ns, dtype=torch.float32, device=wl.out.device)
+    stock = torch.empty(W, Ns, dtype=torch.float32, device=wl.out.device)
+    stock_params = [torch.empty(W * c, dtype=torch.bfloat16, device=wl.out.device) for c in chunks]
+
+    def stock_rs():
+        for k in range(W):
+            torch._chunk_cat(wl.grads[k], dim=0, num_chunks=W, out=stock if k == 0 else pack)
+            if k:
+                stock.add_(pack)
+        stock.mul_(1.0 / W)
+
+    def stock_ag():
+        torch.split_with_sizes_copy(wl.ag.view(W, Ns), chunks, dim=1,
+                                    out=[p.view(W, c) for p, c in zip(stock_params, chunks)])
+
+    rec("stock_torch_pack_reduce", timed_calls(stock_rs, K, stream, flush), B["rs"], 2 * W)
+    rec("stock_torch_copyout", timed_calls(stock_ag, K, stream, flush), B["ag"], 1)
+    wl.plan.rs_reduce(wl.grads, wl.out)
+    wl.plan.ag_place(wl.ag, wl.params)
+    torch.cuda.synchronize()
+    out["stock_torch_pack_reduce"]["same_bits_as_tide"] = bool(
+        torch.equal(stock.view(-1).view(torch.int32), wl.out.view(torch.int32)))
+    # stock copy-out also copies the all-gather buffer's pad slots; compare valid rows only
+    same = True
+    for i, (p, q) in enumerate(zip(stock_params, wl.params)):
+        n = wl.group.numel(i)
+        same &= bool(torch.equal(p[:n].view(torch.int16), q[:n].view(torch.int16)))
+    out["stock_torch_copyout"]["same_valid_bits_as_tide"] = same
+    del pack, stock, stock_params
     wl.drop_slots()
     return out
 

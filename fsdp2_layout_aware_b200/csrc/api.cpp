@@ -7,6 +7,7 @@
 // zero elements), element alignment, buffer sizes against the plan, and
 // overlap between any written buffer and any other buffer of the call.
 #include <algorithm>
+#include <cstdint>
 #include <cstring>
 #include <vector>
 
@@ -136,22 +137,24 @@ bool use_tma(const tide_plan* p, const PtrTable& src, const float* out, int kern
            src.aligned16 && (reinterpret_cast<uintptr_t>(out) & 15) == 0;
 }
 
-// Launch the reduction over `tab` on the chosen kernel and record it in the plan.
+// Launch the reduction over `tab` on the chosen kernel, for the plan's tiles
+// [t0, t1) (t1 < 0: all), and record it in the plan.
 cudaError_t launch_reduce(tide_plan* p, PtrTable& tab, bool slot, int64_t bound, float* out,
                           int64_t out_numel, int32_t scale_mode, int32_t order, int32_t max_ctas,
-                          cudaStream_t s) {
+                          cudaStream_t s, int64_t t0 = 0, int64_t t1 = -1) {
     const int k_tma = slot ? K_SLOT_RS_TMA : K_RS_TMA, k_lsu = slot ? K_SLOT_RS : K_RS;
     const bool tma = use_tma(p, tab, out, k_tma);
     const int kernel = tma ? k_tma : k_lsu;
-    const int grid = grid_for(p, kernel, max_ctas);
+    if (t1 < 0) t1 = (int64_t)p->tiles.size();
+    const int grid = (int)std::min<int64_t>(grid_for(p, kernel, max_ctas), t1 - t0);
     p->last_kernel = kernel;
     p->last_ctas = grid;
     const float scale = inv_world(p->world);
     const bool do_scale = scale_mode == TIDE_SCALE_INV_WORLD;
     return tma ? tide::launch_rs_reduce_tma(p, tab.dev, slot, bound, out, out_numel, scale, do_scale,
-                                            order, grid, s)
+                                            order, grid, s, t0, t1)
                : tide::launch_rs_reduce(p, tab.dev, slot, bound, out, out_numel, scale, do_scale,
-                                        order, grid, s);
+                                        order, grid, s, t0, t1);
 }
 
 tide_status_t stage_impl(tide_plan* p, const void* const* grads, void* const* slots,
@@ -290,6 +293,58 @@ extern "C" tide_status_t tide_rs_reduce_slots(const tide_plan_t* cplan, const vo
     if ((st = launchable(p)) != TIDE_OK) return st;
     return reduce_slots_impl(p, const_cast<void* const*>(slots), slot_numel, out, out_numel, scale_mode,
                              order, max_ctas, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" tide_status_t tide_rs_reduce_pipelined(const tide_plan_t* cplan, const void* const* grads,
+                                                  const int64_t* grad_numel, float* out,
+                                                  int64_t out_numel, int32_t scale_mode,
+                                                  int32_t order, void* const* slots,
+                                                  int64_t slot_numel, int32_t n_segments,
+                                                  int32_t max_ctas, void* stream, void* copy_stream) {
+    tide_plan* p = const_cast<tide_plan*>(cplan);
+    tide_status_t st = check_plan(p);
+    if (st != TIDE_OK) return st;
+    if ((st = check_enums(TIDE_ENGINE_SM, max_ctas)) != TIDE_OK) return st;
+    if ((st = check_reduce_modes(scale_mode, order)) != TIDE_OK) return st;
+    if (n_segments < 1 || n_segments > p->world) return TIDE_ERR_INVALID_ARG;
+    const int64_t W = p->world, n_out = W * p->shard_numel;
+    std::vector<Span> spans;
+    if ((st = check_grads(p, grads, grad_numel, spans)) != TIDE_OK) return st;
+    if ((st = check_buf(out, out_numel, n_out, 4)) != TIDE_OK) return st;
+    add_span(spans, out, 4 * n_out, true);
+    if ((st = check_slots(p, slots, slot_numel, spans)) != TIDE_OK) return st;
+    if (overlaps(spans)) return TIDE_ERR_INVALID_ARG;
+    if ((st = launchable(p)) != TIDE_OK) return st;
+    if (p->tiles.empty()) return TIDE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream), cs = static_cast<cudaStream_t>(copy_stream);
+    // pacing events, one per segment plus one for the start (created once per plan)
+    while ((int64_t)p->seg_events.size() < (int64_t)n_segments + 1) {
+        cudaEvent_t ev = nullptr;
+        if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return TIDE_ERR_CUDA;
+        }
+        p->seg_events.push_back(ev);
+    }
+    if ((st = sync_table(p->slot_tab, const_cast<const void* const*>(slots), W, s)) != TIDE_OK) return st;
+    // the copies may start once everything enqueued on `stream` so far is done
+    cudaEvent_t start = p->seg_events[n_segments];
+    if (cudaEventRecord(start, s) != cudaSuccess || cudaStreamWaitEvent(cs, start, 0) != cudaSuccess)
+        return TIDE_ERR_CUDA;
+    for (int32_t seg = 0; seg < n_segments; ++seg) {
+        const int64_t r0 = W * seg / n_segments, r1 = W * (seg + 1) / n_segments;
+        if (r1 == r0) continue;
+        // phase 1 of these output ranks on the copy engines ...
+        if (tide::ce_slot_stage(p, grads, slots, cs, r0, r1) != cudaSuccess) return TIDE_ERR_CUDA;
+        cudaEvent_t done = p->seg_events[seg];
+        if (cudaEventRecord(done, cs) != cudaSuccess || cudaStreamWaitEvent(s, done, 0) != cudaSuccess)
+            return TIDE_ERR_CUDA;
+        // ... phase 2 of them on the SMs, while the next segment is being copied
+        if (launch_reduce(p, p->slot_tab, true, slot_numel, out, out_numel, scale_mode, order, max_ctas,
+                          s, p->rank_tile_begin[r0], p->rank_tile_begin[r1]) != cudaSuccess)
+            return TIDE_ERR_CUDA;
+    }
+    return TIDE_OK;
 }
 
 extern "C" tide_status_t tide_plan_check(tide_plan_t* p, void* stream) {

@@ -69,9 +69,12 @@ cudaError_t ce_ag_place(const tide_plan* p, const uint16_t* ag, void* const* par
     return cudaSuccess;
 }
 
+// Stage the chunks that output ranks [r0, r1) need (r1 < 0: up to W) from every
+// source rank k into slot k.
 cudaError_t ce_slot_stage(const tide_plan* p, const void* const* grads, void* const* slots,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, int64_t r0, int64_t r1) {
     const int64_t W = p->world, P = p->n_params, Ns = p->shard_numel;
+    if (r1 < 0) r1 = W;
     const size_t max_pitch = device_max_pitch(p->device);
     for (int64_t k = 0; k < W; ++k) {
         uint16_t* slot = static_cast<uint16_t*>(slots[k]);
@@ -80,13 +83,17 @@ cudaError_t ce_slot_stage(const tide_plan* p, const void* const* grads, void* co
             if (c == 0 || n == 0) continue;
             const uint16_t* g = static_cast<const uint16_t*>(grads[k * P + i]);
             uint16_t* dst = slot + p->offset[i];
-            const int64_t full = std::min(W, n / c);
-            cudaError_t e = copy_rows(dst, 2 * Ns, g, 2 * c, 2 * c, full, max_pitch, stream);
-            if (e != cudaSuccess) return e;
-            const int64_t rem = n - full * c;
-            if (rem > 0 && full < W) {
-                e = cudaMemcpyAsync(dst + full * Ns, g + full * c, 2 * rem, cudaMemcpyDeviceToDevice,
-                                    stream);
+            const int64_t full = std::min(W, n / c);  // ranks [0, full) hold whole chunks
+            const int64_t fr1 = std::min(full, r1);
+            if (fr1 > r0) {
+                cudaError_t e = copy_rows(dst + r0 * Ns, 2 * Ns, g + r0 * c, 2 * c, 2 * c, fr1 - r0,
+                                          max_pitch, stream);
+                if (e != cudaSuccess) return e;
+            }
+            const int64_t rem = n - full * c;       // rank `full` holds a partial chunk
+            if (rem > 0 && full < W && full >= r0 && full < r1) {
+                cudaError_t e = cudaMemcpyAsync(dst + full * Ns, g + full * c, 2 * rem,
+                                                cudaMemcpyDeviceToDevice, stream);
                 if (e != cudaSuccess) return e;
             }
         }

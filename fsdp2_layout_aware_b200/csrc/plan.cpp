@@ -145,7 +145,9 @@ extern "C" tide_status_t tide_plan_group(const tide_param_t* params, int32_t n_p
         if (!mul_ok(W, acc)) { delete p; return TIDE_ERR_SIZE; }
         p->shard_numel = acc;
         // tiles in rank-major buffer order: rank, then param, then position
+        p->rank_tile_begin.assign(W + 1, 0);
         for (int64_t r = 0; r < W; ++r) {
+            p->rank_tile_begin[r] = (int64_t)p->tiles.size();
             for (int32_t i = 0; i < n_params; ++i) {
                 const int64_t c = p->chunk[i];
                 const int64_t valid = std::min(c, std::max<int64_t>(0, p->numel[i] - r * c));
@@ -162,6 +164,7 @@ extern "C" tide_status_t tide_plan_group(const tide_param_t* params, int32_t n_p
                 }
             }
         }
+        p->rank_tile_begin[W] = (int64_t)p->tiles.size();
     } catch (const std::bad_alloc&) {
         delete p;
         return TIDE_ERR_NOMEM;
@@ -185,6 +188,8 @@ extern "C" void tide_plan_destroy(tide_plan_t* plan) {
         if (cudaSetDevice(plan->device) == cudaSuccess) {
             cudaDeviceSynchronize();
             free_device(plan);
+            for (cudaEvent_t ev : plan->seg_events) cudaEventDestroy(ev);
+            plan->seg_events.clear();
         }
         if (prev >= 0) cudaSetDevice(prev);
     }

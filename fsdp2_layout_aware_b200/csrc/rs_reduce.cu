@@ -158,11 +158,13 @@ int rs_blocks_per_sm(int world, bool slot, int order) {
 
 cudaError_t launch_rs_reduce(const tide_plan* p, const void* const* d_src_tab, bool slot,
                              int64_t src_bound, float* out, int64_t out_numel, float scale,
-                             bool do_scale, int order, int grid, cudaStream_t stream) {
-    if (p->tiles.empty() || grid <= 0) return cudaSuccess;
+                             bool do_scale, int order, int grid, cudaStream_t stream, int64_t t0,
+                             int64_t t1) {
+    if (t1 < 0) t1 = (int64_t)p->tiles.size();
+    if (t1 <= t0 || grid <= 0) return cudaSuccess;
     RsParams a;
-    a.tiles = p->d_tiles;
-    a.n_tiles = (int64_t)p->tiles.size();
+    a.tiles = p->d_tiles + t0;
+    a.n_tiles = t1 - t0;
     a.src_tab = d_src_tab;
     a.numel = p->d_numel;
     a.slot_numel = src_bound;

@@ -37,7 +37,9 @@ struct tide_plan {
     int64_t shard_numel = 0;             // Ns
     std::vector<int64_t> dim0, inner, numel, rows, chunk, offset;   // per param: d0, inner, d0*inner, S, c, off
     std::vector<tide_tile_t> tiles;
+    std::vector<int64_t> rank_tile_begin;  // [W+1]: the tiles of output rank r are [begin[r], begin[r+1])
     bool tiles_aligned8 = true;          // every tile starts on 8-element boundaries (src and dst)
+    std::vector<cudaEvent_t> seg_events; // pacing events of tide_rs_reduce_pipelined (created on first use)
 
     // device tables (absent for TIDE_PLAN_HOST_ONLY)
     tide_tile_t* d_tiles = nullptr;
@@ -63,12 +65,15 @@ int ag_blocks_per_sm();
 int stage_blocks_per_sm();
 
 // Kernel launches; return the launch's cudaError_t.
+// The RS launchers work on the plan's tiles [t0, t1) (t1 < 0: to the end).
 cudaError_t launch_rs_reduce(const tide_plan* p, const void* const* d_src_tab, bool slot,
                              int64_t src_bound, float* out, int64_t out_numel, float scale,
-                             bool do_scale, int order, int grid, cudaStream_t stream);
+                             bool do_scale, int order, int grid, cudaStream_t stream,
+                             int64_t t0 = 0, int64_t t1 = -1);
 cudaError_t launch_rs_reduce_tma(const tide_plan* p, const void* const* d_src_tab, bool slot,
                                  int64_t src_bound, float* out, int64_t out_numel, float scale,
-                                 bool do_scale, int order, int grid, cudaStream_t stream);
+                                 bool do_scale, int order, int grid, cudaStream_t stream,
+                                 int64_t t0 = 0, int64_t t1 = -1);
 cudaError_t launch_ag_place(const tide_plan* p, const uint16_t* ag, int64_t ag_numel,
                             const void* const* d_param_tab, int grid, cudaStream_t stream);
 cudaError_t launch_slot_stage(const tide_plan* p, const void* const* d_grad_tab,
@@ -79,6 +84,6 @@ cudaError_t launch_slot_stage(const tide_plan* p, const void* const* d_grad_tab,
 cudaError_t ce_ag_place(const tide_plan* p, const uint16_t* ag, void* const* params,
                         cudaStream_t stream);
 cudaError_t ce_slot_stage(const tide_plan* p, const void* const* grads, void* const* slots,
-                          cudaStream_t stream);
+                          cudaStream_t stream, int64_t r0 = 0, int64_t r1 = -1);
 
 }  // namespace tide

@@ -74,6 +74,8 @@ _SIGNATURES = {
     "tide_rs_reduce_slots": (_i32, [_vp, _P(_vp), _i64, _vp, _i64, _i32, _i32, _i32, _vp]),
     "tide_rs_reduce_noalloc": (_i32, [_P(tide_param_t), _i32, _i32, _P(_vp), _P(_i64), _vp, _i64,
                                       _i32, _i32, _vp]),
+    "tide_rs_reduce_pipelined": (_i32, [_vp, _P(_vp), _P(_i64), _vp, _i64, _i32, _i32, _P(_vp),
+                                        _i64, _i32, _i32, _vp, _vp]),
     "tide_plan_check": (_i32, [_vp, _vp]),
     "tide_launch_ctas": (_i32, [_vp, _i32, _i32, _P(_i32)]),
     "tide_plan_last_launch": (_i32, [_vp, _P(_i32), _P(_i32)]),
@@ -204,6 +206,15 @@ def tide_rs_reduce_noalloc(params, world: int, grads, grad_numel, out: int, out_
                                         max_ctas, stream)
 
 
+def tide_rs_reduce_pipelined(plan, grads, grad_numel, out: int, out_numel: int, scale_mode: int,
+                             order: int, slots, slot_numel: int, n_segments: int, max_ctas: int,
+                             stream: int, copy_stream: int) -> int:
+    slot_arr = _ptr_array(slots) if slots is not None else None
+    return lib().tide_rs_reduce_pipelined(plan, _ptr_array(grads), _i64_array(grad_numel), out,
+                                          out_numel, scale_mode, order, slot_arr, slot_numel,
+                                          n_segments, max_ctas, stream, copy_stream)
+
+
 def tide_plan_check(plan, stream: int) -> int:
     return lib().tide_plan_check(plan, stream)
 
@@ -324,6 +335,18 @@ class Plan:
                                   min(s.numel() for s in slots), out.data_ptr(), out.numel(),
                                   scale_mode, order, max_ctas, _stream_handle(stream))
         _check(st, "tide_rs_reduce_slots")
+
+    def rs_reduce_pipelined(self, grads, out, slots, n_segments: int, copy_stream,
+                            scale_mode: int = TIDE_SCALE_INV_WORLD, order: int = TIDE_ORDER_RANK,
+                            max_ctas: int = 0, stream=None) -> None:
+        """Slot-Reuse with copy-engine staging on `copy_stream` overlapping the reduction."""
+        flat = [g for row in grads for g in row]
+        st = tide_rs_reduce_pipelined(self.handle, [g.data_ptr() for g in flat],
+                                      [g.numel() for g in flat], out.data_ptr(), out.numel(),
+                                      scale_mode, order, [s.data_ptr() for s in slots],
+                                      min(s.numel() for s in slots), n_segments, max_ctas,
+                                      _stream_handle(stream), _stream_handle(copy_stream))
+        _check(st, "tide_rs_reduce_pipelined")
 
     def check(self, stream=None) -> None:
         _check(tide_plan_check(self.handle, _stream_handle(stream)), "tide_plan_check")

@@ -192,6 +192,27 @@ TIDE_API tide_status_t tide_rs_reduce_slots(const tide_plan_t* plan, const void*
                                    void* stream);
 
 /*
+ * Slot-Reuse with the two phases overlapped (weekinpapers.com Abstract: the
+ * two-phase pipeline keeps gradient reads apart from the reduction's
+ * progress, and copy engines move the gradients).  Same result as
+ * tide_rs_reduce with the same slots (same bits).  The output ranks are split
+ * into n_segments contiguous groups (1 <= n_segments <= W).  For each group,
+ * phase 1 stages the chunks those ranks need into the slots with copy-engine
+ * memcpys on `copy_stream`, then phase 2 reduces them on `stream` (one kernel
+ * launch per group) while the copy engines already stage the next group.
+ * Work enqueued on `stream` before the call is ordered before the copies;
+ * work enqueued on `stream` after it sees the complete result.  `copy_stream`
+ * may equal `stream` (the phases then run one after the other).  The plan
+ * creates its pacing events (no device memory) on first use.
+ */
+TIDE_API tide_status_t tide_rs_reduce_pipelined(const tide_plan_t* plan, const void* const* grads,
+                                                const int64_t* grad_numel, float* out,
+                                                int64_t out_numel, int32_t scale_mode,
+                                                int32_t order, void* const* slots,
+                                                int64_t slot_numel, int32_t n_segments,
+                                                int32_t max_ctas, void* stream, void* copy_stream);
+
+/*
  * Read and clear the plan's device error word: synchronizes `stream`, then
  * returns TIDE_ERR_KERNEL_CHECK if a kernel enqueued before it rejected a tile
  * (the tile is skipped, nothing outside the buffers is touched), else TIDE_OK.

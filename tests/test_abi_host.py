@@ -202,6 +202,10 @@ def test_valid_arguments_reach_the_device_check(tiny_plan, args):
     assert T.tide_rs_reduce_slots(h, args["slots"], args["n_slot"], args["out"], args["n_out"], 1, 0,
                                   0, 0) == T.TIDE_ERR_DEVICE
     assert T.tide_plan_check(h, 0) == T.TIDE_ERR_DEVICE
+    for n_seg, status in ((1, T.TIDE_ERR_DEVICE), (4, T.TIDE_ERR_DEVICE), (0, T.TIDE_ERR_INVALID_ARG),
+                          (5, T.TIDE_ERR_INVALID_ARG)):
+        assert T.tide_rs_reduce_pipelined(h, args["grads"], args["gnum"], args["out"], args["n_out"], 1,
+                                          0, args["slots"], args["n_slot"], n_seg, 0, 0, 0) == status
     assert T.tide_launch_ctas(h, 0, 0)[0] == T.TIDE_ERR_DEVICE
 
 

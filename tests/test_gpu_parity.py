@@ -176,6 +176,36 @@ def test_slot_reuse_equals_plain_and_oracle(group, engine):
         assert np.array_equal(bits_of(slots[k]), exp)
 
 
+PIPE_GROUPS = [configs.tiny(), degenerate(), mini_wan(), configs.qwen3moe(4), aligned_group(16, 5)]
+
+
+@pytest.mark.parametrize("group", PIPE_GROUPS, ids=[f"{g.name}_w{g.world}" for g in PIPE_GROUPS])
+@pytest.mark.parametrize("segments", ["one", "three", "all"])
+def test_slot_reuse_pipelined(group, segments):
+    """Copy-engine staging on a second stream overlapped with the reduction: same bits."""
+    n_seg = {"one": 1, "three": min(3, group.world), "all": group.world}[segments]
+    grads = synth.grads_host(group, seed=53)
+    ref = oracle.rs_reduce(group.world, group.shapes, grads, 1)
+    L = oracle.layout(group.world, group.shapes)
+    for tma, same_stream in ((False, False), (True, False), (False, True)):
+        plan = T.Plan(group.shapes, group.world, tma=tma)
+        dev = grads_to_dev(group, grads)
+        n = group.world * plan.shard_numel
+        slots = [torch.full((n,), -1, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+                 for _ in range(group.world)]
+        out = torch.full((n,), float("nan"), device="cuda")
+        main = torch.cuda.current_stream()
+        cs = main if same_stream else torch.cuda.Stream()
+        plan.rs_reduce_pipelined(dev, out, slots, n_seg, cs)
+        torch.cuda.synchronize()
+        plan.check()
+        assert np.array_equal(f32_bits(out), ref.view(np.uint32)), (tma, same_stream)
+        for k in range(group.world):
+            exp = np.full(n, 0xFFFF, dtype=np.uint16)
+            oracle.slot_stage(group.world, group.shapes, grads[k], exp)
+            assert np.array_equal(bits_of(slots[k]), exp)
+
+
 def test_slot_phases_separately():
     group = mini_wan()
     grads = synth.grads_host(group, seed=52)
