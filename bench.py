@@ -263,7 +263,7 @@ def run_variants(wl, K, stream, peak, flush):
     tma_plan = T.Plan(wl.group.shapes, wl.group.world, device=wl.out.device, tma=True)
     rec("rs_reduce_tma", timed_calls(lambda: tma_plan.rs_reduce(wl.grads, wl.out), K, stream, flush),
         B["rs"], 1)
-    out["rs_reduce_tma"]["kernel"] = ["lsu", "ag", "stage", "slot_lsu", "tma", "slot_tma"][tma_plan.last_launch()[0]]
+    out["rs_reduce_tma"]["kernel"] = T.KERNEL_NAMES[tma_plan.last_launch()[0]]
     tma_plan.close()
     slots = wl.ensure_slots()
     for eng, name in ((T.TIDE_ENGINE_SM, "sm"), (T.TIDE_ENGINE_CE, "ce")):
@@ -591,7 +591,7 @@ def bench_workload(args, group, rank, world, device, dist_on):
         "kernels": {
             "rs_reduce_kernel": {"ms": round(rs_ms, 4), "GB/s": round(rs_gbs, 1),
                                  "frac_of_peak": round(rs_gbs / peak, 4), "alg_bytes": B["rs"],
-                                 "ctas": rs_ctas, "kernel_id": rs_kernel},
+                                 "ctas": rs_ctas, "kernel": T.KERNEL_NAMES[rs_kernel]},
             "ag_place_kernel": {"ms": round(ag_ms, 4), "GB/s": round(ag_gbs, 1),
                                 "frac_of_peak": round(ag_gbs / peak, 4), "alg_bytes": B["ag"],
                                 "ctas": wl.plan.launch_ctas(T.K_AG, args.max_ctas),

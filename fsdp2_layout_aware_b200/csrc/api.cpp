@@ -110,9 +110,11 @@ tide_status_t sync_table(PtrTable& t, const void* const* ptrs, int64_t n, cudaSt
         std::memcmp(t.host.data(), ptrs, sizeof(void*) * (size_t)n) == 0)
         return TIDE_OK;
     t.host.assign(ptrs, ptrs + n);
-    t.aligned16 = true;
-    for (int64_t j = 0; j < n; ++j)
+    t.aligned16 = t.aligned32 = true;
+    for (int64_t j = 0; j < n; ++j) {
         if ((reinterpret_cast<uintptr_t>(ptrs[j]) & 15) != 0) t.aligned16 = false;
+        if ((reinterpret_cast<uintptr_t>(ptrs[j]) & 31) != 0) t.aligned32 = false;
+    }
     // Pageable source: the runtime stages it before returning, so the host
     // mirror may change afterwards; the device copy is stream-ordered.
     cudaError_t e = cudaMemcpyAsync(t.dev, t.host.data(), sizeof(void*) * (size_t)n,
@@ -137,14 +139,23 @@ bool use_tma(const tide_plan* p, const PtrTable& src, const float* out, int kern
            src.aligned16 && (reinterpret_cast<uintptr_t>(out) & 15) == 0;
 }
 
+// The 32-byte load/store variant needs 32-byte aligned sources and output at
+// every tile: 16-element tile offsets plus 32-byte aligned base pointers.
+bool use_v32(const tide_plan* p, const PtrTable& src, const float* out, int kernel) {
+    return p->tiles_aligned16 && p->blocks_per_sm[kernel] > 0 && src.aligned32 &&
+           (reinterpret_cast<uintptr_t>(out) & 31) == 0;
+}
+
 // Launch the reduction over `tab` on the chosen kernel, for the plan's tiles
 // [t0, t1) (t1 < 0: all), and record it in the plan.
 cudaError_t launch_reduce(tide_plan* p, PtrTable& tab, bool slot, int64_t bound, float* out,
                           int64_t out_numel, int32_t scale_mode, int32_t order, int32_t max_ctas,
                           cudaStream_t s, int64_t t0 = 0, int64_t t1 = -1) {
-    const int k_tma = slot ? K_SLOT_RS_TMA : K_RS_TMA, k_lsu = slot ? K_SLOT_RS : K_RS;
+    const int k_tma = slot ? K_SLOT_RS_TMA : K_RS_TMA;
+    const int k_v32 = slot ? K_SLOT_RS_V32 : K_RS_V32;
     const bool tma = use_tma(p, tab, out, k_tma);
-    const int kernel = tma ? k_tma : k_lsu;
+    const bool v32 = !tma && use_v32(p, tab, out, k_v32);
+    const int kernel = tma ? k_tma : v32 ? k_v32 : (slot ? K_SLOT_RS : K_RS);
     if (t1 < 0) t1 = (int64_t)p->tiles.size();
     const int grid = (int)std::min<int64_t>(grid_for(p, kernel, max_ctas), t1 - t0);
     p->last_kernel = kernel;
@@ -154,7 +165,7 @@ cudaError_t launch_reduce(tide_plan* p, PtrTable& tab, bool slot, int64_t bound,
     return tma ? tide::launch_rs_reduce_tma(p, tab.dev, slot, bound, out, out_numel, scale, do_scale,
                                             order, grid, s, t0, t1)
                : tide::launch_rs_reduce(p, tab.dev, slot, bound, out, out_numel, scale, do_scale,
-                                        order, grid, s, t0, t1);
+                                        order, grid, s, v32, t0, t1);
 }
 
 tide_status_t stage_impl(tide_plan* p, const void* const* grads, void* const* slots,

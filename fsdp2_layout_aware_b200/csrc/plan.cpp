@@ -84,8 +84,12 @@ tide_status_t upload(tide_plan* p) {
         e = cudaDeviceGetAttribute(&p->sm_count, cudaDevAttrMultiProcessorCount, p->device);
     if (st == TIDE_OK && e != cudaSuccess) st = TIDE_ERR_CUDA;
     if (st == TIDE_OK) {
-        p->blocks_per_sm[K_RS] = tide::rs_blocks_per_sm(p->world, false, TIDE_ORDER_RANK);
-        p->blocks_per_sm[K_SLOT_RS] = tide::rs_blocks_per_sm(p->world, true, TIDE_ORDER_RANK);
+        p->blocks_per_sm[K_RS] = tide::rs_blocks_per_sm(p->world, false, TIDE_ORDER_RANK, false);
+        p->blocks_per_sm[K_SLOT_RS] = tide::rs_blocks_per_sm(p->world, true, TIDE_ORDER_RANK, false);
+        if (tide::rs_v32_applies(p->world)) {
+            p->blocks_per_sm[K_RS_V32] = tide::rs_blocks_per_sm(p->world, false, TIDE_ORDER_RANK, true);
+            p->blocks_per_sm[K_SLOT_RS_V32] = tide::rs_blocks_per_sm(p->world, true, TIDE_ORDER_RANK, true);
+        }
         p->blocks_per_sm[K_AG] = tide::ag_blocks_per_sm();
         p->blocks_per_sm[K_STAGE] = tide::stage_blocks_per_sm();
         for (int k = 0; k < K_RS_TMA; ++k)
@@ -160,6 +164,7 @@ extern "C" tide_status_t tide_plan_group(const tide_param_t* params, int32_t n_p
                     t.n_total = (int32_t)std::min<int64_t>(TIDE_TILE_ELEMS, c - e0);
                     t.n_valid = (int32_t)std::min<int64_t>(t.n_total, std::max<int64_t>(0, valid - e0));
                     if ((t.src_off & 7) != 0 || (t.dst_off & 7) != 0) p->tiles_aligned8 = false;
+                    if ((t.src_off & 15) != 0 || (t.dst_off & 15) != 0) p->tiles_aligned16 = false;
                     p->tiles.push_back(t);
                 }
             }
@@ -236,7 +241,7 @@ extern "C" tide_status_t tide_launch_ctas(const tide_plan_t* plan, int32_t kerne
     if (plan->flags & TIDE_PLAN_HOST_ONLY) return TIDE_ERR_DEVICE;
     int64_t units = (int64_t)plan->tiles.size();
     if (kernel == K_STAGE) units *= plan->world;
-    if ((kernel == K_RS_TMA || kernel == K_SLOT_RS_TMA) && plan->blocks_per_sm[kernel] <= 0) {
+    if (kernel >= K_RS_TMA && plan->blocks_per_sm[kernel] <= 0) {
         *ctas = 0;
         return TIDE_OK;
     }

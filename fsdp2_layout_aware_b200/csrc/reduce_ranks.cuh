@@ -21,6 +21,10 @@ __device__ __forceinline__ float lane(const uint4& x, int l) {
     return (l & 1) ? bf16_hi(w) : bf16_lo(w);
 }
 __device__ __forceinline__ float lane(uint32_t x, int) { return __uint_as_float(x << 16); }
+// Lane l (0..15) of a 32-byte vector of 16 bf16.
+__device__ __forceinline__ float lane(const V8& x, int l) {
+    return (l & 1) ? bf16_hi(x.w[l >> 1]) : bf16_lo(x.w[l >> 1]);
+}
 
 // Reduce W ranks for L lanes (L = 8: one 16-byte vector per rank; L = 1: one
 // element).  load(k) returns rank k's raw bf16 bits; loads are issued G ranks

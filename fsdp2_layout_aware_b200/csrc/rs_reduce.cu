@@ -19,7 +19,8 @@
 //   - each thread owns 8 consecutive outputs per step: W independent 16-byte
 //     streaming loads (in groups of G ranks to bound registers), an fp32 sum
 //     with __fadd_rn (no contraction), the optional __fmul_rn scale, two 16-byte
-//     streaming stores;
+//     streaming stores; for 5 <= W <= 16 and 32-byte aligned groups, 16 outputs
+//     per step with 32-byte loads and stores instead;
 //   - tiles whose addresses are not all 16-byte aligned (possible only when
 //     the group's sizes break alignment) fall back to coalesced scalar loads;
 //   - ragged tile ends and pad rows are finished element by element.
@@ -31,12 +32,14 @@
 #include "reduce_ranks.cuh"
 #include "tide_internal.h"
 
-#ifndef TIDE_RS_U8
-#define TIDE_RS_U8 1        // 16-byte vectors per thread per step when W > 4
-#endif
 
 namespace tide {
 namespace {
+
+// The 32-byte path measured faster for 5 <= W <= 16 (70B W=8: 7.03 vs 6.89
+// TB/s; Qwen3 W=8: 7.08 vs 6.87; Wan2.2 W=16: 6.93 vs 6.90) and slower at
+// W=64 (6.90 vs 7.01), where 16-byte loads keep more ranks in flight.
+constexpr int kV32MaxWorld = 16;
 
 struct RsParams {
     const tide_tile_t* tiles;
@@ -53,7 +56,10 @@ struct RsParams {
     int32_t* err;
 };
 
-template <int G, int U, bool SLOT, bool TREE>
+// V32: 32-byte loads and stores (16 outputs per thread per step); the host
+// picks it only when every tile's sources and output are 32-byte aligned
+// (a tile that is not falls back to the element loop, never faults).
+template <int G, int U, bool SLOT, bool TREE, bool V32>
 __global__ void __launch_bounds__(kThreads) rs_reduce_kernel(const RsParams a) {
     // s_src is double-buffered: tile i writes buffer i&1 while no thread can
     // still be reading the same buffer from tile i-2 (a barrier lies between).
@@ -89,12 +95,36 @@ __global__ void __launch_bounds__(kThreads) rs_reduce_kernel(const RsParams a) {
         }
         float* __restrict__ dst = a.out + tl.dst_off;
         misaligned |= (reinterpret_cast<uintptr_t>(dst) & 15) != 0;
+        if (V32) {
+            for (int k = tid; ok && k < W; k += kThreads)
+                misaligned |= (reinterpret_cast<uintptr_t>(srcs[k]) & 31) != 0;
+            misaligned |= (reinterpret_cast<uintptr_t>(dst) & 31) != 0;
+        }
         const bool scalar_only = __syncthreads_or(misaligned);
         if (!ok) continue;  // skipped after the barrier, so every tile keeps exactly one
 
+        int nv;  // 8-element units covered by the vector body
+        if (V32) {
+            // 16 outputs per thread per step: W 32-byte loads, two 32-byte stores.
+            const int nv16 = scalar_only ? 0 : (tl.n_valid >> 4);
+            for (int v = tid; v < nv16; v += kThreads) {
+                float acc[16];
+                auto load = [&](int k) { return ld_stream_v8(srcs[k] + 16 * (int64_t)v); };
+                reduce_ranks<G, 16, TREE, V8>(W, load, acc);
+                if (a.do_scale) {
+#pragma unroll
+                    for (int l = 0; l < 16; ++l) acc[l] = __fmul_rn(acc[l], a.scale);
+                }
+                float* o = dst + 16 * (int64_t)v;
+                st_stream_f8(o, *reinterpret_cast<const float(*)[8]>(&acc[0]));
+                st_stream_f8(o + 8, *reinterpret_cast<const float(*)[8]>(&acc[8]));
+            }
+            nv = 2 * nv16;
+        } else {
+            nv = scalar_only ? 0 : (tl.n_valid >> 3);
+        }
         // Vector body: 8 outputs per thread per unit, U units per step.
-        const int nv = scalar_only ? 0 : (tl.n_valid >> 3);
-        for (int v0 = 0; v0 < nv; v0 += kThreads * U) {
+        for (int v0 = 0; !V32 && v0 < nv; v0 += kThreads * U) {
             float acc[U][8];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
@@ -134,23 +164,26 @@ __global__ void __launch_bounds__(kThreads) rs_reduce_kernel(const RsParams a) {
 using KernelFn = void (*)(const RsParams);
 
 template <bool SLOT, bool TREE>
-KernelFn pick(int world) {
-    if (world <= 2) return rs_reduce_kernel<2, 4, SLOT, TREE>;
-    if (world <= 4) return rs_reduce_kernel<4, 2, SLOT, TREE>;
-    return rs_reduce_kernel<8, TIDE_RS_U8, SLOT, TREE>;
+KernelFn pick(int world, bool v32) {
+    if (world <= 2) return rs_reduce_kernel<2, 4, SLOT, TREE, false>;
+    if (world <= 4) return rs_reduce_kernel<4, 2, SLOT, TREE, false>;
+    if (v32 && world <= kV32MaxWorld) return rs_reduce_kernel<8, 1, SLOT, TREE, true>;
+    return rs_reduce_kernel<8, 1, SLOT, TREE, false>;
 }
 
-KernelFn select(int world, bool slot, int order) {
+KernelFn select(int world, bool slot, int order, bool v32) {
     const bool tree = order == TIDE_ORDER_TREE;
-    if (slot) return tree ? pick<true, true>(world) : pick<true, false>(world);
-    return tree ? pick<false, true>(world) : pick<false, false>(world);
+    if (slot) return tree ? pick<true, true>(world, v32) : pick<true, false>(world, v32);
+    return tree ? pick<false, true>(world, v32) : pick<false, false>(world, v32);
 }
 
 }  // namespace
 
-int rs_blocks_per_sm(int world, bool slot, int order) {
+bool rs_v32_applies(int world) { return world > 4 && world <= kV32MaxWorld; }
+
+int rs_blocks_per_sm(int world, bool slot, int order, bool v32) {
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, select(world, slot, order), kThreads, 0) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, select(world, slot, order, v32), kThreads, 0) !=
         cudaSuccess)
         return 0;
     return n;
@@ -158,8 +191,8 @@ int rs_blocks_per_sm(int world, bool slot, int order) {
 
 cudaError_t launch_rs_reduce(const tide_plan* p, const void* const* d_src_tab, bool slot,
                              int64_t src_bound, float* out, int64_t out_numel, float scale,
-                             bool do_scale, int order, int grid, cudaStream_t stream, int64_t t0,
-                             int64_t t1) {
+                             bool do_scale, int order, int grid, cudaStream_t stream, bool v32,
+                             int64_t t0, int64_t t1) {
     if (t1 < 0) t1 = (int64_t)p->tiles.size();
     if (t1 <= t0 || grid <= 0) return cudaSuccess;
     RsParams a;
@@ -176,7 +209,7 @@ cudaError_t launch_rs_reduce(const tide_plan* p, const void* const* d_src_tab, b
     a.do_scale = do_scale ? 1 : 0;
     a.err = p->d_err;
     (void)cudaGetLastError();  // drop an error left by an earlier failed runtime call
-    select(p->world, slot, order)<<<grid, kThreads, 0, stream>>>(a);
+    select(p->world, slot, order, v32)<<<grid, kThreads, 0, stream>>>(a);
     return cudaGetLastError();
 }
 

@@ -17,7 +17,8 @@ enum : int32_t {
 
 // Kernel ids (match tide_launch_ctas and tide_plan_last_launch).
 enum : int32_t {
-    K_RS = 0, K_AG = 1, K_STAGE = 2, K_SLOT_RS = 3, K_RS_TMA = 4, K_SLOT_RS_TMA = 5, K_COUNT = 6
+    K_RS = 0, K_AG = 1, K_STAGE = 2, K_SLOT_RS = 3, K_RS_TMA = 4, K_SLOT_RS_TMA = 5,
+    K_RS_V32 = 6, K_SLOT_RS_V32 = 7, K_COUNT = 8
 };
 
 // A device pointer table with a host mirror: re-uploaded only when it changes.
@@ -27,6 +28,7 @@ struct PtrTable {
     int64_t capacity = 0;
     bool valid = false;                  // host mirror matches the device copy
     bool aligned16 = false;              // every pointer in it is 16-byte aligned
+    bool aligned32 = false;              // every pointer in it is 32-byte aligned
 };
 
 struct tide_plan {
@@ -39,6 +41,7 @@ struct tide_plan {
     std::vector<tide_tile_t> tiles;
     std::vector<int64_t> rank_tile_begin;  // [W+1]: the tiles of output rank r are [begin[r], begin[r+1])
     bool tiles_aligned8 = true;          // every tile starts on 8-element boundaries (src and dst)
+    bool tiles_aligned16 = true;         // ... and on 16-element boundaries
     std::vector<cudaEvent_t> seg_events; // pacing events of tide_rs_reduce_pipelined (created on first use)
 
     // device tables (absent for TIDE_PLAN_HOST_ONLY)
@@ -49,7 +52,7 @@ struct tide_plan {
     int64_t workspace_bytes = 0;
 
     int32_t sm_count = 0;
-    int32_t blocks_per_sm[K_COUNT] = {0, 0, 0, 0, 0, 0};
+    int32_t blocks_per_sm[K_COUNT] = {0, 0, 0, 0, 0, 0, 0, 0};
     int32_t last_kernel = -1;            // kernel id of the last launch (-1: none or copy engines)
     int32_t last_ctas = 0;
 };
@@ -59,7 +62,8 @@ namespace tide {
 constexpr int kThreads = 256;
 
 // Occupancy (resident CTAs per SM) of each kernel at kThreads threads.
-int rs_blocks_per_sm(int world, bool slot, int order);
+int rs_blocks_per_sm(int world, bool slot, int order, bool v32);
+bool rs_v32_applies(int world);       // whether the 32-byte variant exists for this W
 int rs_tma_blocks_per_sm(int world);  // also opts the TMA kernels in to their shared memory
 int ag_blocks_per_sm();
 int stage_blocks_per_sm();
@@ -69,7 +73,7 @@ int stage_blocks_per_sm();
 cudaError_t launch_rs_reduce(const tide_plan* p, const void* const* d_src_tab, bool slot,
                              int64_t src_bound, float* out, int64_t out_numel, float scale,
                              bool do_scale, int order, int grid, cudaStream_t stream,
-                             int64_t t0 = 0, int64_t t1 = -1);
+                             bool v32 = false, int64_t t0 = 0, int64_t t1 = -1);
 cudaError_t launch_rs_reduce_tma(const tide_plan* p, const void* const* d_src_tab, bool slot,
                                  int64_t src_bound, float* out, int64_t out_numel, float scale,
                                  bool do_scale, int order, int grid, cudaStream_t stream,

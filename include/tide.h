@@ -250,11 +250,14 @@ TIDE_API tide_status_t tide_rs_reduce_noalloc(const tide_param_t* params, int32_
 /* The number of CTAs a kernel call with this max_ctas would launch (0 if that
  * kernel cannot run on this plan).  kernel: 0 = RS reduce (load/store kernel),
  * 1 = AG place, 2 = Slot-Reuse stage, 3 = slot reduce (load/store), 4 = RS
- * reduce with bulk-copy staging, 5 = slot reduce with bulk-copy staging.
+ * reduce with bulk-copy staging, 5 = slot reduce with bulk-copy staging,
+ * 6 = RS reduce with 32-byte loads, 7 = slot reduce with 32-byte loads.
  * The reductions use kernels 4/5 (one CTA per SM, TMA loads into shared memory)
  * when the plan was built with TIDE_PLAN_TMA, every tile starts on an
- * 8-element boundary and every source and the output are 16-byte aligned;
- * otherwise kernels 0/3.  Both give the same bits.  With the whole grid the
+ * 8-element boundary and every source and the output are 16-byte aligned.
+ * Otherwise they use kernels 6/7 when 5 <= W <= 16, every tile starts on a
+ * 16-element boundary and every source and the output are 32-byte aligned,
+ * else kernels 0/3.  All give the same bits.  With the whole grid the
  * load/store kernels are the faster ones on B200; the bulk-copy kernels move
  * more bytes per CTA, which matters when max_ctas is small. */
 TIDE_API tide_status_t tide_launch_ctas(const tide_plan_t* plan, int32_t kernel, int32_t max_ctas,

@@ -58,7 +58,8 @@ def test_rs_rank_order_bit_exact(group, scale, tma):
     assert np.array_equal(f32_bits(out), ref.view(np.uint32))
     kernel, ctas = plan.last_launch()
     if plan.n_tiles:
-        assert kernel in ((T.K_RS, T.K_RS_TMA) if tma else (T.K_RS,)) and ctas > 0
+        lsu = (T.K_RS, T.K_RS_V32)
+        assert kernel in (lsu + (T.K_RS_TMA,) if tma else lsu) and ctas > 0
 
 
 def aligned_group(world, seed):
@@ -174,6 +175,52 @@ def test_slot_reuse_equals_plain_and_oracle(group, engine):
         exp = np.full(group.world * L.Ns, 0xFFFF, dtype=np.uint16)   # slots started as -1 (0xFFFF)
         oracle.slot_stage(group.world, group.shapes, grads[k], exp)
         assert np.array_equal(bits_of(slots[k]), exp)
+
+
+V32_GROUPS = [aligned_group(w, 40 + w) for w in (5, 8, 13, 16)] + [configs.qwen3moe(4)]
+
+
+@pytest.mark.parametrize("group", V32_GROUPS, ids=[f"{g.name}_w{g.world}" for g in V32_GROUPS])
+def test_rs_32_byte_path(group):
+    """5 <= W <= 16 with 32-byte aligned tiles takes the 32-byte variant; same bits."""
+    grads = synth.grads_host(group, seed=34)
+    L = oracle.layout(group.world, group.shapes)
+    aligned16 = all((r * c) % 16 == 0 and (r * L.Ns + o) % 16 == 0
+                    for c, o in zip(L.c, L.off) for r in range(group.world))
+    for scale in (0, 1):
+        ref = oracle.rs_reduce(group.world, group.shapes, grads, scale)
+        for ctas in (0, 5):
+            out, _, plan = run_rs(group, grads, scale=scale, max_ctas=ctas)
+            assert plan.last_launch()[0] == (T.K_RS_V32 if aligned16 else T.K_RS)
+            assert np.array_equal(f32_bits(out), ref.view(np.uint32))
+        out, slots, plan = run_rs(group, grads, scale=scale, slots=True)
+        assert plan.last_launch()[0] == (T.K_SLOT_RS_V32 if aligned16 else T.K_SLOT_RS)
+        assert np.array_equal(f32_bits(out), ref.view(np.uint32))
+    E, A = oracle.exact_f64(group.world, group.shapes, grads)
+    out, _, _ = run_rs(group, grads, scale=0, order=1)
+    assert np.all(np.abs(out.cpu().numpy().astype(np.float64) - E) <= 1e-6 * A)
+
+
+def test_rs_32_byte_path_needs_32_byte_pointers():
+    """Gradients 16- but not 32-byte aligned fall back to the 16-byte kernel, same bits."""
+    group = mini_sweep(8)                                # tiles on 16-element boundaries
+    grads = synth.grads_host(group, seed=35)
+    plan = T.Plan(group.shapes, group.world)
+    keep, dev = [], []
+    for k in range(group.world):
+        row = []
+        for i in range(group.n_params):
+            n = group.numel(i)
+            buf = torch.empty(n + 8, dtype=torch.int16, device="cuda")
+            buf[8:] = to_dev(grads[k][i]).view(torch.int16)
+            keep.append(buf)
+            row.append(buf[8:].view(torch.bfloat16))          # 16-byte offset
+        dev.append(row)
+    out = torch.empty(group.world * plan.shard_numel, device="cuda")
+    plan.rs_reduce(dev, out)
+    torch.cuda.synchronize()
+    assert plan.last_launch()[0] == T.K_RS
+    assert np.array_equal(f32_bits(out), oracle.rs_reduce(8, group.shapes, grads, 1).view(np.uint32))
 
 
 PIPE_GROUPS = [configs.tiny(), degenerate(), mini_wan(), configs.qwen3moe(4), aligned_group(16, 5)]
