@@ -117,6 +117,49 @@ __device__ __forceinline__ void block_copy_bf16(const uint16_t* __restrict__ src
     for (int e = done + tid; e < n; e += NT) dst[e] = ld_stream_u16(src + e);
 }
 
+// 32-byte streaming store of eight 32-bit words; p must be 32-byte aligned.
+__device__ __forceinline__ void st_stream_v8(void* p, const V8& v) {
+    asm volatile("st.global.cs.v8.u32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                 :
+                 : "l"(p), "r"(v.w[0]), "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]),
+                   "r"(v.w[5]), "r"(v.w[6]), "r"(v.w[7])
+                 : "memory");
+}
+
+// As block_copy_bf16 with 32-byte vectors: source and destination must share
+// their offset modulo 32 bytes for the vector body (otherwise the 16-byte copy
+// above takes over).
+template <int U, int NT>
+__device__ __forceinline__ void block_copy_bf16_v32(const uint16_t* __restrict__ src,
+                                                    uint16_t* __restrict__ dst, int n) {
+    const uintptr_t sa = reinterpret_cast<uintptr_t>(src), da = reinterpret_cast<uintptr_t>(dst);
+    if (((sa ^ da) & 31) != 0) {
+        block_copy_bf16<2 * U, NT>(src, dst, n);
+        return;
+    }
+    const int tid = threadIdx.x;
+    int head = (int)(((32 - (da & 31)) & 31) >> 1);
+    if (head > n) head = n;
+    if (tid < head) dst[tid] = ld_stream_u16(src + tid);
+    const int nv = (n - head) >> 4;
+    const uint16_t* s = src + head;
+    uint16_t* d = dst + head;
+    for (int v0 = 0; v0 < nv; v0 += NT * U) {
+        V8 x[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int v = v0 + u * NT + tid;
+            if (v < nv) x[u] = ld_stream_v8(s + 16 * (int64_t)v);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int v = v0 + u * NT + tid;
+            if (v < nv) st_stream_v8(d + 16 * (int64_t)v, x[u]);
+        }
+    }
+    for (int e = head + 16 * nv + tid; e < n; e += NT) dst[e] = ld_stream_u16(src + e);
+}
+
 // Block-wide zero fill of n bf16 elements.
 template <int NT>
 __device__ __forceinline__ void block_zero_bf16(uint16_t* dst, int n) {
