@@ -340,14 +340,25 @@ def run_e2e(wl, K, stream):
     consecutive steps: step i+1's H2D starts once step i's kernels have
     consumed the inputs, while step i's D2H runs on the other copy direction;
     step i+1's kernels wait for step i's D2H before overwriting the outputs.
-    Returns (pipelined ms/step, serial ms/step, h2d bytes, d2h bytes).
+    Returns (pipelined ms/step, serial ms/step, h2d bytes, d2h bytes, pinned?).
     """
     import torch
     dev = wl.out.device
-    g_host = [[t.cpu().pin_memory() for t in row] for row in wl.grads]
-    ag_host = wl.ag.cpu().pin_memory()
-    out_host = torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory()
-    par_host = [torch.empty(p.shape, dtype=p.dtype).pin_memory() for p in wl.params]
+    need = (sum(t.numel() * t.element_size() for row in wl.grads for t in row) + wl.ag.numel() * 2 +
+            wl.out.numel() * 4 + sum(p.numel() * 2 for p in wl.params))
+    # every rank on this node pins its own copy; fall back to pageable host memory
+    # rather than pin more than about half of what the host has free
+    local = int(os.environ.get("LOCAL_WORLD_SIZE", "1"))
+    try:
+        import psutil
+        pin = need * local < 0.5 * psutil.virtual_memory().available
+    except Exception:
+        pin = True
+    host = (lambda t: t.pin_memory()) if pin else (lambda t: t)
+    g_host = [[host(t.cpu()) for t in row] for row in wl.grads]
+    ag_host = host(wl.ag.cpu())
+    out_host = host(torch.empty(wl.out.shape, dtype=wl.out.dtype))
+    par_host = [host(torch.empty(p.shape, dtype=p.dtype)) for p in wl.params]
     h2d = sum(t.numel() * t.element_size() for row in g_host for t in row) + ag_host.numel() * 2
     d2h = out_host.numel() * 4 + sum(p.numel() * 2 for p in par_host)
     s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
@@ -402,7 +413,7 @@ def run_e2e(wl, K, stream):
     pipelined(1)
     ms = pipelined(K)
     del g_host, ag_host, out_host, par_host
-    return ms, serial_ms, h2d, d2h
+    return ms, serial_ms, h2d, d2h, pin
 
 
 def cpu_baseline(group, seed, budget_s):
@@ -605,11 +616,12 @@ def bench_workload(args, group, rank, world, device, dist_on):
     if not args.no_variants:
         res["variants"] = run_variants(wl, max(3, min(K, 20)), stream, peak, flush)
     if not args.no_e2e:
-        e2e_ms, serial_ms, h2d, d2h = run_e2e(wl, max(1, args.e2e_steps), stream)
+        e2e_ms, serial_ms, h2d, d2h, pinned = run_e2e(wl, max(1, args.e2e_steps), stream)
         e2e_ms, serial_ms = max_over_ranks([e2e_ms, serial_ms], device)
         res["e2e"] = {"value": round(replica_throughput(world, step_bytes, e2e_ms), 2), "unit": "GB/s",
                       "serial_value": round(replica_throughput(world, step_bytes, serial_ms), 2),
                       "pipelining": "3 streams: H2D of step i+1 and D2H of step i overlap",
+                      "host_memory": "pinned" if pinned else "pageable (not enough free RAM to pin)",
                       "ms_per_step": round(e2e_ms, 3), "steps": max(1, args.e2e_steps),
                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
     del wl

@@ -111,4 +111,39 @@ __device__ __forceinline__ void reduce_ranks(int W, Load load, float (&acc)[L]) 
     }
 }
 
+// The tree order when all W <= G ranks fit in one group: the same adds as
+// reduce_ranks<G, L, true> makes for such a W (so the same bits), without the
+// group-merge stack.
+template <int G, int L, class Raw, class Load>
+__device__ __forceinline__ void tree_one_group(int W, Load load, float (&acc)[L]) {
+    Raw x[G];
+#pragma unroll
+    for (int j = 0; j < G; ++j) {
+        if (j < W) x[j] = load(j);
+    }
+    constexpr int H = (G + 1) / 2;
+    float f[H][L];
+#pragma unroll
+    for (int j = 0; j < G; j += 2) {
+#pragma unroll
+        for (int l = 0; l < L; ++l) {
+            if (j + 1 < W) f[j / 2][l] = __fadd_rn(lane(x[j], l), lane(x[j + 1], l));
+            else if (j < W) f[j / 2][l] = lane(x[j], l);
+        }
+    }
+    const int n_half = (W + 1) / 2;
+#pragma unroll
+    for (int step = 1; step < H; step <<= 1) {
+#pragma unroll
+        for (int j = 0; j + step < H; j += 2 * step) {
+            if (j + step < n_half) {
+#pragma unroll
+                for (int l = 0; l < L; ++l) f[j][l] = __fadd_rn(f[j][l], f[j + step][l]);
+            }
+        }
+    }
+#pragma unroll
+    for (int l = 0; l < L; ++l) acc[l] = f[0][l];
+}
+
 }  // namespace tide

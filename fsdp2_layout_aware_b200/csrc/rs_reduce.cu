@@ -59,7 +59,8 @@ struct RsParams {
 // V32: 32-byte loads and stores (16 outputs per thread per step); the host
 // picks it only when every tile's sources and output are 32-byte aligned
 // (a tile that is not falls back to the element loop, never faults).
-template <int G, int U, bool SLOT, bool TREE, bool V32>
+// ONE: the tree order for W <= G (a single group), without the merge stack.
+template <int G, int U, bool SLOT, bool TREE, bool V32, bool ONE>
 __global__ void __launch_bounds__(kThreads) rs_reduce_kernel(const RsParams a) {
     // s_src is double-buffered: tile i writes buffer i&1 while no thread can
     // still be reading the same buffer from tile i-2 (a barrier lies between).
@@ -110,7 +111,7 @@ __global__ void __launch_bounds__(kThreads) rs_reduce_kernel(const RsParams a) {
             for (int v = tid; v < nv16; v += kThreads) {
                 float acc[16];
                 auto load = [&](int k) { return ld_stream_v8(srcs[k] + 16 * (int64_t)v); };
-                reduce_ranks<G, 16, TREE, V8>(W, load, acc);
+                reduce_ranks<G, 16, false, V8>(W, load, acc);
                 if (a.do_scale) {
 #pragma unroll
                     for (int l = 0; l < 16; ++l) acc[l] = __fmul_rn(acc[l], a.scale);
@@ -131,7 +132,8 @@ __global__ void __launch_bounds__(kThreads) rs_reduce_kernel(const RsParams a) {
                 const int v = v0 + u * kThreads + tid;
                 if (v < nv) {
                     auto load = [&](int k) { return ld_stream_v4(srcs[k] + 8 * (int64_t)v); };
-                    reduce_ranks<G, 8, TREE, uint4>(W, load, acc[u]);
+                    if constexpr (ONE) tree_one_group<G, 8, uint4>(W, load, acc[u]);
+                    else reduce_ranks<G, 8, TREE, uint4>(W, load, acc[u]);
                 }
             }
 #pragma unroll
@@ -152,7 +154,8 @@ __global__ void __launch_bounds__(kThreads) rs_reduce_kernel(const RsParams a) {
         for (int e = 8 * nv + tid; e < tl.n_valid; e += kThreads) {
             float acc[1];
             auto load = [&](int k) { return (uint32_t)ld_stream_u16(srcs[k] + e); };
-            reduce_ranks<G, 1, TREE, uint32_t>(W, load, acc);
+            if constexpr (ONE) tree_one_group<G, 1, uint32_t>(W, load, acc);
+            else reduce_ranks<G, 1, TREE, uint32_t>(W, load, acc);
             if (a.do_scale) acc[0] = __fmul_rn(acc[0], a.scale);
             dst[e] = acc[0];
         }
@@ -165,10 +168,17 @@ using KernelFn = void (*)(const RsParams);
 
 template <bool SLOT, bool TREE>
 KernelFn pick(int world, bool v32) {
-    if (world <= 2) return rs_reduce_kernel<2, 4, SLOT, TREE, false>;
-    if (world <= 4) return rs_reduce_kernel<4, 2, SLOT, TREE, false>;
-    if (v32 && world <= kV32MaxWorld) return rs_reduce_kernel<8, 1, SLOT, TREE, true>;
-    return rs_reduce_kernel<8, 1, SLOT, TREE, false>;
+    // (in the tree order every W <= G is one group, so G < 8 kernels never merge)
+    if (world <= 2) return rs_reduce_kernel<2, 4, SLOT, TREE, false, TREE>;
+    if (world <= 4) return rs_reduce_kernel<4, 2, SLOT, TREE, false, TREE>;
+    if constexpr (TREE) {
+        // (the 32-byte variant is rank order only: the tree's 16-lane state does not fit)
+        if (world <= 8) return rs_reduce_kernel<8, 1, SLOT, true, false, true>;
+        return rs_reduce_kernel<8, 1, SLOT, true, false, false>;
+    } else {
+        if (v32 && world <= kV32MaxWorld) return rs_reduce_kernel<8, 1, SLOT, false, true, false>;
+        return rs_reduce_kernel<8, 1, SLOT, false, false, false>;
+    }
 }
 
 KernelFn select(int world, bool slot, int order, bool v32) {

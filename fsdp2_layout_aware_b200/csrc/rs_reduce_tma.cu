@@ -217,7 +217,8 @@ __global__ void __launch_bounds__(kTmaThreads, 1) rs_reduce_tma_kernel(const Tma
                     auto load = [&](int k) {
                         return *reinterpret_cast<const uint4*>(sbase + (size_t)k * sub + 8 * v);
                     };
-                    reduce_ranks<8, 8, TREE, uint4>(W, load, acc);
+                    if (TREE && W <= 8) tree_one_group<8, 8, uint4>(W, load, acc);
+                    else reduce_ranks<8, 8, TREE, uint4>(W, load, acc);
                     if (a.do_scale) {
 #pragma unroll
                         for (int l = 0; l < 8; ++l) acc[l] = __fmul_rn(acc[l], a.scale);
@@ -229,7 +230,8 @@ __global__ void __launch_bounds__(kTmaThreads, 1) rs_reduce_tma_kernel(const Tma
                 for (int e = h.n_bulk + ctid; e < h.n_valid; e += kConsumers) {
                     float acc[1];
                     auto load = [&](int k) { return (uint32_t)ld_stream_u16(psrc[k] + e); };
-                    reduce_ranks<8, 1, TREE, uint32_t>(W, load, acc);
+                    if (TREE && W <= 8) tree_one_group<8, 1, uint32_t>(W, load, acc);
+                    else reduce_ranks<8, 1, TREE, uint32_t>(W, load, acc);
                     if (a.do_scale) acc[0] = __fmul_rn(acc[0], a.scale);
                     dst[e] = acc[0];
                 }

@@ -255,9 +255,9 @@ TIDE_API tide_status_t tide_rs_reduce_noalloc(const tide_param_t* params, int32_
  * The reductions use kernels 4/5 (one CTA per SM, TMA loads into shared memory)
  * when the plan was built with TIDE_PLAN_TMA, every tile starts on an
  * 8-element boundary and every source and the output are 16-byte aligned.
- * Otherwise they use kernels 6/7 when 5 <= W <= 16, every tile starts on a
- * 16-element boundary and every source and the output are 32-byte aligned,
- * else kernels 0/3.  All give the same bits.  With the whole grid the
+ * Otherwise, in rank order, they use kernels 6/7 when 5 <= W <= 16, every
+ * tile starts on a 16-element boundary and every source and the output are
+ * 32-byte aligned; else kernels 0/3.  All give the same bits.  With the whole grid the
  * load/store kernels are the faster ones on B200; the bulk-copy kernels move
  * more bytes per CTA, which matters when max_ctas is small. */
 TIDE_API tide_status_t tide_launch_ctas(const tide_plan_t* plan, int32_t kernel, int32_t max_ctas,
