@@ -401,6 +401,54 @@ def test_side_stream_and_empty_groups():
     ep.check()
 
 
+@pytest.mark.parametrize("group", [configs.tiny(), mini_sweep(8)], ids=lambda g: g.name)
+def test_cuda_graph_capture_and_replay(group):
+    """After one uncaptured call with the same buffers (pointer tables on the device), the
+    calls capture into a CUDA graph; replays read the buffers' current contents."""
+    W = group.world
+    plan = T.Plan(group.shapes, W)
+    L = oracle.layout(W, group.shapes)
+    n = W * plan.shard_numel
+    dev = grads_to_dev(group, synth.grads_host(group, seed=94))
+    out = torch.empty(n, device="cuda")
+    out_pipe = torch.empty(n, device="cuda")
+    slots = [torch.empty(n, dtype=torch.bfloat16, device="cuda") for _ in range(W)]
+    ag = to_dev(synth.ag_host(group, L.Ns, seed=95).reshape(-1))
+    params = padded_params(plan, group)
+    cs = torch.cuda.Stream()
+    side = torch.cuda.Stream()
+
+    def step(stream):
+        plan.ag_place(ag, params, stream=stream)
+        plan.rs_reduce(dev, out, stream=stream)
+        plan.rs_reduce_pipelined(dev, out_pipe, slots, min(2, W), cs, stream=stream)
+
+    with torch.cuda.stream(side):
+        step(side)                                   # uploads the pointer tables
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        step(side)
+    for seed in (96, 97):
+        grads = synth.grads_host(group, seed=seed)
+        ag_bits = synth.ag_host(group, L.Ns, seed=seed).reshape(-1)
+        for k in range(W):
+            for i in range(group.n_params):
+                dev[k][i].copy_(to_dev(grads[k][i], group.shapes[i]))
+        ag.copy_(to_dev(ag_bits))
+        out.fill_(float("nan"))
+        out_pipe.fill_(float("nan"))
+        torch.cuda.synchronize()
+        graph.replay()
+        torch.cuda.synchronize()
+        ref = oracle.rs_reduce(W, group.shapes, grads, 1).view(np.uint32)
+        assert np.array_equal(f32_bits(out), ref)
+        assert np.array_equal(f32_bits(out_pipe), ref)
+        for p, r in zip(params, oracle.ag_copyout(W, group.shapes, ag_bits)):
+            assert np.array_equal(bits_of(p), r)
+    plan.check()
+
+
 def test_wrong_device_index_rejected():
     group = configs.tiny()
     st, h = T.tide_plan_group([(s[0], int(np.prod(s[1:]))) for s in group.shapes], 4,
