@@ -39,7 +39,8 @@ __device__ __forceinline__ V8 ld_stream_v8(const void* p) {
     return v;
 }
 
-// 32-byte streaming store of 8 floats; p must be 32-byte aligned.
+// 32-byte streaming store of 8 floats; p must be 32-byte aligned.  (Plain and
+// L1::no_allocate stores measured within 1 % of this on B200.)
 __device__ __forceinline__ void st_stream_f8(float* p, const float (&f)[8]) {
     asm volatile("st.global.cs.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
                  :
@@ -74,12 +75,6 @@ __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w 
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 __device__ __forceinline__ float bf16_one(uint16_t h) { return __uint_as_float((uint32_t)h << 16); }
 
-__device__ __forceinline__ void unpack8(const uint4& x, float f[8]) {
-    f[0] = bf16_lo(x.x); f[1] = bf16_hi(x.x);
-    f[2] = bf16_lo(x.y); f[3] = bf16_hi(x.y);
-    f[4] = bf16_lo(x.z); f[5] = bf16_hi(x.z);
-    f[6] = bf16_lo(x.w); f[7] = bf16_hi(x.w);
-}
 
 // Block-wide copy of n bf16 elements.  When source and destination share
 // their offset modulo 16 bytes, a short scalar head brings both to a 16-byte

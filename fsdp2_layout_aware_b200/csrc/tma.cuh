@@ -76,34 +76,4 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
         : "memory");
 }
 
-// Bulk copy of `bytes` (multiple of 16) from shared `src` to global `dst`
-// (both 16-byte aligned), tracked by the issuing thread's bulk group.
-__device__ __forceinline__ void bulk_s2g(void* dst, const void* src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
-                 :
-                 : "l"(dst), "r"(smem_addr(src)), "r"(bytes)
-                 : "memory");
-}
-
-__device__ __forceinline__ void bulk_commit() {
-    asm volatile("cp.async.bulk.commit_group;" : : : "memory");
-}
-
-// Wait until at most N of this thread's committed bulk groups still read shared memory.
-template <int N>
-__device__ __forceinline__ void bulk_wait_read() {
-    asm volatile("cp.async.bulk.wait_group.read %0;" : : "n"(N) : "memory");
-}
-
-// Wait until all of this thread's committed bulk groups have completed.
-__device__ __forceinline__ void bulk_wait_all() {
-    asm volatile("cp.async.bulk.wait_group 0;" : : : "memory");
-}
-
-// Order this thread's generic-proxy shared-memory accesses before later
-// async-proxy (bulk copy) accesses.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" : : : "memory");
-}
-
 }  // namespace tide
