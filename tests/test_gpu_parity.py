@@ -449,6 +449,35 @@ def test_cuda_graph_capture_and_replay(group):
     plan.check()
 
 
+def test_copy_engine_paths_launch_no_kernel():
+    """AG placement and Slot-Reuse staging on the copy engines use no SM: the CUDA
+    activity trace of those calls holds memcpy/memset records and no kernel."""
+    from torch.profiler import ProfilerActivity, profile
+    group = configs.tiny()
+    W = group.world
+    plan = T.Plan(group.shapes, W)
+    L = oracle.layout(W, group.shapes)
+    ag = to_dev(synth.ag_host(group, L.Ns, seed=98).reshape(-1))
+    params = padded_params(plan, group)
+    dev = grads_to_dev(group, synth.grads_host(group, seed=99))
+    slots = [torch.empty(W * L.Ns, dtype=torch.bfloat16, device="cuda") for _ in range(W)]
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        plan.ag_place(ag, params, engine=T.TIDE_ENGINE_CE)
+        plan.rs_stage(dev, slots, engine=T.TIDE_ENGINE_CE)
+        torch.cuda.synchronize()
+    names = [e.name for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA]
+    assert names, "no CUDA activity recorded"
+    assert all(("emcpy" in n) or ("emset" in n) for n in names), names
+    assert plan.last_launch()[0] == -1
+    # and the SM engine really launches kernels (the trace would show them)
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        plan.ag_place(ag, params, engine=T.TIDE_ENGINE_SM)
+        torch.cuda.synchronize()
+    names = [e.name for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA]
+    assert any("ag_place_kernel" in n for n in names), names
+
+
 def test_wrong_device_index_rejected():
     group = configs.tiny()
     st, h = T.tide_plan_group([(s[0], int(np.prod(s[1:]))) for s in group.shapes], 4,
