@@ -195,6 +195,10 @@ extern "C" void tide_plan_destroy(tide_plan_t* plan) {
             free_device(plan);
             for (cudaEvent_t ev : plan->seg_events) cudaEventDestroy(ev);
             plan->seg_events.clear();
+            for (cudaStream_t st : plan->ce_streams) cudaStreamDestroy(st);
+            for (cudaEvent_t ev : plan->ce_events) cudaEventDestroy(ev);
+            plan->ce_streams.clear();
+            plan->ce_events.clear();
         }
         if (prev >= 0) cudaSetDevice(prev);
     }

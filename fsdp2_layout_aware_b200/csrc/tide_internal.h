@@ -43,6 +43,8 @@ struct tide_plan {
     bool tiles_aligned8 = true;          // every tile starts on 8-element boundaries (src and dst)
     bool tiles_aligned16 = true;         // ... and on 16-element boundaries
     std::vector<cudaEvent_t> seg_events; // pacing events of tide_rs_reduce_pipelined (created on first use)
+    std::vector<cudaStream_t> ce_streams;  // copy-engine fan-out streams (created on first use)
+    std::vector<cudaEvent_t> ce_events;    // their fork event [0] and join events [1..]
 
     // device tables (absent for TIDE_PLAN_HOST_ONLY)
     tide_tile_t* d_tiles = nullptr;
@@ -85,9 +87,9 @@ cudaError_t launch_slot_stage(const tide_plan* p, const void* const* d_grad_tab,
                               cudaStream_t stream);
 
 // Copy-engine variants (no kernels).
-cudaError_t ce_ag_place(const tide_plan* p, const uint16_t* ag, void* const* params,
+cudaError_t ce_ag_place(tide_plan* p, const uint16_t* ag, void* const* params,
                         cudaStream_t stream);
-cudaError_t ce_slot_stage(const tide_plan* p, const void* const* grads, void* const* slots,
+cudaError_t ce_slot_stage(tide_plan* p, const void* const* grads, void* const* slots,
                           cudaStream_t stream, int64_t r0 = 0, int64_t r1 = -1);
 
 }  // namespace tide

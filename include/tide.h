@@ -42,8 +42,13 @@
  *     tide_rs_reduce_slots, tide_rs_reduce_pipelined) can be captured into a
  *     CUDA graph once the same buffers have been used in an uncaptured call on
  *     the same plan (that call uploads the pointer tables and creates the
- *     pipeline's events; a capture that needs an upload fails with
- *     TIDE_ERR_CUDA).  Replays read the buffers' current contents.
+ *     pipeline's events and the copy-engine streams; a capture that needs an
+ *     upload fails with TIDE_ERR_CUDA).  Replays read the buffers' current
+ *     contents.
+ *   - TIDE_ENGINE_CE calls spread their memcpys over 8 streams that the plan
+ *     creates on first use (no device memory), forked from the call's stream
+ *     with an event and joined back to it before the call returns; work
+ *     enqueued on the call's stream afterwards sees every copy.
  */
 #ifndef TIDE_H
 #define TIDE_H
