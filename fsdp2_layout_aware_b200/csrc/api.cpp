@@ -199,6 +199,32 @@ tide_status_t reduce_slots_impl(tide_plan* p, void* const* slots, int64_t slot_n
     return e == cudaSuccess ? TIDE_OK : TIDE_ERR_CUDA;
 }
 
+// Cut the chunks, in tile order (chunk i*W + r), into n contiguous segments
+// that hold about equal numbers of valid elements, so that the copy engines
+// stage about the same bytes for each.  Segment s is [b[s], b[s+1]).  Cut this
+// way, a segment copies only the params it holds: about W*(P + n) copies in
+// all, where cutting by output ranks would copy every param in every segment
+// (W*P*n copies, which is what limits groups of many small params).
+std::vector<int64_t> segment_bounds(const tide_plan* p, int32_t n) {
+    const int64_t W = p->world, J = (int64_t)p->n_params * W;
+    auto valid = [&](int64_t j) {
+        const int64_t i = j / W, r = j % W, c = p->chunk[i];
+        return std::min(c, std::max<int64_t>(0, p->numel[i] - r * c));
+    };
+    long double total = 0;
+    for (int64_t i = 0; i < p->n_params; ++i) total += (long double)p->numel[i];
+    std::vector<int64_t> b((size_t)n + 1, J);
+    b[0] = 0;
+    long double acc = 0;
+    int64_t j = 0;
+    for (int32_t s = 1; s < n; ++s) {
+        const long double target = total * s / n;
+        while (j < J && acc < target) acc += (long double)valid(j++);
+        b[s] = j;
+    }
+    return b;
+}
+
 }  // namespace
 
 extern "C" tide_status_t tide_ag_place(const tide_plan_t* cplan, const void* ag_buf,
@@ -342,17 +368,18 @@ extern "C" tide_status_t tide_rs_reduce_pipelined(const tide_plan_t* cplan, cons
     cudaEvent_t start = p->seg_events[n_segments];
     if (cudaEventRecord(start, s) != cudaSuccess || cudaStreamWaitEvent(cs, start, 0) != cudaSuccess)
         return TIDE_ERR_CUDA;
+    const std::vector<int64_t> bounds = segment_bounds(p, n_segments);
     for (int32_t seg = 0; seg < n_segments; ++seg) {
-        const int64_t r0 = W * seg / n_segments, r1 = W * (seg + 1) / n_segments;
-        if (r1 == r0) continue;
-        // phase 1 of these output ranks on the copy engines ...
-        if (tide::ce_slot_stage(p, grads, slots, cs, r0, r1) != cudaSuccess) return TIDE_ERR_CUDA;
+        const int64_t j0 = bounds[seg], j1 = bounds[seg + 1];
+        if (j1 == j0) continue;
+        // phase 1 of these chunks on the copy engines ...
+        if (tide::ce_slot_stage(p, grads, slots, cs, j0, j1) != cudaSuccess) return TIDE_ERR_CUDA;
         cudaEvent_t done = p->seg_events[seg];
         if (cudaEventRecord(done, cs) != cudaSuccess || cudaStreamWaitEvent(s, done, 0) != cudaSuccess)
             return TIDE_ERR_CUDA;
         // ... phase 2 of them on the SMs, while the next segment is being copied
         if (launch_reduce(p, p->slot_tab, true, slot_numel, out, out_numel, scale_mode, order, max_ctas,
-                          s, p->rank_tile_begin[r0], p->rank_tile_begin[r1]) != cudaSuccess)
+                          s, p->chunk_tile_begin[j0], p->chunk_tile_begin[j1]) != cudaSuccess)
             return TIDE_ERR_CUDA;
     }
     return TIDE_OK;

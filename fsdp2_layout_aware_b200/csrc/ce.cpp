@@ -22,13 +22,22 @@
 namespace tide {
 namespace {
 
-// Copy `rows` rows of `width` bytes; falls back to one 1-D copy per row when a
-// pitch exceeds the device limit.
+// Rows at least this wide go as one 1-D copy each.  Measured on B200: 2-D
+// device-to-device copies stay near 3.4 TB/s whatever the number of streams,
+// while 1-D copies on several streams reach HBM bandwidth; below a few MB a row,
+// the fixed cost of each extra copy call (about 3 us) outweighs that.  Staging
+// for Slot-Reuse (70B / Qwen3 / Wan2.2 groups, ms): all 2-D 7.72 / 10.78 / 6.63;
+// split from 256 KB 4.31 / 79.4 / 10.9; from 1 MB 4.31 / 11.3 / 11.1; from
+// 4 MB 4.38 / 10.8 / 5.57.
+constexpr size_t kRowSplitBytes = size_t(4) << 20;
+
+// Copy `rows` rows of `width` bytes: one 2-D copy, or one 1-D copy per row when
+// the rows are wide or a pitch exceeds the device limit.
 cudaError_t copy_rows(void* dst, size_t dpitch, const void* src, size_t spitch, size_t width,
                       int64_t rows, size_t max_pitch, cudaStream_t stream) {
     if (rows <= 0 || width == 0) return cudaSuccess;
     if (rows == 1) return cudaMemcpyAsync(dst, src, width, cudaMemcpyDeviceToDevice, stream);
-    if (dpitch <= max_pitch && spitch <= max_pitch)
+    if (dpitch <= max_pitch && spitch <= max_pitch && width < kRowSplitBytes)
         return cudaMemcpy2DAsync(dst, dpitch, src, spitch, width, (size_t)rows,
                                  cudaMemcpyDeviceToDevice, stream);
     for (int64_t r = 0; r < rows; ++r) {
@@ -119,12 +128,15 @@ cudaError_t ce_ag_place(tide_plan* p, const uint16_t* ag, void* const* params, c
     return e != cudaSuccess ? e : j;
 }
 
-// Stage the chunks that output ranks [r0, r1) need (r1 < 0: up to W) from every
-// source rank k into slot k.
+// Stage the chunks [j0, j1) (chunk i*W + r: rank r's rows of param i) from
+// every source rank k into slot k.  Within one param the chunks of a range are
+// consecutive ranks, so each (k, param) pair takes one 2-D copy plus at most
+// one 1-D copy for a partial chunk.
 cudaError_t ce_slot_stage(tide_plan* p, const void* const* grads, void* const* slots,
-                          cudaStream_t caller, int64_t r0, int64_t r1) {
+                          cudaStream_t caller, int64_t j0, int64_t j1) {
     const int64_t W = p->world, P = p->n_params, Ns = p->shard_numel;
-    if (r1 < 0) r1 = W;
+    if (j1 < 0) j1 = P * W;
+    if (j1 <= j0) return cudaSuccess;
     const size_t max_pitch = device_max_pitch(p->device);
     cudaError_t fe = fork(p, caller);
     if (fe != cudaSuccess) return fe;
@@ -132,9 +144,10 @@ cudaError_t ce_slot_stage(tide_plan* p, const void* const* grads, void* const* s
     for (int64_t k = 0; res == cudaSuccess && k < W; ++k) {
         cudaStream_t stream = p->ce_streams[k % kFanout];  // one source rank per stream at a time
         uint16_t* slot = static_cast<uint16_t*>(slots[k]);
-        for (int64_t i = 0; i < P; ++i) {
+        for (int64_t i = j0 / W; i <= (j1 - 1) / W; ++i) {
             const int64_t c = p->chunk[i], n = p->numel[i];
             if (c == 0 || n == 0) continue;
+            const int64_t r0 = std::max<int64_t>(0, j0 - i * W), r1 = std::min<int64_t>(W, j1 - i * W);
             const uint16_t* g = static_cast<const uint16_t*>(grads[k * P + i]);
             uint16_t* dst = slot + p->offset[i];
             const int64_t full = std::min(W, n / c);  // ranks [0, full) hold whole chunks

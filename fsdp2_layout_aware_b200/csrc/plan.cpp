@@ -148,11 +148,12 @@ extern "C" tide_status_t tide_plan_group(const tide_param_t* params, int32_t n_p
         }
         if (!mul_ok(W, acc)) { delete p; return TIDE_ERR_SIZE; }
         p->shard_numel = acc;
-        // tiles in rank-major buffer order: rank, then param, then position
-        p->rank_tile_begin.assign(W + 1, 0);
-        for (int64_t r = 0; r < W; ++r) {
-            p->rank_tile_begin[r] = (int64_t)p->tiles.size();
-            for (int32_t i = 0; i < n_params; ++i) {
+        // tiles in chunk order: param, then rank, then position; the chunk
+        // (i, r) is number i*W + r and holds tiles [begin[i*W+r], begin[i*W+r+1])
+        p->chunk_tile_begin.assign((size_t)n_params * W + 1, 0);
+        for (int32_t i = 0; i < n_params; ++i) {
+            for (int64_t r = 0; r < W; ++r) {
+                p->chunk_tile_begin[(size_t)i * W + r] = (int64_t)p->tiles.size();
                 const int64_t c = p->chunk[i];
                 const int64_t valid = std::min(c, std::max<int64_t>(0, p->numel[i] - r * c));
                 for (int64_t e0 = 0; e0 < c; e0 += TIDE_TILE_ELEMS) {
@@ -169,7 +170,7 @@ extern "C" tide_status_t tide_plan_group(const tide_param_t* params, int32_t n_p
                 }
             }
         }
-        p->rank_tile_begin[W] = (int64_t)p->tiles.size();
+        p->chunk_tile_begin[(size_t)n_params * W] = (int64_t)p->tiles.size();
     } catch (const std::bad_alloc&) {
         delete p;
         return TIDE_ERR_NOMEM;

@@ -39,7 +39,7 @@ struct tide_plan {
     int64_t shard_numel = 0;             // Ns
     std::vector<int64_t> dim0, inner, numel, rows, chunk, offset;   // per param: d0, inner, d0*inner, S, c, off
     std::vector<tide_tile_t> tiles;
-    std::vector<int64_t> rank_tile_begin;  // [W+1]: the tiles of output rank r are [begin[r], begin[r+1])
+    std::vector<int64_t> chunk_tile_begin;  // [P*W+1]: chunk (i, r) holds tiles [begin[i*W+r], begin[i*W+r+1])
     bool tiles_aligned8 = true;          // every tile starts on 8-element boundaries (src and dst)
     bool tiles_aligned16 = true;         // ... and on 16-element boundaries
     std::vector<cudaEvent_t> seg_events; // pacing events of tide_rs_reduce_pipelined (created on first use)
@@ -89,7 +89,9 @@ cudaError_t launch_slot_stage(const tide_plan* p, const void* const* d_grad_tab,
 // Copy-engine variants (no kernels).
 cudaError_t ce_ag_place(tide_plan* p, const uint16_t* ag, void* const* params,
                         cudaStream_t stream);
+// Stages the chunks [j0, j1) (numbered i*W + r as in chunk_tile_begin; j1 < 0:
+// all) from every source rank k into slot k.
 cudaError_t ce_slot_stage(tide_plan* p, const void* const* grads, void* const* slots,
-                          cudaStream_t stream, int64_t r0 = 0, int64_t r1 = -1);
+                          cudaStream_t stream, int64_t j0 = 0, int64_t j1 = -1);
 
 }  // namespace tide

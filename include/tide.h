@@ -206,9 +206,11 @@ TIDE_API tide_status_t tide_rs_reduce_slots(const tide_plan_t* plan, const void*
  * Slot-Reuse with the two phases overlapped (weekinpapers.com Abstract: the
  * two-phase pipeline keeps gradient reads apart from the reduction's
  * progress, and copy engines move the gradients).  Same result as
- * tide_rs_reduce with the same slots (same bits).  The output ranks are split
- * into n_segments contiguous groups (1 <= n_segments <= W).  For each group,
- * phase 1 stages the chunks those ranks need into the slots with copy-engine
+ * tide_rs_reduce with the same slots (same bits).  The (param, rank) chunks,
+ * taken param by param and within a param rank by rank, are cut into
+ * n_segments contiguous groups of about equal valid elements
+ * (1 <= n_segments <= W; a group may be empty).  For each group, phase 1
+ * stages its chunks from every source rank into the slots with copy-engine
  * memcpys on `copy_stream`, then phase 2 reduces them on `stream` (one kernel
  * launch per group) while the copy engines already stage the next group.
  * Work enqueued on `stream` before the call is ordered before the copies;

@@ -69,7 +69,7 @@ def check_tiles(group):
     assert len(tiles) == plan.n_tiles
     W, Ns = group.world, L.Ns
     cover = np.zeros(W * Ns, dtype=np.int32)
-    last = -1
+    last = (-1, -1, -1)
     for t in tiles:
         i, r = t.param, t.rank
         assert 0 <= i < group.n_params and 0 <= r < W
@@ -77,8 +77,9 @@ def check_tiles(group):
         e0 = t.src_off - r * L.c[i]
         assert e0 % T.TIDE_TILE_ELEMS == 0 and 0 <= e0 < L.c[i]
         assert t.dst_off == r * Ns + L.off[i] + e0
-        assert t.dst_off > last                      # sorted by output position
-        last = t.dst_off
+        key = (i, r, e0)                             # chunk order: param, rank, position
+        assert key > last
+        last = key
         assert t.n_valid == min(t.n_total, max(0, group.numel(i) - t.src_off))
         cover[t.dst_off: t.dst_off + t.n_total] += 1
         # validity agrees with the oracle's per-position locate, at both ends

@@ -223,7 +223,10 @@ def test_rs_32_byte_path_needs_32_byte_pointers():
     assert np.array_equal(f32_bits(out), oracle.rs_reduce(8, group.shapes, grads, 1).view(np.uint32))
 
 
-PIPE_GROUPS = [configs.tiny(), degenerate(), mini_wan(), configs.qwen3moe(4), aligned_group(16, 5)]
+# pad_tail: with 4 segments, the cut by valid elements leaves two groups empty
+# and a last group of all-pad chunks and empty params (nothing to stage).
+PIPE_GROUPS = [configs.tiny(), degenerate(), mini_wan(), configs.qwen3moe(4), aligned_group(16, 5),
+               configs.Group("pad_tail", 4, ((8, 4), (1, 1000), (0, 3)))]
 
 
 @pytest.mark.parametrize("group", PIPE_GROUPS, ids=[f"{g.name}_w{g.world}" for g in PIPE_GROUPS])
