@@ -155,7 +155,9 @@ cudaError_t launch_reduce(tide_plan* p, PtrTable& tab, bool slot, int64_t bound,
     const int k_v32 = slot ? K_SLOT_RS_V32 : K_RS_V32;
     const bool tma = use_tma(p, tab, out, k_tma);
     const bool v32 = !tma && order == TIDE_ORDER_RANK && use_v32(p, tab, out, k_v32);
-    const int kernel = tma ? k_tma : v32 ? k_v32 : (slot ? K_SLOT_RS : K_RS);
+    const bool tree = order == TIDE_ORDER_TREE;
+    const int kernel = tma ? k_tma : v32 ? k_v32 : tree ? (slot ? K_SLOT_RS_TREE : K_RS_TREE)
+                                                        : (slot ? K_SLOT_RS : K_RS);
     if (t1 < 0) t1 = (int64_t)p->tiles.size();
     const int grid = (int)std::min<int64_t>(grid_for(p, kernel, max_ctas), t1 - t0);
     p->last_kernel = kernel;

@@ -90,9 +90,11 @@ tide_status_t upload(tide_plan* p) {
             p->blocks_per_sm[K_RS_V32] = tide::rs_blocks_per_sm(p->world, false, TIDE_ORDER_RANK, true);
             p->blocks_per_sm[K_SLOT_RS_V32] = tide::rs_blocks_per_sm(p->world, true, TIDE_ORDER_RANK, true);
         }
+        p->blocks_per_sm[K_RS_TREE] = tide::rs_blocks_per_sm(p->world, false, TIDE_ORDER_TREE, false);
+        p->blocks_per_sm[K_SLOT_RS_TREE] = tide::rs_blocks_per_sm(p->world, true, TIDE_ORDER_TREE, false);
         p->blocks_per_sm[K_AG] = tide::ag_blocks_per_sm();
         p->blocks_per_sm[K_STAGE] = tide::stage_blocks_per_sm();
-        for (int k = 0; k < K_RS_TMA; ++k)
+        for (int k : {K_RS, K_AG, K_STAGE, K_SLOT_RS, K_RS_TREE, K_SLOT_RS_TREE})
             if (p->blocks_per_sm[k] <= 0) st = TIDE_ERR_CUDA;
         // 0 here (not enough shared memory) only disables the bulk-copy path
         p->blocks_per_sm[K_RS_TMA] = p->blocks_per_sm[K_SLOT_RS_TMA] = tide::rs_tma_blocks_per_sm(p->world);

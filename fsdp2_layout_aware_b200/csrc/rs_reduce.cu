@@ -60,8 +60,14 @@ struct RsParams {
 // picks it only when every tile's sources and output are 32-byte aligned
 // (a tile that is not falls back to the element loop, never faults).
 // ONE: the tree order for W <= G (a single group), without the merge stack.
+// The single-group tree kernels are held to 3 CTAs per SM (80 registers, a
+// spill of 88 bytes per thread at G = 8): left free they take 128 registers
+// and 2 CTAs per SM, 4 % slower on B200 (70B W=8: 6.52 vs 6.28 TB/s; Qwen3:
+// 6.47 vs 6.19).  The others keep the compiler's choice (an explicit minimum
+// of 1 CTA raised the rank-order kernels' registers and cost bandwidth).
 template <int G, int U, bool SLOT, bool TREE, bool V32, bool ONE>
-__global__ void __launch_bounds__(kThreads) rs_reduce_kernel(const RsParams a) {
+__global__ void __launch_bounds__(kThreads, (TREE && ONE) ? 3 : 0)
+rs_reduce_kernel(const RsParams a) {
     // s_src is double-buffered: tile i writes buffer i&1 while no thread can
     // still be reading the same buffer from tile i-2 (a barrier lies between).
     __shared__ const uint16_t* s_src[2][TIDE_MAX_WORLD];

@@ -18,7 +18,7 @@ enum : int32_t {
 // Kernel ids (match tide_launch_ctas and tide_plan_last_launch).
 enum : int32_t {
     K_RS = 0, K_AG = 1, K_STAGE = 2, K_SLOT_RS = 3, K_RS_TMA = 4, K_SLOT_RS_TMA = 5,
-    K_RS_V32 = 6, K_SLOT_RS_V32 = 7, K_COUNT = 8
+    K_RS_V32 = 6, K_SLOT_RS_V32 = 7, K_RS_TREE = 8, K_SLOT_RS_TREE = 9, K_COUNT = 10
 };
 
 // A device pointer table with a host mirror: re-uploaded only when it changes.
@@ -54,7 +54,7 @@ struct tide_plan {
     int64_t workspace_bytes = 0;
 
     int32_t sm_count = 0;
-    int32_t blocks_per_sm[K_COUNT] = {0, 0, 0, 0, 0, 0, 0, 0};
+    int32_t blocks_per_sm[K_COUNT] = {};
     int32_t last_kernel = -1;            // kernel id of the last launch (-1: none or copy engines)
     int32_t last_ctas = 0;
 };

@@ -37,8 +37,10 @@ TIDE_MAX_WORLD = 256
 TIDE_TILE_ELEMS = 8192
 TIDE_NOALLOC_SCRATCH_BYTES = 1 << 20
 
-K_RS, K_AG, K_STAGE, K_SLOT_RS, K_RS_TMA, K_SLOT_RS_TMA, K_RS_V32, K_SLOT_RS_V32 = range(8)
-KERNEL_NAMES = ("rs", "ag", "stage", "slot_rs", "rs_tma", "slot_rs_tma", "rs_v32", "slot_rs_v32")
+(K_RS, K_AG, K_STAGE, K_SLOT_RS, K_RS_TMA, K_SLOT_RS_TMA, K_RS_V32, K_SLOT_RS_V32, K_RS_TREE,
+ K_SLOT_RS_TREE) = range(10)
+KERNEL_NAMES = ("rs", "ag", "stage", "slot_rs", "rs_tma", "slot_rs_tma", "rs_v32", "slot_rs_v32",
+                "rs_tree", "slot_rs_tree")
 
 
 class tide_param_t(ctypes.Structure):

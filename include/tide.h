@@ -264,13 +264,15 @@ TIDE_API tide_status_t tide_rs_reduce_noalloc(const tide_param_t* params, int32_
  * kernel cannot run on this plan).  kernel: 0 = RS reduce (load/store kernel),
  * 1 = AG place, 2 = Slot-Reuse stage, 3 = slot reduce (load/store), 4 = RS
  * reduce with bulk-copy staging, 5 = slot reduce with bulk-copy staging,
- * 6 = RS reduce with 32-byte loads, 7 = slot reduce with 32-byte loads.
+ * 6 = RS reduce with 32-byte loads, 7 = slot reduce with 32-byte loads,
+ * 8 = RS reduce in tree order, 9 = slot reduce in tree order.
  * The reductions use kernels 4/5 (one CTA per SM, TMA loads into shared memory)
  * when the plan was built with TIDE_PLAN_TMA, every tile starts on an
  * 8-element boundary and every source and the output are 16-byte aligned.
  * Otherwise, in rank order, they use kernels 6/7 when 5 <= W <= 16, every
  * tile starts on a 16-element boundary and every source and the output are
- * 32-byte aligned; else kernels 0/3.  All give the same bits.  With the whole grid the
+ * 32-byte aligned; else kernels 0/3.  In tree order they use kernels 8/9.
+ * Kernels of the same order give the same bits.  With the whole grid the
  * load/store kernels are the faster ones on B200; the bulk-copy kernels move
  * more bytes per CTA, which matters when max_ctas is small. */
 TIDE_API tide_status_t tide_launch_ctas(const tide_plan_t* plan, int32_t kernel, int32_t max_ctas,

@@ -106,7 +106,9 @@ def test_rs_tiny_all_seeds(seed):
 @pytest.mark.parametrize("group", GROUPS, ids=IDS)
 def test_rs_tree_order_within_tolerance(group):
     grads = synth.grads_host(group, seed=32)
-    out, _, _ = run_rs(group, grads, scale=0, order=1)
+    out, _, plan = run_rs(group, grads, scale=0, order=1)
+    if plan.n_tiles:   # the tree kernel, on the grid its own occupancy gives
+        assert plan.last_launch() == (T.K_RS_TREE, plan.launch_ctas(T.K_RS_TREE, 0))
     E, A = oracle.exact_f64(group.world, group.shapes, grads)
     got = out.cpu().numpy().astype(np.float64)
     assert np.all(np.abs(got - E) <= 1e-6 * A)
@@ -115,6 +117,20 @@ def test_rs_tree_order_within_tolerance(group):
     ref = oracle.rs_reduce(group.world, group.shapes, grads, 0)
     pad[np.nonzero(A)[0]] = False
     assert np.all(f32_bits(out)[A == 0] == ref.view(np.uint32)[A == 0])   # zeros / pads agree bitwise
+
+
+@pytest.mark.parametrize("group", GROUPS, ids=IDS)
+def test_tree_order_kernels_agree_bitwise(group):
+    """Every tree-order kernel adds in the same tree: pairwise by levels, an odd one carried.
+    Load/store (groups of 2, 4 or 8 ranks merged pairwise), bulk-copy, Slot-Reuse on SMs or
+    copy engines, and any CTA count give the same bits."""
+    grads = synth.grads_host(group, seed=35)
+    ref, _, _ = run_rs(group, grads, scale=1, order=1)
+    ref = f32_bits(ref)
+    for kw in (dict(max_ctas=3), dict(tma=True), dict(slots=True),
+               dict(slots=True, engine=T.TIDE_ENGINE_CE)):
+        out, _, _ = run_rs(group, grads, scale=1, order=1, **kw)
+        assert np.array_equal(f32_bits(out), ref), kw
 
 
 @pytest.mark.parametrize("W", [2, 4, 8, 16, 64, 256])
@@ -268,6 +284,7 @@ def test_slot_phases_separately():
     for order in (0, 1):
         plan.rs_reduce_slots(slots, out, scale_mode=0, order=order)
         torch.cuda.synchronize()
+        assert plan.last_launch()[0] == (T.K_SLOT_RS_TREE if order else T.K_SLOT_RS)
         if order == 0:
             assert np.array_equal(f32_bits(out),
                                   oracle.rs_reduce(group.world, group.shapes, grads, 0).view(np.uint32))
