@@ -387,7 +387,8 @@ extern "C" tide_status_t tide_rs_reduce_pipelined(const tide_plan_t* cplan, cons
     return TIDE_OK;
 }
 
-extern "C" tide_status_t tide_plan_check(tide_plan_t* p, void* stream) {
+extern "C" tide_status_t tide_plan_errors(tide_plan_t* p, void* stream, int32_t* bits) {
+    if (bits != nullptr) *bits = 0;
     tide_status_t st = check_plan(p);
     if (st != TIDE_OK) return st;
     if ((st = launchable(p)) != TIDE_OK) return st;
@@ -396,9 +397,14 @@ extern "C" tide_status_t tide_plan_check(tide_plan_t* p, void* stream) {
     if (cudaMemcpyAsync(&h, p->d_err, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
         cudaStreamSynchronize(s) != cudaSuccess)
         return TIDE_ERR_CUDA;
+    if (bits != nullptr) *bits = h;
     if (h == 0) return TIDE_OK;
     if (cudaMemsetAsync(p->d_err, 0, sizeof(int32_t), s) != cudaSuccess ||
         cudaStreamSynchronize(s) != cudaSuccess)
         return TIDE_ERR_CUDA;
     return TIDE_ERR_KERNEL_CHECK;
+}
+
+extern "C" tide_status_t tide_plan_check(tide_plan_t* p, void* stream) {
+    return tide_plan_errors(p, stream, nullptr);
 }

@@ -116,7 +116,8 @@ extern "C" tide_status_t tide_plan_group(const tide_param_t* params, int32_t n_p
     *out_plan = nullptr;
     if (n_params < 0 || (n_params > 0 && params == nullptr)) return TIDE_ERR_INVALID_ARG;
     if (world < 1 || world > TIDE_MAX_WORLD) return TIDE_ERR_INVALID_ARG;
-    if ((flags & ~(uint32_t)(TIDE_PLAN_HOST_ONLY | TIDE_PLAN_TMA)) != 0) return TIDE_ERR_INVALID_ARG;
+    if ((flags & ~(uint32_t)(TIDE_PLAN_HOST_ONLY | TIDE_PLAN_TMA | TIDE_PLAN_TEST_TMA_TIMEOUT)) != 0)
+        return TIDE_ERR_INVALID_ARG;
     if (!(flags & TIDE_PLAN_HOST_ONLY) && device < 0) return TIDE_ERR_DEVICE;
 
     tide_plan* p = new (std::nothrow) tide_plan;

@@ -67,6 +67,7 @@ struct TmaParams {
     int32_t sub;                 // elements per rank per stage (multiple of 8)
     float scale;
     int32_t do_scale;
+    int32_t withhold;            // test hook: CTA 0 withholds its first stage (its wait then runs out)
     int32_t* err;
 };
 
@@ -108,6 +109,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1) rs_reduce_tma_kernel(const Tma
         uint32_t pending = 0;     // stages whose last issue carried bulk bytes
         uint32_t pend_par = 0;    // parity of that issue, per stage bit
         bool aborted = false;
+        bool withhold = a.withhold != 0 && blockIdx.x == 0;  // warp-uniform
         int64_t t = blockIdx.x;
         tide_tile_t next = t < a.n_tiles ? a.tiles[t] : tide_tile_t{};
         for (; t < a.n_tiles && !aborted; t += gridDim.x) {
@@ -158,12 +160,12 @@ __global__ void __launch_bounds__(kTmaThreads, 1) rs_reduce_tma_kernel(const Tma
                     hdr[stage] = h;
                 }
                 __syncwarp();
-                if (lane == 0) {
+                if (lane == 0 && !withhold) {
                     if (n_bulk > 0) mbar_arrive_expect_tx(&full[stage], (uint32_t)(W * n_bulk * 2));
                     else mbar_arrive(&full[stage]);
                 }
                 __syncwarp();
-                if (n_bulk > 0) {
+                if (n_bulk > 0 && !withhold) {
 #pragma unroll
                     for (int j = 0; j < kPtrsPerLane; ++j) {
                         const int k = lane + 32 * j;
@@ -176,6 +178,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1) rs_reduce_tma_kernel(const Tma
                 } else {
                     pending &= ~(1u << stage);
                 }
+                withhold = false;
                 if (++stage == kStages) {
                     stage = 0;
                     phase ^= 1;
@@ -316,6 +319,7 @@ cudaError_t launch_rs_reduce_tma(const tide_plan* p, const void* const* d_src_ta
     a.sub = sub_for(p->world);
     a.scale = scale;
     a.do_scale = do_scale ? 1 : 0;
+    a.withhold = (p->flags & TIDE_PLAN_TEST_TMA_TIMEOUT) ? 1 : 0;
     a.err = p->d_err;
     (void)cudaGetLastError();  // drop an error left by an earlier failed runtime call
     select_tma(slot, order)<<<grid, kTmaThreads, smem_for(p->world), stream>>>(a);

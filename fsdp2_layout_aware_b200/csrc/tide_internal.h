@@ -9,12 +9,6 @@
 
 #include "tide.h"
 
-// Bits of the device error word.
-enum : int32_t {
-    TIDE_KCHECK_TILE = 1,     // a tile descriptor pointed outside its buffers
-    TIDE_KCHECK_TIMEOUT = 2,  // a bounded mbarrier wait gave up
-};
-
 // Kernel ids (match tide_launch_ctas and tide_plan_last_launch).
 enum : int32_t {
     K_RS = 0, K_AG = 1, K_STAGE = 2, K_SLOT_RS = 3, K_RS_TMA = 4, K_SLOT_RS_TMA = 5,

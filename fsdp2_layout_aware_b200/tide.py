@@ -33,6 +33,8 @@ TIDE_SCALE_NONE = 0
 TIDE_SCALE_INV_WORLD = 1
 TIDE_PLAN_HOST_ONLY = 1
 TIDE_PLAN_TMA = 2
+TIDE_PLAN_TEST_TMA_TIMEOUT = 4
+TIDE_KCHECK_TILE, TIDE_KCHECK_TIMEOUT = 1, 2
 TIDE_MAX_WORLD = 256
 TIDE_TILE_ELEMS = 8192
 TIDE_NOALLOC_SCRATCH_BYTES = 1 << 20
@@ -80,6 +82,7 @@ _SIGNATURES = {
     "tide_rs_reduce_pipelined": (_i32, [_vp, _P(_vp), _P(_i64), _vp, _i64, _i32, _i32, _P(_vp),
                                         _i64, _i32, _i32, _vp, _vp]),
     "tide_plan_check": (_i32, [_vp, _vp]),
+    "tide_plan_errors": (_i32, [_vp, _vp, _P(_i32)]),
     "tide_launch_ctas": (_i32, [_vp, _i32, _i32, _P(_i32)]),
     "tide_plan_last_launch": (_i32, [_vp, _P(_i32), _P(_i32)]),
     "tide_status_string": (ctypes.c_char_p, [_i32]),
@@ -222,6 +225,12 @@ def tide_plan_check(plan, stream: int) -> int:
     return lib().tide_plan_check(plan, stream)
 
 
+def tide_plan_errors(plan, stream: int):
+    bits = ctypes.c_int32(0)
+    st = lib().tide_plan_errors(plan, stream, ctypes.byref(bits))
+    return st, bits.value
+
+
 def tide_plan_last_launch(plan):
     k, n = _i32(), _i32()
     st = lib().tide_plan_last_launch(plan, ctypes.byref(k), ctypes.byref(n))
@@ -252,7 +261,7 @@ class Plan:
     """
 
     def __init__(self, shapes, world: int, device=None, host_only: bool = False,
-                 tma: bool = False):
+                 tma: bool = False, test_tma_timeout: bool = False):
         self.shapes = [tuple(int(d) for d in s) for s in shapes]
         self.world = int(world)
         if host_only:
@@ -262,7 +271,8 @@ class Plan:
             dev = torch.cuda.current_device() if device is None else torch.device(device).index
             dev = 0 if dev is None else dev
         params = [(s[0], _prod(s[1:])) for s in self.shapes]
-        flags = (TIDE_PLAN_HOST_ONLY if host_only else 0) | (TIDE_PLAN_TMA if tma else 0)
+        flags = ((TIDE_PLAN_HOST_ONLY if host_only else 0) | (TIDE_PLAN_TMA if tma else 0) |
+                 (TIDE_PLAN_TEST_TMA_TIMEOUT if test_tma_timeout else 0))
         st, handle = tide_plan_group(params, self.world, dev, flags)
         _check(st, "tide_plan_group")
         self.handle = handle
@@ -353,6 +363,13 @@ class Plan:
 
     def check(self, stream=None) -> None:
         _check(tide_plan_check(self.handle, _stream_handle(stream)), "tide_plan_check")
+
+    def errors(self, stream=None) -> int:
+        """Read and clear the device error word; its TIDE_KCHECK_* bits (0 if none)."""
+        st, bits = tide_plan_errors(self.handle, _stream_handle(stream))
+        if st not in (TIDE_OK, TIDE_ERR_KERNEL_CHECK):
+            _check(st, "tide_plan_errors")
+        return bits
 
 
 def _prod(dims) -> int:

@@ -81,7 +81,13 @@ enum { TIDE_ORDER_RANK = 0, TIDE_ORDER_TREE = 1 };
 enum { TIDE_SCALE_NONE = 0, TIDE_SCALE_INV_WORLD = 1 };
 enum {
     TIDE_PLAN_HOST_ONLY = 1, /* flag: build the tables on the host only (no CUDA calls) */
-    TIDE_PLAN_TMA = 2        /* flag: reduce with the bulk-copy (TMA) kernel where it applies */
+    TIDE_PLAN_TMA = 2,       /* flag: reduce with the bulk-copy (TMA) kernel where it applies */
+    /* flag, test hook for the timeout path: with TIDE_PLAN_TMA, CTA 0 of every
+     * bulk-copy launch withholds its first stage (no arrival, no copy), so its
+     * consumers' bounded wait gives up after about 1 s; the CTA stops, the
+     * launch sets TIDE_KCHECK_TIMEOUT and its result is incomplete.  Nothing
+     * faults or hangs.  Not for use outside tests. */
+    TIDE_PLAN_TEST_TMA_TIMEOUT = 4
 };
 
 #define TIDE_MAX_WORLD 256
@@ -225,12 +231,23 @@ TIDE_API tide_status_t tide_rs_reduce_pipelined(const tide_plan_t* plan, const v
                                                 int64_t slot_numel, int32_t n_segments,
                                                 int32_t max_ctas, void* stream, void* copy_stream);
 
+/* Bits of a plan's device error word. */
+enum {
+    TIDE_KCHECK_TILE = 1,    /* a tile descriptor pointed outside its buffers; the tile was skipped */
+    TIDE_KCHECK_TIMEOUT = 2  /* a bounded wait of the bulk-copy kernel gave up (about 1 s); that CTA stopped */
+};
+
 /*
  * Read and clear the plan's device error word: synchronizes `stream`, then
- * returns TIDE_ERR_KERNEL_CHECK if a kernel enqueued before it rejected a tile
- * (the tile is skipped, nothing outside the buffers is touched), else TIDE_OK.
+ * returns TIDE_ERR_KERNEL_CHECK if a kernel enqueued before it set any bit
+ * (a rejected tile is skipped, nothing outside the buffers is touched; a
+ * timed-out CTA leaves its remaining tiles unwritten), else TIDE_OK.
  */
 TIDE_API tide_status_t tide_plan_check(tide_plan_t* plan, void* stream);
+
+/* tide_plan_check that also stores the bits it read (TIDE_KCHECK_*, 0 if none)
+ * in *bits. */
+TIDE_API tide_status_t tide_plan_errors(tide_plan_t* plan, void* stream, int32_t* bits);
 
 /*
  * Allocation-free rank-order reduction.  The paper has no counterpart: this

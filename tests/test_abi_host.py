@@ -127,6 +127,11 @@ def test_plan_group_rejects(world, params, status):
 def test_plan_group_rejects_unknown_flag_and_empty_group_ok():
     st, _ = T.tide_plan_group([(4, 4)], 2, 0, 0x80)
     assert st == T.TIDE_ERR_INVALID_ARG
+    flags = T.TIDE_PLAN_HOST_ONLY | T.TIDE_PLAN_TMA | T.TIDE_PLAN_TEST_TMA_TIMEOUT
+    st, h = T.tide_plan_group([(4, 4)], 2, 0, flags)
+    assert st == T.TIDE_OK
+    assert T.tide_plan_errors(h, 0) == (T.TIDE_ERR_DEVICE, 0)   # host-only: no error word
+    T.tide_plan_destroy(h)
     st, h = T.tide_plan_group([], 4, 0, T.TIDE_PLAN_HOST_ONLY)
     assert st == T.TIDE_OK
     st, info = T.tide_plan_info(h)

@@ -5,6 +5,8 @@ RS within 1e-6 * sum|terms| of the exact fp64 sum.  Sizes are small enough for
 the oracle to finish in seconds but span many tiles, ragged tile ends,
 misaligned chunk offsets, pad rows and all-pad chunks.
 """
+import time
+
 import numpy as np
 import pytest
 import torch
@@ -131,6 +133,42 @@ def test_tree_order_kernels_agree_bitwise(group):
                dict(slots=True, engine=T.TIDE_ENGINE_CE)):
         out, _, _ = run_rs(group, grads, scale=1, order=1, **kw)
         assert np.array_equal(f32_bits(out), ref), kw
+
+
+@pytest.mark.parametrize("slots", [False, True], ids=["plain", "slot"])
+def test_bulk_copy_wait_timeout_is_reported_and_recovered(slots):
+    """A bounded wait that runs out.  Test hook: CTA 0 of the bulk-copy kernel withholds its
+    first stage, so its consumers' wait gives up after about 1 s. The CTA then stops and waits
+    for its own copies in flight. The launch reports TIDE_KCHECK_TIMEOUT in the error word,
+    and the context stays usable."""
+    group = aligned_group(8, 3)
+    grads = synth.grads_host(group, seed=36)
+    ref = oracle.rs_reduce(group.world, group.shapes, grads, 1)
+    plan = T.Plan(group.shapes, group.world, tma=True, test_tma_timeout=True)
+    assert plan.n_tiles > 0
+    dev = grads_to_dev(group, grads)
+    n = group.world * plan.shard_numel
+    slot_bufs = ([torch.empty(n, dtype=torch.bfloat16, device="cuda") for _ in range(group.world)]
+                 if slots else None)
+    out = torch.full((n,), float("nan"), device="cuda")
+    torch.cuda.synchronize()
+    t0 = time.monotonic()
+    plan.rs_reduce(dev, out, slots=slot_bufs)
+    torch.cuda.synchronize()
+    elapsed = time.monotonic() - t0
+    assert plan.last_launch()[0] == (T.K_SLOT_RS_TMA if slots else T.K_RS_TMA)
+    assert plan.errors() == T.TIDE_KCHECK_TIMEOUT
+    assert plan.errors() == 0                       # read and cleared
+    assert 0.5 < elapsed < 60
+    # CTAs other than 0 finished their tiles: those outputs are the oracle's
+    got = f32_bits(out)
+    done = got == ref.view(np.uint32)
+    assert done.mean() > 0.5
+    # the context is intact: a plan without the hook gives the oracle's bits
+    plan.close()
+    out2, _, plan2 = run_rs(group, grads, scale=1, tma=True, slots=slots)
+    assert plan2.last_launch()[0] == (T.K_SLOT_RS_TMA if slots else T.K_RS_TMA)
+    assert np.array_equal(f32_bits(out2), ref.view(np.uint32))
 
 
 @pytest.mark.parametrize("W", [2, 4, 8, 16, 64, 256])
