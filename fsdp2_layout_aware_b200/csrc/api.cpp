@@ -11,9 +11,20 @@
 #include <cstring>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "tide_internal.h"
 
 namespace {
+
+// An NVTX range over one API call, named after it, for Nsight Systems
+// timelines (with no tool attached it costs a check of a function pointer).
+struct ApiRange {
+    explicit ApiRange(const char* name) { nvtxRangePushA(name); }
+    ~ApiRange() { nvtxRangePop(); }
+    ApiRange(const ApiRange&) = delete;
+    ApiRange& operator=(const ApiRange&) = delete;
+};
 
 struct Span {
     uintptr_t lo, hi;
@@ -233,6 +244,7 @@ extern "C" tide_status_t tide_ag_place(const tide_plan_t* cplan, const void* ag_
                                        int64_t ag_numel, void* const* param_storage,
                                        const int64_t* param_numel, int32_t engine,
                                        int32_t max_ctas, void* stream) {
+    ApiRange range("tide_ag_place");
     tide_plan* p = const_cast<tide_plan*>(cplan);
     tide_status_t st = check_plan(p);
     if (st != TIDE_OK) return st;
@@ -271,6 +283,7 @@ extern "C" tide_status_t tide_rs_reduce(const tide_plan_t* cplan, const void* co
                                         int32_t scale_mode, int32_t order, void* const* slots,
                                         int64_t slot_numel, int32_t engine, int32_t max_ctas,
                                         void* stream) {
+    ApiRange range("tide_rs_reduce");
     tide_plan* p = const_cast<tide_plan*>(cplan);
     tide_status_t st = check_plan(p);
     if (st != TIDE_OK) return st;
@@ -300,6 +313,7 @@ extern "C" tide_status_t tide_rs_stage(const tide_plan_t* cplan, const void* con
                                        const int64_t* grad_numel, void* const* slots,
                                        int64_t slot_numel, int32_t engine, int32_t max_ctas,
                                        void* stream) {
+    ApiRange range("tide_rs_stage");
     tide_plan* p = const_cast<tide_plan*>(cplan);
     tide_status_t st = check_plan(p);
     if (st != TIDE_OK) return st;
@@ -316,6 +330,7 @@ extern "C" tide_status_t tide_rs_reduce_slots(const tide_plan_t* cplan, const vo
                                               int64_t slot_numel, float* out, int64_t out_numel,
                                               int32_t scale_mode, int32_t order, int32_t max_ctas,
                                               void* stream) {
+    ApiRange range("tide_rs_reduce_slots");
     tide_plan* p = const_cast<tide_plan*>(cplan);
     tide_status_t st = check_plan(p);
     if (st != TIDE_OK) return st;
@@ -340,6 +355,7 @@ extern "C" tide_status_t tide_rs_reduce_pipelined(const tide_plan_t* cplan, cons
                                                   int32_t order, void* const* slots,
                                                   int64_t slot_numel, int32_t n_segments,
                                                   int32_t max_ctas, void* stream, void* copy_stream) {
+    ApiRange range("tide_rs_reduce_pipelined");
     tide_plan* p = const_cast<tide_plan*>(cplan);
     tide_status_t st = check_plan(p);
     if (st != TIDE_OK) return st;
