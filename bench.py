@@ -55,6 +55,8 @@ def parse_args():
     ap.add_argument("--interference", action="store_true",
                     help="also run the concurrent-GEMM interference sweep")
     ap.add_argument("--suite", action="store_true", help="one JSON line per workload")
+    ap.add_argument("--jsonl", default=None,
+                    help="also append one flat row per (workload, op, mode, ctas) to this file")
     ap.add_argument("--profile-small", action="store_true",
                     help="a short run of the sweep_w8 workload, sized for an ncu capture")
     return ap.parse_args()
@@ -223,11 +225,21 @@ class Workload:
     def drop_slots(self):
         self.slots = None
 
+    def params_poison(self):
+        """Fill the parameter storage (pads included) with a bit pattern no call writes."""
+        import torch
+        for p in self.params:
+            p.view(torch.int16).fill_(-1)
 
-def timed_calls(fn, K, stream, flush=None):
-    """Mean device time of fn() over K calls, each bracketed by events on `stream`."""
+
+def timed_calls(fn, K, stream, flush=None, warmup=2):
+    """Mean device time of fn() over K calls, each bracketed by events on `stream`,
+    after `warmup` untimed calls (first-call costs: streams and events a plan
+    creates on first use, allocator growth in torch's own kernels)."""
     import torch
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for _ in range(warmup):
+        fn()
     torch.cuda.synchronize()
     for a, b in evs:
         if flush is not None:
@@ -252,43 +264,71 @@ def make_flush(device, nbytes):
 
 
 def run_variants(wl, K, stream, peak, flush):
-    """The other hot-path modes on the same workload, each timed on its own."""
+    """The other hot-path modes on the same workload, each timed on its own.
+
+    Every mode meant to give the plain call's bits is compared, on the device,
+    with the plain tide_rs_reduce / tide_ag_place output of the same inputs
+    ("same_bits_as_plain"); the plain calls are pinned to the CPU oracle by the
+    test suite.  Tree order has its own bits and is not compared."""
+    import torch
     from fsdp2_layout_aware_b200 import tide as T
     B = alg_bytes(wl.group, oracle_free_layout(wl))
     out = {}
+    wl.plan.rs_reduce(wl.grads, wl.out)
+    wl.plan.ag_place(wl.ag, wl.params)
+    torch.cuda.synchronize()
+    ref_out = wl.out.view(torch.int32).clone()
+    ref_params = [p.view(torch.int16).clone() for p in wl.params]
 
-    def rec(name, ms, nbytes, launches):
+    def same_rs():
+        torch.cuda.synchronize()
+        return bool(torch.equal(wl.out.view(torch.int32), ref_out))
+
+    def same_ag():
+        torch.cuda.synchronize()
+        return all(bool(torch.equal(p.view(torch.int16), q)) for p, q in zip(wl.params, ref_params))
+
+    def rec(name, ms, nbytes, launches, plan=None, same=None):
         gbs = nbytes / (ms * 1e-3) / 1e9
         out[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_of_peak": round(gbs / peak, 4),
                      "alg_bytes": nbytes, "kernel_launches": launches}
+        if plan is not None:
+            k, n = plan.last_launch()
+            out[name]["kernel"] = T.KERNEL_NAMES[k] if k >= 0 else "copy engines"
+            out[name]["ctas"] = n if k >= 0 else 0
+        if same is not None:
+            out[name]["same_bits_as_plain"] = same()
 
+    wl.params_poison()
     rec("ag_place_ce", timed_calls(lambda: wl.plan.ag_place(wl.ag, wl.params, engine=T.TIDE_ENGINE_CE),
-                                   K, stream, flush), B["ag"], 0)
+                                   K, stream, flush), B["ag"], 0, wl.plan, same_ag)
     rec("rs_reduce_tree", timed_calls(lambda: wl.plan.rs_reduce(wl.grads, wl.out, order=T.TIDE_ORDER_TREE),
-                                      K, stream, flush), B["rs"], 1)
+                                      K, stream, flush), B["rs"], 1, wl.plan)
     tma_plan = T.Plan(wl.group.shapes, wl.group.world, device=wl.out.device, tma=True)
+    wl.out.fill_(float("nan"))
     rec("rs_reduce_tma", timed_calls(lambda: tma_plan.rs_reduce(wl.grads, wl.out), K, stream, flush),
-        B["rs"], 1)
-    out["rs_reduce_tma"]["kernel"] = T.KERNEL_NAMES[tma_plan.last_launch()[0]]
+        B["rs"], 1, tma_plan, same_rs)
     tma_plan.close()
     slots = wl.ensure_slots()
     for eng, name in ((T.TIDE_ENGINE_SM, "sm"), (T.TIDE_ENGINE_CE, "ce")):
         rec(f"slot_stage_{name}", timed_calls(lambda: wl.plan.rs_stage(wl.grads, slots, engine=eng),
-                                              K, stream, flush), B["stage"], 1 if eng == 0 else 0)
+                                              K, stream, flush), B["stage"], 1 if eng == 0 else 0, wl.plan)
+    wl.out.fill_(float("nan"))
     rec("slot_reduce", timed_calls(lambda: wl.plan.rs_reduce_slots(slots, wl.out), K, stream, flush),
-        B["slot_rs"], 1)
+        B["slot_rs"], 1, wl.plan, same_rs)
     # both phases: one after the other (CE staging, then the reduce kernel) ...
+    wl.out.fill_(float("nan"))
     rec("slot_reuse_serial_ce",
         timed_calls(lambda: wl.plan.rs_reduce(wl.grads, wl.out, slots=slots, engine=T.TIDE_ENGINE_CE),
-                    K, stream, flush), B["stage"] + B["slot_rs"], 1)
-    # ... and overlapped: the copy engines stage group s+1 while the SMs reduce group s
-    import torch
+                    K, stream, flush), B["stage"] + B["slot_rs"], 1, wl.plan, same_rs)
+    # ... and overlapped: the copy engines stage run s+1 while the SMs reduce run s
     cs = torch.cuda.Stream(wl.out.device)
     W = wl.group.world
     for nseg in sorted({1, min(4, W), W}):
+        wl.out.fill_(float("nan"))
         rec(f"slot_reuse_pipelined_seg{nseg}",
             timed_calls(lambda: wl.plan.rs_reduce_pipelined(wl.grads, wl.out, slots, nseg, cs),
-                        K, stream, flush), B["stage"] + B["slot_rs"], nseg)
+                        K, stream, flush), B["stage"] + B["slot_rs"], nseg, wl.plan, same_rs)
     wl.drop_slots()
     del slots
     # Context: the stock FSDP2 layout conversion with torch's own kernels on the same GPU
@@ -325,9 +365,48 @@ def run_variants(wl, K, stream, peak, flush):
         n = wl.group.numel(i)
         same &= bool(torch.equal(p[:n].view(torch.int16), q[:n].view(torch.int16)))
     out["stock_torch_copyout"]["same_valid_bits_as_tide"] = same
-    del pack, stock, stock_params
+    del pack, stock, stock_params, ref_out, ref_params
     wl.drop_slots()
     return out
+
+
+# (op, mode) of each timed entry of a bench line, for the flat JSONL log
+ROW_KINDS = {
+    "rs_reduce_kernel": ("rs_reduce", "SM, rank order"),
+    "ag_place_kernel": ("ag_place", "SM"),
+    "ag_place_ce": ("ag_place", "copy engines"),
+    "rs_reduce_tree": ("rs_reduce", "SM, tree order"),
+    "rs_reduce_tma": ("rs_reduce", "SM bulk-copy kernel, rank order"),
+    "slot_stage_sm": ("slot_stage", "SM"),
+    "slot_stage_ce": ("slot_stage", "copy engines"),
+    "slot_reduce": ("slot_reduce", "SM, rank order"),
+    "slot_reuse_serial_ce": ("slot_reuse", "copy-engine staging, then reduce"),
+    "stock_torch_pack_reduce": ("stock_rs", "torch _chunk_cat pack + add"),
+    "stock_torch_copyout": ("stock_ag", "torch split_with_sizes_copy"),
+}
+
+
+def jsonl_rows(res, group_name, world):
+    """One flat row per (config, op, mode, ctas) of a bench line."""
+    rows = []
+    cpu = res.get("cpu_baseline") or {}
+    entries = list(res.get("kernels", {}).items()) + list(res.get("variants", {}).items())
+    for name, e in entries:
+        op, mode = ROW_KINDS.get(name, (name, ""))
+        if name.startswith("slot_reuse_pipelined_seg"):
+            op, mode = "slot_reuse", f"pipelined, {name.rsplit('seg', 1)[1]} segments"
+        same = e.get("same_bits_as_plain", e.get("same_bits_as_tide", e.get("same_valid_bits_as_tide")))
+        rows.append({
+            "config": group_name, "world": world, "op": op, "mode": mode, "entry": name,
+            "kernel": e.get("kernel"), "ctas": e.get("ctas"), "alg_bytes": e["alg_bytes"],
+            "ms": e["ms"], "GB/s": e["GB/s"], "frac_of_measured_peak": e["frac_of_peak"],
+            "dram_bytes_per_launch": e.get("traffic"),
+            "same_bits_as_plain": same,
+            "oracle_GB/s": cpu.get("value"), "oracle_cores": cpu.get("cores"),
+            "host_cores": len(os.sched_getaffinity(0)),
+            "sm_mhz": (res.get("clocks") or {}).get("sm_mhz"),
+        })
+    return rows
 
 
 def oracle_free_layout(wl):
@@ -663,6 +742,10 @@ def run_ours(args):
                 res["interference"] = run_interference(device, args.seed)
             if rank == 0:
                 print(json.dumps(res), flush=True)
+                if args.jsonl:
+                    with open(args.jsonl, "a") as f:
+                        for row in jsonl_rows(res, name, configs.by_name(name).world):
+                            f.write(json.dumps(row) + "\n")
     finally:
         if dist_on:
             torch.distributed.destroy_process_group()

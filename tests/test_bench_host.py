@@ -74,3 +74,34 @@ def test_reference_arm_rank0_prints_one_line_other_ranks_exit_quietly():
     assert d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["higher_is_better"] is True
+
+
+def test_jsonl_rows_flatten_a_bench_line():
+    """One row per timed entry, with (op, mode, ctas), bytes, time and the bit check."""
+    res = {
+        "kernels": {
+            "rs_reduce_kernel": {"ms": 2.5, "GB/s": 6900.0, "frac_of_peak": 1.05, "alg_bytes": 17,
+                                 "ctas": 296, "kernel": "rs_v32", "traffic": 17},
+            "ag_place_kernel": {"ms": 0.5, "GB/s": 6600.0, "frac_of_peak": 1.0, "alg_bytes": 3,
+                                "ctas": 592, "traffic": None}},
+        "variants": {
+            "ag_place_ce": {"ms": 0.7, "GB/s": 5000.0, "frac_of_peak": 0.76, "alg_bytes": 3,
+                            "kernel_launches": 0, "kernel": "copy engines", "ctas": 0,
+                            "same_bits_as_plain": True},
+            "slot_reuse_pipelined_seg4": {"ms": 6.8, "GB/s": 6500.0, "frac_of_peak": 0.99,
+                                          "alg_bytes": 44, "kernel_launches": 4, "kernel": "slot_rs_v32",
+                                          "ctas": 296, "same_bits_as_plain": False}},
+        "cpu_baseline": {"value": 1.9, "cores": 1},
+        "clocks": {"sm_mhz": 1965},
+    }
+    rows = bench.jsonl_rows(res, "llama70b", 8)
+    assert [r["entry"] for r in rows] == ["rs_reduce_kernel", "ag_place_kernel", "ag_place_ce",
+                                          "slot_reuse_pipelined_seg4"]
+    by = {r["entry"]: r for r in rows}
+    assert by["rs_reduce_kernel"]["op"] == "rs_reduce" and by["rs_reduce_kernel"]["ctas"] == 296
+    assert by["rs_reduce_kernel"]["dram_bytes_per_launch"] == 17
+    assert by["ag_place_ce"]["mode"] == "copy engines" and by["ag_place_ce"]["same_bits_as_plain"] is True
+    assert by["slot_reuse_pipelined_seg4"]["mode"] == "pipelined, 4 segments"
+    assert by["slot_reuse_pipelined_seg4"]["same_bits_as_plain"] is False
+    assert all(r["config"] == "llama70b" and r["world"] == 8 and r["oracle_GB/s"] == 1.9 for r in rows)
+    assert all(json.loads(json.dumps(r)) == r for r in rows)
