@@ -43,8 +43,8 @@ def sample_positions(group, L, n_random, rng):
     return sorted(pos)
 
 
-def expected_rs(group, L, positions, scale):
-    """Oracle value at each sampled output position, from host-regenerated inputs."""
+def rank_values(group, positions):
+    """(located, vals): the oracle's locate() of each position and the W bf16 inputs there."""
     W = group.world
     zero = [synth.zero_grad_params(group, SEED, k) for k in range(W)]
     located = [oracle.locate(W, group.shapes, r, j) for r, j in positions]
@@ -60,6 +60,12 @@ def expected_rs(group, L, positions, scale):
             if i in zero[k]:
                 continue
             vals[rows, k] = synth.gather_bf16(idx, SEED, synth.STREAM_GRAD, k, i, group.grad_sigma)
+    return located, vals
+
+
+def expected_rs(group, L, positions, scale):
+    """Oracle value at each sampled output position, from host-regenerated inputs."""
+    located, vals = rank_values(group, positions)
     out = np.zeros(len(positions), dtype=np.float32)
     for n, (st, _, _) in enumerate(located):
         out[n] = oracle.sum_ranks(vals[n], scale) if st == 1 else np.float32(0.0)
@@ -143,6 +149,63 @@ def test_full_size_rs_and_ag(name):
         for p in params:
             p.view(torch.int16).fill_(0x7777)
     del ag, params
+    torch.cuda.empty_cache()
+
+
+def bf16_to_f64(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+@pytest.mark.parametrize("name", ["llama70b", "qwen3moe"])
+def test_full_size_other_modes(name):
+    """At full size: tree order within 1e-6 * sum|terms| of the exact sum at sampled
+    positions; the bulk-copy kernel and the pipelined Slot-Reuse (W segments, copy engines on
+    a second stream) give the plain call's bits."""
+    group = configs.by_name(name)
+    W = group.world
+    rng = np.random.default_rng(8)
+    torch.cuda.empty_cache()
+    plan = T.Plan(group.shapes, W)
+    L = oracle.layout(W, group.shapes)
+    grads = synth.dev_grads(group, SEED)
+    n = W * L.Ns
+    ref = torch.full((n,), float("nan"), device="cuda")
+    plan.rs_reduce(grads, ref, scale_mode=T.TIDE_SCALE_INV_WORLD)
+    torch.cuda.synchronize()
+    check_rs(group, ref, L, 1, rng, n_random=5000)
+    out = torch.full((n,), float("nan"), device="cuda")
+    # tree order, unscaled: exact sums at sampled positions (W <= 64 bf16 terms: exact in fp64)
+    plan.rs_reduce(grads, out, scale_mode=T.TIDE_SCALE_NONE, order=T.TIDE_ORDER_TREE)
+    torch.cuda.synchronize()
+    plan.check()
+    assert plan.last_launch()[0] == T.K_RS_TREE
+    pos = sample_positions(group, L, 20000, rng)
+    located, vals = rank_values(group, pos)
+    terms = bf16_to_f64(vals)
+    E, A = terms.sum(axis=1), np.abs(terms).sum(axis=1)
+    flat = torch.tensor([r * L.Ns + j for r, j in pos], dtype=torch.int64, device="cuda")
+    got = out[flat].cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - E) <= 1e-6 * A)
+    pads = np.array([st != 1 for st, _, _ in located])
+    assert np.all(got[pads] == 0.0)
+    # the bulk-copy kernel
+    tma = T.Plan(group.shapes, W, tma=True)
+    out.fill_(float("nan"))
+    tma.rs_reduce(grads, out, scale_mode=T.TIDE_SCALE_INV_WORLD)
+    torch.cuda.synchronize()
+    tma.check()
+    assert tma.last_launch()[0] == T.K_RS_TMA
+    assert torch.equal(out.view(torch.int32), ref.view(torch.int32))
+    tma.close()
+    # pipelined Slot-Reuse, W segments
+    slots = [torch.empty(n, dtype=torch.bfloat16, device="cuda") for _ in range(W)]
+    cs = torch.cuda.Stream()
+    out.fill_(float("nan"))
+    plan.rs_reduce_pipelined(grads, out, slots, W, cs)
+    torch.cuda.synchronize()
+    plan.check()
+    assert torch.equal(out.view(torch.int32), ref.view(torch.int32))
+    del slots, grads, out, ref
     torch.cuda.empty_cache()
 
 
