@@ -56,15 +56,16 @@ def _load():
         for name in ("orc_ag_copyout", "orc_pack_f32", "orc_slot_stage"):
             getattr(lib, name).argtypes = [i64, i64, vp, vp, vp, vp]
             getattr(lib, name).restype = ctypes.c_int
-        for name in ("orc_rs_reduce", "orc_rs_reduce_slots"):
+        for name in ("orc_rs_reduce", "orc_rs_reduce_slots", "orc_rs_reduce_tree"):
             getattr(lib, name).argtypes = [i64, i64, vp, vp, vp, i32, vp]
             getattr(lib, name).restype = ctypes.c_int
         lib.orc_exact_f64.argtypes = [i64, i64, vp, vp, vp, vp, vp]
         lib.orc_exact_f64.restype = ctypes.c_int
         lib.orc_locate.argtypes = [i64, i64, vp, vp, i64, i64, p64, p64]
         lib.orc_locate.restype = ctypes.c_int
-        lib.orc_sum_ranks.argtypes = [i64, vp, i32]
-        lib.orc_sum_ranks.restype = ctypes.c_float
+        for name in ("orc_sum_ranks", "orc_sum_ranks_tree"):
+            getattr(lib, name).argtypes = [i64, vp, i32]
+            getattr(lib, name).restype = ctypes.c_float
         lib.orc_ag_source.argtypes = [i64, i64, vp, vp, i64, i64, p64]
         lib.orc_ag_source.restype = ctypes.c_int
         _lib = lib
@@ -109,6 +110,20 @@ def rs_reduce(world: int, shapes, grads, scale_mode: int) -> np.ndarray:
     flat = [np.ascontiguousarray(grads[k][i], dtype=np.uint16) for k in range(world) for i in range(P)]
     rc = _load().orc_rs_reduce(world, P, d0.ctypes.data, inner.ctypes.data, _ptrs(flat),
                                scale_mode, out.ctypes.data)
+    if rc != 0:
+        raise MemoryError("oracle allocation failed")
+    return out
+
+
+def rs_reduce_tree(world: int, shapes, grads, scale_mode: int) -> np.ndarray:
+    """The reduce-scatter in tree order (pairs level by level, odd one carried).  fp32 [W*Ns]."""
+    d0, inner = _dims(shapes)
+    P = len(shapes)
+    Ns = layout(world, shapes).Ns
+    out = np.empty(world * Ns, dtype=np.float32)
+    flat = [np.ascontiguousarray(grads[k][i], dtype=np.uint16) for k in range(world) for i in range(P)]
+    rc = _load().orc_rs_reduce_tree(world, P, d0.ctypes.data, inner.ctypes.data, _ptrs(flat),
+                                    scale_mode, out.ctypes.data)
     if rc != 0:
         raise MemoryError("oracle allocation failed")
     return out
@@ -180,6 +195,11 @@ def locate(world: int, shapes, r: int, j: int):
 def sum_ranks(vals, scale_mode: int) -> np.float32:
     v = np.ascontiguousarray(vals, dtype=np.uint16)
     return np.float32(_load().orc_sum_ranks(v.size, v.ctypes.data, scale_mode))
+
+
+def sum_ranks_tree(vals, scale_mode: int) -> np.float32:
+    v = np.ascontiguousarray(vals, dtype=np.uint16)
+    return np.float32(_load().orc_sum_ranks_tree(v.size, v.ctypes.data, scale_mode))
 
 
 def ag_source(world: int, shapes, i: int, q: int):

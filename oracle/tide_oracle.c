@@ -33,6 +33,10 @@
  *   - Sum: rank order 0..W-1 starting from fp32(g_0), IEEE fp32
  *     round-to-nearest-even, no fused multiply-add; bf16 -> fp32 is exact.
  *   - Optional scale: after the sum, one fp32 multiply by fl32(1/W).
+ *   - Tree order (an optional mode of the reduction, not on the pages): the W
+ *     fp32 values of a position are added in adjacent pairs, level by level,
+ *     an odd last value carried unchanged to the next level, until one is
+ *     left; then the optional scale.
  *   - Pads: +0.0 in the fp32 shards and in padded parameter rows; source pads
  *     of the all-gather buffer are never read.
  *
@@ -203,6 +207,59 @@ int orc_rs_reduce_slots(int64_t W, int64_t P, const int64_t* d0, const int64_t* 
                 out[j] = scale_mode == 1 ? acc * s : acc;
             }
     free(S); free(c); free(off);
+    return 0;
+}
+
+/*
+ * The tree order on one position: v[0..n) are replaced, level by level, by the
+ * sums of adjacent pairs (v[0]+v[1], v[2]+v[3], ...), an odd last value carried
+ * unchanged, until one value is left.  fp32 adds, round-to-nearest-even.
+ */
+static float tree_of(float* v, int64_t n) {
+    while (n > 1) {
+        int64_t m = 0;
+        for (int64_t j = 0; j + 1 < n; j += 2) v[m++] = v[j] + v[j + 1];
+        if (n % 2 == 1) v[m++] = v[n - 1];
+        n = m;
+    }
+    return v[0];
+}
+
+/* Tree-order sum of one position's W bf16 values, then the optional scale. */
+float orc_sum_ranks_tree(int64_t W, const uint16_t* vals, int32_t scale_mode) {
+    float* v = malloc(sizeof(float) * (size_t)(W > 0 ? W : 1));
+    if (!v) return 0.0f;
+    for (int64_t k = 0; k < W; ++k) v[k] = bf16_to_f32(vals[k]);
+    float acc = tree_of(v, W);
+    free(v);
+    if (scale_mode == 1) acc = acc * (1.0f / (float)W);
+    return acc;
+}
+
+/*
+ * The reduce-scatter in tree order, position by position straight from the
+ * per-parameter gradients (the definition written out; no packed buffer):
+ *   out[r*Ns + off_i + e] = s * tree_k(fp32(g_{k,i}[r*c_i + e])) for valid
+ * positions, +0.0 at pads.
+ */
+int orc_rs_reduce_tree(int64_t W, int64_t P, const int64_t* d0, const int64_t* inner,
+                       const uint16_t* const* grads, int32_t scale_mode, float* out) {
+    int64_t *S = malloc(sizeof(int64_t) * (P + 1)), *c = malloc(sizeof(int64_t) * (P + 1)),
+            *off = malloc(sizeof(int64_t) * (P + 1)), Ns = 0;
+    float* v = malloc(sizeof(float) * (size_t)(W > 0 ? W : 1));
+    if (!S || !c || !off || !v) { free(S); free(c); free(off); free(v); return -1; }
+    orc_layout(W, P, d0, inner, S, c, off, &Ns);
+    const float s = 1.0f / (float)W;
+    for (int64_t r = 0; r < W; ++r)
+        for (int64_t i = 0; i < P; ++i)
+            for (int64_t e = 0; e < c[i]; ++e) {
+                int64_t j = r * Ns + off[i] + e, src = r * c[i] + e;
+                if (src >= d0[i] * inner[i]) { out[j] = 0.0f; continue; }
+                for (int64_t k = 0; k < W; ++k) v[k] = bf16_to_f32(grads[k * P + i][src]);
+                float acc = tree_of(v, W);
+                out[j] = scale_mode == 1 ? acc * s : acc;
+            }
+    free(S); free(c); free(off); free(v);
     return 0;
 }
 

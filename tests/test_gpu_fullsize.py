@@ -158,9 +158,10 @@ def bf16_to_f64(bits):
 
 @pytest.mark.parametrize("name", ["llama70b", "qwen3moe"])
 def test_full_size_other_modes(name):
-    """At full size: tree order within 1e-6 * sum|terms| of the exact sum at sampled
-    positions; the bulk-copy kernel and the pipelined Slot-Reuse (W segments, copy engines on
-    a second stream) give the plain call's bits."""
+    """At full size: tree order bit-exact against the oracle's tree (and within 1e-6 *
+    sum|terms| of the exact sum) at sampled positions; the bulk-copy kernel and the
+    pipelined Slot-Reuse (W segments, copy engines on a second stream) give the plain call's
+    bits."""
     group = configs.by_name(name)
     W = group.world
     rng = np.random.default_rng(8)
@@ -184,10 +185,14 @@ def test_full_size_other_modes(name):
     terms = bf16_to_f64(vals)
     E, A = terms.sum(axis=1), np.abs(terms).sum(axis=1)
     flat = torch.tensor([r * L.Ns + j for r, j in pos], dtype=torch.int64, device="cuda")
-    got = out[flat].cpu().numpy().astype(np.float64)
+    got32 = out[flat].cpu().numpy()
+    got = got32.astype(np.float64)
     assert np.all(np.abs(got - E) <= 1e-6 * A)
     pads = np.array([st != 1 for st, _, _ in located])
     assert np.all(got[pads] == 0.0)
+    want = np.array([oracle.sum_ranks_tree(vals[n], 0) if st == 1 else np.float32(0.0)
+                     for n, (st, _, _) in enumerate(located)], dtype=np.float32)
+    assert np.array_equal(got32.view(np.uint32), want.view(np.uint32))
     # the bulk-copy kernel
     tma = T.Plan(group.shapes, W, tma=True)
     out.fill_(float("nan"))

@@ -1,7 +1,7 @@
 """GPU parity: the CUDA path through the C-ABI against the CPU oracle, element by element.
 
-Bars: AG placement, Slot-Reuse staging and rank-order RS bit-exact; tree-order
-RS within 1e-6 * sum|terms| of the exact fp64 sum.  Sizes are small enough for
+Bars: AG placement, Slot-Reuse staging, rank-order RS and tree-order RS bit-exact
+against the oracle (tree order also within 1e-6 * sum|terms| of the exact fp64 sum).  Sizes are small enough for
 the oracle to finish in seconds but span many tiles, ragged tile ends,
 misaligned chunk offsets, pad rows and all-pad chunks.
 """
@@ -91,6 +91,8 @@ def test_rs_bulk_copy_path(group):
     out, _, plan = run_rs(group, grads, scale=0, order=1, tma=True)
     assert plan.last_launch()[0] == T.K_RS_TMA
     assert np.all(np.abs(out.cpu().numpy().astype(np.float64) - E) <= 1e-6 * A)
+    tree = oracle.rs_reduce_tree(group.world, group.shapes, grads, 0)
+    assert np.array_equal(f32_bits(out), tree.view(np.uint32))
     for engine in (T.TIDE_ENGINE_SM, T.TIDE_ENGINE_CE):
         out, _, plan = run_rs(group, grads, scale=1, slots=True, engine=engine, tma=True)
         assert plan.last_launch()[0] == T.K_SLOT_RS_TMA
@@ -111,6 +113,8 @@ def test_rs_tree_order_within_tolerance(group):
     out, _, plan = run_rs(group, grads, scale=0, order=1)
     if plan.n_tiles:   # the tree kernel, on the grid its own occupancy gives
         assert plan.last_launch() == (T.K_RS_TREE, plan.launch_ctas(T.K_RS_TREE, 0))
+    assert np.array_equal(f32_bits(out),
+                          oracle.rs_reduce_tree(group.world, group.shapes, grads, 0).view(np.uint32))
     E, A = oracle.exact_f64(group.world, group.shapes, grads)
     got = out.cpu().numpy().astype(np.float64)
     assert np.all(np.abs(got - E) <= 1e-6 * A)
@@ -129,6 +133,7 @@ def test_tree_order_kernels_agree_bitwise(group):
     grads = synth.grads_host(group, seed=35)
     ref, _, _ = run_rs(group, grads, scale=1, order=1)
     ref = f32_bits(ref)
+    assert np.array_equal(ref, oracle.rs_reduce_tree(group.world, group.shapes, grads, 1).view(np.uint32))
     for kw in (dict(max_ctas=3), dict(tma=True), dict(slots=True),
                dict(slots=True, engine=T.TIDE_ENGINE_CE)):
         out, _, _ = run_rs(group, grads, scale=1, order=1, **kw)
@@ -200,6 +205,23 @@ def test_rs_rank_order_pin_on_gpu():
         assert np.all(valid == np.float32(exp))
 
 
+@pytest.mark.parametrize("vals,exp", [
+    ([1.0, 2.0 ** -24, 2.0 ** -24, 2.0 ** -24], 1.0 + 2.0 ** -23),    # rank order gives 1
+    ([1.0] + [2.0 ** -24] * 4, 1.0 + 2.0 ** -22),                       # a tie rounded to even
+    ([1.0] + [2.0 ** -24] * 9, 1.0 + 2.0 ** -21),                       # W=10, two groups on the GPU
+])
+def test_rs_tree_order_pin_on_gpu(vals, exp):
+    """Worked values of the tree order (pairs by levels, odd one carried) on every tree kernel."""
+    W = len(vals)
+    shapes = ((64 * W, 8),)
+    g = configs.Group("tree_pin", W, shapes)
+    grads = [[np.full(64 * W * 8, np.array([v], np.float32).view(np.uint32)[0] >> 16, np.uint16)]
+             for v in vals]
+    for kw in (dict(), dict(tma=True), dict(slots=True)):
+        out, _, _ = run_rs(g, grads, scale=0, order=1, **kw)
+        assert np.all(out.cpu().numpy() == np.float32(exp)), kw
+
+
 @pytest.mark.parametrize("group", GROUPS, ids=IDS)
 @pytest.mark.parametrize("engine", [T.TIDE_ENGINE_SM, T.TIDE_ENGINE_CE])
 def test_ag_place_bit_exact(group, engine):
@@ -253,6 +275,8 @@ def test_rs_32_byte_path(group):
     E, A = oracle.exact_f64(group.world, group.shapes, grads)
     out, _, _ = run_rs(group, grads, scale=0, order=1)
     assert np.all(np.abs(out.cpu().numpy().astype(np.float64) - E) <= 1e-6 * A)
+    assert np.array_equal(f32_bits(out),
+                          oracle.rs_reduce_tree(group.world, group.shapes, grads, 0).view(np.uint32))
 
 
 def test_rs_32_byte_path_needs_32_byte_pointers():
@@ -327,8 +351,8 @@ def test_slot_phases_separately():
             assert np.array_equal(f32_bits(out),
                                   oracle.rs_reduce(group.world, group.shapes, grads, 0).view(np.uint32))
         else:
-            E, A = oracle.exact_f64(group.world, group.shapes, grads)
-            assert np.all(np.abs(out.cpu().numpy() - E) <= 1e-6 * A)
+            tree = oracle.rs_reduce_tree(group.world, group.shapes, grads, 0)
+            assert np.array_equal(f32_bits(out), tree.view(np.uint32))
 
 
 @pytest.mark.parametrize("group", [configs.tiny(), mini_sweep(8), configs.qwen3moe(4)],

@@ -27,6 +27,9 @@ MUTANTS = {
     "ag_pad_rows_not_zeroed": ("for (int64_t t = 0; t < inner[i]; ++t) dst[t] = 0;", ";"),
     "ag_source_stride_dropped": ("const uint16_t* src = ag + r * Ns + off[i] + s * inner[i];",
                                  "const uint16_t* src = ag + r * Ns + off[i] + s;"),
+    "tree_pairs_mirrored": ("for (int64_t j = 0; j + 1 < n; j += 2) v[m++] = v[j] + v[j + 1];",
+                            "for (int64_t j = 0; j + 1 < n; j += 2) v[m++] = v[j] + v[n - 1 - j];"),
+    "tree_odd_one_dropped": ("if (n % 2 == 1) v[m++] = v[n - 1];", "if (n % 2 == 1) m += 0;"),
     "ranks_added_in_reverse": ("pack_f32(W, P, d0, inner, S, off, Ns, grads + k * P, packed);",
                                "pack_f32(W, P, d0, inner, S, off, Ns, grads + (W - k) * P, packed);"),
 }

@@ -361,3 +361,88 @@ def test_locate_and_ag_source_agree_with_bulk(grp):
         for q in rng.integers(0, max(1, W * L.c[i]), size=min(50, W * L.c[i])):
             st, a = oracle.ag_source(W, grp.shapes, i, int(q))
             assert placed[i][q] == (ag[a] if st == 1 else 0)
+
+
+# --------------------------------------------------------------------------- tree order
+# The tree order is an optional mode of the reduction: adjacent pairs level by level, an
+# odd last value carried.  Pinned by worked values where it differs from the rank order,
+# by a top-down formulation of the same tree, by closed forms and by its error bound.
+
+E24 = 2.0 ** -24
+
+
+def _tree_bits(vals):
+    return [int(bf16_bits(np.float32(v))) for v in vals]
+
+
+@pytest.mark.parametrize("vals,tree,rank", [
+    ([1.0, E24, E24, E24], 1.0 + 2.0 ** -23, 1.0),        # (1+e) + (e+e): the pair of e's survives
+    ([E24, E24, 1.0], 1.0 + 2.0 ** -23, 1.0 + 2.0 ** -23),
+    ([1.0, E24, E24], 1.0, 1.0),                           # (1+e) rounds to 1, then + e rounds to 1
+    # [1, 2e, e] -> [1+2^-23, e] -> 1 + 3e, a tie, rounds to the even 1 + 2^-22
+    ([1.0, E24, E24, E24, E24], 1.0 + 2.0 ** -22, 1.0),
+    ([-0.0, -0.0, -0.0], -0.0, -0.0),
+])
+def test_tree_worked_values(vals, tree, rank):
+    bits = np.array(_tree_bits(vals), dtype=np.uint16)
+    got = oracle.sum_ranks_tree(bits, 0)
+    assert got.view(np.uint32) == np.float32(tree).view(np.uint32)
+    assert oracle.sum_ranks(bits, 0).view(np.uint32) == np.float32(rank).view(np.uint32)
+
+
+def _top_down(v):
+    """The same tree written top-down: split at the largest power of two below n."""
+    n = len(v)
+    if n == 1:
+        return v[0]
+    p = 1
+    while 2 * p < n:
+        p *= 2
+    return np.float32(_top_down(v[:p]) + _top_down(v[p:]))
+
+
+@pytest.mark.parametrize("W", list(range(1, 34)) + [63, 64, 65, 100])
+def test_tree_matches_top_down_split(W):
+    rng = np.random.default_rng(W)
+    for _ in range(40):
+        # wide exponent range and mixed signs, so that the grouping changes the rounding
+        mant = rng.integers(128, 256, size=W).astype(np.float32) / np.float32(128.0)
+        exps = rng.integers(-30, 2, size=W)
+        sign = np.where(rng.random(W) < 0.3, -1.0, 1.0).astype(np.float32)
+        f = (sign * mant * np.float32(2.0) ** exps).astype(np.float32)
+        bits = bf16_bits(f)
+        want = _top_down([np.float32(x) for x in f32_of(bits)])
+        assert oracle.sum_ranks_tree(bits, 0).view(np.uint32) == np.float32(want).view(np.uint32)
+        scaled = np.float32(np.float32(want) * np.float32(1.0 / W))
+        assert oracle.sum_ranks_tree(bits, 1).view(np.uint32) == scaled.view(np.uint32)
+
+
+@pytest.mark.parametrize("grp", groups_for_agreement(), ids=lambda g: f"{g.name}_w{g.world}")
+def test_tree_reduce_matches_numpy_levels(grp):
+    """The C tree reduce-scatter against the numpy levels tree, chunk by chunk (pads +0)."""
+    W = grp.world
+    grads = synth.grads_host(grp, seed=23)
+    out = oracle.rs_reduce_tree(W, grp.shapes, grads, 1)
+    L = oracle.layout(W, grp.shapes)
+    ref = np.zeros(W * L.Ns, dtype=np.float32)
+    for i in range(grp.n_params):
+        for r in range(W):
+            lo, hi = r * L.c[i], min((r + 1) * L.c[i], grp.numel(i))
+            if hi > lo:
+                s = r * L.Ns + L.off[i]
+                tree = oracle_np.tree_sum([f32_of(grads[k][i][lo:hi]) for k in range(W)])
+                ref[s: s + hi - lo] = tree * np.float32(1.0 / W)
+    assert np.array_equal(out.view(np.uint32), ref.view(np.uint32))
+
+
+@pytest.mark.parametrize("W", [1, 2, 3, 8, 16, 64])
+def test_tree_closed_forms_and_bound(W):
+    grp = configs.Group("treecf", W, ((37, 16), (1000,), (7, 3)))
+    g = synth.grads_host(configs.Group("src", 1, grp.shapes), seed=2)[0]
+    same = oracle.rs_reduce_tree(W, grp.shapes, [g for _ in range(W)], 0).astype(np.float64)
+    plain = oracle.rs_reduce(W, grp.shapes, [g for _ in range(W)], 0).astype(np.float64)
+    assert np.array_equal(same, plain)             # k*g is exact for k <= 64: any order agrees
+    grads = synth.grads_host(grp, seed=22)
+    E, A = oracle.exact_f64(W, grp.shapes, grads)
+    tree = oracle.rs_reduce_tree(W, grp.shapes, grads, 0).astype(np.float64)
+    assert np.all(np.abs(tree - E) <= max(1, math.ceil(math.log2(W))) * E24 * A)
