@@ -513,7 +513,9 @@ def cpu_baseline(group, seed, budget_s):
     import synth
     from synth import configs
     W = group.world
-    spent, nbytes, names = 0.0, 0, []
+    rs_s = ag_s = 0.0
+    rs_b = ag_b = 0
+    names = []
     for i in range(group.n_params):
         sub = configs.Group("sample", W, (group.shapes[i],))
         grads = [[synth.grad_host(group, seed, k, i)] for k in range(W)]
@@ -521,20 +523,44 @@ def cpu_baseline(group, seed, budget_s):
         ag = synth.fill_bf16(W * L.Ns, seed, synth.STREAM_AG, 0, i, group.param_sigma)
         t0 = time.perf_counter()
         oracle.rs_reduce(W, sub.shapes, grads, 1)
+        t1 = time.perf_counter()
         oracle.ag_copyout(W, sub.shapes, ag)
-        spent += time.perf_counter() - t0
+        t2 = time.perf_counter()
+        rs_s += t1 - t0
+        ag_s += t2 - t1
         n = sub.numel(0)
-        nbytes += (2 * W * n + 4 * W * L.Ns) + (2 * n + 2 * W * L.Ns)
+        rs_b += 2 * W * n + 4 * W * L.Ns
+        ag_b += 2 * n + 2 * W * L.Ns
         names.append(group.names[i] if group.names else str(i))
         del grads, ag
-        if spent >= budget_s:
+        if rs_s + ag_s >= budget_s:
             break
+    spent, nbytes = rs_s + ag_s, rs_b + ag_b
     cores = 1
     return {"value": round(nbytes / spent / 1e9, 3), "unit": "GB/s", "cores": cores, "kind": "oracle",
             "sample": f"{group.name}: params {names} (each as a one-param group, W={W}), "
                       f"RS x fl32(1/W) + AG copy-out, {nbytes / 1e9:.2f} GB algorithmic, "
                       f"{spent:.1f} s single-thread C oracle, generation excluded",
-            "seconds": round(spent, 2)}
+            "seconds": round(spent, 2),
+            # the two oracle steps timed apart: pack + reduce, and the all-gather copy-out
+            "rs_pack_reduce": {"GB/s": round(rs_b / rs_s / 1e9, 3), "seconds": round(rs_s, 2)},
+            "ag_copyout": {"GB/s": round(ag_b / ag_s / 1e9, 3) if ag_s > 0 else None,
+                           "seconds": round(ag_s, 3)},
+            "host": host_cpu()}
+
+
+def host_cpu():
+    """CPU model and the cores this process may run on."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"model": model, "cores_available": len(os.sched_getaffinity(0))}
 
 
 def run_interference(device, seed):
