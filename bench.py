@@ -212,6 +212,9 @@ class Workload:
         self.out = torch.empty(W * self.Ns, dtype=torch.float32, device=device)
         self.params = [torch.empty(self.plan.query(i)["padded_numel"], dtype=torch.bfloat16,
                                    device=device) for i in range(group.n_params)]
+        # pointer tables marshalled once, as a training loop would per bucket
+        self.grads_t = T.TensorTable([g for row in self.grads for g in row])
+        self.params_t = T.TensorTable(self.params)
         self.slots = None
 
     def ensure_slots(self):
@@ -274,8 +277,8 @@ def run_variants(wl, K, stream, peak, flush):
     from fsdp2_layout_aware_b200 import tide as T
     B = alg_bytes(wl.group, oracle_free_layout(wl))
     out = {}
-    wl.plan.rs_reduce(wl.grads, wl.out)
-    wl.plan.ag_place(wl.ag, wl.params)
+    wl.plan.rs_reduce(wl.grads_t, wl.out)
+    wl.plan.ag_place(wl.ag, wl.params_t)
     torch.cuda.synchronize()
     ref_out = wl.out.view(torch.int32).clone()
     ref_params = [p.view(torch.int16).clone() for p in wl.params]
@@ -300,18 +303,18 @@ def run_variants(wl, K, stream, peak, flush):
             out[name]["same_bits_as_plain"] = same()
 
     wl.params_poison()
-    rec("ag_place_ce", timed_calls(lambda: wl.plan.ag_place(wl.ag, wl.params, engine=T.TIDE_ENGINE_CE),
+    rec("ag_place_ce", timed_calls(lambda: wl.plan.ag_place(wl.ag, wl.params_t, engine=T.TIDE_ENGINE_CE),
                                    K, stream, flush), B["ag"], 0, wl.plan, same_ag)
-    rec("rs_reduce_tree", timed_calls(lambda: wl.plan.rs_reduce(wl.grads, wl.out, order=T.TIDE_ORDER_TREE),
+    rec("rs_reduce_tree", timed_calls(lambda: wl.plan.rs_reduce(wl.grads_t, wl.out, order=T.TIDE_ORDER_TREE),
                                       K, stream, flush), B["rs"], 1, wl.plan)
     tma_plan = T.Plan(wl.group.shapes, wl.group.world, device=wl.out.device, tma=True)
     wl.out.fill_(float("nan"))
-    rec("rs_reduce_tma", timed_calls(lambda: tma_plan.rs_reduce(wl.grads, wl.out), K, stream, flush),
+    rec("rs_reduce_tma", timed_calls(lambda: tma_plan.rs_reduce(wl.grads_t, wl.out), K, stream, flush),
         B["rs"], 1, tma_plan, same_rs)
     tma_plan.close()
     slots = wl.ensure_slots()
     for eng, name in ((T.TIDE_ENGINE_SM, "sm"), (T.TIDE_ENGINE_CE, "ce")):
-        rec(f"slot_stage_{name}", timed_calls(lambda: wl.plan.rs_stage(wl.grads, slots, engine=eng),
+        rec(f"slot_stage_{name}", timed_calls(lambda: wl.plan.rs_stage(wl.grads_t, slots, engine=eng),
                                               K, stream, flush), B["stage"], 1 if eng == 0 else 0, wl.plan)
     wl.out.fill_(float("nan"))
     rec("slot_reduce", timed_calls(lambda: wl.plan.rs_reduce_slots(slots, wl.out), K, stream, flush),
@@ -319,7 +322,7 @@ def run_variants(wl, K, stream, peak, flush):
     # both phases: one after the other (CE staging, then the reduce kernel) ...
     wl.out.fill_(float("nan"))
     rec("slot_reuse_serial_ce",
-        timed_calls(lambda: wl.plan.rs_reduce(wl.grads, wl.out, slots=slots, engine=T.TIDE_ENGINE_CE),
+        timed_calls(lambda: wl.plan.rs_reduce(wl.grads_t, wl.out, slots=slots, engine=T.TIDE_ENGINE_CE),
                     K, stream, flush), B["stage"] + B["slot_rs"], 1, wl.plan, same_rs)
     # ... and overlapped: the copy engines stage run s+1 while the SMs reduce run s
     cs = torch.cuda.Stream(wl.out.device)
@@ -327,7 +330,7 @@ def run_variants(wl, K, stream, peak, flush):
     for nseg in sorted({1, min(4, W), W}):
         wl.out.fill_(float("nan"))
         rec(f"slot_reuse_pipelined_seg{nseg}",
-            timed_calls(lambda: wl.plan.rs_reduce_pipelined(wl.grads, wl.out, slots, nseg, cs),
+            timed_calls(lambda: wl.plan.rs_reduce_pipelined(wl.grads_t, wl.out, slots, nseg, cs),
                         K, stream, flush), B["stage"] + B["slot_rs"], nseg, wl.plan, same_rs)
     wl.drop_slots()
     del slots
@@ -354,8 +357,8 @@ def run_variants(wl, K, stream, peak, flush):
 
     rec("stock_torch_pack_reduce", timed_calls(stock_rs, K, stream, flush), B["rs"], 2 * W)
     rec("stock_torch_copyout", timed_calls(stock_ag, K, stream, flush), B["ag"], 1)
-    wl.plan.rs_reduce(wl.grads, wl.out)
-    wl.plan.ag_place(wl.ag, wl.params)
+    wl.plan.rs_reduce(wl.grads_t, wl.out)
+    wl.plan.ag_place(wl.ag, wl.params_t)
     torch.cuda.synchronize()
     out["stock_torch_pack_reduce"]["same_bits_as_tide"] = bool(
         torch.equal(stock.view(-1).view(torch.int32), wl.out.view(torch.int32)))
@@ -455,8 +458,8 @@ def run_e2e(wl, K, stream):
         wl.ag.copy_(ag_host, non_blocking=True)
 
     def kernels(st):
-        wl.plan.ag_place(wl.ag, wl.params, stream=st)
-        wl.plan.rs_reduce(wl.grads, wl.out, stream=st)
+        wl.plan.ag_place(wl.ag, wl.params_t, stream=st)
+        wl.plan.rs_reduce(wl.grads_t, wl.out, stream=st)
 
     def d2h_copies(st):
         out_host.copy_(wl.out, non_blocking=True)
@@ -606,7 +609,7 @@ def run_interference(device, seed):
         g = {"gemm": f"bf16 {m}x{n}x{k} torch.matmul (cuBLAS), {n_gemm} per batch", "points": []}
         for kind, plan in plans.items():
             for ctas in (8, 16, 32, 0):
-                rs_ms = timed_calls(lambda: plan.rs_reduce(wl.grads, wl.out, max_ctas=ctas, stream=s_rs),
+                rs_ms = timed_calls(lambda: plan.rs_reduce(wl.grads_t, wl.out, max_ctas=ctas, stream=s_rs),
                                     5, s_rs)
                 _, n_ctas = plan.last_launch()
                 alone, conc, rs_conc = [], [], []
@@ -619,7 +622,7 @@ def run_interference(device, seed):
                     with torch.cuda.stream(s_rs):
                         r0.record(s_rs)
                         for _ in range(reps):
-                            plan.rs_reduce(wl.grads, wl.out, max_ctas=ctas, stream=s_rs)
+                            plan.rs_reduce(wl.grads_t, wl.out, max_ctas=ctas, stream=s_rs)
                         r1.record(s_rs)
                     with torch.cuda.stream(s_gemm):
                         e0.record(s_gemm); gemm_batch(); e1.record(s_gemm)
@@ -653,8 +656,8 @@ def bench_workload(args, group, rank, world, device, dist_on):
     flush = None if in_bytes > 4 * L2_BYTES else make_flush(device, 2 * L2_BYTES)
 
     def step():
-        wl.plan.ag_place(wl.ag, wl.params, max_ctas=args.max_ctas)
-        wl.plan.rs_reduce(wl.grads, wl.out, max_ctas=args.max_ctas)
+        wl.plan.ag_place(wl.ag, wl.params_t, max_ctas=args.max_ctas)
+        wl.plan.rs_reduce(wl.grads_t, wl.out, max_ctas=args.max_ctas)
 
     for _ in range(args.warmup):
         step()
@@ -673,9 +676,9 @@ def bench_workload(args, group, rank, world, device, dist_on):
             if flush is not None:
                 flush()
             e[0].record(stream)
-            wl.plan.ag_place(wl.ag, wl.params, max_ctas=args.max_ctas)
+            wl.plan.ag_place(wl.ag, wl.params_t, max_ctas=args.max_ctas)
             e[1].record(stream)
-            wl.plan.rs_reduce(wl.grads, wl.out, max_ctas=args.max_ctas)
+            wl.plan.rs_reduce(wl.grads_t, wl.out, max_ctas=args.max_ctas)
             e[2].record(stream)
         end.record(stream)
         torch.cuda.synchronize()

@@ -191,6 +191,7 @@ extern "C" tide_status_t tide_plan_group(const tide_param_t* params, int32_t n_p
 
 extern "C" void tide_plan_destroy(tide_plan_t* plan) {
     if (plan == nullptr) return;
+    tide::ce_release(plan);
     if (!(plan->flags & TIDE_PLAN_HOST_ONLY)) {
         int prev = -1;
         cudaGetDevice(&prev);

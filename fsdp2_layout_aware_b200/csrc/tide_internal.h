@@ -39,6 +39,7 @@ struct tide_plan {
     std::vector<cudaEvent_t> seg_events; // pacing events of tide_rs_reduce_pipelined (created on first use)
     std::vector<cudaStream_t> ce_streams;  // copy-engine fan-out streams (created on first use)
     std::vector<cudaEvent_t> ce_events;    // their fork event [0] and join events [1..]
+    struct CeIssuer* ce_issuer = nullptr;  // host threads that issue the copies (created on first use)
 
     // device tables (absent for TIDE_PLAN_HOST_ONLY)
     tide_tile_t* d_tiles = nullptr;
@@ -87,5 +88,7 @@ cudaError_t ce_ag_place(tide_plan* p, const uint16_t* ag, void* const* params,
 // all) from every source rank k into slot k.
 cudaError_t ce_slot_stage(tide_plan* p, const void* const* grads, void* const* slots,
                           cudaStream_t stream, int64_t j0 = 0, int64_t j1 = -1);
+// Stops and frees the plan's copy-issuing threads (nothing if there are none).
+void ce_release(tide_plan* p);
 
 }  // namespace tide

@@ -107,17 +107,44 @@ def lib():
 
 
 def _ptr_array(ptrs):
-    arr = (_vp * max(1, len(ptrs)))()
-    for j, p in enumerate(ptrs):
-        arr[j] = p
-    return arr
+    """A ctypes void* array of the given addresses (an existing ctypes array passes through)."""
+    if isinstance(ptrs, ctypes.Array):
+        return ptrs
+    return (_vp * max(1, len(ptrs)))(*ptrs)
 
 
 def _i64_array(vals):
-    arr = (_i64 * max(1, len(vals)))()
-    for j, v in enumerate(vals):
-        arr[j] = int(v)
-    return arr
+    if isinstance(vals, ctypes.Array):
+        return vals
+    return (_i64 * max(1, len(vals)))(*[int(v) for v in vals])
+
+
+class TensorTable:
+    """Device pointers and element counts of a fixed list of tensors, marshalled once.
+
+    Passing one to the Plan methods in place of a list skips the per-call
+    collection of pointers and sizes (for a group of 393 params at W=8 that is
+    3144 tensors).  The table holds references to the tensors; their storage
+    must not be replaced while the table is in use.
+    """
+
+    def __init__(self, tensors):
+        self.tensors = list(tensors)
+        self.ptrs = _ptr_array([t.data_ptr() for t in self.tensors])
+        self.numels = _i64_array([t.numel() for t in self.tensors])
+        self.min_numel = min((t.numel() for t in self.tensors), default=0)
+
+    def __len__(self):
+        return len(self.tensors)
+
+
+def _table(tensors) -> TensorTable:
+    """A TensorTable as is, or one built now from a (possibly nested per rank) list."""
+    if isinstance(tensors, TensorTable):
+        return tensors
+    flat = [t for row in tensors for t in row] if tensors and isinstance(tensors[0], (list, tuple)) \
+        else list(tensors)
+    return TensorTable(flat)
 
 
 def _check(status: int, where: str) -> None:
@@ -316,36 +343,38 @@ class Plan:
         _check(st, "tide_plan_last_launch")
         return k, n
 
+    # grads: rank k's gradient of param i at grads[k][i], or a TensorTable of the W*P
+    # gradients in that order; params and slots: a list or a TensorTable.
+
     def ag_place(self, ag, params, engine: int = TIDE_ENGINE_SM, max_ctas: int = 0,
                  stream=None) -> None:
-        st = tide_ag_place(self.handle, ag.data_ptr(), ag.numel(), [p.data_ptr() for p in params],
-                           [p.numel() for p in params], engine, max_ctas, _stream_handle(stream))
+        p = _table(params)
+        st = tide_ag_place(self.handle, ag.data_ptr(), ag.numel(), p.ptrs, p.numels, engine,
+                           max_ctas, _stream_handle(stream))
         _check(st, "tide_ag_place")
 
     def rs_reduce(self, grads, out, scale_mode: int = TIDE_SCALE_INV_WORLD,
                   order: int = TIDE_ORDER_RANK, slots=None, engine: int = TIDE_ENGINE_SM,
                   max_ctas: int = 0, stream=None) -> None:
         """grads[k][i]: rank k's gradient of param i; out: fp32 [W*Ns]."""
-        flat = [g for row in grads for g in row]
-        st = tide_rs_reduce(self.handle, [g.data_ptr() for g in flat], [g.numel() for g in flat],
-                            out.data_ptr(), out.numel(), scale_mode, order,
-                            None if slots is None else [s.data_ptr() for s in slots],
-                            0 if slots is None else min(s.numel() for s in slots),
+        g = _table(grads)
+        s = None if slots is None else _table(slots)
+        st = tide_rs_reduce(self.handle, g.ptrs, g.numels, out.data_ptr(), out.numel(), scale_mode,
+                            order, None if s is None else s.ptrs, 0 if s is None else s.min_numel,
                             engine, max_ctas, _stream_handle(stream))
         _check(st, "tide_rs_reduce")
 
     def rs_stage(self, grads, slots, engine: int = TIDE_ENGINE_SM, max_ctas: int = 0,
                  stream=None) -> None:
-        flat = [g for row in grads for g in row]
-        st = tide_rs_stage(self.handle, [g.data_ptr() for g in flat], [g.numel() for g in flat],
-                           [s.data_ptr() for s in slots], min(s.numel() for s in slots), engine,
-                           max_ctas, _stream_handle(stream))
+        g, s = _table(grads), _table(slots)
+        st = tide_rs_stage(self.handle, g.ptrs, g.numels, s.ptrs, s.min_numel, engine, max_ctas,
+                           _stream_handle(stream))
         _check(st, "tide_rs_stage")
 
     def rs_reduce_slots(self, slots, out, scale_mode: int = TIDE_SCALE_INV_WORLD,
                         order: int = TIDE_ORDER_RANK, max_ctas: int = 0, stream=None) -> None:
-        st = tide_rs_reduce_slots(self.handle, [s.data_ptr() for s in slots],
-                                  min(s.numel() for s in slots), out.data_ptr(), out.numel(),
+        s = _table(slots)
+        st = tide_rs_reduce_slots(self.handle, s.ptrs, s.min_numel, out.data_ptr(), out.numel(),
                                   scale_mode, order, max_ctas, _stream_handle(stream))
         _check(st, "tide_rs_reduce_slots")
 
@@ -353,11 +382,9 @@ class Plan:
                             scale_mode: int = TIDE_SCALE_INV_WORLD, order: int = TIDE_ORDER_RANK,
                             max_ctas: int = 0, stream=None) -> None:
         """Slot-Reuse with copy-engine staging on `copy_stream` overlapping the reduction."""
-        flat = [g for row in grads for g in row]
-        st = tide_rs_reduce_pipelined(self.handle, [g.data_ptr() for g in flat],
-                                      [g.numel() for g in flat], out.data_ptr(), out.numel(),
-                                      scale_mode, order, [s.data_ptr() for s in slots],
-                                      min(s.numel() for s in slots), n_segments, max_ctas,
+        g, s = _table(grads), _table(slots)
+        st = tide_rs_reduce_pipelined(self.handle, g.ptrs, g.numels, out.data_ptr(), out.numel(),
+                                      scale_mode, order, s.ptrs, s.min_numel, n_segments, max_ctas,
                                       _stream_handle(stream), _stream_handle(copy_stream))
         _check(st, "tide_rs_reduce_pipelined")
 

@@ -48,7 +48,10 @@
  *   - TIDE_ENGINE_CE calls spread their memcpys over 8 streams that the plan
  *     creates on first use (no device memory), forked from the call's stream
  *     with an event and joined back to it before the call returns; work
- *     enqueued on the call's stream afterwards sees every copy.
+ *     enqueued on the call's stream afterwards sees every copy.  The copies
+ *     are issued by the calling thread and 3 host threads that the plan starts
+ *     on its first copy-engine call (they sleep between calls and are joined
+ *     by tide_plan_destroy); the call returns once every copy is enqueued.
  */
 #ifndef TIDE_H
 #define TIDE_H

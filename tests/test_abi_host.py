@@ -269,3 +269,29 @@ def test_null_allowed_only_for_empty_buffers():
         for i in empty:
             grads[k * g.n_params + i] = 0
     assert rs(plan, a, grads=grads) == T.TIDE_ERR_DEVICE
+
+
+def test_tensor_table_marshals_once_in_rank_major_order():
+    import torch
+    grads = [[torch.zeros(n, dtype=torch.bfloat16) for n in (5, 7, 3)] for _ in range(2)]
+    t = T._table(grads)
+    flat = [g for row in grads for g in row]
+    assert len(t) == 6 and t.min_numel == 3
+    assert [t.ptrs[j] for j in range(6)] == [g.data_ptr() for g in flat]
+    assert [t.numels[j] for j in range(6)] == [5, 7, 3, 5, 7, 3]
+    assert T._table(t) is t                                  # a table passes through
+    slots = [torch.zeros(4, dtype=torch.bfloat16), torch.zeros(9, dtype=torch.bfloat16)]
+    s = T._table(slots)
+    assert [s.ptrs[j] for j in range(2)] == [x.data_ptr() for x in slots] and s.min_numel == 4
+    assert len(T._table([])) == 0 and T._table([]).min_numel == 0
+    # the marshalled arrays go straight to the C ABI, which validates them (sizes and
+    # overlaps) before it finds that a host-only plan has no device
+    st, h = T.tide_plan_group([(5, 1), (7, 1), (3, 1)], 2, 0, T.TIDE_PLAN_HOST_ONLY)
+    assert st == T.TIDE_OK
+    out = torch.zeros(2 * (3 + 4 + 2), dtype=torch.float32)
+    assert T.tide_rs_reduce(h, t.ptrs, t.numels, out.data_ptr(), out.numel(), 1, 0, None, 0, 0, 0,
+                            0) == T.TIDE_ERR_DEVICE
+    short = T.TensorTable([g[:2] for g in flat])
+    assert T.tide_rs_reduce(h, short.ptrs, short.numels, out.data_ptr(), out.numel(), 1, 0, None, 0,
+                            0, 0, 0) == T.TIDE_ERR_SIZE
+    T.tide_plan_destroy(h)
