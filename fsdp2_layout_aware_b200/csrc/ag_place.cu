@@ -31,14 +31,21 @@ constexpr int kCopyU = 2;  // 32-byte vectors in flight per thread (64 bytes, as
 struct AgParams {
     const tide_tile_t* tiles;
     int64_t n_tiles;
-    const uint16_t* ag;
-    int64_t ag_numel;
+    const uint16_t* ag;            // rank-major source [W][Ns] (placement)
+    int64_t ag_numel;              // its length; for gathering, each shard's length
+    const void* const* shard_tab;  // gathering: [W] per-rank shards of Ns elements
+    int64_t shard_numel;           // Ns
+    int32_t world;
     const void* const* param_tab;  // [P] padded param storage
     const int64_t* numel;          // [2P]: unpadded numel, then padded numel
     int32_t n_params;
     int32_t* err;
 };
 
+// GATHER: the source of rank r's chunk is rank r's own shard (shard_tab[r], of
+// which the chunk starts at off_i), not row r of one rank-major buffer; the
+// shards may live in other processes' or GPUs' memory (peer pointers).
+template <bool GATHER>
 __global__ void __launch_bounds__(kThreads) ag_place_kernel(const AgParams a) {
     __shared__ tide_tile_t s_tile;
     for (int64_t t = blockIdx.x; t < a.n_tiles; t += gridDim.x) {
@@ -47,15 +54,19 @@ __global__ void __launch_bounds__(kThreads) ag_place_kernel(const AgParams a) {
         __syncthreads();
         const tide_tile_t tl = s_tile;
         const bool param_ok = tl.param >= 0 && tl.param < a.n_params;
+        // offset of the tile's first element in its source buffer
+        const int64_t src = GATHER ? tl.dst_off - (int64_t)tl.rank * a.shard_numel : tl.dst_off;
         const bool ok = param_ok && tl.n_valid >= 0 && tl.n_valid <= tl.n_total &&
                         tl.src_off >= 0 && tl.src_off + tl.n_total <= a.numel[a.n_params + tl.param] &&
-                        tl.dst_off >= 0 && tl.dst_off + tl.n_valid <= a.ag_numel;
+                        (!GATHER || (tl.rank >= 0 && tl.rank < a.world)) &&
+                        src >= 0 && src + tl.n_valid <= a.ag_numel;
         if (!ok) {
             if (threadIdx.x == 0) atomicOr(a.err, TIDE_KCHECK_TILE);
             continue;
         }
+        const uint16_t* from = GATHER ? static_cast<const uint16_t*>(a.shard_tab[tl.rank]) + src : a.ag + src;
         uint16_t* dst = static_cast<uint16_t*>(const_cast<void*>(a.param_tab[tl.param])) + tl.src_off;
-        block_copy_bf16_v32<kCopyU, kThreads>(a.ag + tl.dst_off, dst, tl.n_valid);
+        block_copy_bf16_v32<kCopyU, kThreads>(from, dst, tl.n_valid);
         if (tl.n_total > tl.n_valid) block_zero_bf16<kThreads>(dst + tl.n_valid, tl.n_total - tl.n_valid);
     }
 }
@@ -102,9 +113,10 @@ __global__ void __launch_bounds__(kThreads) slot_stage_kernel(const StageParams 
 
 }  // namespace
 
-int ag_blocks_per_sm() {
+int ag_blocks_per_sm(bool gather) {
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, ag_place_kernel, kThreads, 0) != cudaSuccess)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &n, gather ? ag_place_kernel<true> : ag_place_kernel<false>, kThreads, 0) != cudaSuccess)
         return 0;
     return n;
 }
@@ -124,12 +136,35 @@ cudaError_t launch_ag_place(const tide_plan* p, const uint16_t* ag, int64_t ag_n
     a.n_tiles = (int64_t)p->tiles.size();
     a.ag = ag;
     a.ag_numel = ag_numel;
+    a.shard_tab = nullptr;
+    a.shard_numel = p->shard_numel;
+    a.world = p->world;
     a.param_tab = d_param_tab;
     a.numel = p->d_numel;
     a.n_params = p->n_params;
     a.err = p->d_err;
     (void)cudaGetLastError();  // drop an error left by an earlier failed runtime call
-    ag_place_kernel<<<grid, kThreads, 0, stream>>>(a);
+    ag_place_kernel<false><<<grid, kThreads, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_ag_gather(const tide_plan* p, const void* const* d_shard_tab, int64_t shard_numel,
+                             const void* const* d_param_tab, int grid, cudaStream_t stream) {
+    if (p->tiles.empty() || grid <= 0) return cudaSuccess;
+    AgParams a;
+    a.tiles = p->d_tiles;
+    a.n_tiles = (int64_t)p->tiles.size();
+    a.ag = nullptr;
+    a.ag_numel = shard_numel;
+    a.shard_tab = d_shard_tab;
+    a.shard_numel = p->shard_numel;
+    a.world = p->world;
+    a.param_tab = d_param_tab;
+    a.numel = p->d_numel;
+    a.n_params = p->n_params;
+    a.err = p->d_err;
+    (void)cudaGetLastError();  // drop an error left by an earlier failed runtime call
+    ag_place_kernel<true><<<grid, kThreads, 0, stream>>>(a);
     return cudaGetLastError();
 }
 

@@ -66,6 +66,9 @@ tide_status_t launchable(const tide_plan* p) {
     return (p->flags & TIDE_PLAN_HOST_ONLY) ? TIDE_ERR_DEVICE : TIDE_OK;
 }
 
+// Calls that need every rank's tiles refuse a one-rank plan.
+tide_status_t all_ranks(const tide_plan* p) { return p->rank >= 0 ? TIDE_ERR_INVALID_ARG : TIDE_OK; }
+
 // A device buffer of `need` elements of size `esize` at `ptr` with `have` elements.
 tide_status_t check_buf(const void* ptr, int64_t have, int64_t need, int esize) {
     if (need == 0) return TIDE_OK;
@@ -248,6 +251,7 @@ extern "C" tide_status_t tide_ag_place(const tide_plan_t* cplan, const void* ag_
     tide_plan* p = const_cast<tide_plan*>(cplan);
     tide_status_t st = check_plan(p);
     if (st != TIDE_OK) return st;
+    if ((st = all_ranks(p)) != TIDE_OK) return st;
     if ((st = check_enums(engine, max_ctas)) != TIDE_OK) return st;
     const int64_t W = p->world, P = p->n_params;
     std::vector<Span> spans;
@@ -278,6 +282,48 @@ extern "C" tide_status_t tide_ag_place(const tide_plan_t* cplan, const void* ag_
     return e == cudaSuccess ? TIDE_OK : TIDE_ERR_CUDA;
 }
 
+extern "C" tide_status_t tide_ag_gather_place(const tide_plan_t* cplan, const void* const* shards,
+                                              int64_t shard_numel, void* const* param_storage,
+                                              const int64_t* param_numel, int32_t engine,
+                                              int32_t max_ctas, void* stream) {
+    ApiRange range("tide_ag_gather_place");
+    tide_plan* p = const_cast<tide_plan*>(cplan);
+    tide_status_t st = check_plan(p);
+    if (st != TIDE_OK) return st;
+    if ((st = all_ranks(p)) != TIDE_OK) return st;
+    if ((st = check_enums(engine, max_ctas)) != TIDE_OK) return st;
+    const int64_t W = p->world, P = p->n_params, Ns = p->shard_numel;
+    std::vector<Span> spans;
+    if (W > 0 && shards == nullptr) return TIDE_ERR_INVALID_ARG;
+    for (int64_t r = 0; r < W; ++r) {
+        if ((st = check_buf(shards[r], shard_numel, Ns, 2)) != TIDE_OK) return st;
+        add_span(spans, shards[r], 2 * Ns, false);
+    }
+    if (P > 0 && (param_storage == nullptr || param_numel == nullptr)) return TIDE_ERR_INVALID_ARG;
+    for (int64_t i = 0; i < P; ++i) {
+        if ((st = check_buf(param_storage[i], param_numel[i], W * p->chunk[i], 2)) != TIDE_OK) return st;
+        add_span(spans, param_storage[i], 2 * W * p->chunk[i], true);
+    }
+    if (overlaps(spans)) return TIDE_ERR_INVALID_ARG;
+    if ((st = launchable(p)) != TIDE_OK) return st;
+    if (p->tiles.empty()) return TIDE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (engine == TIDE_ENGINE_CE) {
+        p->last_kernel = -1;
+        p->last_ctas = 0;
+        e = tide::ce_ag_gather(p, shards, param_storage, s);
+    } else {
+        if ((st = sync_table(p->shard_tab, shards, W, s)) != TIDE_OK) return st;
+        if ((st = sync_table(p->param_tab, const_cast<const void* const*>(param_storage), P, s)) != TIDE_OK)
+            return st;
+        p->last_kernel = K_AG_GATHER;
+        p->last_ctas = grid_for(p, K_AG_GATHER, max_ctas);
+        e = tide::launch_ag_gather(p, p->shard_tab.dev, shard_numel, p->param_tab.dev, p->last_ctas, s);
+    }
+    return e == cudaSuccess ? TIDE_OK : TIDE_ERR_CUDA;
+}
+
 extern "C" tide_status_t tide_rs_reduce(const tide_plan_t* cplan, const void* const* grads,
                                         const int64_t* grad_numel, float* out, int64_t out_numel,
                                         int32_t scale_mode, int32_t order, void* const* slots,
@@ -289,7 +335,9 @@ extern "C" tide_status_t tide_rs_reduce(const tide_plan_t* cplan, const void* co
     if (st != TIDE_OK) return st;
     if ((st = check_enums(engine, max_ctas)) != TIDE_OK) return st;
     if ((st = check_reduce_modes(scale_mode, order)) != TIDE_OK) return st;
-    const int64_t W = p->world, P = p->n_params, n_out = W * p->shard_numel;
+    if (slots != nullptr && (st = all_ranks(p)) != TIDE_OK) return st;
+    // a one-rank plan writes only its own shard
+    const int64_t W = p->world, P = p->n_params, n_out = (p->rank >= 0 ? 1 : W) * p->shard_numel;
     std::vector<Span> spans;
     if ((st = check_grads(p, grads, grad_numel, spans)) != TIDE_OK) return st;
     if ((st = check_buf(out, out_numel, n_out, 4)) != TIDE_OK) return st;
@@ -317,6 +365,7 @@ extern "C" tide_status_t tide_rs_stage(const tide_plan_t* cplan, const void* con
     tide_plan* p = const_cast<tide_plan*>(cplan);
     tide_status_t st = check_plan(p);
     if (st != TIDE_OK) return st;
+    if ((st = all_ranks(p)) != TIDE_OK) return st;
     if ((st = check_enums(engine, max_ctas)) != TIDE_OK) return st;
     std::vector<Span> spans;
     if ((st = check_grads(p, grads, grad_numel, spans)) != TIDE_OK) return st;
@@ -334,6 +383,7 @@ extern "C" tide_status_t tide_rs_reduce_slots(const tide_plan_t* cplan, const vo
     tide_plan* p = const_cast<tide_plan*>(cplan);
     tide_status_t st = check_plan(p);
     if (st != TIDE_OK) return st;
+    if ((st = all_ranks(p)) != TIDE_OK) return st;
     if ((st = check_enums(TIDE_ENGINE_SM, max_ctas)) != TIDE_OK) return st;
     if ((st = check_reduce_modes(scale_mode, order)) != TIDE_OK) return st;
     const int64_t n_out = (int64_t)p->world * p->shard_numel;
@@ -359,6 +409,7 @@ extern "C" tide_status_t tide_rs_reduce_pipelined(const tide_plan_t* cplan, cons
     tide_plan* p = const_cast<tide_plan*>(cplan);
     tide_status_t st = check_plan(p);
     if (st != TIDE_OK) return st;
+    if ((st = all_ranks(p)) != TIDE_OK) return st;
     if ((st = check_enums(TIDE_ENGINE_SM, max_ctas)) != TIDE_OK) return st;
     if ((st = check_reduce_modes(scale_mode, order)) != TIDE_OK) return st;
     if (n_segments < 1 || n_segments > p->world) return TIDE_ERR_INVALID_ARG;

@@ -262,6 +262,37 @@ cudaError_t ce_ag_place(tide_plan* p, const uint16_t* ag, void* const* params, c
     return e != cudaSuccess ? e : j;
 }
 
+// Gathering placement: rank r's chunk of param i comes from rank r's own shard
+// (shards[r] + off_i), one 1-D copy per chunk with data, on the fan-out stream
+// of its source rank; each param's pad tail is one memset.
+cudaError_t ce_ag_gather(tide_plan* p, const void* const* shards, void* const* params,
+                         cudaStream_t stream) {
+    const int64_t W = p->world;
+    const size_t max_pitch = device_max_pitch(p->device);
+    CeIssuer* q = issuer(p);
+    if (q == nullptr) return cudaErrorMemoryAllocation;
+    for (auto& l : q->lists) l.clear();
+    for (int32_t i = 0; i < p->n_params; ++i) {
+        const int64_t c = p->chunk[i], n = p->numel[i];
+        if (c == 0) continue;
+        uint16_t* dst = static_cast<uint16_t*>(params[i]);
+        for (int64_t r = 0; r < W; ++r) {
+            const int64_t valid = std::min(c, std::max<int64_t>(0, n - r * c));
+            if (valid == 0) break;  // later ranks hold only pad rows
+            const uint16_t* src = static_cast<const uint16_t*>(shards[r]) + p->offset[i];
+            q->lists[r % kFanout].push_back(rows_op(dst + r * c, 0, src, 0, 2 * valid, 1));
+        }
+        if (W * c > n)
+            q->lists[i % kFanout].push_back(
+                CeOp{CeOp::kMemset, dst + n, 0, nullptr, 0, (size_t)(2 * (W * c - n)), 0});
+    }
+    cudaError_t e = fork(p, stream);
+    if (e != cudaSuccess) return e;
+    e = issue_all(p, q, max_pitch);
+    cudaError_t j = join(p, stream);
+    return e != cudaSuccess ? e : j;
+}
+
 // Stage the chunks [j0, j1) (chunk i*W + r: rank r's rows of param i) from
 // every source rank k into slot k.  Within one param the chunks of a range are
 // consecutive ranks, so each (k, param) pair takes one 2-D copy plus at most

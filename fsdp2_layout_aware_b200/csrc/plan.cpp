@@ -37,10 +37,11 @@ void free_device(tide_plan* p) {
     cudaFree(p->grad_tab.dev);
     cudaFree(p->param_tab.dev);
     cudaFree(p->slot_tab.dev);
+    cudaFree(p->shard_tab.dev);
     p->d_tiles = nullptr;
     p->d_numel = nullptr;
     p->d_err = nullptr;
-    p->grad_tab.dev = p->param_tab.dev = p->slot_tab.dev = nullptr;
+    p->grad_tab.dev = p->param_tab.dev = p->slot_tab.dev = p->shard_tab.dev = nullptr;
 }
 
 tide_status_t upload(tide_plan* p) {
@@ -63,12 +64,14 @@ tide_status_t upload(tide_plan* p) {
     if (e == cudaSuccess) e = dev_alloc(&p->grad_tab.dev, W * P, &total);
     if (e == cudaSuccess) e = dev_alloc(&p->param_tab.dev, P, &total);
     if (e == cudaSuccess) e = dev_alloc(&p->slot_tab.dev, W, &total);
+    if (e == cudaSuccess) e = dev_alloc(&p->shard_tab.dev, W, &total);
     if (e != cudaSuccess) {
         st = (e == cudaErrorMemoryAllocation) ? TIDE_ERR_NOMEM : TIDE_ERR_CUDA;
     }
     p->grad_tab.capacity = W * P;
     p->param_tab.capacity = P;
     p->slot_tab.capacity = W;
+    p->shard_tab.capacity = W;
     if (st == TIDE_OK && T > 0)
         e = cudaMemcpy(p->d_tiles, p->tiles.data(), sizeof(tide_tile_t) * T, cudaMemcpyHostToDevice);
     if (st == TIDE_OK && e == cudaSuccess && P > 0) {
@@ -92,9 +95,10 @@ tide_status_t upload(tide_plan* p) {
         }
         p->blocks_per_sm[K_RS_TREE] = tide::rs_blocks_per_sm(p->world, false, TIDE_ORDER_TREE, false);
         p->blocks_per_sm[K_SLOT_RS_TREE] = tide::rs_blocks_per_sm(p->world, true, TIDE_ORDER_TREE, false);
-        p->blocks_per_sm[K_AG] = tide::ag_blocks_per_sm();
+        p->blocks_per_sm[K_AG] = tide::ag_blocks_per_sm(false);
+        p->blocks_per_sm[K_AG_GATHER] = tide::ag_blocks_per_sm(true);
         p->blocks_per_sm[K_STAGE] = tide::stage_blocks_per_sm();
-        for (int k : {K_RS, K_AG, K_STAGE, K_SLOT_RS, K_RS_TREE, K_SLOT_RS_TREE})
+        for (int k : {K_RS, K_AG, K_STAGE, K_SLOT_RS, K_RS_TREE, K_SLOT_RS_TREE, K_AG_GATHER})
             if (p->blocks_per_sm[k] <= 0) st = TIDE_ERR_CUDA;
         // 0 here (not enough shared memory) only disables the bulk-copy path
         p->blocks_per_sm[K_RS_TMA] = p->blocks_per_sm[K_SLOT_RS_TMA] = tide::rs_tma_blocks_per_sm(p->world);
@@ -107,15 +111,14 @@ tide_status_t upload(tide_plan* p) {
     return st;
 }
 
-}  // namespace
-
-extern "C" tide_status_t tide_plan_group(const tide_param_t* params, int32_t n_params,
-                                         int32_t world, int32_t device, uint32_t flags,
-                                         tide_plan_t** out_plan) {
+// Builds a plan for all ranks (rank < 0) or for one output rank.
+tide_status_t make_plan(const tide_param_t* params, int32_t n_params, int32_t world, int32_t rank,
+                        int32_t device, uint32_t flags, tide_plan_t** out_plan) {
     if (out_plan == nullptr) return TIDE_ERR_INVALID_ARG;
     *out_plan = nullptr;
     if (n_params < 0 || (n_params > 0 && params == nullptr)) return TIDE_ERR_INVALID_ARG;
     if (world < 1 || world > TIDE_MAX_WORLD) return TIDE_ERR_INVALID_ARG;
+    if (rank >= world) return TIDE_ERR_INVALID_ARG;
     if ((flags & ~(uint32_t)(TIDE_PLAN_HOST_ONLY | TIDE_PLAN_TMA | TIDE_PLAN_TEST_TMA_TIMEOUT)) != 0)
         return TIDE_ERR_INVALID_ARG;
     if (!(flags & TIDE_PLAN_HOST_ONLY) && device < 0) return TIDE_ERR_DEVICE;
@@ -124,6 +127,7 @@ extern "C" tide_status_t tide_plan_group(const tide_param_t* params, int32_t n_p
     if (p == nullptr) return TIDE_ERR_NOMEM;
     p->device = device;
     p->world = world;
+    p->rank = rank;
     p->n_params = n_params;
     p->flags = flags;
     const int64_t W = world;
@@ -152,17 +156,19 @@ extern "C" tide_status_t tide_plan_group(const tide_param_t* params, int32_t n_p
         if (!mul_ok(W, acc)) { delete p; return TIDE_ERR_SIZE; }
         p->shard_numel = acc;
         // tiles in chunk order: param, then rank, then position; the chunk
-        // (i, r) is number i*W + r and holds tiles [begin[i*W+r], begin[i*W+r+1])
+        // (i, r) is number i*W + r and holds tiles [begin[i*W+r], begin[i*W+r+1]).
+        // A one-rank plan keeps only its rank's chunks, at offsets in its shard.
         p->chunk_tile_begin.assign((size_t)n_params * W + 1, 0);
         for (int32_t i = 0; i < n_params; ++i) {
             for (int64_t r = 0; r < W; ++r) {
                 p->chunk_tile_begin[(size_t)i * W + r] = (int64_t)p->tiles.size();
+                if (rank >= 0 && r != rank) continue;
                 const int64_t c = p->chunk[i];
                 const int64_t valid = std::min(c, std::max<int64_t>(0, p->numel[i] - r * c));
                 for (int64_t e0 = 0; e0 < c; e0 += TIDE_TILE_ELEMS) {
                     tide_tile_t t;
                     t.src_off = r * c + e0;
-                    t.dst_off = r * acc + p->offset[i] + e0;
+                    t.dst_off = (rank >= 0 ? 0 : r * acc) + p->offset[i] + e0;
                     t.param = i;
                     t.rank = (int32_t)r;
                     t.n_total = (int32_t)std::min<int64_t>(TIDE_TILE_ELEMS, c - e0);
@@ -187,6 +193,24 @@ extern "C" tide_status_t tide_plan_group(const tide_param_t* params, int32_t n_p
     }
     *out_plan = p;
     return TIDE_OK;
+}
+
+}  // namespace
+
+extern "C" tide_status_t tide_plan_group(const tide_param_t* params, int32_t n_params,
+                                         int32_t world, int32_t device, uint32_t flags,
+                                         tide_plan_t** out_plan) {
+    return make_plan(params, n_params, world, -1, device, flags, out_plan);
+}
+
+extern "C" tide_status_t tide_plan_group_rank(const tide_param_t* params, int32_t n_params,
+                                              int32_t world, int32_t rank, int32_t device,
+                                              uint32_t flags, tide_plan_t** out_plan) {
+    if (rank < 0) {
+        if (out_plan != nullptr) *out_plan = nullptr;
+        return TIDE_ERR_INVALID_ARG;
+    }
+    return make_plan(params, n_params, world, rank, device, flags, out_plan);
 }
 
 extern "C" void tide_plan_destroy(tide_plan_t* plan) {

@@ -12,7 +12,7 @@
 // Kernel ids (match tide_launch_ctas and tide_plan_last_launch).
 enum : int32_t {
     K_RS = 0, K_AG = 1, K_STAGE = 2, K_SLOT_RS = 3, K_RS_TMA = 4, K_SLOT_RS_TMA = 5,
-    K_RS_V32 = 6, K_SLOT_RS_V32 = 7, K_RS_TREE = 8, K_SLOT_RS_TREE = 9, K_COUNT = 10
+    K_RS_V32 = 6, K_SLOT_RS_V32 = 7, K_RS_TREE = 8, K_SLOT_RS_TREE = 9, K_AG_GATHER = 10, K_COUNT = 11
 };
 
 // A device pointer table with a host mirror: re-uploaded only when it changes.
@@ -28,6 +28,7 @@ struct PtrTable {
 struct tide_plan {
     int32_t device = -1;
     int32_t world = 0;
+    int32_t rank = -1;                   // >= 0: the plan covers only this output rank's shard
     int32_t n_params = 0;
     uint32_t flags = 0;
     int64_t shard_numel = 0;             // Ns
@@ -45,7 +46,7 @@ struct tide_plan {
     tide_tile_t* d_tiles = nullptr;
     int64_t* d_numel = nullptr;
     int32_t* d_err = nullptr;
-    PtrTable grad_tab, param_tab, slot_tab;
+    PtrTable grad_tab, param_tab, slot_tab, shard_tab;
     int64_t workspace_bytes = 0;
 
     int32_t sm_count = 0;
@@ -62,7 +63,7 @@ constexpr int kThreads = 256;
 int rs_blocks_per_sm(int world, bool slot, int order, bool v32);
 bool rs_v32_applies(int world);       // whether the 32-byte variant exists for this W
 int rs_tma_blocks_per_sm(int world);  // also opts the TMA kernels in to their shared memory
-int ag_blocks_per_sm();
+int ag_blocks_per_sm(bool gather);
 int stage_blocks_per_sm();
 
 // Kernel launches; return the launch's cudaError_t.
@@ -77,6 +78,9 @@ cudaError_t launch_rs_reduce_tma(const tide_plan* p, const void* const* d_src_ta
                                  int64_t t0 = 0, int64_t t1 = -1);
 cudaError_t launch_ag_place(const tide_plan* p, const uint16_t* ag, int64_t ag_numel,
                             const void* const* d_param_tab, int grid, cudaStream_t stream);
+// Placement from W per-rank shards (d_shard_tab[r]: rank r's [Ns] shard).
+cudaError_t launch_ag_gather(const tide_plan* p, const void* const* d_shard_tab, int64_t shard_numel,
+                             const void* const* d_param_tab, int grid, cudaStream_t stream);
 cudaError_t launch_slot_stage(const tide_plan* p, const void* const* d_grad_tab,
                               const void* const* d_slot_tab, int64_t slot_numel, int grid,
                               cudaStream_t stream);
@@ -84,6 +88,9 @@ cudaError_t launch_slot_stage(const tide_plan* p, const void* const* d_grad_tab,
 // Copy-engine variants (no kernels).
 cudaError_t ce_ag_place(tide_plan* p, const uint16_t* ag, void* const* params,
                         cudaStream_t stream);
+// Placement from W per-rank shards (shards[r]: rank r's [Ns] shard).
+cudaError_t ce_ag_gather(tide_plan* p, const void* const* shards, void* const* params,
+                         cudaStream_t stream);
 // Stages the chunks [j0, j1) (numbered i*W + r as in chunk_tile_begin; j1 < 0:
 // all) from every source rank k into slot k.
 cudaError_t ce_slot_stage(tide_plan* p, const void* const* grads, void* const* slots,

@@ -40,9 +40,9 @@ TIDE_TILE_ELEMS = 8192
 TIDE_NOALLOC_SCRATCH_BYTES = 1 << 20
 
 (K_RS, K_AG, K_STAGE, K_SLOT_RS, K_RS_TMA, K_SLOT_RS_TMA, K_RS_V32, K_SLOT_RS_V32, K_RS_TREE,
- K_SLOT_RS_TREE) = range(10)
+ K_SLOT_RS_TREE, K_AG_GATHER) = range(11)
 KERNEL_NAMES = ("rs", "ag", "stage", "slot_rs", "rs_tma", "slot_rs_tma", "rs_v32", "slot_rs_v32",
-                "rs_tree", "slot_rs_tree")
+                "rs_tree", "slot_rs_tree", "ag_gather")
 
 
 class tide_param_t(ctypes.Structure):
@@ -68,6 +68,8 @@ _P = ctypes.POINTER
 
 _SIGNATURES = {
     "tide_plan_group": (_i32, [_P(tide_param_t), _i32, _i32, _i32, _u32, _P(_vp)]),
+    "tide_plan_group_rank": (_i32, [_P(tide_param_t), _i32, _i32, _i32, _i32, _u32, _P(_vp)]),
+    "tide_ag_gather_place": (_i32, [_vp, _P(_vp), _i64, _P(_vp), _P(_i64), _i32, _i32, _vp]),
     "tide_plan_destroy": (None, [_vp]),
     "tide_plan_info": (_i32, [_vp, _P(_i32), _P(_i32), _P(_i64), _P(_i64), _P(_i64)]),
     "tide_plan_query": (_i32, [_vp, _i32, _P(_i64), _P(_i64), _P(_i64), _P(_i64)]),
@@ -173,6 +175,16 @@ def tide_plan_group(params, world: int, device: int, flags: int = 0):
     return st, (out.value if st == TIDE_OK else None)
 
 
+def tide_plan_group_rank(params, world: int, rank: int, device: int, flags: int = 0):
+    """A plan for one output rank.  Returns (status, plan handle or None)."""
+    arr = (tide_param_t * max(1, len(params)))()
+    for j, (d0, inner) in enumerate(params):
+        arr[j].dim0, arr[j].inner = int(d0), int(inner)
+    out = _vp()
+    st = lib().tide_plan_group_rank(arr, len(params), world, rank, device, flags, ctypes.byref(out))
+    return st, (out.value if st == TIDE_OK else None)
+
+
 def tide_plan_destroy(plan) -> None:
     lib().tide_plan_destroy(plan)
 
@@ -205,6 +217,12 @@ def tide_ag_place(plan, ag_buf: int, ag_numel: int, param_storage, param_numel, 
                   max_ctas: int, stream: int) -> int:
     return lib().tide_ag_place(plan, ag_buf, ag_numel, _ptr_array(param_storage),
                                _i64_array(param_numel), engine, max_ctas, stream)
+
+
+def tide_ag_gather_place(plan, shards, shard_numel: int, param_storage, param_numel, engine: int,
+                         max_ctas: int, stream: int) -> int:
+    return lib().tide_ag_gather_place(plan, _ptr_array(shards), shard_numel, _ptr_array(param_storage),
+                                      _i64_array(param_numel), engine, max_ctas, stream)
 
 
 def tide_rs_reduce(plan, grads, grad_numel, out: int, out_numel: int, scale_mode: int, order: int,
@@ -288,7 +306,9 @@ class Plan:
     """
 
     def __init__(self, shapes, world: int, device=None, host_only: bool = False,
-                 tma: bool = False, test_tma_timeout: bool = False):
+                 tma: bool = False, test_tma_timeout: bool = False, rank=None):
+        """rank: None for the whole group (all W output shards), or one output rank r, whose
+        rs_reduce then writes only its own [Ns] shard."""
         self.shapes = [tuple(int(d) for d in s) for s in shapes]
         self.world = int(world)
         if host_only:
@@ -300,7 +320,11 @@ class Plan:
         params = [(s[0], _prod(s[1:])) for s in self.shapes]
         flags = ((TIDE_PLAN_HOST_ONLY if host_only else 0) | (TIDE_PLAN_TMA if tma else 0) |
                  (TIDE_PLAN_TEST_TMA_TIMEOUT if test_tma_timeout else 0))
-        st, handle = tide_plan_group(params, self.world, dev, flags)
+        self.rank = None if rank is None else int(rank)
+        if self.rank is None:
+            st, handle = tide_plan_group(params, self.world, dev, flags)
+        else:
+            st, handle = tide_plan_group_rank(params, self.world, self.rank, dev, flags)
         _check(st, "tide_plan_group")
         self.handle = handle
         self.device_index = dev
@@ -352,6 +376,14 @@ class Plan:
         st = tide_ag_place(self.handle, ag.data_ptr(), ag.numel(), p.ptrs, p.numels, engine,
                            max_ctas, _stream_handle(stream))
         _check(st, "tide_ag_place")
+
+    def ag_gather_place(self, shards, params, engine: int = TIDE_ENGINE_SM, max_ctas: int = 0,
+                        stream=None) -> None:
+        """Place every rank's shard (shards[r]: bf16 [Ns], possibly a peer's memory)."""
+        s, p = _table(shards), _table(params)
+        st = tide_ag_gather_place(self.handle, s.ptrs, s.min_numel, p.ptrs, p.numels, engine,
+                                  max_ctas, _stream_handle(stream))
+        _check(st, "tide_ag_gather_place")
 
     def rs_reduce(self, grads, out, scale_mode: int = TIDE_SCALE_INV_WORLD,
                   order: int = TIDE_ORDER_RANK, slots=None, engine: int = TIDE_ENGINE_SM,

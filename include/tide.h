@@ -134,6 +134,23 @@ typedef struct tide_plan tide_plan_t;
 TIDE_API tide_status_t tide_plan_group(const tide_param_t* params, int32_t n_params, int32_t world,
                               int32_t device, uint32_t flags, tide_plan_t** out_plan);
 
+/*
+ * A plan for ONE output rank of a group (0 <= rank < world): the same layout,
+ * but only rank `rank`'s tiles, with output offsets inside its own shard.  It
+ * is the plan a real data-parallel rank uses to reduce-scatter (weekinpapers.com
+ * Abstract, TIDE-RS: each rank's shard is reduced from every rank's
+ * gradients): tide_rs_reduce with it reads chunk `rank` of every rank's
+ * gradients, which may be peer pointers (other processes' or GPUs' memory
+ * mapped into this one), and writes out[0 .. Ns):
+ *   out[off_i + e] = s * fl32(sum_k fp32(g_{k,i}[rank*c_i + e])),  +0.0 at pads,
+ * the same bits as rows [rank*Ns, (rank+1)*Ns) of the all-rank call.  Only
+ * tide_rs_reduce without slots accepts such a plan; the other data calls
+ * return TIDE_ERR_INVALID_ARG for it.  Arguments and errors as tide_plan_group.
+ */
+TIDE_API tide_status_t tide_plan_group_rank(const tide_param_t* params, int32_t n_params,
+                                            int32_t world, int32_t rank, int32_t device,
+                                            uint32_t flags, tide_plan_t** out_plan);
+
 /* Free a plan (NULL is accepted).  Synchronizes the plan's device first, so
  * that no enqueued call can still read the tables. */
 TIDE_API void tide_plan_destroy(tide_plan_t* plan);
@@ -166,6 +183,24 @@ TIDE_API tide_status_t tide_plan_tiles(const tide_plan_t* plan, tide_tile_t* out
 TIDE_API tide_status_t tide_ag_place(const tide_plan_t* plan, const void* ag_buf, int64_t ag_numel,
                             void* const* param_storage, const int64_t* param_numel,
                             int32_t engine, int32_t max_ctas, void* stream);
+
+/*
+ * TIDE-AG placement from per-rank shards (weekinpapers.com Abstract, TIDE-AG:
+ * shards land in parameter storage; kongchang.com "TIDE's Design Approach"):
+ * the same result as tide_ag_place, but rank r's shard is its own buffer
+ * shards[r] (bf16, shard_numel >= Ns elements each) instead of row r of one
+ * rank-major buffer, so each rank can place every peer's shard straight from
+ * that peer's memory (peer pointers):
+ *   param_i[r*c_i + e] = shards[r][off_i + e]  for valid rows, +0 for pad rows.
+ * shards is a host array of W device pointers; shards are only read, and no
+ * shard may overlap any parameter storage.  engine: TIDE_ENGINE_SM (one kernel
+ * launch) or TIDE_ENGINE_CE (one copy per (param, rank) chunk with data plus
+ * one memset per padded param).  Needs an all-rank plan.
+ */
+TIDE_API tide_status_t tide_ag_gather_place(const tide_plan_t* plan, const void* const* shards,
+                                            int64_t shard_numel, void* const* param_storage,
+                                            const int64_t* param_numel, int32_t engine,
+                                            int32_t max_ctas, void* stream);
 
 /*
  * TIDE-RS (weekinpapers.com Abstract, TIDE-RS and the two-phase pipeline;
@@ -285,7 +320,8 @@ TIDE_API tide_status_t tide_rs_reduce_noalloc(const tide_param_t* params, int32_
  * 1 = AG place, 2 = Slot-Reuse stage, 3 = slot reduce (load/store), 4 = RS
  * reduce with bulk-copy staging, 5 = slot reduce with bulk-copy staging,
  * 6 = RS reduce with 32-byte loads, 7 = slot reduce with 32-byte loads,
- * 8 = RS reduce in tree order, 9 = slot reduce in tree order.
+ * 8 = RS reduce in tree order, 9 = slot reduce in tree order,
+ * 10 = AG placement from per-rank shards (tide_ag_gather_place).
  * The reductions use kernels 4/5 (one CTA per SM, TMA loads into shared memory)
  * when the plan was built with TIDE_PLAN_TMA, every tile starts on an
  * 8-element boundary and every source and the output are 16-byte aligned.

@@ -295,3 +295,76 @@ def test_tensor_table_marshals_once_in_rank_major_order():
     assert T.tide_rs_reduce(h, short.ptrs, short.numels, out.data_ptr(), out.numel(), 1, 0, None, 0,
                             0, 0, 0) == T.TIDE_ERR_SIZE
     T.tide_plan_destroy(h)
+
+
+# --------------------------------------------------------------------------- one-rank plans, gathering
+
+
+@pytest.mark.parametrize("group", [configs.tiny(), degenerate(), mini_wan(), configs.qwen3moe(4)],
+                         ids=lambda g: g.name)
+def test_rank_plan_tiles_are_that_ranks_tiles_inside_its_shard(group):
+    W = group.world
+    full = host_plan(group)
+    L = oracle.layout(W, group.shapes)
+    all_tiles = full.tiles()
+    for r in range(W):
+        plan = T.Plan(group.shapes, W, host_only=True, rank=r)
+        assert plan.rank == r and plan.shard_numel == L.Ns
+        mine = [t for t in all_tiles if t.rank == r]
+        tiles = plan.tiles()
+        assert len(tiles) == len(mine) == plan.n_tiles
+        cover = np.zeros(L.Ns, dtype=np.int32)
+        for t, u in zip(tiles, mine):
+            assert (t.param, t.rank, t.src_off, t.n_valid, t.n_total) == \
+                   (u.param, u.rank, u.src_off, u.n_valid, u.n_total)
+            assert t.dst_off == u.dst_off - r * L.Ns
+            cover[t.dst_off: t.dst_off + t.n_total] += 1
+        assert np.all(cover == 1)                    # the rank's shard, each position once
+
+
+def test_rank_plan_arguments():
+    g = configs.tiny()
+    params = [(s[0], int(np.prod(s[1:])) if len(s) > 1 else 1) for s in g.shapes]
+    for rank in (-1, g.world, 99):
+        st, h = T.tide_plan_group_rank(params, g.world, rank, 0, T.TIDE_PLAN_HOST_ONLY)
+        assert st == T.TIDE_ERR_INVALID_ARG and h is None
+    plan = T.Plan(g.shapes, g.world, host_only=True, rank=2)
+    a = fake_args(g)
+    L = oracle.layout(g.world, g.shapes)
+    # its output is one shard: Ns elements are enough, fewer are not
+    assert rs(plan, a, n_out=L.Ns) == T.TIDE_ERR_DEVICE
+    assert rs(plan, a, n_out=L.Ns - 1) == T.TIDE_ERR_SIZE
+    # calls that need every rank's tiles refuse it
+    assert rs(plan, a, use_slots=a["slots"]) == T.TIDE_ERR_INVALID_ARG
+    assert ag(plan, a) == T.TIDE_ERR_INVALID_ARG
+    assert T.tide_rs_stage(plan.handle, a["grads"], a["gnum"], a["slots"], a["n_slot"], 0, 0,
+                           0) == T.TIDE_ERR_INVALID_ARG
+    assert T.tide_rs_reduce_slots(plan.handle, a["slots"], a["n_slot"], a["out"], a["n_out"], 1, 0,
+                                  0, 0) == T.TIDE_ERR_INVALID_ARG
+    assert T.tide_rs_reduce_pipelined(plan.handle, a["grads"], a["gnum"], a["out"], a["n_out"], 1, 0,
+                                      a["slots"], a["n_slot"], 1, 0, 0, 0) == T.TIDE_ERR_INVALID_ARG
+    assert T.tide_ag_gather_place(plan.handle, a["slots"], L.Ns, a["params"], a["pnum"], 0, 0,
+                                  0) == T.TIDE_ERR_INVALID_ARG
+
+
+def test_gather_place_validation(tiny_plan, args):
+    g = configs.tiny()
+    W = g.world
+    L = oracle.layout(W, g.shapes)
+    f = Fake()
+    f.next = BASE + (1 << 40)                        # clear of the other fake buffers
+    shards = [f.buf(2 * L.Ns) for _ in range(W)]
+
+    def gather(sh=shards, n=L.Ns, params=None, engine=0):
+        return T.tide_ag_gather_place(tiny_plan.handle, sh, n, params or args["params"], args["pnum"],
+                                      engine, 0, 0)
+    assert gather() == T.TIDE_ERR_DEVICE             # valid: stops at the host-only plan
+    assert gather(engine=1) == T.TIDE_ERR_DEVICE
+    assert gather(n=L.Ns - 1) == T.TIDE_ERR_SIZE
+    assert gather(sh=[shards[0] + 1] + shards[1:]) == T.TIDE_ERR_ALIGNMENT
+    assert gather(sh=[0] + shards[1:]) == T.TIDE_ERR_INVALID_ARG
+    assert gather(engine=7) == T.TIDE_ERR_INVALID_ARG
+    # a parameter storage overlapping a shard is refused
+    assert gather(params=[shards[1]] + args["params"][1:]) == T.TIDE_ERR_INVALID_ARG
+    # shards may overlap one another (they are only read)
+    assert gather(sh=[shards[0]] * W) == T.TIDE_ERR_DEVICE
