@@ -312,6 +312,24 @@ def run_variants(wl, K, stream, peak, flush):
     rec("rs_reduce_tma", timed_calls(lambda: tma_plan.rs_reduce(wl.grads_t, wl.out), K, stream, flush),
         B["rs"], 1, tma_plan, same_rs)
     tma_plan.close()
+    # the exchange as one rank runs it: rank 0 reduces its own shard ...
+    rank0 = T.Plan(wl.group.shapes, wl.group.world, device=wl.out.device, rank=0)
+    n0 = sum(min(rank0.query(i)["chunk_numel"], wl.group.numel(i)) for i in range(wl.group.n_params))
+    shard0 = torch.full((wl.Ns,), float("nan"), device=wl.out.device)
+    rec("rs_reduce_one_rank", timed_calls(lambda: rank0.rs_reduce(wl.grads_t, shard0), K, stream, flush),
+        2 * wl.group.world * n0 + 4 * wl.Ns, 1, rank0,
+        lambda: bool(torch.equal(shard0.view(torch.int32), ref_out[: wl.Ns])))
+    rank0.close()
+    del shard0
+    # ... and places every rank's shard, each from its own buffer (here: row r of the input)
+    flat_ag = wl.ag.reshape(-1)
+    shards = T.TensorTable([flat_ag[r * wl.Ns: (r + 1) * wl.Ns] for r in range(wl.group.world)])
+    for eng, name in ((T.TIDE_ENGINE_SM, "sm"), (T.TIDE_ENGINE_CE, "ce")):
+        wl.params_poison()
+        rec(f"ag_gather_place_{name}",
+            timed_calls(lambda: wl.plan.ag_gather_place(shards, wl.params_t, engine=eng), K, stream, flush),
+            B["ag"], 1 if eng == 0 else 0, wl.plan, same_ag)
+    del shards, flat_ag
     slots = wl.ensure_slots()
     for eng, name in ((T.TIDE_ENGINE_SM, "sm"), (T.TIDE_ENGINE_CE, "ce")):
         rec(f"slot_stage_{name}", timed_calls(lambda: wl.plan.rs_stage(wl.grads_t, slots, engine=eng),
@@ -384,6 +402,9 @@ ROW_KINDS = {
     "slot_stage_ce": ("slot_stage", "copy engines"),
     "slot_reduce": ("slot_reduce", "SM, rank order"),
     "slot_reuse_serial_ce": ("slot_reuse", "copy-engine staging, then reduce"),
+    "rs_reduce_one_rank": ("rs_reduce", "one rank's shard (one-rank plan), rank order"),
+    "ag_gather_place_sm": ("ag_gather_place", "SM, from per-rank shards"),
+    "ag_gather_place_ce": ("ag_gather_place", "copy engines, from per-rank shards"),
     "stock_torch_pack_reduce": ("stock_rs", "torch _chunk_cat pack + add"),
     "stock_torch_copyout": ("stock_ag", "torch split_with_sizes_copy"),
 }
@@ -728,7 +749,12 @@ def bench_workload(args, group, rank, world, device, dist_on):
         "stock_fp32_buffer_bytes": 4 * group.world * wl.Ns,
     }
     if not args.no_variants:
-        res["variants"] = run_variants(wl, max(3, min(K, 20)), stream, peak, flush)
+        # the step's figures above stand even if a variant fails: record the error instead
+        try:
+            res["variants"] = run_variants(wl, max(3, min(K, 20)), stream, peak, flush)
+        except Exception as e:  # noqa: BLE001
+            res["variants_error"] = f"{type(e).__name__}: {e}"
+            wl.drop_slots()
     if not args.no_e2e:
         e2e_ms, serial_ms, h2d, d2h, pinned = run_e2e(wl, max(1, args.e2e_steps), stream)
         e2e_ms, serial_ms = max_over_ranks([e2e_ms, serial_ms], device)

@@ -576,5 +576,6 @@ def test_workspace_is_tables_only():
         g = configs.by_name(name)
         plan = T.Plan(g.shapes, g.world)
         W, P = g.world, g.n_params
-        expect = plan.n_tiles * 32 + 2 * P * 8 + 4 + W * P * 8 + P * 8 + W * 8
+        # tiles, numel table, error word, pointer tables: grads, params, slots, shards
+        expect = plan.n_tiles * 32 + 2 * P * 8 + 4 + W * P * 8 + P * 8 + W * 8 + W * 8
         assert plan.workspace_bytes == expect
