@@ -108,6 +108,7 @@ typedef struct {
  * `param` that rank `rank` owns, with e0 a multiple of TIDE_TILE_ELEMS.
  *   src_off = rank*c_i + e0        offset into the param's own tensor
  *   dst_off = rank*Ns + off_i + e0 offset into a rank-major [W][Ns] buffer
+ *             (off_i + e0, inside the rank's own shard, in a one-rank plan)
  *   the first n_valid elements hold data; the remaining ones are padding.
  */
 typedef struct {
@@ -164,7 +165,9 @@ TIDE_API tide_status_t tide_plan_info(const tide_plan_t* plan, int32_t* world, i
 TIDE_API tide_status_t tide_plan_query(const tide_plan_t* plan, int32_t param, int64_t* shard_rows,
                               int64_t* shard_offset, int64_t* padded_numel, int64_t* chunk_numel);
 
-/* Copy up to `capacity` tiles into out (host array); *n_written gets the count. */
+/* Copy up to `capacity` tiles into out (host array); *n_written gets the count.
+ * Tiles are listed chunk by chunk: param 0's chunks of ranks 0..W-1, then
+ * param 1's, and so on; within a chunk by position. */
 TIDE_API tide_status_t tide_plan_tiles(const tide_plan_t* plan, tide_tile_t* out, int64_t capacity,
                               int64_t* n_written);
 
