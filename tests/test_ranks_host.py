@@ -7,7 +7,6 @@ import os
 import pytest
 import torch.multiprocessing as mp
 
-
 from _dist_helpers import free_port
 
 SHAPES = ((37, 16), (1000,), (7, 3), (5, 130), (0, 4), (64, 64))
