@@ -34,7 +34,8 @@
  *   - A plan keeps small device tables (tile list, pointer tables, an error
  *     word).  A pointer table is re-uploaded, stream-ordered, only when its
  *     contents change.  One plan must be used from one stream at a time (or the
- *     caller orders the streams).
+ *     caller orders the streams) and from one host thread at a time; different
+ *     plans are independent.
  *   - bf16 buffers must be 2-byte aligned and fp32 buffers 4-byte aligned; any
  *     such alignment is accepted (16-byte alignment gives the fast path).
  *   - No call allocates device memory except tide_plan_group.
