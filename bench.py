@@ -594,8 +594,10 @@ def run_interference(device, seed):
     B200, i.e. not single-wave) and 3072x3072x16384, whose kernel fits in one
     wave.  Per point, three trials of: the GEMM batch alone, then concurrently
     with back-to-back RS launches on a second stream (started first, enough of
-    them to outlast the GEMMs); slowdown = median(concurrent) / median(alone)
-    - 1.  Done for the load/store RS kernel and for the bulk-copy (TMA) one.
+    them to outlast the GEMMs twice over); slowdown = median(concurrent) / median(alone)
+    - 1.  Done for the load/store RS kernel and for the bulk-copy (TMA) one,
+    and for the Slot-Reuse staging on the copy engines (no SM; its bytes are
+    the staging's).
     """
     import torch
     from synth import configs
@@ -628,38 +630,43 @@ def run_interference(device, seed):
         for _ in range(5):
             gemm_alone()
         g = {"gemm": f"bf16 {m}x{n}x{k} torch.matmul (cuBLAS), {n_gemm} per batch", "points": []}
-        for kind, plan in plans.items():
-            for ctas in (8, 16, 32, 0):
-                rs_ms = timed_calls(lambda: plan.rs_reduce(wl.grads_t, wl.out, max_ctas=ctas, stream=s_rs),
-                                    5, s_rs)
-                _, n_ctas = plan.last_launch()
-                alone, conc, rs_conc = [], [], []
-                for _ in range(3):
-                    alone.append(gemm_alone())
-                    reps = int((alone[-1] * n_gemm * 1.2) / max(rs_ms, 1e-3)) + 2
-                    torch.cuda.synchronize()
-                    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                    with torch.cuda.stream(s_rs):
-                        r0.record(s_rs)
-                        for _ in range(reps):
-                            plan.rs_reduce(wl.grads_t, wl.out, max_ctas=ctas, stream=s_rs)
-                        r1.record(s_rs)
-                    with torch.cuda.stream(s_gemm):
-                        e0.record(s_gemm); gemm_batch(); e1.record(s_gemm)
-                    torch.cuda.synchronize()
-                    conc.append(e0.elapsed_time(e1) / n_gemm)
-                    rs_conc.append(r0.elapsed_time(r1) / reps)
-                ga, gc = statistics.median(alone), statistics.median(conc)
-                g["points"].append({
-                    "rs_kernel": kind, "max_ctas": ctas, "ctas": n_ctas, "rs_ms_alone": round(rs_ms, 4),
-                    "rs_GBps_alone": round(B["rs"] / (rs_ms * 1e-3) / 1e9, 1),
-                    "rs_ms_concurrent": round(statistics.median(rs_conc), 4),
-                    "gemm_ms_alone": round(ga, 4), "gemm_ms_concurrent": round(gc, 4),
-                    "gemm_slowdown": round(gc / ga - 1.0, 4),
-                    "rs_cta_ms_per_call": round(n_ctas * rs_ms, 2)})
+        points = [(kind, plan, ctas, B["rs"],
+                   lambda plan=plan, ctas=ctas: plan.rs_reduce(wl.grads_t, wl.out, max_ctas=ctas, stream=s_rs))
+                  for kind, plan in plans.items() for ctas in (8, 16, 32, 0)]
+        slots = T.TensorTable(wl.ensure_slots())
+        points.append(("ce_stage", wl.plan, 0, B["stage"],
+                       lambda: wl.plan.rs_stage(wl.grads_t, slots, engine=T.TIDE_ENGINE_CE, stream=s_rs)))
+        for kind, plan, ctas, nbytes, call in points:
+            rs_ms = timed_calls(call, 5, s_rs)
+            n_ctas = max(0, plan.last_launch()[1]) if kind != "ce_stage" else 0
+            alone, conc, rs_conc = [], [], []
+            for _ in range(3):
+                alone.append(gemm_alone())
+                reps = int((alone[-1] * n_gemm * 2.0) / max(rs_ms, 1e-3)) + 2
+                torch.cuda.synchronize()
+                r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                with torch.cuda.stream(s_rs):
+                    r0.record(s_rs)
+                    for _ in range(reps):
+                        call()
+                    r1.record(s_rs)
+                with torch.cuda.stream(s_gemm):
+                    e0.record(s_gemm); gemm_batch(); e1.record(s_gemm)
+                torch.cuda.synchronize()
+                conc.append(e0.elapsed_time(e1) / n_gemm)
+                rs_conc.append(r0.elapsed_time(r1) / reps)
+            ga, gc = statistics.median(alone), statistics.median(conc)
+            g["points"].append({
+                "rs_kernel": kind, "max_ctas": ctas, "ctas": n_ctas, "rs_ms_alone": round(rs_ms, 4),
+                "rs_GBps_alone": round(nbytes / (rs_ms * 1e-3) / 1e9, 1),
+                "rs_ms_concurrent": round(statistics.median(rs_conc), 4),
+                "gemm_ms_alone": round(ga, 4), "gemm_ms_concurrent": round(gc, 4),
+                "gemm_slowdown": round(gc / ga - 1.0, 4),
+                "rs_cta_ms_per_call": round(n_ctas * rs_ms, 2)})
         res["gemms"].append(g)
-        del a, b, c
+        del a, b, c, slots
+        wl.drop_slots()
     plans["tma"].close()
     del wl
     torch.cuda.empty_cache()
