@@ -33,6 +33,20 @@ struct Span {
 
 // True if a written span overlaps any other span (read spans may overlap each other).
 bool overlaps(std::vector<Span>& spans) {
+    size_t n_write = 0;
+    for (const Span& s : spans) n_write += (s.write && s.lo != s.hi) ? 1 : 0;
+    if (n_write <= 16) {
+        // few written spans (one output, or a few slots): test each against every span
+        for (size_t i = 0; i < spans.size(); ++i) {
+            const Span& w = spans[i];
+            if (!w.write || w.lo == w.hi) continue;
+            for (size_t j = 0; j < spans.size(); ++j) {
+                const Span& o = spans[j];
+                if (j != i && o.lo != o.hi && o.lo < w.hi && w.lo < o.hi) return true;
+            }
+        }
+        return false;
+    }
     std::sort(spans.begin(), spans.end(), [](const Span& a, const Span& b) { return a.lo < b.lo; });
     uintptr_t max_hi = 0, max_hi_write = 0;
     for (const Span& s : spans) {
@@ -255,6 +269,7 @@ extern "C" tide_status_t tide_ag_place(const tide_plan_t* cplan, const void* ag_
     if ((st = check_enums(engine, max_ctas)) != TIDE_OK) return st;
     const int64_t W = p->world, P = p->n_params;
     std::vector<Span> spans;
+    spans.reserve((size_t)p->world * (p->n_params + 1) + p->n_params + 2);
     if ((st = check_buf(ag_buf, ag_numel, W * p->shard_numel, 2)) != TIDE_OK) return st;
     add_span(spans, ag_buf, 2 * W * p->shard_numel, false);
     if (P > 0 && (param_storage == nullptr || param_numel == nullptr)) return TIDE_ERR_INVALID_ARG;
@@ -294,6 +309,7 @@ extern "C" tide_status_t tide_ag_gather_place(const tide_plan_t* cplan, const vo
     if ((st = check_enums(engine, max_ctas)) != TIDE_OK) return st;
     const int64_t W = p->world, P = p->n_params, Ns = p->shard_numel;
     std::vector<Span> spans;
+    spans.reserve((size_t)p->world * (p->n_params + 1) + p->n_params + 2);
     if (W > 0 && shards == nullptr) return TIDE_ERR_INVALID_ARG;
     for (int64_t r = 0; r < W; ++r) {
         if ((st = check_buf(shards[r], shard_numel, Ns, 2)) != TIDE_OK) return st;
@@ -339,6 +355,7 @@ extern "C" tide_status_t tide_rs_reduce(const tide_plan_t* cplan, const void* co
     // a one-rank plan writes only its own shard
     const int64_t W = p->world, P = p->n_params, n_out = (p->rank >= 0 ? 1 : W) * p->shard_numel;
     std::vector<Span> spans;
+    spans.reserve((size_t)p->world * (p->n_params + 1) + p->n_params + 2);
     if ((st = check_grads(p, grads, grad_numel, spans)) != TIDE_OK) return st;
     if ((st = check_buf(out, out_numel, n_out, 4)) != TIDE_OK) return st;
     add_span(spans, out, 4 * n_out, true);
@@ -368,6 +385,7 @@ extern "C" tide_status_t tide_rs_stage(const tide_plan_t* cplan, const void* con
     if ((st = all_ranks(p)) != TIDE_OK) return st;
     if ((st = check_enums(engine, max_ctas)) != TIDE_OK) return st;
     std::vector<Span> spans;
+    spans.reserve((size_t)p->world * (p->n_params + 1) + p->n_params + 2);
     if ((st = check_grads(p, grads, grad_numel, spans)) != TIDE_OK) return st;
     if ((st = check_slots(p, slots, slot_numel, spans)) != TIDE_OK) return st;
     if (overlaps(spans)) return TIDE_ERR_INVALID_ARG;
@@ -388,6 +406,7 @@ extern "C" tide_status_t tide_rs_reduce_slots(const tide_plan_t* cplan, const vo
     if ((st = check_reduce_modes(scale_mode, order)) != TIDE_OK) return st;
     const int64_t n_out = (int64_t)p->world * p->shard_numel;
     std::vector<Span> spans;
+    spans.reserve((size_t)p->world * (p->n_params + 1) + p->n_params + 2);
     if ((st = check_slots(p, const_cast<void* const*>(slots), slot_numel, spans)) != TIDE_OK) return st;
     // slots are only read in this phase: re-tag them as read spans
     for (Span& sp : spans) sp.write = false;
@@ -415,6 +434,7 @@ extern "C" tide_status_t tide_rs_reduce_pipelined(const tide_plan_t* cplan, cons
     if (n_segments < 1 || n_segments > p->world) return TIDE_ERR_INVALID_ARG;
     const int64_t W = p->world, n_out = W * p->shard_numel;
     std::vector<Span> spans;
+    spans.reserve((size_t)p->world * (p->n_params + 1) + p->n_params + 2);
     if ((st = check_grads(p, grads, grad_numel, spans)) != TIDE_OK) return st;
     if ((st = check_buf(out, out_numel, n_out, 4)) != TIDE_OK) return st;
     add_span(spans, out, 4 * n_out, true);

@@ -368,3 +368,39 @@ def test_gather_place_validation(tiny_plan, args):
     assert gather(params=[shards[1]] + args["params"][1:]) == T.TIDE_ERR_INVALID_ARG
     # shards may overlap one another (they are only read)
     assert gather(sh=[shards[0]] * W) == T.TIDE_ERR_DEVICE
+
+
+@pytest.mark.parametrize("W", [4, 32])   # 5 written spans (direct check), 33 (sorted check)
+def test_overlap_verdict_matches_brute_force(W):
+    """Gradients (read), the output and the slots (written) at random addresses: the call is
+    refused exactly when a written buffer overlaps any other buffer."""
+    g = configs.Group("ov", W, ((3 * W, 4), (2 * W + 1,), (5, 8)))
+    L = oracle.layout(W, g.shapes)
+    P = g.n_params
+    plan = T.Plan(g.shapes, W, host_only=True)
+    sizes = ([2 * g.numel(i) for _ in range(W) for i in range(P)] + [4 * W * L.Ns] +
+             [2 * W * L.Ns] * W)
+    writes = [False] * (W * P) + [True] * (1 + W)
+    window = 4 * sum(sizes)
+    rng = np.random.default_rng(W)
+    seen = set()
+    for trial in range(300):
+        if trial % 2:
+            lo = [BASE + 16 * int(rng.integers(0, window // 16)) for _ in sizes]
+        else:
+            # packed in a random order with random gaps (no overlap), then sometimes one
+            # buffer moved to start inside another
+            lo, at = [0] * len(sizes), BASE
+            for k in rng.permutation(len(sizes)):
+                lo[k] = at
+                at += (sizes[k] + 15) // 16 * 16 + 16 * int(rng.integers(0, 4))
+            if rng.random() < 0.5:
+                a, b = rng.choice(len(sizes), size=2, replace=False)
+                lo[a] = lo[b] + 16 * int(rng.integers(0, max(1, sizes[b] // 16)))
+        bad = any((writes[a] or writes[b]) and lo[a] < lo[b] + sizes[b] and lo[b] < lo[a] + sizes[a]
+                  for a in range(len(sizes)) for b in range(a + 1, len(sizes)))
+        st = T.tide_rs_reduce(plan.handle, lo[: W * P], [g.numel(i) for _ in range(W) for i in range(P)],
+                              lo[W * P], W * L.Ns, 1, 0, lo[W * P + 1:], W * L.Ns, 0, 0, 0)
+        assert st == (T.TIDE_ERR_INVALID_ARG if bad else T.TIDE_ERR_DEVICE)
+        seen.add(bad)
+    assert seen == {True, False}
