@@ -1,0 +1,57 @@
+"""The layout readings pinned against FSDP2 itself (CPU, gloo).
+
+A real FSDP2 job (fully_shard, bf16 parameters, fp32 reduction) runs over W processes.
+Its collectives are wrapped to capture the buffers FSDP2 builds. The checks:
+- FSDP2's all-gather buffer, put through the oracle's copy-out, gives back the full
+  parameters. Its length is the plan's W*Ns.
+- FSDP2's packed fp32 gradient buffer of each rank equals the oracle's pack.
+- Its reduce-scatter output equals the oracle's reduce-scatter. The inputs are exactly
+  summable, so the collective's order of adds does not matter.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+import oracle
+from fsdp2_layout_aware_b200 import tide as T
+
+from _dist_helpers import free_port
+from _fsdp2_workers import fsdp2_worker, integer_grads, param_values
+
+pytest.importorskip("torch.distributed.fsdp._fully_shard._fsdp_collectives")
+
+SHAPES = ((37, 16), (1000,), (7, 3), (5, 130), (64, 8))
+
+
+def bf16_bits(a):
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+    assert np.all((u & 0xFFFF) == 0)
+    return (u >> 16).astype(np.uint16)
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_fsdp2_buffers_match_the_layout_and_the_oracle(world, tmp_path):
+    mp.spawn(fsdp2_worker, args=(world, free_port(), SHAPES, str(tmp_path)), nprocs=world, join=True)
+    L = oracle.layout(world, SHAPES)
+    plan = T.Plan(SHAPES, world, host_only=True)
+    assert plan.shard_numel == L.Ns
+    full = param_values(SHAPES)
+    grads = [[bf16_bits(g).reshape(-1) for g in integer_grads(SHAPES, k)] for k in range(world)]
+    rs = oracle.rs_reduce(world, SHAPES, grads, 0).reshape(world, L.Ns)
+    for r in range(world):
+        ag = np.load(tmp_path / f"ag_{r}.npy")
+        assert ag.size == world * L.Ns                       # FSDP2's buffer is [W][Ns]
+        placed = oracle.ag_copyout(world, SHAPES, ag)
+        for i, p in enumerate(full):
+            n = p.size
+            assert np.array_equal(placed[i][:n], bf16_bits(p).reshape(-1)), (r, i)
+        packed = np.load(tmp_path / f"rs_in_{r}.npy")
+        assert np.array_equal(packed.view(np.uint32),
+                              oracle.pack_f32(world, SHAPES, grads[r]).view(np.uint32)), r
+        out = np.load(tmp_path / f"rs_out_{r}.npy")
+        assert np.array_equal(out.view(np.uint32), rs[r].view(np.uint32)), r
+    # TIDE's tiles cover exactly those shards
+    for t in plan.tiles():
+        assert 0 <= t.dst_off - t.rank * L.Ns < L.Ns
