@@ -28,7 +28,7 @@
  *     numel arrays are host arrays that are only read during the call.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and never synchronize the device, except tide_plan_group,
- *     tide_plan_destroy and tide_plan_check where stated.
+ *     tide_plan_destroy, tide_plan_check and tide_plan_errors where stated.
  *   - All arguments are validated on the host before anything is enqueued; on
  *     any error status nothing has been enqueued.
  *   - A plan keeps small device tables (tile list, pointer tables, an error
@@ -39,8 +39,8 @@
  *   - bf16 buffers must be 2-byte aligned and fp32 buffers 4-byte aligned; any
  *     such alignment is accepted (16-byte alignment gives the fast path).
  *   - No call allocates device memory except tide_plan_group.
- *   - The plan-based calls (tide_ag_place, tide_rs_reduce, tide_rs_stage,
- *     tide_rs_reduce_slots, tide_rs_reduce_pipelined) can be captured into a
+ *   - The plan-based calls (tide_ag_place, tide_ag_gather_place, tide_rs_reduce,
+ *     tide_rs_stage, tide_rs_reduce_slots, tide_rs_reduce_pipelined) can be captured into a
  *     CUDA graph once the same buffers have been used in an uncaptured call on
  *     the same plan (that call uploads the pointer tables and creates the
  *     pipeline's events and the copy-engine streams; a capture that needs an
@@ -217,8 +217,11 @@ TIDE_API tide_status_t tide_ag_gather_place(const tide_plan_t* plan, const void*
  * for r*c_i + e < d0_i*inner_i, and +0.0 at pad positions.  scale_mode
  * TIDE_SCALE_INV_WORLD multiplies once by fl32(1/W) after the sum; NONE skips it.
  * order TIDE_ORDER_RANK adds in rank order 0..W-1 (bit-exact against the stock
- * pack-then-reduce result); TIDE_ORDER_TREE adds pairwise (within
- * |err| <= 1e-6 * sum|terms| of the exact sum).
+ * pack-then-reduce result); TIDE_ORDER_TREE adds adjacent ranks pairwise, level
+ * by level, an odd last one carried to the next level (every kernel gives the
+ * same bits; within |err| <= 1e-6 * sum|terms| of the exact sum for W <= 64).
+ * With a one-rank plan (tide_plan_group_rank) out is that rank's shard only:
+ * fp32 [Ns], out_numel >= Ns.
  * slots == NULL: one kernel launch.  slots != NULL: Slot-Reuse, the two phases
  * of tide_rs_stage (with `engine`) and tide_rs_reduce_slots run back to back;
  * slots is a host array of W device pointers to bf16 [W][Ns] buffers
