@@ -39,8 +39,8 @@
  *   - bf16 buffers must be 2-byte aligned and fp32 buffers 4-byte aligned; any
  *     such alignment is accepted (16-byte alignment gives the fast path).
  *   - No call allocates device memory except tide_plan_group.
- *   - The plan-based calls (tide_ag_place, tide_ag_gather_place, tide_rs_reduce,
- *     tide_rs_stage, tide_rs_reduce_slots, tide_rs_reduce_pipelined) can be captured into a
+ *   - The plan-based calls (tide_ag_place, tide_rs_reduce, tide_rs_stage,
+ *     tide_rs_reduce_slots, tide_rs_reduce_pipelined; tested) can be captured into a
  *     CUDA graph once the same buffers have been used in an uncaptured call on
  *     the same plan (that call uploads the pointer tables and creates the
  *     pipeline's events and the copy-engine streams; a capture that needs an
