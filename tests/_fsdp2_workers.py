@@ -22,7 +22,7 @@ def param_values(shapes):
             .reshape(s) for s in shapes]
 
 
-def fsdp2_worker(rank, world, port, shapes, out_dir):
+def fsdp2_worker(rank, world, port, shapes, out_dir, reduce_fp32=True):
     import torch
     import torch.distributed as dist
     from torch.distributed.device_mesh import init_device_mesh
@@ -62,8 +62,9 @@ def fsdp2_worker(rank, world, port, shapes, out_dir):
         model = Group()
         mesh = init_device_mesh("cpu", (world,))
         fully_shard(model, mesh=mesh,
-                    mp_policy=MixedPrecisionPolicy(param_dtype=torch.bfloat16,
-                                                   reduce_dtype=torch.float32))
+                    mp_policy=MixedPrecisionPolicy(
+                        param_dtype=torch.bfloat16,
+                        reduce_dtype=torch.float32 if reduce_fp32 else torch.bfloat16))
         model.set_custom_all_gather(CaptureAllGather())
         model.set_custom_reduce_scatter(CaptureReduceScatter())
         model.set_gradient_divide_factor(1.0)
@@ -72,7 +73,10 @@ def fsdp2_worker(rank, world, port, shapes, out_dir):
         model(gs).backward()
         np.save(os.path.join(out_dir, f"ag_{rank}.npy"),
                 captured["ag"].view(torch.int16).numpy().view(np.uint16))
-        np.save(os.path.join(out_dir, f"rs_in_{rank}.npy"), captured["rs_in"].float().numpy())
+        rs_in = captured["rs_in"]
+        if rs_in.dtype == torch.bfloat16:
+            np.save(os.path.join(out_dir, f"rs_in_bf16_{rank}.npy"), rs_in.view(torch.int16).numpy().view(np.uint16))
+        np.save(os.path.join(out_dir, f"rs_in_{rank}.npy"), rs_in.float().numpy())
         np.save(os.path.join(out_dir, f"rs_out_{rank}.npy"), captured["rs_out"].float().numpy())
     finally:
         dist.destroy_process_group()

@@ -55,3 +55,17 @@ def test_fsdp2_buffers_match_the_layout_and_the_oracle(world, tmp_path):
     # TIDE's tiles cover exactly those shards
     for t in plan.tiles():
         assert 0 <= t.dst_off - t.rank * L.Ns < L.Ns
+
+
+def test_fsdp2_bf16_pack_is_the_slot_reuse_staging(tmp_path):
+    """With a bf16 reduction FSDP2 packs each rank's gradients, still bf16, into the
+    rank-major layout: that is Slot-Reuse staging (the oracle's slot_stage), pads as +0."""
+    world = 3
+    mp.spawn(fsdp2_worker, args=(world, free_port(), SHAPES, str(tmp_path), False), nprocs=world,
+             join=True)
+    L = oracle.layout(world, SHAPES)
+    for r in range(world):
+        grads = [bf16_bits(g).reshape(-1) for g in integer_grads(SHAPES, r)]
+        slot = np.zeros(world * L.Ns, dtype=np.uint16)           # FSDP2 pads with +0
+        oracle.slot_stage(world, SHAPES, grads, slot)
+        assert np.array_equal(np.load(tmp_path / f"rs_in_bf16_{r}.npy"), slot), r
