@@ -22,7 +22,7 @@ def param_values(shapes):
             .reshape(s) for s in shapes]
 
 
-def fsdp2_worker(rank, world, port, shapes, out_dir, reduce_fp32=True):
+def fsdp2_worker(rank, world, port, shapes, out_dir, reduce_fp32=True, average=False):
     import torch
     import torch.distributed as dist
     from torch.distributed.device_mesh import init_device_mesh
@@ -67,8 +67,9 @@ def fsdp2_worker(rank, world, port, shapes, out_dir, reduce_fp32=True):
                         reduce_dtype=torch.float32 if reduce_fp32 else torch.bfloat16))
         model.set_custom_all_gather(CaptureAllGather())
         model.set_custom_reduce_scatter(CaptureReduceScatter())
-        model.set_gradient_divide_factor(1.0)
-        model.set_force_sum_reduction_for_comms(True)
+        if not average:
+            model.set_gradient_divide_factor(1.0)   # a plain sum
+        model.set_force_sum_reduction_for_comms(True)   # gloo: SUM, then FSDP2's own division
         gs = [torch.from_numpy(g).to(torch.bfloat16) for g in integer_grads(shapes, rank)]
         model(gs).backward()
         np.save(os.path.join(out_dir, f"ag_{rank}.npy"),
@@ -78,5 +79,7 @@ def fsdp2_worker(rank, world, port, shapes, out_dir, reduce_fp32=True):
             np.save(os.path.join(out_dir, f"rs_in_bf16_{rank}.npy"), rs_in.view(torch.int16).numpy().view(np.uint16))
         np.save(os.path.join(out_dir, f"rs_in_{rank}.npy"), rs_in.float().numpy())
         np.save(os.path.join(out_dir, f"rs_out_{rank}.npy"), captured["rs_out"].float().numpy())
+        for i, p in enumerate(model.ps):          # the reduced gradient FSDP2 hands to the optimizer
+            np.save(os.path.join(out_dir, f"grad_{rank}_{i}.npy"), p.grad.to_local().float().numpy())
     finally:
         dist.destroy_process_group()

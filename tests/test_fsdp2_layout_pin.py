@@ -69,3 +69,40 @@ def test_fsdp2_bf16_pack_is_the_slot_reuse_staging(tmp_path):
         slot = np.zeros(world * L.Ns, dtype=np.uint16)           # FSDP2 pads with +0
         oracle.slot_stage(world, SHAPES, grads, slot)
         assert np.array_equal(np.load(tmp_path / f"rs_in_bf16_{r}.npy"), slot), r
+
+
+def _averaged(world, tmp_path):
+    mp.spawn(fsdp2_worker, args=(world, free_port(), SHAPES, str(tmp_path), True, True),
+             nprocs=world, join=True)
+    L = oracle.layout(world, SHAPES)
+    grads = [[bf16_bits(g).reshape(-1) for g in integer_grads(SHAPES, k)] for k in range(world)]
+    got, total = [], oracle.rs_reduce(world, SHAPES, grads, 0)
+    for r in range(world):
+        for i in range(len(SHAPES)):
+            c, n = L.c[i], int(np.prod(SHAPES[i]))
+            valid = max(0, min(c, n - r * c))
+            local = np.load(tmp_path / f"grad_{r}_{i}.npy").reshape(-1)
+            assert local.size >= valid
+            start = r * L.Ns + L.off[i]
+            got.append((local[:valid], start, valid))
+    return got, total
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_fsdp2_average_is_the_scaled_reduction(world, tmp_path):
+    """FSDP2's averaged gradient shard (sum, then its division by W) equals the oracle's
+    sum times fl32(1/W) bit for bit: for power-of-two W the two are the same operation."""
+    got, _ = _averaged(world, tmp_path)
+    grads = [[bf16_bits(g).reshape(-1) for g in integer_grads(SHAPES, k)] for k in range(world)]
+    ref = oracle.rs_reduce(world, SHAPES, grads, 1)
+    for local, start, valid in got:
+        assert np.array_equal(local.view(np.uint32), ref[start: start + valid].view(np.uint32))
+
+
+def test_fsdp2_average_divides_for_other_world_sizes(tmp_path):
+    """For W = 3 FSDP2 divides the sum by 3 (correctly rounded); the oracle's reading
+    multiplies by fl32(1/3), which may differ in the last bit."""
+    got, total = _averaged(3, tmp_path)
+    for local, start, valid in got:
+        want = (total[start: start + valid].astype(np.float32) / np.float32(3)).astype(np.float32)
+        assert np.array_equal(local.view(np.uint32), want.view(np.uint32))
