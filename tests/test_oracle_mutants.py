@@ -30,6 +30,7 @@ MUTANTS = {
     "tree_pairs_mirrored": ("for (int64_t j = 0; j + 1 < n; j += 2) v[m++] = v[j] + v[j + 1];",
                             "for (int64_t j = 0; j + 1 < n; j += 2) v[m++] = v[j] + v[n - 1 - j];"),
     "tree_odd_one_dropped": ("if (n % 2 == 1) v[m++] = v[n - 1];", "if (n % 2 == 1) m += 0;"),
+    "exact_magnitude_keeps_sign": ("mag += v < 0 ? -v : v;", "mag += v;"),
     "ranks_added_in_reverse": ("pack_f32(W, P, d0, inner, S, off, Ns, grads + k * P, packed);",
                                "pack_f32(W, P, d0, inner, S, off, Ns, grads + (W - k) * P, packed);"),
 }

@@ -446,3 +446,20 @@ def test_tree_closed_forms_and_bound(W):
     E, A = oracle.exact_f64(W, grp.shapes, grads)
     tree = oracle.rs_reduce_tree(W, grp.shapes, grads, 0).astype(np.float64)
     assert np.all(np.abs(tree - E) <= max(1, math.ceil(math.log2(W))) * E24 * A)
+
+
+@pytest.mark.parametrize("W", [2, 3, 8, 64])
+def test_exact_sums_against_integer_brute_force(W):
+    """The exact fp64 sums behind every tolerance check: small integers times 2^-10, summed
+    in int64 and laid out with torch.chunk, give E and A exactly; pads give 0."""
+    grp = configs.Group("exact", W, ((65, 9), (301,), (3, 3)))
+    rng = np.random.default_rng(100 + W)
+    ints = [[rng.integers(-8, 9, size=grp.numel(i)) for i in range(grp.n_params)] for _ in range(W)]
+    grads = [[bf16_bits(m.astype(np.float32) * np.float32(2.0 ** -10)) for m in rk] for rk in ints]
+    E, A = oracle.exact_f64(W, grp.shapes, grads)
+    tot = [sum(ints[k][i] for k in range(W)).astype(np.int64) for i in range(grp.n_params)]
+    mag = [sum(np.abs(ints[k][i]) for k in range(W)).astype(np.int64) for i in range(grp.n_params)]
+    e_ref = torch_rank_major(W, grp.shapes, [torch.from_numpy(t) for t in tot], 0).numpy()
+    a_ref = torch_rank_major(W, grp.shapes, [torch.from_numpy(t) for t in mag], 0).numpy()
+    assert np.array_equal(E, e_ref.astype(np.float64) * 2.0 ** -10)
+    assert np.array_equal(A, a_ref.astype(np.float64) * 2.0 ** -10)
