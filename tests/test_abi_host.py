@@ -371,7 +371,7 @@ def test_gather_place_validation(tiny_plan, args):
 
 
 @pytest.mark.parametrize("W", [4, 32])   # 5 written spans (direct check), 33 (sorted check)
-def test_overlap_verdict_matches_brute_force(W):
+def test_overlap_decision_matches_brute_force(W):
     """Gradients (read), the output and the slots (written) at random addresses: the call is
     refused exactly when a written buffer overlaps any other buffer."""
     g = configs.Group("ov", W, ((3 * W, 4), (2 * W + 1,), (5, 8)))
