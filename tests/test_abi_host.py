@@ -300,8 +300,10 @@ def test_tensor_table_marshals_once_in_rank_major_order():
 # --------------------------------------------------------------------------- one-rank plans, gathering
 
 
-@pytest.mark.parametrize("group", [configs.tiny(), degenerate(), mini_wan(), configs.qwen3moe(4)],
-                         ids=lambda g: g.name)
+@pytest.mark.parametrize("group", [configs.tiny(), degenerate(), mini_wan(), configs.qwen3moe(4),
+                                   mini_sweep(64),
+                                   configs.Group("w256", 256, ((300, 3), (255,), (1000, 2)))],
+                         ids=lambda g: f"{g.name}_w{g.world}")
 def test_rank_plan_tiles_are_that_ranks_tiles_inside_its_shard(group):
     W = group.world
     full = host_plan(group)
