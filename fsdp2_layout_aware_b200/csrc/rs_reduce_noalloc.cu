@@ -18,7 +18,13 @@
 //     groups are rejected with TIDE_ERR_SIZE before anything happens.
 //   - The first call on each device looks up that device's address of the
 //     array (cudaGetSymbolAddress, with the device current) and caches it; make
-//     that first call before any stream capture.
+//     that first call before any stream capture.  The cached address lives as
+//     long as the process; after cudaDeviceReset on a device (which unloads
+//     this module there) the entry point must not be called on that device.
+//   - A call on a stream that is being captured is refused with
+//     TIDE_ERR_INVALID_ARG before anything is enqueued: the tables are copied
+//     from one host array that every later call overwrites, so a recorded copy
+//     would replay another call's tables.
 //   - Every call rewrites every byte of the array that its kernel reads (the
 //     previous call's tables are left beyond that and never read), so nothing
 //     depends on earlier contents.  Calls that may overlap on the GPU
@@ -205,6 +211,14 @@ extern "C" tide_status_t tide_rs_reduce_noalloc(const tide_param_t* params, int3
         }
     if (n_tiles == 0) return TIDE_OK;
 
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &capture) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return TIDE_ERR_CUDA;
+    }
+    if (capture != cudaStreamCaptureStatusNone) return TIDE_ERR_INVALID_ARG;
+
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return TIDE_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return TIDE_ERR_DEVICE;
@@ -237,7 +251,6 @@ extern "C" tide_status_t tide_rs_reduce_noalloc(const tide_param_t* params, int3
     const void** tab = reinterpret_cast<const void**>(prm + P);
     for (int64_t j = 0; j < W * P; ++j) tab[j] = grads[j];
     const size_t bytes = (size_t)(P * (int64_t)sizeof(NaParam) + W * P * 8);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (cudaMemcpyAsync(scratch, g_host_stage, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
         (void)cudaGetLastError();
         return TIDE_ERR_CUDA;

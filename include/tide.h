@@ -311,10 +311,14 @@ TIDE_API tide_status_t tide_plan_errors(tide_plan_t* plan, void* stream, int32_t
  * holds until the process exits; a larger group is rejected with
  * TIDE_ERR_SIZE before anything is enqueued.  The first call on each device
  * looks up that device's address of the array; make that first call before
- * any stream capture.  Every call rewrites the tables its kernel reads, so no
- * state carries over, but all calls share the one array: calls that may
- * overlap on the GPU (on streams the caller does not order) race and must not
- * be issued.
+ * any stream capture.  That address is kept for the life of the process:
+ * after cudaDeviceReset on a device, do not call this entry point on that
+ * device again.  The tables are copied in from one host array that the next
+ * call reuses, so a call on a stream that is being captured is refused with
+ * TIDE_ERR_INVALID_ARG (nothing enqueued).  Every call rewrites the tables its
+ * kernel reads, so no state carries over, but all calls share the one array:
+ * calls that may overlap on the GPU (on streams the caller does not order)
+ * race and must not be issued.
  */
 TIDE_API tide_status_t tide_rs_reduce_noalloc(const tide_param_t* params, int32_t n_params,
                                               int32_t world, const void* const* grads,
