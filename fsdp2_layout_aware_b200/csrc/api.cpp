@@ -118,9 +118,11 @@ tide_status_t check_slots(const tide_plan* p, void* const* slots, int64_t slot_n
     return TIDE_OK;
 }
 
-tide_status_t check_enums(int32_t engine, int32_t max_ctas) {
+tide_status_t check_enums(const tide_plan* p, int32_t engine, int32_t max_ctas) {
     if (engine != TIDE_ENGINE_SM && engine != TIDE_ENGINE_CE) return TIDE_ERR_INVALID_ARG;
     if (max_ctas < 0) return TIDE_ERR_INVALID_ARG;
+    // short-lived CTAs: one per unit of work, so no cap on the grid
+    if ((p->flags & TIDE_PLAN_SHORT_CTAS) && max_ctas != 0) return TIDE_ERR_INVALID_ARG;
     return TIDE_OK;
 }
 
@@ -179,11 +181,11 @@ bool use_v32(const tide_plan* p, const PtrTable& src, const float* out, int kern
 cudaError_t launch_reduce(tide_plan* p, PtrTable& tab, bool slot, int64_t bound, float* out,
                           int64_t out_numel, int32_t scale_mode, int32_t order, int32_t max_ctas,
                           cudaStream_t s, int64_t t0 = 0, int64_t t1 = -1) {
-    const int k_tma = slot ? K_SLOT_RS_TMA : K_RS_TMA;
-    const int k_v32 = slot ? K_SLOT_RS_V32 : K_RS_V32;
-    const bool tma = use_tma(p, tab, out, k_tma);
-    const bool v32 = !tma && order == TIDE_ORDER_RANK && use_v32(p, tab, out, k_v32);
     const bool tree = order == TIDE_ORDER_TREE;
+    const int k_tma = slot ? K_SLOT_RS_TMA : K_RS_TMA;
+    const int k_v32 = tree ? (slot ? K_SLOT_RS_TREE_V32 : K_RS_TREE_V32) : (slot ? K_SLOT_RS_V32 : K_RS_V32);
+    const bool tma = use_tma(p, tab, out, k_tma);
+    const bool v32 = !tma && use_v32(p, tab, out, k_v32);
     const int kernel = tma ? k_tma : v32 ? k_v32 : tree ? (slot ? K_SLOT_RS_TREE : K_RS_TREE)
                                                         : (slot ? K_SLOT_RS : K_RS);
     if (t1 < 0) t1 = (int64_t)p->tiles.size();
@@ -266,7 +268,7 @@ extern "C" tide_status_t tide_ag_place(const tide_plan_t* cplan, const void* ag_
     tide_status_t st = check_plan(p);
     if (st != TIDE_OK) return st;
     if ((st = all_ranks(p)) != TIDE_OK) return st;
-    if ((st = check_enums(engine, max_ctas)) != TIDE_OK) return st;
+    if ((st = check_enums(p, engine, max_ctas)) != TIDE_OK) return st;
     const int64_t W = p->world, P = p->n_params;
     std::vector<Span> spans;
     spans.reserve((size_t)p->world * (p->n_params + 1) + p->n_params + 2);
@@ -306,7 +308,7 @@ extern "C" tide_status_t tide_ag_gather_place(const tide_plan_t* cplan, const vo
     tide_status_t st = check_plan(p);
     if (st != TIDE_OK) return st;
     if ((st = all_ranks(p)) != TIDE_OK) return st;
-    if ((st = check_enums(engine, max_ctas)) != TIDE_OK) return st;
+    if ((st = check_enums(p, engine, max_ctas)) != TIDE_OK) return st;
     const int64_t W = p->world, P = p->n_params, Ns = p->shard_numel;
     std::vector<Span> spans;
     spans.reserve((size_t)p->world * (p->n_params + 1) + p->n_params + 2);
@@ -349,7 +351,7 @@ extern "C" tide_status_t tide_rs_reduce(const tide_plan_t* cplan, const void* co
     tide_plan* p = const_cast<tide_plan*>(cplan);
     tide_status_t st = check_plan(p);
     if (st != TIDE_OK) return st;
-    if ((st = check_enums(engine, max_ctas)) != TIDE_OK) return st;
+    if ((st = check_enums(p, engine, max_ctas)) != TIDE_OK) return st;
     if ((st = check_reduce_modes(scale_mode, order)) != TIDE_OK) return st;
     if (slots != nullptr && (st = all_ranks(p)) != TIDE_OK) return st;
     // a one-rank plan writes only its own shard
@@ -383,7 +385,7 @@ extern "C" tide_status_t tide_rs_stage(const tide_plan_t* cplan, const void* con
     tide_status_t st = check_plan(p);
     if (st != TIDE_OK) return st;
     if ((st = all_ranks(p)) != TIDE_OK) return st;
-    if ((st = check_enums(engine, max_ctas)) != TIDE_OK) return st;
+    if ((st = check_enums(p, engine, max_ctas)) != TIDE_OK) return st;
     std::vector<Span> spans;
     spans.reserve((size_t)p->world * (p->n_params + 1) + p->n_params + 2);
     if ((st = check_grads(p, grads, grad_numel, spans)) != TIDE_OK) return st;
@@ -402,7 +404,7 @@ extern "C" tide_status_t tide_rs_reduce_slots(const tide_plan_t* cplan, const vo
     tide_status_t st = check_plan(p);
     if (st != TIDE_OK) return st;
     if ((st = all_ranks(p)) != TIDE_OK) return st;
-    if ((st = check_enums(TIDE_ENGINE_SM, max_ctas)) != TIDE_OK) return st;
+    if ((st = check_enums(p, TIDE_ENGINE_SM, max_ctas)) != TIDE_OK) return st;
     if ((st = check_reduce_modes(scale_mode, order)) != TIDE_OK) return st;
     const int64_t n_out = (int64_t)p->world * p->shard_numel;
     std::vector<Span> spans;
@@ -429,7 +431,7 @@ extern "C" tide_status_t tide_rs_reduce_pipelined(const tide_plan_t* cplan, cons
     tide_status_t st = check_plan(p);
     if (st != TIDE_OK) return st;
     if ((st = all_ranks(p)) != TIDE_OK) return st;
-    if ((st = check_enums(TIDE_ENGINE_SM, max_ctas)) != TIDE_OK) return st;
+    if ((st = check_enums(p, TIDE_ENGINE_SM, max_ctas)) != TIDE_OK) return st;
     if ((st = check_reduce_modes(scale_mode, order)) != TIDE_OK) return st;
     if (n_segments < 1 || n_segments > p->world) return TIDE_ERR_INVALID_ARG;
     const int64_t W = p->world, n_out = W * p->shard_numel;

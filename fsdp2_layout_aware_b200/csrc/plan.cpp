@@ -10,6 +10,7 @@
 // round-robin over CTAs balances thousands of small MoE chunks and a few huge
 // dense ones alike.
 #include <algorithm>
+#include <cstdint>
 #include <cstring>
 #include <new>
 
@@ -89,9 +90,14 @@ tide_status_t upload(tide_plan* p) {
     if (st == TIDE_OK) {
         p->blocks_per_sm[K_RS] = tide::rs_blocks_per_sm(p->world, false, TIDE_ORDER_RANK, false);
         p->blocks_per_sm[K_SLOT_RS] = tide::rs_blocks_per_sm(p->world, true, TIDE_ORDER_RANK, false);
-        if (tide::rs_v32_applies(p->world)) {
+        if (tide::rs_v32_applies(p->world, TIDE_ORDER_RANK)) {
             p->blocks_per_sm[K_RS_V32] = tide::rs_blocks_per_sm(p->world, false, TIDE_ORDER_RANK, true);
             p->blocks_per_sm[K_SLOT_RS_V32] = tide::rs_blocks_per_sm(p->world, true, TIDE_ORDER_RANK, true);
+        }
+        if (tide::rs_v32_applies(p->world, TIDE_ORDER_TREE)) {
+            p->blocks_per_sm[K_RS_TREE_V32] = tide::rs_blocks_per_sm(p->world, false, TIDE_ORDER_TREE, true);
+            p->blocks_per_sm[K_SLOT_RS_TREE_V32] =
+                tide::rs_blocks_per_sm(p->world, true, TIDE_ORDER_TREE, true);
         }
         p->blocks_per_sm[K_RS_TREE] = tide::rs_blocks_per_sm(p->world, false, TIDE_ORDER_TREE, false);
         p->blocks_per_sm[K_SLOT_RS_TREE] = tide::rs_blocks_per_sm(p->world, true, TIDE_ORDER_TREE, false);
@@ -119,7 +125,8 @@ tide_status_t make_plan(const tide_param_t* params, int32_t n_params, int32_t wo
     if (n_params < 0 || (n_params > 0 && params == nullptr)) return TIDE_ERR_INVALID_ARG;
     if (world < 1 || world > TIDE_MAX_WORLD) return TIDE_ERR_INVALID_ARG;
     if (rank >= world) return TIDE_ERR_INVALID_ARG;
-    if ((flags & ~(uint32_t)(TIDE_PLAN_HOST_ONLY | TIDE_PLAN_TMA | TIDE_PLAN_TEST_TMA_TIMEOUT)) != 0)
+    if ((flags & ~(uint32_t)(TIDE_PLAN_HOST_ONLY | TIDE_PLAN_TMA | TIDE_PLAN_TEST_TMA_TIMEOUT |
+                             TIDE_PLAN_SHORT_CTAS)) != 0)
         return TIDE_ERR_INVALID_ARG;
     if (!(flags & TIDE_PLAN_HOST_ONLY) && device < 0) return TIDE_ERR_DEVICE;
 
@@ -276,6 +283,11 @@ extern "C" tide_status_t tide_launch_ctas(const tide_plan_t* plan, int32_t kerne
     if (kernel == K_STAGE) units *= plan->world;
     if (kernel >= K_RS_TMA && plan->blocks_per_sm[kernel] <= 0) {
         *ctas = 0;
+        return TIDE_OK;
+    }
+    if ((plan->flags & TIDE_PLAN_SHORT_CTAS) && kernel != K_RS_TMA && kernel != K_SLOT_RS_TMA) {
+        // one short-lived CTA per unit of work
+        *ctas = (int32_t)std::min<int64_t>(units, INT32_MAX);
         return TIDE_OK;
     }
     int64_t grid = (int64_t)plan->blocks_per_sm[kernel] * plan->sm_count;

@@ -146,4 +146,19 @@ __device__ __forceinline__ void tree_one_group(int W, Load load, float (&acc)[L]
     for (int l = 0; l < L; ++l) acc[l] = f[0][l];
 }
 
+// The tree order when G < W <= 2G: the two groups' trees, then one add that
+// joins them -- the adds reduce_ranks<G, L, true> makes for such a W (its
+// binary counter holds group 0's sum on level 0 and merges group 1's into it),
+// so the same bits, without the six-level merge stack.  The second group is
+// loaded only after the first is reduced, which keeps two groups' raw vectors
+// from being live at once.
+template <int G, int L, class Raw, class Load>
+__device__ __forceinline__ void tree_two_groups(int W, Load load, float (&acc)[L]) {
+    float first[L];
+    tree_one_group<G, L, Raw>(G, load, first);
+    tree_one_group<G, L, Raw>(W - G, [&](int k) { return load(G + k); }, acc);
+#pragma unroll
+    for (int l = 0; l < L; ++l) acc[l] = __fadd_rn(first[l], acc[l]);
+}
+
 }  // namespace tide

@@ -60,13 +60,19 @@ struct RsParams {
 // picks it only when every tile's sources and output are 32-byte aligned
 // (a tile that is not falls back to the element loop, never faults).
 // ONE: the tree order for W <= G (a single group), without the merge stack.
-// The single-group tree kernels are held to 3 CTAs per SM (80 registers, a
-// spill of 88 bytes per thread at G = 8): left free they take 128 registers
-// and 2 CTAs per SM, 4 % slower on B200 (70B W=8: 6.52 vs 6.28 TB/s; Qwen3:
-// 6.47 vs 6.19).  The others keep the compiler's choice (an explicit minimum
-// of 1 CTA raised the rank-order kernels' registers and cost bandwidth).
+// In tree order the 32-byte kernels serve W = G (ONE) and W = 2G (not ONE: two
+// groups joined by one add, tree_two_groups), with the tree fixed at compile
+// time and no merge stack: a runtime W kept up to 8 ranks' unpacked lanes live
+// and spilled (276 and 708 bytes) at the 128 registers of 2 CTAs per SM.
+// The 16-byte single-group tree kernels are held to 3 CTAs per SM (80
+// registers, a spill of 88 bytes per thread at G = 8): left free they take 128
+// registers and 2 CTAs per SM, 4 % slower on B200 (70B W=8: 6.52 vs 6.28 TB/s;
+// Qwen3: 6.47 vs 6.19).  The 32-byte tree kernels are held to 2 CTAs per SM,
+// the rank-order 32-byte kernel's occupancy.  The others keep the compiler's
+// choice (an explicit minimum of 1 CTA raised the rank-order kernels'
+// registers and cost bandwidth).
 template <int G, int U, bool SLOT, bool TREE, bool V32, bool ONE>
-__global__ void __launch_bounds__(kThreads, (TREE && ONE) ? 3 : 0)
+__global__ void __launch_bounds__(kThreads, (TREE && V32) ? 2 : (TREE && ONE) ? 3 : 0)
 rs_reduce_kernel(const RsParams a) {
     // s_src is double-buffered: tile i writes buffer i&1 while no thread can
     // still be reading the same buffer from tile i-2 (a barrier lies between).
@@ -117,7 +123,11 @@ rs_reduce_kernel(const RsParams a) {
             for (int v = tid; v < nv16; v += kThreads) {
                 float acc[16];
                 auto load = [&](int k) { return ld_stream_v8(srcs[k] + 16 * (int64_t)v); };
-                reduce_ranks<G, 16, false, V8>(W, load, acc);
+                // (the 32-byte tree kernels run only for W = G and W = 2G, so their
+                // trees are fixed at compile time)
+                if constexpr (!TREE) reduce_ranks<G, 16, false, V8>(W, load, acc);
+                else if constexpr (ONE) tree_one_group<G, 16, V8>(G, load, acc);
+                else tree_two_groups<G, 16, V8>(2 * G, load, acc);
                 if (a.do_scale) {
 #pragma unroll
                     for (int l = 0; l < 16; ++l) acc[l] = __fmul_rn(acc[l], a.scale);
@@ -161,6 +171,7 @@ rs_reduce_kernel(const RsParams a) {
             float acc[1];
             auto load = [&](int k) { return (uint32_t)ld_stream_u16(srcs[k] + e); };
             if constexpr (ONE) tree_one_group<G, 1, uint32_t>(W, load, acc);
+            else if constexpr (TREE && V32) tree_two_groups<G, 1, uint32_t>(2 * G, load, acc);
             else reduce_ranks<G, 1, TREE, uint32_t>(W, load, acc);
             if (a.do_scale) acc[0] = __fmul_rn(acc[0], a.scale);
             dst[e] = acc[0];
@@ -178,7 +189,10 @@ KernelFn pick(int world, bool v32) {
     if (world <= 2) return rs_reduce_kernel<2, 4, SLOT, TREE, false, TREE>;
     if (world <= 4) return rs_reduce_kernel<4, 2, SLOT, TREE, false, TREE>;
     if constexpr (TREE) {
-        // (the 32-byte variant is rank order only: the tree's 16-lane state does not fit)
+        // 32-byte tree kernels: exactly one group (W = 8) or two groups (W = 16) of 8
+        if (v32 && (world == 8 || world == 16))
+            return world == 8 ? rs_reduce_kernel<8, 1, SLOT, true, true, true>
+                              : rs_reduce_kernel<8, 1, SLOT, true, true, false>;
         if (world <= 8) return rs_reduce_kernel<8, 1, SLOT, true, false, true>;
         return rs_reduce_kernel<8, 1, SLOT, true, false, false>;
     } else {
@@ -195,7 +209,9 @@ KernelFn select(int world, bool slot, int order, bool v32) {
 
 }  // namespace
 
-bool rs_v32_applies(int world) { return world > 4 && world <= kV32MaxWorld; }
+bool rs_v32_applies(int world, int order) {
+    return order == TIDE_ORDER_TREE ? (world == 8 || world == 16) : (world > 4 && world <= kV32MaxWorld);
+}
 
 int rs_blocks_per_sm(int world, bool slot, int order, bool v32) {
     int n = 0;

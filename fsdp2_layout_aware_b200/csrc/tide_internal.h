@@ -12,7 +12,8 @@
 // Kernel ids (match tide_launch_ctas and tide_plan_last_launch).
 enum : int32_t {
     K_RS = 0, K_AG = 1, K_STAGE = 2, K_SLOT_RS = 3, K_RS_TMA = 4, K_SLOT_RS_TMA = 5,
-    K_RS_V32 = 6, K_SLOT_RS_V32 = 7, K_RS_TREE = 8, K_SLOT_RS_TREE = 9, K_AG_GATHER = 10, K_COUNT = 11
+    K_RS_V32 = 6, K_SLOT_RS_V32 = 7, K_RS_TREE = 8, K_SLOT_RS_TREE = 9, K_AG_GATHER = 10,
+    K_RS_TREE_V32 = 11, K_SLOT_RS_TREE_V32 = 12, K_COUNT = 13
 };
 
 // A device pointer table with a host mirror: re-uploaded only when it changes.
@@ -61,7 +62,7 @@ constexpr int kThreads = 256;
 
 // Occupancy (resident CTAs per SM) of each kernel at kThreads threads.
 int rs_blocks_per_sm(int world, bool slot, int order, bool v32);
-bool rs_v32_applies(int world);       // whether the 32-byte variant exists for this W
+bool rs_v32_applies(int world, int order);  // whether a 32-byte variant exists for this W and order
 int rs_tma_blocks_per_sm(int world);  // also opts the TMA kernels in to their shared memory
 int ag_blocks_per_sm(bool gather);
 int stage_blocks_per_sm();

@@ -34,15 +34,17 @@ TIDE_SCALE_INV_WORLD = 1
 TIDE_PLAN_HOST_ONLY = 1
 TIDE_PLAN_TMA = 2
 TIDE_PLAN_TEST_TMA_TIMEOUT = 4
+TIDE_PLAN_SHORT_CTAS = 8
 TIDE_KCHECK_TILE, TIDE_KCHECK_TIMEOUT = 1, 2
 TIDE_MAX_WORLD = 256
 TIDE_TILE_ELEMS = 8192
 TIDE_NOALLOC_SCRATCH_BYTES = 1 << 20
+TIDE_IPC_HANDLE_BYTES = 64
 
 (K_RS, K_AG, K_STAGE, K_SLOT_RS, K_RS_TMA, K_SLOT_RS_TMA, K_RS_V32, K_SLOT_RS_V32, K_RS_TREE,
- K_SLOT_RS_TREE, K_AG_GATHER) = range(11)
+ K_SLOT_RS_TREE, K_AG_GATHER, K_RS_TREE_V32, K_SLOT_RS_TREE_V32) = range(13)
 KERNEL_NAMES = ("rs", "ag", "stage", "slot_rs", "rs_tma", "slot_rs_tma", "rs_v32", "slot_rs_v32",
-                "rs_tree", "slot_rs_tree", "ag_gather")
+                "rs_tree", "slot_rs_tree", "ag_gather", "rs_tree_v32", "slot_rs_tree_v32")
 
 
 class tide_param_t(ctypes.Structure):
@@ -306,9 +308,11 @@ class Plan:
     """
 
     def __init__(self, shapes, world: int, device=None, host_only: bool = False,
-                 tma: bool = False, test_tma_timeout: bool = False, rank=None):
+                 tma: bool = False, test_tma_timeout: bool = False, rank=None,
+                 short_ctas: bool = False):
         """rank: None for the whole group (all W output shards), or one output rank r, whose
-        rs_reduce then writes only its own [Ns] shard."""
+        rs_reduce then writes only its own [Ns] shard.  short_ctas: one short-lived CTA per
+        unit of work instead of a persistent grid (TIDE_PLAN_SHORT_CTAS)."""
         self.shapes = [tuple(int(d) for d in s) for s in shapes]
         self.world = int(world)
         if host_only:
@@ -319,7 +323,8 @@ class Plan:
             dev = 0 if dev is None else dev
         params = [(s[0], _prod(s[1:])) for s in self.shapes]
         flags = ((TIDE_PLAN_HOST_ONLY if host_only else 0) | (TIDE_PLAN_TMA if tma else 0) |
-                 (TIDE_PLAN_TEST_TMA_TIMEOUT if test_tma_timeout else 0))
+                 (TIDE_PLAN_TEST_TMA_TIMEOUT if test_tma_timeout else 0) |
+                 (TIDE_PLAN_SHORT_CTAS if short_ctas else 0))
         self.rank = None if rank is None else int(rank)
         if self.rank is None:
             st, handle = tide_plan_group(params, self.world, dev, flags)

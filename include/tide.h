@@ -91,7 +91,17 @@ enum {
      * consumers' bounded wait gives up after about 1 s; the CTA stops, the
      * launch sets TIDE_KCHECK_TIMEOUT and its result is incomplete.  Nothing
      * faults or hangs.  Not for use outside tests. */
-    TIDE_PLAN_TEST_TMA_TIMEOUT = 4
+    TIDE_PLAN_TEST_TMA_TIMEOUT = 4,
+    /* flag: short-lived CTAs (kongchang.com, "TIDE's Design Approach": node-local
+     * accumulation by short-lived CTAs; weekinpapers.com Abstract).  The SM
+     * kernels (every kernel but the bulk-copy ones) launch one CTA per unit of
+     * work -- per tile, or per (tile, rank) for Slot-Reuse staging -- that does
+     * that unit and exits, instead of a persistent grid; max_ctas must then be
+     * 0 (TIDE_ERR_INVALID_ARG otherwise).  Each CTA holds its SM for a few
+     * microseconds, so when work of a higher-priority stream (say a GEMM) is
+     * waiting for SMs it gets them as CTAs finish, instead of waiting for the
+     * whole reduction.  Same results, same bits. */
+    TIDE_PLAN_SHORT_CTAS = 8
 };
 
 #define TIDE_MAX_WORLD 256
@@ -327,18 +337,21 @@ TIDE_API tide_status_t tide_rs_reduce_noalloc(const tide_param_t* params, int32_
                                               int32_t max_ctas, void* stream);
 
 /* The number of CTAs a kernel call with this max_ctas would launch (0 if that
- * kernel cannot run on this plan).  kernel: 0 = RS reduce (load/store kernel),
+ * kernel cannot run on this plan; the unit count under TIDE_PLAN_SHORT_CTAS).  kernel: 0 = RS reduce (load/store kernel),
  * 1 = AG place, 2 = Slot-Reuse stage, 3 = slot reduce (load/store), 4 = RS
  * reduce with bulk-copy staging, 5 = slot reduce with bulk-copy staging,
  * 6 = RS reduce with 32-byte loads, 7 = slot reduce with 32-byte loads,
  * 8 = RS reduce in tree order, 9 = slot reduce in tree order,
- * 10 = AG placement from per-rank shards (tide_ag_gather_place).
+ * 10 = AG placement from per-rank shards (tide_ag_gather_place),
+ * 11 = RS reduce in tree order with 32-byte loads, 12 = slot reduce in tree
+ * order with 32-byte loads.
  * The reductions use kernels 4/5 (one CTA per SM, TMA loads into shared memory)
  * when the plan was built with TIDE_PLAN_TMA, every tile starts on an
  * 8-element boundary and every source and the output are 16-byte aligned.
- * Otherwise, in rank order, they use kernels 6/7 when 5 <= W <= 16, every
- * tile starts on a 16-element boundary and every source and the output are
- * 32-byte aligned; else kernels 0/3.  In tree order they use kernels 8/9.
+ * Otherwise they use the 32-byte kernels (rank order 6/7 when 5 <= W <= 16,
+ * tree order 11/12 when W is 8 or 16) if every tile starts on a 16-element
+ * boundary and every source and the output are 32-byte aligned; else kernels
+ * 0/3 (rank order) or 8/9 (tree order).
  * Kernels of the same order give the same bits.  With the whole grid the
  * load/store kernels are the faster ones on B200; the bulk-copy kernels move
  * more bytes per CTA, which matters when max_ctas is small. */

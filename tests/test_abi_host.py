@@ -406,3 +406,21 @@ def test_overlap_decision_matches_brute_force(W):
         assert st == (T.TIDE_ERR_INVALID_ARG if bad else T.TIDE_ERR_DEVICE)
         seen.add(bad)
     assert seen == {True, False}
+
+
+def test_short_lived_ctas_take_no_cta_cap(args):
+    """Under TIDE_PLAN_SHORT_CTAS the grid is one CTA per unit of work: a CTA cap is refused
+    before the device check, and without one the call validates as usual."""
+    plan = T.Plan(configs.tiny().shapes, 4, host_only=True, short_ctas=True)
+    assert rs(plan, args, max_ctas=8) == T.TIDE_ERR_INVALID_ARG
+    assert ag(plan, args, max_ctas=8) == T.TIDE_ERR_INVALID_ARG
+    assert rs(plan, args) == T.TIDE_ERR_DEVICE
+    assert ag(plan, args, engine=1) == T.TIDE_ERR_DEVICE
+    h = plan.handle
+    assert T.tide_rs_stage(h, args["grads"], args["gnum"], args["slots"], args["n_slot"], 0, 4, 0) \
+        == T.TIDE_ERR_INVALID_ARG
+    assert T.tide_rs_reduce_slots(h, args["slots"], args["n_slot"], args["out"], args["n_out"], 1, 0,
+                                  4, 0) == T.TIDE_ERR_INVALID_ARG
+    # unknown flag bits are still refused
+    st, _ = T.tide_plan_group([(4, 4)], 4, 0, T.TIDE_PLAN_HOST_ONLY | 64)
+    assert st == T.TIDE_ERR_INVALID_ARG

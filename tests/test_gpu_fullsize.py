@@ -156,7 +156,7 @@ def bf16_to_f64(bits):
     return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
-@pytest.mark.parametrize("name", ["llama70b", "qwen3moe"])
+@pytest.mark.parametrize("name", ["llama70b", "qwen3moe", "wan14b"])
 def test_full_size_other_modes(name):
     """At full size: tree order bit-exact against the oracle's tree (and within 1e-6 *
     sum|terms| of the exact sum) at sampled positions; the bulk-copy kernel and the
@@ -179,7 +179,7 @@ def test_full_size_other_modes(name):
     plan.rs_reduce(grads, out, scale_mode=T.TIDE_SCALE_NONE, order=T.TIDE_ORDER_TREE)
     torch.cuda.synchronize()
     plan.check()
-    assert plan.last_launch()[0] == T.K_RS_TREE
+    assert plan.last_launch()[0] == T.K_RS_TREE_V32          # W = 8 or 16: the 32-byte tree kernel
     pos = sample_positions(group, L, 20000, rng)
     located, vals = rank_values(group, pos)
     terms = bf16_to_f64(vals)

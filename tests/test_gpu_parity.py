@@ -35,10 +35,14 @@ GROUPS = parity_groups()
 IDS = [f"{g.name}_w{g.world}" for g in GROUPS]
 
 
-def run_rs(group, grads_host, scale=1, order=0, max_ctas=0, slots=False, engine=0, tma=False):
-    plan = T.Plan(group.shapes, group.world, tma=tma)
+def run_rs(group, grads_host, scale=1, order=0, max_ctas=0, slots=False, engine=0, tma=False,
+           out_shift=0, short_ctas=False):
+    """out_shift > 0 places the output that many floats past a 512-byte boundary (4: 16-byte but
+    not 32-byte aligned, which rules out the 32-byte kernels)."""
+    plan = T.Plan(group.shapes, group.world, tma=tma, short_ctas=short_ctas)
     grads = grads_to_dev(group, grads_host)
-    out = torch.full((group.world * plan.shard_numel,), float("nan"), device="cuda")
+    n = group.world * plan.shard_numel
+    out = torch.full((n + out_shift,), float("nan"), device="cuda")[out_shift:]
     slot_bufs = None
     if slots:
         slot_bufs = [torch.full((group.world * plan.shard_numel,), -1, dtype=torch.int16,
@@ -111,8 +115,11 @@ def test_rs_tiny_all_seeds(seed):
 def test_rs_tree_order_within_tolerance(group):
     grads = synth.grads_host(group, seed=32)
     out, _, plan = run_rs(group, grads, scale=0, order=1)
-    if plan.n_tiles:   # the tree kernel, on the grid its own occupancy gives
-        assert plan.last_launch() == (T.K_RS_TREE, plan.launch_ctas(T.K_RS_TREE, 0))
+    if plan.n_tiles:   # a tree kernel, on the grid its own occupancy gives
+        k, ctas = plan.last_launch()
+        assert k in (T.K_RS_TREE, T.K_RS_TREE_V32) and ctas == plan.launch_ctas(k, 0)
+        if k == T.K_RS_TREE_V32:
+            assert group.world in (8, 16)
     assert np.array_equal(f32_bits(out),
                           oracle.rs_reduce_tree(group.world, group.shapes, grads, 0).view(np.uint32))
     E, A = oracle.exact_f64(group.world, group.shapes, grads)
@@ -128,16 +135,18 @@ def test_rs_tree_order_within_tolerance(group):
 @pytest.mark.parametrize("group", GROUPS, ids=IDS)
 def test_tree_order_kernels_agree_bitwise(group):
     """Every tree-order kernel adds in the same tree: pairwise by levels, an odd one carried.
-    Load/store (groups of 2, 4 or 8 ranks merged pairwise), bulk-copy, Slot-Reuse on SMs or
-    copy engines, and any CTA count give the same bits."""
+    Load/store (groups of 2, 4 or 8 ranks merged pairwise; 16- or 32-byte loads), bulk-copy,
+    Slot-Reuse on SMs or copy engines, and any CTA count give the same bits."""
     grads = synth.grads_host(group, seed=35)
     ref, _, _ = run_rs(group, grads, scale=1, order=1)
     ref = f32_bits(ref)
     assert np.array_equal(ref, oracle.rs_reduce_tree(group.world, group.shapes, grads, 1).view(np.uint32))
     for kw in (dict(max_ctas=3), dict(tma=True), dict(slots=True),
-               dict(slots=True, engine=T.TIDE_ENGINE_CE)):
-        out, _, _ = run_rs(group, grads, scale=1, order=1, **kw)
+               dict(slots=True, engine=T.TIDE_ENGINE_CE), dict(out_shift=4)):
+        out, _, plan = run_rs(group, grads, scale=1, order=1, **kw)
         assert np.array_equal(f32_bits(out), ref), kw
+        if kw == dict(out_shift=4) and plan.n_tiles:
+            assert plan.last_launch()[0] == T.K_RS_TREE     # the 16-byte tree kernel
 
 
 @pytest.mark.parametrize("slots", [False, True], ids=["plain", "slot"])
@@ -209,17 +218,24 @@ def test_rs_rank_order_pin_on_gpu():
     ([1.0, 2.0 ** -24, 2.0 ** -24, 2.0 ** -24], 1.0 + 2.0 ** -23),    # rank order gives 1
     ([1.0] + [2.0 ** -24] * 4, 1.0 + 2.0 ** -22),                       # a tie rounded to even
     ([1.0] + [2.0 ** -24] * 9, 1.0 + 2.0 ** -21),                       # W=10, two groups on the GPU
+    ([1.0] + [2.0 ** -24] * 7, 1.0 + 3 * 2.0 ** -23),                   # W=8, 32-byte kernel
+    ([1.0] + [2.0 ** -24] * 15, 1.0 + 7 * 2.0 ** -23),                  # W=16, 32-byte kernel
 ])
 def test_rs_tree_order_pin_on_gpu(vals, exp):
-    """Worked values of the tree order (pairs by levels, odd one carried) on every tree kernel."""
+    """Worked values of the tree order (pairs by levels, odd one carried) on every tree kernel.
+    W=8: [1, e, e, e, e, e, e, e] with e = 2^-24 gives (1+e) = 1 (tie to even), 2e, 2e, 2e;
+    then 1 + 2^-23 and 2^-22; then 1 + 3*2^-23.  W=16 likewise gives 1 + 7*2^-23.  Rank
+    order gives 1 for both."""
     W = len(vals)
     shapes = ((64 * W, 8),)
     g = configs.Group("tree_pin", W, shapes)
     grads = [[np.full(64 * W * 8, np.array([v], np.float32).view(np.uint32)[0] >> 16, np.uint16)]
              for v in vals]
-    for kw in (dict(), dict(tma=True), dict(slots=True)):
-        out, _, _ = run_rs(g, grads, scale=0, order=1, **kw)
+    for kw in (dict(), dict(tma=True), dict(slots=True), dict(out_shift=4)):
+        out, _, plan = run_rs(g, grads, scale=0, order=1, **kw)
         assert np.all(out.cpu().numpy() == np.float32(exp)), kw
+        if not kw and W in (8, 16):
+            assert plan.last_launch()[0] == T.K_RS_TREE_V32
 
 
 @pytest.mark.parametrize("group", GROUPS, ids=IDS)
@@ -579,3 +595,34 @@ def test_workspace_is_tables_only():
         # tiles, numel table, error word, pointer tables: grads, params, slots, shards
         expect = plan.n_tiles * 32 + 2 * P * 8 + 4 + W * P * 8 + P * 8 + W * 8 + W * 8
         assert plan.workspace_bytes == expect
+
+
+@pytest.mark.parametrize("group", [configs.tiny(), mini_wan(), mini_sweep(8), configs.qwen3moe(4),
+                                   degenerate()], ids=lambda g: f"{g.name}_w{g.world}")
+def test_short_lived_ctas_give_the_same_bits(group):
+    """TIDE_PLAN_SHORT_CTAS: one CTA per tile (per tile and rank when staging) that does its
+    unit and exits.  Rank and tree order, Slot-Reuse on both engines and AG placement give the
+    oracle's bits, with as many CTAs as units."""
+    grads = synth.grads_host(group, seed=91)
+    W = group.world
+    ref = oracle.rs_reduce(W, group.shapes, grads, 1).view(np.uint32)
+    out, _, plan = run_rs(group, grads, scale=1, short_ctas=True)
+    assert np.array_equal(f32_bits(out), ref)
+    if plan.n_tiles:
+        assert plan.last_launch()[1] == plan.n_tiles
+    out, _, _ = run_rs(group, grads, scale=1, order=1, short_ctas=True)
+    assert np.array_equal(f32_bits(out), oracle.rs_reduce_tree(W, group.shapes, grads, 1).view(np.uint32))
+    for engine in (T.TIDE_ENGINE_SM, T.TIDE_ENGINE_CE):
+        out, _, plan = run_rs(group, grads, scale=1, slots=True, engine=engine, short_ctas=True)
+        assert np.array_equal(f32_bits(out), ref)
+    L = oracle.layout(W, group.shapes)
+    ag_bits = poison_pads(synth.ag_host(group, L.Ns, seed=92).reshape(-1), group, L)
+    params = padded_params(plan, group)
+    plan.ag_place(to_dev(ag_bits), params)
+    torch.cuda.synchronize()
+    plan.check()
+    for p, r in zip(params, oracle.ag_copyout(W, group.shapes, ag_bits)):
+        assert np.array_equal(bits_of(p), r)
+    if plan.n_tiles:
+        assert plan.last_launch()[1] == plan.n_tiles
+        assert plan.launch_ctas(T.K_STAGE, 0) == plan.n_tiles * W
