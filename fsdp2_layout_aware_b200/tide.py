@@ -89,6 +89,10 @@ _SIGNATURES = {
     "tide_plan_errors": (_i32, [_vp, _vp, _P(_i32)]),
     "tide_launch_ctas": (_i32, [_vp, _i32, _i32, _P(_i32)]),
     "tide_plan_last_launch": (_i32, [_vp, _P(_i32), _P(_i32)]),
+    "tide_ipc_export": (_i32, [_vp, _vp, _P(_i64), _P(_i32)]),
+    "tide_ipc_open": (_i32, [_vp, _i32, _P(_vp)]),
+    "tide_ipc_close": (_i32, [_vp, _i32]),
+    "tide_peer_access": (_i32, [_i32, _i32, _P(_i32)]),
     "tide_status_string": (ctypes.c_char_p, [_i32]),
     "tide_abi_version": (_i32, []),
 }
@@ -140,6 +144,22 @@ class TensorTable:
 
     def __len__(self):
         return len(self.tensors)
+
+
+class PointerTable(TensorTable):
+    """A table of raw device addresses and element counts (for example peers' buffers mapped
+    through tide_ipc_open), usable wherever the Plan methods accept a TensorTable.  `keep`
+    holds references to whatever owns the memory."""
+
+    def __init__(self, ptrs, numels, keep=()):
+        self.tensors = list(keep)
+        self.ptrs = _ptr_array([int(p) for p in ptrs])
+        self.numels = _i64_array(numels)
+        self.min_numel = min((int(n) for n in numels), default=0)
+        self._n = len(ptrs)
+
+    def __len__(self):
+        return self._n
 
 
 def _table(tensors) -> TensorTable:
@@ -288,6 +308,34 @@ def tide_launch_ctas(plan, kernel: int, max_ctas: int):
     n = _i32()
     st = lib().tide_launch_ctas(plan, kernel, max_ctas, ctypes.byref(n))
     return st, n.value
+
+
+def tide_ipc_export(dev_ptr: int):
+    """(status, handle bytes, offset, device) of the allocation holding dev_ptr."""
+    h = ctypes.create_string_buffer(TIDE_IPC_HANDLE_BYTES)
+    off, dev = _i64(0), _i32(-1)
+    st = lib().tide_ipc_export(dev_ptr, h, ctypes.byref(off), ctypes.byref(dev))
+    return st, h.raw, off.value, dev.value
+
+
+def tide_ipc_open(handle: bytes, device: int):
+    """(status, base pointer) of another process's exported allocation, mapped for `device`."""
+    if len(handle) != TIDE_IPC_HANDLE_BYTES:
+        return TIDE_ERR_INVALID_ARG, 0
+    h = ctypes.create_string_buffer(handle, TIDE_IPC_HANDLE_BYTES)
+    base = _vp(0)
+    st = lib().tide_ipc_open(h, device, ctypes.byref(base))
+    return st, base.value or 0
+
+
+def tide_ipc_close(base: int, device: int) -> int:
+    return lib().tide_ipc_close(base, device)
+
+
+def tide_peer_access(device: int, peer: int):
+    v = _i32(0)
+    st = lib().tide_peer_access(device, peer, ctypes.byref(v))
+    return st, v.value
 
 
 # --------------------------------------------------------------------------- torch convenience

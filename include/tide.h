@@ -363,6 +363,42 @@ TIDE_API tide_status_t tide_launch_ctas(const tide_plan_t* plan, int32_t kernel,
 TIDE_API tide_status_t tide_plan_last_launch(const tide_plan_t* plan, int32_t* kernel,
                                              int32_t* ctas);
 
+/*
+ * Peer buffers across processes (CUDA IPC), for the exchange between ranks that
+ * run as one process per GPU: each rank reduces its own shard from every
+ * rank's gradients and places every rank's shard (weekinpapers.com Abstract,
+ * TIDE-RS and TIDE-AG; kongchang.com "TIDE's Design Approach"), so the
+ * pointer tables of tide_rs_reduce / tide_ag_gather_place name other ranks'
+ * buffers.  The allocation must come from cudaMalloc (PyTorch's default
+ * caching allocator qualifies; its expandable segments do not).
+ *
+ * tide_ipc_export: for the device buffer dev_ptr, writes the IPC handle of the
+ * allocation that holds it (TIDE_IPC_HANDLE_BYTES bytes into the host buffer
+ * `handle`), dev_ptr's byte offset inside that allocation (*offset), and, if
+ * device is not NULL, the allocation's device (*device).  The handle stays
+ * valid while the allocation lives.  TIDE_ERR_INVALID_ARG for a NULL or
+ * non-device pointer.
+ * tide_ipc_open: in another process, maps the exported allocation for use by
+ * kernels on `device` (made current for the call, then restored), enabling
+ * peer access from `device` to the owner's GPU as needed; *base receives the
+ * mapping's address, to which the exporter's offset is added.  The same
+ * allocation may be opened once per process and device.  TIDE_ERR_CUDA when the
+ * runtime refuses (no peer access between the two GPUs, a handle from this
+ * same process, an expired allocation).
+ * tide_ipc_close: unmaps a base returned by tide_ipc_open (same device), after
+ * every call that reads it has completed.
+ * tide_peer_access: *can_access = 1 when kernels on `device` can read `peer`'s
+ * memory directly (always for device == peer), else 0.
+ * None of these synchronizes other processes: the caller orders ranks' writes
+ * and reads with host barriers.
+ */
+#define TIDE_IPC_HANDLE_BYTES 64
+TIDE_API tide_status_t tide_ipc_export(const void* dev_ptr, void* handle, int64_t* offset,
+                                       int32_t* device);
+TIDE_API tide_status_t tide_ipc_open(const void* handle, int32_t device, void** base);
+TIDE_API tide_status_t tide_ipc_close(void* base, int32_t device);
+TIDE_API tide_status_t tide_peer_access(int32_t device, int32_t peer, int32_t* can_access);
+
 TIDE_API const char* tide_status_string(tide_status_t status);
 TIDE_API int32_t tide_abi_version(void);
 
