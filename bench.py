@@ -825,9 +825,7 @@ def run_interference(device, seed, quick=False):
     t_start = time.perf_counter()
     group = configs.sweep(8)
     wl = Workload(group, seed, device)
-    plans = {"lsu": wl.plan}
-    if not quick:
-        plans["tma"] = T.Plan(group.shapes, group.world, device=device, tma=True)
+    plans = {"lsu": wl.plan, "tma": T.Plan(group.shapes, group.world, device=device, tma=True)}
     trials = 1 if quick else 3
     B = alg_bytes(group, oracle_free_layout(wl))
     short = T.Plan(group.shapes, group.world, device=device, short_ctas=True)
@@ -862,22 +860,27 @@ def run_interference(device, seed, quick=False):
         g = {"gemm": f"bf16 {m}x{n}x{k} torch.matmul (cuBLAS), {n_gemm} per batch",
              "kernel": launch["kernel"], "grid": launch["grid"], "ctas": launch["ctas"],
              "single_wave": (launch["ctas"] <= sms) if launch["ctas"] else None, "points": []}
-        points = [(kind, plan, ctas, B["rs"],
-                   lambda plan=plan, ctas=ctas: plan.rs_reduce(wl.grads_t, wl.out, max_ctas=ctas, stream=s_rs),
+        # CTA caps: the single-wave GEMM leaves sm_count - 144 = 4 SMs idle on B200, so caps of
+        # 2 and 4 fit beside it and 8 and more do not
+        caps = {"lsu": (2, 4, 8, 16, 32, 0), "tma": (4,) if quick else (2, 4, 8, 16, 32, 0)}
+        points = [(kind, plans[kind], ctas, B["rs"],
+                   lambda plan=plans[kind], ctas=ctas: plan.rs_reduce(wl.grads_t, wl.out, max_ctas=ctas,
+                                                                      stream=s_rs),
                    s_gemm)
-                  for kind, plan in plans.items() for ctas in (8, 16, 32, 0)]
+                  for kind in ("lsu", "tma") for ctas in caps[kind]]
         slots = T.TensorTable(wl.ensure_slots())
         points.append(("ce_stage", wl.plan, 0, B["stage"],
                        lambda: wl.plan.rs_stage(wl.grads_t, slots, engine=T.TIDE_ENGINE_CE, stream=s_rs),
                        s_gemm))
         # short-lived CTAs (one per tile), with the GEMM's stream at the default priority and
         # at the highest; the persistent full grid with the high-priority GEMM for contrast
-        points.append(("lsu_short", short, 0, B["rs"],
-                       lambda: short.rs_reduce(wl.grads_t, wl.out, stream=s_rs), s_gemm))
         points.append(("lsu_short_gemm_high_priority", short, 0, B["rs"],
                        lambda: short.rs_reduce(wl.grads_t, wl.out, stream=s_rs), s_gemm_hi))
-        points.append(("lsu_gemm_high_priority", wl.plan, 0, B["rs"],
-                       lambda: wl.plan.rs_reduce(wl.grads_t, wl.out, stream=s_rs), s_gemm_hi))
+        if not quick:
+            points.append(("lsu_short", short, 0, B["rs"],
+                           lambda: short.rs_reduce(wl.grads_t, wl.out, stream=s_rs), s_gemm))
+            points.append(("lsu_gemm_high_priority", wl.plan, 0, B["rs"],
+                           lambda: wl.plan.rs_reduce(wl.grads_t, wl.out, stream=s_rs), s_gemm_hi))
         for kind, plan, ctas, nbytes, call, sg in points:
             rs_ms = timed_calls(call, 3 if quick else 5, s_rs)
             n_ctas = max(0, plan.last_launch()[1]) if kind != "ce_stage" else 0
@@ -909,8 +912,7 @@ def run_interference(device, seed, quick=False):
         res["gemms"].append(g)
         del a, b, c, slots
         wl.drop_slots()
-    if "tma" in plans:
-        plans["tma"].close()
+    plans["tma"].close()
     short.close()
     del wl
     torch.cuda.empty_cache()
@@ -1342,13 +1344,14 @@ def run_exchange(args, group, proc, n_procs, device, shared_device):
             short_plans = {k: T.Plan(group.shapes, W, device=device, rank=k, short_ctas=True)
                            for k in mine}
 
-            def rs_on(st, pl):
+            def rs_on(st, pl, cap=0):
                 for k in mine:
-                    pl[k].rs_reduce(gtab, outs[k], stream=st)
+                    pl[k].rs_reduce(gtab, outs[k], stream=st, max_ctas=cap)
 
             try:
                 nccl = run_nccl_compare(group, lay, mine, n_procs, device, grads,
-                                        lambda st: rs_on(st, plans), lambda st: rs_on(st, short_plans))
+                                        lambda st, cap=0: rs_on(st, plans, cap),
+                                        lambda st: rs_on(st, short_plans))
             except Exception as e:  # noqa: BLE001  (the step's figures stand)
                 nccl = {"error": f"{type(e).__name__}: {e}"}
             for pl in short_plans.values():
@@ -1514,13 +1517,16 @@ def run_nccl_compare(group, lay, mine, n_procs, device, grads, rs_tide, short_rs
         r = int(cover / max(t, 1e-3)) + 2
         return int(max_over_ranks([r], device)[0])      # the same count on every process
 
-    r_nccl, r_tide, r_short = reps_for(t_nccl), reps_for(t_tide), reps_for(t_short)
+    t_cap = ev_ms(lambda: rs_tide(s_comm, 4), s_comm, 2)
+    t_cap = max_over_ranks([t_cap], device)[0]
+    r_nccl, r_tide, r_short, r_cap = reps_for(t_nccl), reps_for(t_tide), reps_for(t_short), reps_for(t_cap)
     with_nccl = concurrent(s_gemm, stock_rs, r_nccl)
     with_tide = concurrent(s_gemm, lambda: rs_tide(s_comm), r_tide)
     with_short = concurrent(s_gemm_hi, lambda: short_rs(s_comm), r_short)
+    with_cap = concurrent(s_gemm, lambda: rs_tide(s_comm, 4), r_cap)
     dist.barrier()
-    alone, alone_hi, with_nccl, with_tide, with_short = max_over_ranks(
-        [alone, alone_hi, with_nccl, with_tide, with_short], device)
+    alone, alone_hi, with_nccl, with_tide, with_short, with_cap = max_over_ranks(
+        [alone, alone_hi, with_nccl, with_tide, with_short, with_cap], device)
     del pack, acc, out, a, b, c
     torch.cuda.empty_cache()
     return {
@@ -1528,12 +1534,14 @@ def run_nccl_compare(group, lay, mine, n_procs, device, grads, rs_tide, short_rs
                  "over the processes, x 1/W",
         "stock_ms": {"pack": round(t_pack, 4), "nccl_reduce_scatter": round(t_nccl, 4)},
         "tide_rs_ms": round(t_tide, 4), "tide_rs_short_ctas_ms": round(t_short, 4),
+        "tide_rs_4_ctas_ms": round(t_cap, 4),
         "gemm": "bf16 3072x3072x16384 torch.matmul, single wave",
         "gemm_ms_alone": round(alone, 4),
         "gemm_slowdown": {"nccl_reduce_scatter": round(with_nccl / alone - 1, 4),
                           "tide_rs": round(with_tide / alone - 1, 4),
-                          "tide_rs_short_ctas_gemm_high_priority": round(with_short / alone_hi - 1, 4)},
-        "reps": {"nccl": r_nccl, "tide": r_tide, "tide_short": r_short},
+                          "tide_rs_short_ctas_gemm_high_priority": round(with_short / alone_hi - 1, 4),
+                          "tide_rs_4_ctas": round(with_cap / alone - 1, 4)},
+        "reps": {"nccl": r_nccl, "tide": r_tide, "tide_short": r_short, "tide_4_ctas": r_cap},
     }
 
 

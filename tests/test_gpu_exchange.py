@@ -108,4 +108,4 @@ def test_bench_exchange_mode_one_process_with_nccl():
     assert "error" not in nc, nc
     assert nc["stock_ms"]["nccl_reduce_scatter"] > 0 and nc["tide_rs_ms"] > 0
     assert set(nc["gemm_slowdown"]) == {"nccl_reduce_scatter", "tide_rs",
-                                        "tide_rs_short_ctas_gemm_high_priority"}
+                                        "tide_rs_short_ctas_gemm_high_priority", "tide_rs_4_ctas"}
