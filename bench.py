@@ -1623,7 +1623,8 @@ def run_reference(args):
     sample = describe_sample(group, items, nbytes) + f"; {workers} processes, one pass per step"
     res = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s",
            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-           "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+           "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
+           "scaling": "strong" if args.gpus > 1 else "weak",
            "vs_baseline": None, "dtype": "bf16/f32", "data": "synthetic",
            "config": {"workload": f"{group.name} layer group, W={group.world} simulated ranks, "
                                   f"{group.n_params} params, {total} elements",
