@@ -424,3 +424,15 @@ def test_short_lived_ctas_take_no_cta_cap(args):
     # unknown flag bits are still refused
     st, _ = T.tide_plan_group([(4, 4)], 4, 0, T.TIDE_PLAN_HOST_ONLY | 64)
     assert st == T.TIDE_ERR_INVALID_ARG
+
+
+def test_ipc_calls_validate_their_arguments_on_the_host():
+    """The peer-mapping calls refuse NULL pointers and negative devices before any CUDA call."""
+    st, handle, off, dev = T.tide_ipc_export(0)
+    assert st == T.TIDE_ERR_INVALID_ARG and len(handle) == T.TIDE_IPC_HANDLE_BYTES
+    assert T.tide_ipc_open(bytes(T.TIDE_IPC_HANDLE_BYTES), -1) == (T.TIDE_ERR_INVALID_ARG, 0)
+    assert T.tide_ipc_open(b"short", 0)[0] == T.TIDE_ERR_INVALID_ARG
+    assert T.tide_ipc_close(0, 0) == T.TIDE_ERR_INVALID_ARG
+    assert T.tide_ipc_close(1 << 40, -1) == T.TIDE_ERR_INVALID_ARG
+    assert T.tide_peer_access(3, 3) == (T.TIDE_OK, 1)        # a device always reads itself
+    assert T.tide_peer_access(-1, 0)[0] == T.TIDE_ERR_INVALID_ARG
