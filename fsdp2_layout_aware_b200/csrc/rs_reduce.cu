@@ -38,7 +38,10 @@ namespace {
 
 // The 32-byte path measured faster for 5 <= W <= 16 (70B W=8: 7.03 vs 6.89
 // TB/s; Qwen3 W=8: 7.08 vs 6.87; Wan2.2 W=16: 6.93 vs 6.90) and slower at
-// W=64 (6.90 vs 7.01), where 16-byte loads keep more ranks in flight.
+// W=64 (6.90 vs 7.01), where 16-byte loads keep more ranks in flight.  At W = 2
+// it beats the 16-byte two-rank kernel by 20-27 % (67 MB to 1.1 GB groups:
+// 3.41 vs 2.73, 5.02 vs 3.95, 5.31 vs 4.45 TB/s); at W = 3 and 4 it does not
+// (5.34 vs 5.39, 6.18 vs 6.16 and 5.64 vs 5.78), so they keep 16-byte loads.
 constexpr int kV32MaxWorld = 16;
 
 struct RsParams {
@@ -186,6 +189,10 @@ using KernelFn = void (*)(const RsParams);
 template <bool SLOT, bool TREE>
 KernelFn pick(int world, bool v32) {
     // (in the tree order every W <= G is one group, so G < 8 kernels never merge)
+    if constexpr (!TREE) {
+        // W = 2 in rank order: the 32-byte kernel (one group, two ranks loaded)
+        if (v32 && world == 2) return rs_reduce_kernel<8, 1, SLOT, false, true, false>;
+    }
     if (world <= 2) return rs_reduce_kernel<2, 4, SLOT, TREE, false, TREE>;
     if (world <= 4) return rs_reduce_kernel<4, 2, SLOT, TREE, false, TREE>;
     if constexpr (TREE) {
@@ -210,7 +217,8 @@ KernelFn select(int world, bool slot, int order, bool v32) {
 }  // namespace
 
 bool rs_v32_applies(int world, int order) {
-    return order == TIDE_ORDER_TREE ? (world == 8 || world == 16) : (world > 4 && world <= kV32MaxWorld);
+    if (order == TIDE_ORDER_TREE) return world == 8 || world == 16;
+    return world == 2 || (world > 4 && world <= kV32MaxWorld);
 }
 
 int rs_blocks_per_sm(int world, bool slot, int order, bool v32) {
