@@ -24,6 +24,17 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
     return v;
 }
 
+// ld_stream_v4 that the compiler keeps in program order with other volatile asm
+// (a wide tree loads one group of ranks at a time this way, so registers hold
+// one group's raw vectors, not all of them).
+__device__ __forceinline__ uint4 ld_stream_v4_ordered(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
 // 32 bytes (16 bf16) as eight 32-bit words.
 struct V8 {
     uint32_t w[8];

@@ -146,19 +146,30 @@ __device__ __forceinline__ void tree_one_group(int W, Load load, float (&acc)[L]
     for (int l = 0; l < L; ++l) acc[l] = f[0][l];
 }
 
-// The tree order when G < W <= 2G: the two groups' trees, then one add that
-// joins them -- the adds reduce_ranks<G, L, true> makes for such a W (its
-// binary counter holds group 0's sum on level 0 and merges group 1's into it),
-// so the same bits, without the six-level merge stack.  The second group is
-// loaded only after the first is reduced, which keeps two groups' raw vectors
-// from being live at once.
-template <int G, int L, class Raw, class Load>
-__device__ __forceinline__ void tree_two_groups(int W, Load load, float (&acc)[L]) {
-    float first[L];
-    tree_one_group<G, L, Raw>(G, load, first);
-    tree_one_group<G, L, Raw>(W - G, [&](int k) { return load(G + k); }, acc);
+// The tree order when W = NG * G exactly, NG a power of two, fixed at compile
+// time: the two halves' trees, then one add that joins them, recursively down
+// to single groups.  For W a power of two this is the balanced binary tree,
+// which is what adjacent pairs level by level make (no odd one is ever carried)
+// and what reduce_ranks<G, L, true> makes by merging group sums through its
+// binary counter -- the same bits, with no merge stack and no run-time W.  The
+// second half is loaded only after the first is reduced, so at most one
+// group's raw vectors are live beside log2(NG) partial sums.
+template <int G, int NG, int L, class Raw, class Load>
+__device__ __forceinline__ void tree_groups(Load load, float (&acc)[L]) {
+    static_assert(NG >= 1 && (NG & (NG - 1)) == 0, "group count must be a power of two");
+    if constexpr (NG == 1) {
+        tree_one_group<G, L, Raw>(G, load, acc);
+    } else {
+        float first[L];
+        tree_groups<G, NG / 2, L, Raw>(load, first);
+        // the first half's sums exist before the second half's loads are issued (with
+        // ordered loads, see ld_stream_v4_ordered, the compiler cannot hoist them above)
 #pragma unroll
-    for (int l = 0; l < L; ++l) acc[l] = __fadd_rn(first[l], acc[l]);
+        for (int l = 0; l < L; ++l) asm volatile("" : "+f"(first[l]));
+        tree_groups<G, NG / 2, L, Raw>([&](int k) { return load(NG / 2 * G + k); }, acc);
+#pragma unroll
+        for (int l = 0; l < L; ++l) acc[l] = __fadd_rn(first[l], acc[l]);
+    }
 }
 
 }  // namespace tide

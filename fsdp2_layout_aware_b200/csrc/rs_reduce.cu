@@ -62,20 +62,23 @@ struct RsParams {
 // V32: 32-byte loads and stores (16 outputs per thread per step); the host
 // picks it only when every tile's sources and output are 32-byte aligned
 // (a tile that is not falls back to the element loop, never faults).
-// ONE: the tree order for W <= G (a single group), without the merge stack.
-// In tree order the 32-byte kernels serve W = G (ONE) and W = 2G (not ONE: two
-// groups joined by one add, tree_two_groups), with the tree fixed at compile
-// time and no merge stack: a runtime W kept up to 8 ranks' unpacked lanes live
+// NG selects how the tree order is formed (rank order ignores it):
+//   NG = -1: W <= G at run time, one group (tree_one_group), no merge stack;
+//   NG =  0: any W at run time, groups of G merged through reduce_ranks' stack;
+//   NG >= 1: W = NG * G exactly, the whole tree fixed at compile time
+//            (tree_groups): no merge stack and no run-time W.
+// The 32-byte tree kernels are NG = 1 and 2 (W = 8, 16).  A first 32-byte
+// version kept W at run time; up to 8 ranks' unpacked lanes then stayed live
 // and spilled (276 and 708 bytes) at the 128 registers of 2 CTAs per SM.
-// The 16-byte single-group tree kernels are held to 3 CTAs per SM (80
-// registers, a spill of 88 bytes per thread at G = 8): left free they take 128
-// registers and 2 CTAs per SM, 4 % slower on B200 (70B W=8: 6.52 vs 6.28 TB/s;
-// Qwen3: 6.47 vs 6.19).  The 32-byte tree kernels are held to 2 CTAs per SM,
-// the rank-order 32-byte kernel's occupancy.  The others keep the compiler's
+// The 16-byte NG = -1 kernels are held to 3 CTAs per SM (80 registers, a
+// spill of 88 bytes per thread at G = 8): left free they take 128 registers
+// and 2 CTAs per SM, 4 % slower on B200 (70B W=8: 6.52 vs 6.28 TB/s; Qwen3:
+// 6.47 vs 6.19).  The 32-byte tree kernels are held to 2 CTAs per SM, the
+// rank-order 32-byte kernel's occupancy.  The others keep the compiler's
 // choice (an explicit minimum of 1 CTA raised the rank-order kernels'
 // registers and cost bandwidth).
-template <int G, int U, bool SLOT, bool TREE, bool V32, bool ONE>
-__global__ void __launch_bounds__(kThreads, (TREE && V32) ? 2 : (TREE && ONE) ? 3 : 0)
+template <int G, int U, bool SLOT, bool TREE, bool V32, int NG>
+__global__ void __launch_bounds__(kThreads, (TREE && (V32 || NG >= 4)) ? 2 : (TREE && NG == -1) ? 3 : 0)
 rs_reduce_kernel(const RsParams a) {
     // s_src is double-buffered: tile i writes buffer i&1 while no thread can
     // still be reading the same buffer from tile i-2 (a barrier lies between).
@@ -126,11 +129,9 @@ rs_reduce_kernel(const RsParams a) {
             for (int v = tid; v < nv16; v += kThreads) {
                 float acc[16];
                 auto load = [&](int k) { return ld_stream_v8(srcs[k] + 16 * (int64_t)v); };
-                // (the 32-byte tree kernels run only for W = G and W = 2G, so their
-                // trees are fixed at compile time)
+                // (the 32-byte tree kernels run only for W = NG * G, tree fixed at compile time)
                 if constexpr (!TREE) reduce_ranks<G, 16, false, V8>(W, load, acc);
-                else if constexpr (ONE) tree_one_group<G, 16, V8>(G, load, acc);
-                else tree_two_groups<G, 16, V8>(2 * G, load, acc);
+                else tree_groups<G, (NG > 0 ? NG : 1), 16, V8>(load, acc);
                 if (a.do_scale) {
 #pragma unroll
                     for (int l = 0; l < 16; ++l) acc[l] = __fmul_rn(acc[l], a.scale);
@@ -150,8 +151,18 @@ rs_reduce_kernel(const RsParams a) {
             for (int u = 0; u < U; ++u) {
                 const int v = v0 + u * kThreads + tid;
                 if (v < nv) {
-                    auto load = [&](int k) { return ld_stream_v4(srcs[k] + 8 * (int64_t)v); };
-                    if constexpr (ONE) tree_one_group<G, 8, uint4>(W, load, acc[u]);
+                    // (the wide trees re-read each source address from shared memory at its
+                    // use, in order, rather than keeping all W addresses in registers)
+                    auto load = [&](int k) {
+                        if constexpr (TREE && NG >= 4) {
+                            const uint16_t* p = const_cast<const uint16_t* const volatile*>(srcs)[k];
+                            return ld_stream_v4_ordered(p + 8 * (int64_t)v);
+                        } else {
+                            return ld_stream_v4(srcs[k] + 8 * (int64_t)v);
+                        }
+                    };
+                    if constexpr (TREE && NG == -1) tree_one_group<G, 8, uint4>(W, load, acc[u]);
+                    else if constexpr (TREE && NG > 0) tree_groups<G, NG, 8, uint4>(load, acc[u]);
                     else reduce_ranks<G, 8, TREE, uint4>(W, load, acc[u]);
                 }
             }
@@ -173,8 +184,8 @@ rs_reduce_kernel(const RsParams a) {
         for (int e = 8 * nv + tid; e < tl.n_valid; e += kThreads) {
             float acc[1];
             auto load = [&](int k) { return (uint32_t)ld_stream_u16(srcs[k] + e); };
-            if constexpr (ONE) tree_one_group<G, 1, uint32_t>(W, load, acc);
-            else if constexpr (TREE && V32) tree_two_groups<G, 1, uint32_t>(2 * G, load, acc);
+            if constexpr (TREE && NG == -1) tree_one_group<G, 1, uint32_t>(W, load, acc);
+            else if constexpr (TREE && NG > 0) tree_groups<G, NG, 1, uint32_t>(load, acc);
             else reduce_ranks<G, 1, TREE, uint32_t>(W, load, acc);
             if (a.do_scale) acc[0] = __fmul_rn(acc[0], a.scale);
             dst[e] = acc[0];
@@ -191,20 +202,24 @@ KernelFn pick(int world, bool v32) {
     // (in the tree order every W <= G is one group, so G < 8 kernels never merge)
     if constexpr (!TREE) {
         // W = 2 in rank order: the 32-byte kernel (one group, two ranks loaded)
-        if (v32 && world == 2) return rs_reduce_kernel<8, 1, SLOT, false, true, false>;
+        if (v32 && world == 2) return rs_reduce_kernel<8, 1, SLOT, false, true, 0>;
     }
-    if (world <= 2) return rs_reduce_kernel<2, 4, SLOT, TREE, false, TREE>;
-    if (world <= 4) return rs_reduce_kernel<4, 2, SLOT, TREE, false, TREE>;
+    if (world <= 2) return rs_reduce_kernel<2, 4, SLOT, TREE, false, TREE ? -1 : 0>;
+    if (world <= 4) return rs_reduce_kernel<4, 2, SLOT, TREE, false, TREE ? -1 : 0>;
     if constexpr (TREE) {
         // 32-byte tree kernels: exactly one group (W = 8) or two groups (W = 16) of 8
         if (v32 && (world == 8 || world == 16))
-            return world == 8 ? rs_reduce_kernel<8, 1, SLOT, true, true, true>
-                              : rs_reduce_kernel<8, 1, SLOT, true, true, false>;
-        if (world <= 8) return rs_reduce_kernel<8, 1, SLOT, true, false, true>;
-        return rs_reduce_kernel<8, 1, SLOT, true, false, false>;
+            return world == 8 ? rs_reduce_kernel<8, 1, SLOT, true, true, 1>
+                              : rs_reduce_kernel<8, 1, SLOT, true, true, 2>;
+        if (world <= 8) return rs_reduce_kernel<8, 1, SLOT, true, false, -1>;
+        // 16-byte trees fixed at compile time for W = 16 and 32 (at W = 64 the eight
+        // groups' partial sums and addresses spill at 2 CTAs per SM)
+        if (world == 16) return rs_reduce_kernel<8, 1, SLOT, true, false, 2>;
+        if (world == 32) return rs_reduce_kernel<8, 1, SLOT, true, false, 4>;
+        return rs_reduce_kernel<8, 1, SLOT, true, false, 0>;
     } else {
-        if (v32 && world <= kV32MaxWorld) return rs_reduce_kernel<8, 1, SLOT, false, true, false>;
-        return rs_reduce_kernel<8, 1, SLOT, false, false, false>;
+        if (v32 && world <= kV32MaxWorld) return rs_reduce_kernel<8, 1, SLOT, false, true, 0>;
+        return rs_reduce_kernel<8, 1, SLOT, false, false, 0>;
     }
 }
 
