@@ -390,11 +390,17 @@ def run_variants(wl, K, stream, peak, flush):
     # ... and overlapped: the copy engines stage run s+1 while the SMs reduce run s
     cs = torch.cuda.Stream(wl.out.device)
     W = wl.group.world
+    # (a full-grid reduction keeps the copy engines from progressing beside it, so the
+    # overlapped runs cap the reduction at one CTA per SM; one segment is the serial order)
+    sms = torch.cuda.get_device_properties(wl.out.device).multi_processor_count
     for nseg in sorted({1, min(4, W), W}):
+        cap = 0 if nseg == 1 else sms
         wl.out.fill_(float("nan"))
         rec(f"slot_reuse_pipelined_seg{nseg}",
-            timed_calls(lambda: wl.plan.rs_reduce_pipelined(wl.grads_t, wl.out, slots, nseg, cs),
+            timed_calls(lambda: wl.plan.rs_reduce_pipelined(wl.grads_t, wl.out, slots, nseg, cs,
+                                                            max_ctas=cap),
                         K, stream, flush), B["stage"] + B["slot_rs"], nseg, wl.plan, same_rs)
+        out[f"slot_reuse_pipelined_seg{nseg}"]["max_ctas"] = cap
     wl.drop_slots()
     del slots
     # Context: the stock FSDP2 layout conversion with torch's own kernels on the same GPU

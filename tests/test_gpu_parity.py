@@ -28,6 +28,8 @@ def parity_groups():
            configs.qwen3moe(4), configs.Group("long_chunk", 3, ((30011, 7), (5,), (40000,)))]
     for w in (1, 2, 3, 5, 8, 16, 64):
         out.append(random_group(rng, w, int(rng.integers(1, 8)), max_rows=1500, name=f"rand_w{w}"))
+    # W = 32: the tree order's compile-time four-group kernel
+    out.append(random_group(np.random.default_rng(32), 32, 5, max_rows=1500, name="rand_w32"))
     return out
 
 
@@ -220,12 +222,13 @@ def test_rs_rank_order_pin_on_gpu():
     ([1.0] + [2.0 ** -24] * 9, 1.0 + 2.0 ** -21),                       # W=10, two groups on the GPU
     ([1.0] + [2.0 ** -24] * 7, 1.0 + 3 * 2.0 ** -23),                   # W=8, 32-byte kernel
     ([1.0] + [2.0 ** -24] * 15, 1.0 + 7 * 2.0 ** -23),                  # W=16, 32-byte kernel
+    ([1.0] + [2.0 ** -24] * 31, 1.0 + 15 * 2.0 ** -23),                 # W=32, four groups fixed
 ])
 def test_rs_tree_order_pin_on_gpu(vals, exp):
     """Worked values of the tree order (pairs by levels, odd one carried) on every tree kernel.
     W=8: [1, e, e, e, e, e, e, e] with e = 2^-24 gives (1+e) = 1 (tie to even), 2e, 2e, 2e;
-    then 1 + 2^-23 and 2^-22; then 1 + 3*2^-23.  W=16 likewise gives 1 + 7*2^-23.  Rank
-    order gives 1 for both."""
+    then 1 + 2^-23 and 2^-22; then 1 + 3*2^-23.  W=16 and 32 likewise give 1 + 7*2^-23 and
+    1 + 15*2^-23.  Rank order gives 1 for all three."""
     W = len(vals)
     shapes = ((64 * W, 8),)
     g = configs.Group("tree_pin", W, shapes)
