@@ -70,6 +70,10 @@ struct RsParams {
 // The 32-byte tree kernels are NG = 1 and 2 (W = 8, 16).  A first 32-byte
 // version kept W at run time; up to 8 ranks' unpacked lanes then stayed live
 // and spilled (276 and 708 bytes) at the 128 registers of 2 CTAs per SM.
+// The 16-byte NG = 4 (W = 32) kernel keeps 2 CTAs per SM by loading one group
+// at a time; NG = 8 (W = 64) spilled 300-320 bytes that way and runs at one
+// CTA per SM instead (153 registers, no spill): 6.74 TB/s against 6.18 for the
+// merge-stack kernel on the sweep's W = 64 group.
 // The 16-byte NG = -1 kernels are held to 3 CTAs per SM (80 registers, a
 // spill of 88 bytes per thread at G = 8): left free they take 128 registers
 // and 2 CTAs per SM, 4 % slower on B200 (70B W=8: 6.52 vs 6.28 TB/s; Qwen3:
@@ -78,7 +82,7 @@ struct RsParams {
 // choice (an explicit minimum of 1 CTA raised the rank-order kernels'
 // registers and cost bandwidth).
 template <int G, int U, bool SLOT, bool TREE, bool V32, int NG>
-__global__ void __launch_bounds__(kThreads, (TREE && (V32 || NG >= 4)) ? 2 : (TREE && NG == -1) ? 3 : 0)
+__global__ void __launch_bounds__(kThreads, (TREE && NG == 8) ? 1 : (TREE && (V32 || NG == 4)) ? 2 : (TREE && NG == -1) ? 3 : 0)
 rs_reduce_kernel(const RsParams a) {
     // s_src is double-buffered: tile i writes buffer i&1 while no thread can
     // still be reading the same buffer from tile i-2 (a barrier lies between).
@@ -151,10 +155,10 @@ rs_reduce_kernel(const RsParams a) {
             for (int u = 0; u < U; ++u) {
                 const int v = v0 + u * kThreads + tid;
                 if (v < nv) {
-                    // (the wide trees re-read each source address from shared memory at its
-                    // use, in order, rather than keeping all W addresses in registers)
+                    // (the four-group tree re-reads each source address from shared memory at
+                    // its use, in order, rather than keeping all W addresses in registers)
                     auto load = [&](int k) {
-                        if constexpr (TREE && NG >= 4) {
+                        if constexpr (TREE && NG == 4) {
                             const uint16_t* p = const_cast<const uint16_t* const volatile*>(srcs)[k];
                             return ld_stream_v4_ordered(p + 8 * (int64_t)v);
                         } else {
@@ -212,10 +216,10 @@ KernelFn pick(int world, bool v32) {
             return world == 8 ? rs_reduce_kernel<8, 1, SLOT, true, true, 1>
                               : rs_reduce_kernel<8, 1, SLOT, true, true, 2>;
         if (world <= 8) return rs_reduce_kernel<8, 1, SLOT, true, false, -1>;
-        // 16-byte trees fixed at compile time for W = 16 and 32 (at W = 64 the eight
-        // groups' partial sums and addresses spill at 2 CTAs per SM)
+        // 16-byte trees fixed at compile time for W = 16, 32 and 64
         if (world == 16) return rs_reduce_kernel<8, 1, SLOT, true, false, 2>;
         if (world == 32) return rs_reduce_kernel<8, 1, SLOT, true, false, 4>;
+        if (world == 64) return rs_reduce_kernel<8, 1, SLOT, true, false, 8>;
         return rs_reduce_kernel<8, 1, SLOT, true, false, 0>;
     } else {
         if (v32 && world <= kV32MaxWorld) return rs_reduce_kernel<8, 1, SLOT, false, true, 0>;

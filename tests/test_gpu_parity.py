@@ -223,12 +223,13 @@ def test_rs_rank_order_pin_on_gpu():
     ([1.0] + [2.0 ** -24] * 7, 1.0 + 3 * 2.0 ** -23),                   # W=8, 32-byte kernel
     ([1.0] + [2.0 ** -24] * 15, 1.0 + 7 * 2.0 ** -23),                  # W=16, 32-byte kernel
     ([1.0] + [2.0 ** -24] * 31, 1.0 + 15 * 2.0 ** -23),                 # W=32, four groups fixed
+    ([1.0] + [2.0 ** -24] * 63, 1.0 + 31 * 2.0 ** -23),                 # W=64, eight groups fixed
 ])
 def test_rs_tree_order_pin_on_gpu(vals, exp):
     """Worked values of the tree order (pairs by levels, odd one carried) on every tree kernel.
     W=8: [1, e, e, e, e, e, e, e] with e = 2^-24 gives (1+e) = 1 (tie to even), 2e, 2e, 2e;
-    then 1 + 2^-23 and 2^-22; then 1 + 3*2^-23.  W=16 and 32 likewise give 1 + 7*2^-23 and
-    1 + 15*2^-23.  Rank order gives 1 for all three."""
+    then 1 + 2^-23 and 2^-22; then 1 + 3*2^-23.  W=16, 32 and 64 likewise give 1 + 7*2^-23,
+    1 + 15*2^-23 and 1 + 31*2^-23.  Rank order gives 1 for all of them."""
     W = len(vals)
     shapes = ((64 * W, 8),)
     g = configs.Group("tree_pin", W, shapes)
