@@ -464,7 +464,7 @@ extern "C" tide_status_t tide_rs_reduce_pipelined(const tide_plan_t* cplan, cons
         const int64_t j0 = bounds[seg], j1 = bounds[seg + 1];
         if (j1 == j0) continue;
         // phase 1 of these chunks on the copy engines ...
-        if (tide::ce_slot_stage(p, grads, slots, cs, j0, j1) != cudaSuccess) return TIDE_ERR_CUDA;
+        if (tide::ce_slot_stage(p, grads, slots, cs, j0, j1, false) != cudaSuccess) return TIDE_ERR_CUDA;
         cudaEvent_t done = p->seg_events[seg];
         if (cudaEventRecord(done, cs) != cudaSuccess || cudaStreamWaitEvent(s, done, 0) != cudaSuccess)
             return TIDE_ERR_CUDA;

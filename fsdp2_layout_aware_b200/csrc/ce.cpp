@@ -15,6 +15,18 @@
 // caller's stream with an event and joined back before the call returns), so
 // that several copy engines work at once: on one stream the copies run one
 // after another, which holds them to about half of HBM bandwidth.
+//
+// Issuing a copy costs the host about 3 us, which bounds the calls on groups of
+// many small parameters.  So the first placement call with a given set of
+// buffers (outside any stream capture) records its copies once as a CUDA graph,
+// on a private stream, and every call with the same buffers launches that graph
+// on the caller's stream: one launch instead of hundreds of copy calls.  A call
+// on a stream that is being captured issues its copies directly, into the
+// caller's capture.  Measured on B200 against direct issue (TB/s): placement
+// 6.55 / 3.29 / 3.72 against 6.27 / 3.25 / 3.68 on the 70B / Qwen3 / Wan2.2
+// groups; placement from per-rank shards (one copy per chunk) 6.48 / 1.90 /
+// 4.55 against 6.12 / 0.70 / 2.60.  Slot-Reuse staging stays on direct issue
+// (see ce_slot_stage).
 #include <algorithm>
 #include <condition_variable>
 #include <functional>
@@ -226,40 +238,117 @@ CeOp rows_op(void* dst, size_t dpitch, const void* src, size_t spitch, size_t wi
     return CeOp{CeOp::kRows, dst, dpitch, src, spitch, width, rows};
 }
 
-}  // namespace
+// Recorded graphs kept per plan (the least recently used one is replaced).
+constexpr size_t kMaxCeGraphs = 4;
 
-cudaError_t ce_ag_place(tide_plan* p, const uint16_t* ag, void* const* params, cudaStream_t stream) {
-    const int64_t W = p->world, Ns = p->shard_numel;
-    const size_t max_pitch = device_max_pitch(p->device);
+enum { kCallPlace = 1, kCallGather = 2, kCallStage = 3 };
+
+// Issue the planned lists (q->lists) as one call on `stream`: replay the graph
+// recorded for (kind, j0, j1, key) if there is one, else record it now and
+// replay it; if the stream is being captured, or recording fails, fork, issue
+// and join directly on `stream`.  `plan` fills q->lists; it runs only when the
+// copies are issued or recorded.
+cudaError_t run_call(tide_plan* p, cudaStream_t stream, int kind, int64_t j0, int64_t j1,
+                     std::vector<const void*>&& key, bool record,
+                     const std::function<void(CeIssuer*)>& plan) {
     CeIssuer* q = issuer(p);
     if (q == nullptr) return cudaErrorMemoryAllocation;
-    for (auto& l : q->lists) l.clear();
-    int next = 0;  // round-robin over the fan-out streams for whole (small) params
-    for (int32_t i = 0; i < p->n_params; ++i) {
-        const int64_t c = p->chunk[i], n = p->numel[i];
-        if (c == 0) continue;
-        uint16_t* dst = static_cast<uint16_t*>(params[i]);
-        const uint16_t* src = ag + p->offset[i];
-        const int64_t full = std::min(W, n / c);
-        // ranks [0, full) hold whole chunks: one 2-D copy, cut by ranks over the streams if large
-        const int parts = (2 * n >= kSplitBytes) ? (int)std::min<int64_t>(kFanout, full) : 1;
-        for (int j = 0; j < parts; ++j) {
-            const int64_t r0 = full * j / parts, r1 = full * (j + 1) / parts;
-            if (r1 > r0)
-                q->lists[(next + j) % kFanout].push_back(
-                    rows_op(dst + r0 * c, 2 * c, src + r0 * Ns, 2 * Ns, 2 * c, r1 - r0));
-        }
-        auto& l = q->lists[next % kFanout];
-        next = (next + parts) % kFanout;
-        const int64_t rem = n - full * c;
-        if (rem > 0 && full < W) l.push_back(rows_op(dst + full * c, 0, src + full * Ns, 0, 2 * rem, 1));
-        if (W * c > n) l.push_back(CeOp{CeOp::kMemset, dst + n, 0, nullptr, 0, (size_t)(2 * (W * c - n)), 0});
+    const size_t max_pitch = device_max_pitch(p->device);
+    cudaStreamCaptureStatus capturing = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &capturing) != cudaSuccess) {
+        (void)cudaGetLastError();
+        capturing = cudaStreamCaptureStatusActive;  // treat as captured: issue directly
     }
+    if (record && capturing == cudaStreamCaptureStatusNone) {
+        for (auto& g : p->ce_graphs) {
+            if (g.kind == kind && g.j0 == j0 && g.j1 == j1 && g.key == key) {
+                g.last_use = ++p->ce_clock;
+                return cudaGraphLaunch(g.exec, stream);
+            }
+        }
+        // record the call on the private stream: fork, issue, join, as below
+        bool ok = p->ce_capture_stream != nullptr ||
+                  cudaStreamCreateWithFlags(&p->ce_capture_stream, cudaStreamNonBlocking) == cudaSuccess;
+        cudaGraph_t graph = nullptr;
+        cudaGraphExec_t exec = nullptr;
+        if (ok) {
+            for (auto& l : q->lists) l.clear();
+            plan(q);
+            cudaStream_t cap = p->ce_capture_stream;
+            ok = cudaStreamBeginCapture(cap, cudaStreamCaptureModeRelaxed) == cudaSuccess;
+            if (ok) {
+                cudaError_t e = fork(p, cap);
+                if (e == cudaSuccess) e = issue_all(p, q, max_pitch);
+                cudaError_t j = join(p, cap);
+                cudaError_t end = cudaStreamEndCapture(cap, &graph);  // ends the capture in every case
+                ok = e == cudaSuccess && j == cudaSuccess && end == cudaSuccess && graph != nullptr &&
+                     cudaGraphInstantiate(&exec, graph, 0) == cudaSuccess;
+                if (graph != nullptr) cudaGraphDestroy(graph);
+            }
+        }
+        if (ok) {
+            if (p->ce_graphs.size() >= kMaxCeGraphs) {
+                auto lru = std::min_element(p->ce_graphs.begin(), p->ce_graphs.end(),
+                                            [](const tide_plan::CeGraph& a, const tide_plan::CeGraph& b) {
+                                                return a.last_use < b.last_use;
+                                            });
+                cudaGraphExecDestroy(lru->exec);
+                p->ce_graphs.erase(lru);
+            }
+            tide_plan::CeGraph g;
+            g.kind = kind;
+            g.j0 = j0;
+            g.j1 = j1;
+            g.key = std::move(key);
+            g.exec = exec;
+            g.last_use = ++p->ce_clock;
+            p->ce_graphs.push_back(std::move(g));
+            return cudaGraphLaunch(exec, stream);
+        }
+        if (exec != nullptr) cudaGraphExecDestroy(exec);
+        (void)cudaGetLastError();  // fall back to issuing the copies directly
+    }
+    for (auto& l : q->lists) l.clear();
+    plan(q);
     cudaError_t e = fork(p, stream);
     if (e != cudaSuccess) return e;
     e = issue_all(p, q, max_pitch);
     cudaError_t j = join(p, stream);
     return e != cudaSuccess ? e : j;
+}
+
+}  // namespace
+
+cudaError_t ce_ag_place(tide_plan* p, const uint16_t* ag, void* const* params, cudaStream_t stream) {
+    const int64_t W = p->world, Ns = p->shard_numel;
+    std::vector<const void*> key;
+    key.reserve((size_t)p->n_params + 1);
+    key.push_back(ag);
+    for (int32_t i = 0; i < p->n_params; ++i) key.push_back(params[i]);
+    return run_call(p, stream, kCallPlace, 0, 0, std::move(key), true, [&](CeIssuer* q) {
+        int next = 0;  // round-robin over the fan-out streams for whole (small) params
+        for (int32_t i = 0; i < p->n_params; ++i) {
+            const int64_t c = p->chunk[i], n = p->numel[i];
+            if (c == 0) continue;
+            uint16_t* dst = static_cast<uint16_t*>(params[i]);
+            const uint16_t* src = ag + p->offset[i];
+            const int64_t full = std::min(W, n / c);
+            // ranks [0, full) hold whole chunks: one 2-D copy, cut by ranks over the streams if large
+            const int parts = (2 * n >= kSplitBytes) ? (int)std::min<int64_t>(kFanout, full) : 1;
+            for (int j = 0; j < parts; ++j) {
+                const int64_t r0 = full * j / parts, r1 = full * (j + 1) / parts;
+                if (r1 > r0)
+                    q->lists[(next + j) % kFanout].push_back(
+                        rows_op(dst + r0 * c, 2 * c, src + r0 * Ns, 2 * Ns, 2 * c, r1 - r0));
+            }
+            auto& l = q->lists[next % kFanout];
+            next = (next + parts) % kFanout;
+            const int64_t rem = n - full * c;
+            if (rem > 0 && full < W) l.push_back(rows_op(dst + full * c, 0, src + full * Ns, 0, 2 * rem, 1));
+            if (W * c > n)
+                l.push_back(CeOp{CeOp::kMemset, dst + n, 0, nullptr, 0, (size_t)(2 * (W * c - n)), 0});
+        }
+    });
 }
 
 // Gathering placement: rank r's chunk of param i comes from rank r's own shard
@@ -268,29 +357,26 @@ cudaError_t ce_ag_place(tide_plan* p, const uint16_t* ag, void* const* params, c
 cudaError_t ce_ag_gather(tide_plan* p, const void* const* shards, void* const* params,
                          cudaStream_t stream) {
     const int64_t W = p->world;
-    const size_t max_pitch = device_max_pitch(p->device);
-    CeIssuer* q = issuer(p);
-    if (q == nullptr) return cudaErrorMemoryAllocation;
-    for (auto& l : q->lists) l.clear();
-    for (int32_t i = 0; i < p->n_params; ++i) {
-        const int64_t c = p->chunk[i], n = p->numel[i];
-        if (c == 0) continue;
-        uint16_t* dst = static_cast<uint16_t*>(params[i]);
-        for (int64_t r = 0; r < W; ++r) {
-            const int64_t valid = std::min(c, std::max<int64_t>(0, n - r * c));
-            if (valid == 0) break;  // later ranks hold only pad rows
-            const uint16_t* src = static_cast<const uint16_t*>(shards[r]) + p->offset[i];
-            q->lists[r % kFanout].push_back(rows_op(dst + r * c, 0, src, 0, 2 * valid, 1));
+    std::vector<const void*> key;
+    key.reserve((size_t)(W + p->n_params));
+    for (int64_t r = 0; r < W; ++r) key.push_back(shards[r]);
+    for (int32_t i = 0; i < p->n_params; ++i) key.push_back(params[i]);
+    return run_call(p, stream, kCallGather, 0, 0, std::move(key), true, [&](CeIssuer* q) {
+        for (int32_t i = 0; i < p->n_params; ++i) {
+            const int64_t c = p->chunk[i], n = p->numel[i];
+            if (c == 0) continue;
+            uint16_t* dst = static_cast<uint16_t*>(params[i]);
+            for (int64_t r = 0; r < W; ++r) {
+                const int64_t valid = std::min(c, std::max<int64_t>(0, n - r * c));
+                if (valid == 0) break;  // later ranks hold only pad rows
+                const uint16_t* src = static_cast<const uint16_t*>(shards[r]) + p->offset[i];
+                q->lists[r % kFanout].push_back(rows_op(dst + r * c, 0, src, 0, 2 * valid, 1));
+            }
+            if (W * c > n)
+                q->lists[i % kFanout].push_back(
+                    CeOp{CeOp::kMemset, dst + n, 0, nullptr, 0, (size_t)(2 * (W * c - n)), 0});
         }
-        if (W * c > n)
-            q->lists[i % kFanout].push_back(
-                CeOp{CeOp::kMemset, dst + n, 0, nullptr, 0, (size_t)(2 * (W * c - n)), 0});
-    }
-    cudaError_t e = fork(p, stream);
-    if (e != cudaSuccess) return e;
-    e = issue_all(p, q, max_pitch);
-    cudaError_t j = join(p, stream);
-    return e != cudaSuccess ? e : j;
+    });
 }
 
 // Stage the chunks [j0, j1) (chunk i*W + r: rank r's rows of param i) from
@@ -298,41 +384,44 @@ cudaError_t ce_ag_gather(tide_plan* p, const void* const* shards, void* const* p
 // consecutive ranks, so each (k, param) pair takes one 2-D copy plus at most
 // one 1-D copy for a partial chunk.
 cudaError_t ce_slot_stage(tide_plan* p, const void* const* grads, void* const* slots,
-                          cudaStream_t caller, int64_t j0, int64_t j1) {
+                          cudaStream_t caller, int64_t j0, int64_t j1, bool record) {
     const int64_t W = p->world, P = p->n_params, Ns = p->shard_numel;
     if (j1 < 0) j1 = P * W;
     if (j1 <= j0) return cudaSuccess;
-    const size_t max_pitch = device_max_pitch(p->device);
-    CeIssuer* q = issuer(p);
-    if (q == nullptr) return cudaErrorMemoryAllocation;
-    for (auto& l : q->lists) l.clear();
-    for (int64_t k = 0; k < W; ++k) {
-        auto& l = q->lists[k % kFanout];  // one source rank per stream at a time
-        uint16_t* slot = static_cast<uint16_t*>(slots[k]);
-        for (int64_t i = j0 / W; i <= (j1 - 1) / W; ++i) {
-            const int64_t c = p->chunk[i], n = p->numel[i];
-            if (c == 0 || n == 0) continue;
-            const int64_t r0 = std::max<int64_t>(0, j0 - i * W), r1 = std::min<int64_t>(W, j1 - i * W);
-            const uint16_t* g = static_cast<const uint16_t*>(grads[k * P + i]);
-            uint16_t* dst = slot + p->offset[i];
-            const int64_t full = std::min(W, n / c);  // ranks [0, full) hold whole chunks
-            const int64_t fr1 = std::min(full, r1);
-            if (fr1 > r0) l.push_back(rows_op(dst + r0 * Ns, 2 * Ns, g + r0 * c, 2 * c, 2 * c, fr1 - r0));
-            const int64_t rem = n - full * c;       // rank `full` holds a partial chunk
-            if (rem > 0 && full < W && full >= r0 && full < r1)
-                l.push_back(rows_op(dst + full * Ns, 0, g + full * c, 0, 2 * rem, 1));
-        }
+    std::vector<const void*> key;
+    if (record) {
+        key.reserve((size_t)(W * P + W));
+        for (int64_t j = 0; j < W * P; ++j) key.push_back(grads[j]);
+        for (int64_t k = 0; k < W; ++k) key.push_back(slots[k]);
     }
-    cudaError_t e = fork(p, caller);
-    if (e != cudaSuccess) return e;
-    e = issue_all(p, q, max_pitch);
-    cudaError_t je = join(p, caller);
-    return e != cudaSuccess ? e : je;
+    return run_call(p, caller, kCallStage, j0, j1, std::move(key), record, [&](CeIssuer* q) {
+        for (int64_t k = 0; k < W; ++k) {
+            auto& l = q->lists[k % kFanout];  // one source rank per stream at a time
+            uint16_t* slot = static_cast<uint16_t*>(slots[k]);
+            for (int64_t i = j0 / W; i <= (j1 - 1) / W; ++i) {
+                const int64_t c = p->chunk[i], n = p->numel[i];
+                if (c == 0 || n == 0) continue;
+                const int64_t r0 = std::max<int64_t>(0, j0 - i * W), r1 = std::min<int64_t>(W, j1 - i * W);
+                const uint16_t* g = static_cast<const uint16_t*>(grads[k * P + i]);
+                uint16_t* dst = slot + p->offset[i];
+                const int64_t full = std::min(W, n / c);  // ranks [0, full) hold whole chunks
+                const int64_t fr1 = std::min(full, r1);
+                if (fr1 > r0) l.push_back(rows_op(dst + r0 * Ns, 2 * Ns, g + r0 * c, 2 * c, 2 * c, fr1 - r0));
+                const int64_t rem = n - full * c;       // rank `full` holds a partial chunk
+                if (rem > 0 && full < W && full >= r0 && full < r1)
+                    l.push_back(rows_op(dst + full * Ns, 0, g + full * c, 0, 2 * rem, 1));
+            }
+        }
+    });
 }
 
 void ce_release(tide_plan* p) {
     delete p->ce_issuer;
     p->ce_issuer = nullptr;
+    for (auto& g : p->ce_graphs) cudaGraphExecDestroy(g.exec);
+    p->ce_graphs.clear();
+    if (p->ce_capture_stream != nullptr) cudaStreamDestroy(p->ce_capture_stream);
+    p->ce_capture_stream = nullptr;
 }
 
 }  // namespace tide

@@ -53,6 +53,15 @@
  *     are issued by the calling thread and 3 host threads that the plan starts
  *     on its first copy-engine call (they sleep between calls and are joined
  *     by tide_plan_destroy); the call returns once every copy is enqueued.
+ *   - A TIDE_ENGINE_CE placement (tide_ag_place, tide_ag_gather_place) made
+ *     outside any stream capture records its copies once as a CUDA graph (on a
+ *     private stream of the plan) the first time its set of buffer addresses
+ *     is seen, and then launches that graph on the call's stream, for this
+ *     call and every later one with the same addresses: one graph launch
+ *     instead of one host call per copy.  The plan keeps the 4 most recently
+ *     used recordings and frees them in tide_plan_destroy.  A call on a stream
+ *     that is being captured issues its copies directly into that capture.
+ *     Slot-Reuse staging on the copy engines always issues its copies directly.
  */
 #ifndef TIDE_H
 #define TIDE_H

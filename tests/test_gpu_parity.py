@@ -517,11 +517,15 @@ def test_cuda_graph_capture_and_replay(group):
     slots = [torch.empty(n, dtype=torch.bfloat16, device="cuda") for _ in range(W)]
     ag = to_dev(synth.ag_host(group, L.Ns, seed=95).reshape(-1))
     params = padded_params(plan, group)
+    params_ce = padded_params(plan, group)
     cs = torch.cuda.Stream()
     side = torch.cuda.Stream()
 
     def step(stream):
         plan.ag_place(ag, params, stream=stream)
+        # (uncaptured, the copy-engine call records and replays its own graph; inside the
+        # capture it issues its copies into the caller's capture)
+        plan.ag_place(ag, params_ce, engine=T.TIDE_ENGINE_CE, stream=stream)
         plan.rs_reduce(dev, out, stream=stream)
         plan.rs_reduce_pipelined(dev, out_pipe, slots, min(2, W), cs, stream=stream)
 
@@ -546,8 +550,9 @@ def test_cuda_graph_capture_and_replay(group):
         ref = oracle.rs_reduce(W, group.shapes, grads, 1).view(np.uint32)
         assert np.array_equal(f32_bits(out), ref)
         assert np.array_equal(f32_bits(out_pipe), ref)
-        for p, r in zip(params, oracle.ag_copyout(W, group.shapes, ag_bits)):
+        for p, pc, r in zip(params, params_ce, oracle.ag_copyout(W, group.shapes, ag_bits)):
             assert np.array_equal(bits_of(p), r)
+            assert np.array_equal(bits_of(pc), r)
     plan.check()
 
 
@@ -630,3 +635,45 @@ def test_short_lived_ctas_give_the_same_bits(group):
     if plan.n_tiles:
         assert plan.last_launch()[1] == plan.n_tiles
         assert plan.launch_ctas(T.K_STAGE, 0) == plan.n_tiles * W
+
+
+@pytest.mark.parametrize("group", [configs.tiny(), mini_wan(), configs.qwen3moe(4)],
+                         ids=lambda g: f"{g.name}_w{g.world}")
+def test_copy_engine_calls_replay_recorded_graphs(group):
+    """A copy-engine placement records its copies as a graph the first time a set of buffers
+    is used and replays it when the same buffers come back.  Placement and gather placement
+    give the oracle's bits on the recording call, on replays (outputs poisoned in between),
+    with a second set of buffers, and back on the first; Slot-Reuse staging (issued
+    directly) likewise on repeated calls."""
+    W = group.world
+    L = oracle.layout(W, group.shapes)
+    plan = T.Plan(group.shapes, W)
+    ag_bits = poison_pads(synth.ag_host(group, L.Ns, seed=93).reshape(-1), group, L)
+    ag = to_dev(ag_bits)
+    ref = oracle.ag_copyout(W, group.shapes, ag_bits)
+    sets = [padded_params(plan, group), padded_params(plan, group)]
+    rows = ag_bits.reshape(W, L.Ns)
+    shards = [to_dev(rows[r]) for r in range(W)]
+    for params in (sets[0], sets[0], sets[1], sets[0]):
+        for fn in (lambda p: plan.ag_place(ag, p, engine=T.TIDE_ENGINE_CE),
+                   lambda p: plan.ag_gather_place(shards, p, engine=T.TIDE_ENGINE_CE)):
+            for t in params:
+                t.view(torch.int16).fill_(0x7777)
+            fn(params)
+            torch.cuda.synchronize()
+            for t, r in zip(params, ref):
+                assert np.array_equal(bits_of(t), r)
+    grads = synth.grads_host(group, seed=94)
+    dev = grads_to_dev(group, grads)
+    n = W * L.Ns
+    slot_sets = [[torch.empty(n, dtype=torch.bfloat16, device="cuda") for _ in range(W)] for _ in range(2)]
+    for slots in (slot_sets[0], slot_sets[0], slot_sets[1], slot_sets[0]):
+        for sl in slots:
+            sl.view(torch.int16).fill_(-1)
+        plan.rs_stage(dev, slots, engine=T.TIDE_ENGINE_CE)
+        torch.cuda.synchronize()
+        for k in range(W):
+            exp = np.full(n, 0xFFFF, dtype=np.uint16)
+            oracle.slot_stage(W, group.shapes, grads[k], exp)
+            assert np.array_equal(bits_of(slots[k]), exp)
+    plan.check()
