@@ -123,7 +123,8 @@ def ncu_traffic(kernel: str, sources, alg_read: int, alg_write: int):
 
     profiles/ncu_traffic.txt holds, per kernel, one ncu capture on the sweep_w8 group (inputs
     larger than L2, under 1 GB on the device): dram__bytes_read.sum, dram__bytes_write.sum,
-    lts__t_sectors_op_write.sum x 32 B, and that launch's algorithmic read and write bytes.
+    the bytes its SMs wrote into L2 ((lts__t_sectors_op_write.sum - the ltcfabric share) x
+    32 B), and that launch's algorithmic read and write bytes.
     Reads scale by read/alg_read.  The small case ends with part of its output still dirty in
     L2 (not yet in dram__bytes_write), so writes scale by the bytes the kernel wrote into L2,
     all of which reach DRAM.  Returns (traffic bytes or None, source note).  None when the
