@@ -34,3 +34,22 @@ def run_gloo_reduce_scatter(packed, tmp_dir):
         np.save(os.path.join(tmp_dir, f"packed_{k}.npy"), p)
     mp.spawn(_rs_worker, args=(world, free_port(), str(tmp_dir)), nprocs=world, join=True)
     return [np.load(os.path.join(tmp_dir, f"shard_{k}.npy")) for k in range(world)]
+
+
+def run_procs(target, n, args):
+    """Run target(p, *args(port)) in n spawned processes (p = 0..n-1) and require each to exit
+    0 within 300 s."""
+    import torch
+    ctx = torch.multiprocessing.get_context("spawn")
+    port = free_port()
+    procs = [ctx.Process(target=target, args=(p, *args(port))) for p in range(n)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=300)
+    alive = [p for p in procs if p.is_alive()]
+    for p in alive:
+        p.terminate()
+        p.join(timeout=30)
+    assert not alive, "a process did not finish"
+    assert [p.exitcode for p in procs] == [0] * n

@@ -21,7 +21,7 @@ import oracle
 import synth
 from synth import configs
 
-from _dist_helpers import free_port
+from _dist_helpers import free_port, run_procs
 
 pytestmark = pytest.mark.gpu
 
@@ -29,25 +29,9 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SHAPES = ((37, 16), (1000,), (7, 3), (5, 130), (64, 64), (8 * 4 + 3, 40), (0, 5), (256, 256))
 
 
-def _run(target, n, args):
-    ctx = torch.multiprocessing.get_context("spawn")
-    port = free_port()
-    procs = [ctx.Process(target=target, args=(p, *args(port))) for p in range(n)]
-    for p in procs:
-        p.start()
-    for p in procs:
-        p.join(timeout=300)
-    alive = [p for p in procs if p.is_alive()]
-    for p in alive:
-        p.terminate()
-        p.join(timeout=30)
-    assert not alive, "a process did not finish"
-    assert [p.exitcode for p in procs] == [0] * n
-
-
 def test_ipc_export_open_read_write(tmp_path):
     from _exchange_workers import ipc_worker
-    _run(ipc_worker, 2, lambda port: (port, str(tmp_path)))
+    run_procs(ipc_worker, 2, lambda port: (port, str(tmp_path)))
     assert np.array_equal(np.load(tmp_path / "peer_read.npy"), np.arange(1000, 1016, dtype=np.int32))
     after = np.load(tmp_path / "owner_after.npy")
     want = np.arange(2048, dtype=np.int32)
@@ -59,7 +43,7 @@ def test_ipc_export_open_read_write(tmp_path):
 def test_exchange_over_ipc_matches_oracle(world, n_procs, tmp_path):
     from _exchange_workers import exchange_worker
     seed = 74
-    _run(exchange_worker, n_procs,
+    run_procs(exchange_worker, n_procs,
          lambda port: (n_procs, port, SHAPES, world, seed, str(tmp_path)))
     group = configs.Group("exchange", world, SHAPES)
     L = oracle.layout(world, group.shapes)
