@@ -74,11 +74,11 @@ __global__ void __launch_bounds__(kThreads) ag_place_kernel(const AgParams a) {
 struct StageParams {
     const tide_tile_t* tiles;
     int64_t n_tiles;
-    const void* const* grad_tab;  // [W*P], k*P + i
-    const void* const* slot_tab;  // [W]
+    const void* const* grad_tab;  // [world*P], k*P + i
+    const void* const* slot_tab;  // [world]
     const int64_t* numel;         // [P] unpadded numel
     int64_t slot_numel;
-    int32_t world;
+    int32_t world;                // source ranks in the tables: W, or 1 for one rank's gradients
     int32_t n_params;
     int32_t* err;
 };
@@ -170,7 +170,7 @@ cudaError_t launch_ag_gather(const tide_plan* p, const void* const* d_shard_tab,
 
 cudaError_t launch_slot_stage(const tide_plan* p, const void* const* d_grad_tab,
                               const void* const* d_slot_tab, int64_t slot_numel, int grid,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, int32_t sources) {
     if (p->tiles.empty() || grid <= 0) return cudaSuccess;
     StageParams a;
     a.tiles = p->d_tiles;
@@ -179,7 +179,7 @@ cudaError_t launch_slot_stage(const tide_plan* p, const void* const* d_grad_tab,
     a.slot_tab = d_slot_tab;
     a.numel = p->d_numel;
     a.slot_numel = slot_numel;
-    a.world = p->world;
+    a.world = sources;  // the kernel's source ranks: its units are (tile, source) pairs
     a.n_params = p->n_params;
     a.err = p->d_err;
     (void)cudaGetLastError();  // drop an error left by an earlier failed runtime call

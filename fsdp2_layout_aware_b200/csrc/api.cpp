@@ -215,7 +215,8 @@ tide_status_t stage_impl(tide_plan* p, const void* const* grads, void* const* sl
         if (st != TIDE_OK) return st;
         p->last_kernel = K_STAGE;
         p->last_ctas = grid_for(p, K_STAGE, max_ctas);
-        e = tide::launch_slot_stage(p, p->grad_tab.dev, p->slot_tab.dev, slot_numel, p->last_ctas, s);
+        e = tide::launch_slot_stage(p, p->grad_tab.dev, p->slot_tab.dev, slot_numel, p->last_ctas, s,
+                                    p->world);
     }
     return e == cudaSuccess ? TIDE_OK : TIDE_ERR_CUDA;
 }
@@ -224,10 +225,15 @@ tide_status_t reduce_slots_impl(tide_plan* p, void* const* slots, int64_t slot_n
                                 int64_t out_numel, int32_t scale_mode, int32_t order,
                                 int32_t max_ctas, cudaStream_t s) {
     if (p->tiles.empty()) return TIDE_OK;
-    tide_status_t st = sync_table(p->slot_tab, const_cast<const void* const*>(slots), p->world, s);
+    // A one-rank plan's tiles address its shard from 0; its rows of every slot start at
+    // rank * Ns, so the kernel gets each slot from there on.
+    const int64_t row0 = p->rank >= 0 ? (int64_t)p->rank * p->shard_numel : 0;
+    std::vector<const void*> from((size_t)p->world);
+    for (int64_t k = 0; k < p->world; ++k) from[k] = static_cast<const uint16_t*>(slots[k]) + row0;
+    tide_status_t st = sync_table(p->slot_tab, from.data(), p->world, s);
     if (st != TIDE_OK) return st;
-    cudaError_t e = launch_reduce(p, p->slot_tab, true, slot_numel, out, out_numel, scale_mode, order,
-                                  max_ctas, s);
+    cudaError_t e = launch_reduce(p, p->slot_tab, true, slot_numel - row0, out, out_numel, scale_mode,
+                                  order, max_ctas, s);
     return e == cudaSuccess ? TIDE_OK : TIDE_ERR_CUDA;
 }
 
@@ -395,6 +401,47 @@ extern "C" tide_status_t tide_rs_stage(const tide_plan_t* cplan, const void* con
     return stage_impl(p, grads, slots, slot_numel, engine, max_ctas, static_cast<cudaStream_t>(stream));
 }
 
+extern "C" tide_status_t tide_rs_stage_one(const tide_plan_t* cplan, const void* const* grads,
+                                           const int64_t* grad_numel, void* slot, int64_t slot_numel,
+                                           int32_t engine, int32_t max_ctas, void* stream) {
+    ApiRange range("tide_rs_stage_one");
+    tide_plan* p = const_cast<tide_plan*>(cplan);
+    tide_status_t st = check_plan(p);
+    if (st != TIDE_OK) return st;
+    if ((st = all_ranks(p)) != TIDE_OK) return st;
+    if ((st = check_enums(p, engine, max_ctas)) != TIDE_OK) return st;
+    const int64_t W = p->world, P = p->n_params;
+    std::vector<Span> spans;
+    spans.reserve((size_t)P + 1);
+    if (P > 0 && (grads == nullptr || grad_numel == nullptr)) return TIDE_ERR_INVALID_ARG;
+    for (int64_t i = 0; i < P; ++i) {
+        if ((st = check_buf(grads[i], grad_numel[i], p->numel[i], 2)) != TIDE_OK) return st;
+        add_span(spans, grads[i], 2 * p->numel[i], false);
+    }
+    if ((st = check_buf(slot, slot_numel, W * p->shard_numel, 2)) != TIDE_OK) return st;
+    add_span(spans, slot, 2 * W * p->shard_numel, true);
+    if (overlaps(spans)) return TIDE_ERR_INVALID_ARG;
+    if ((st = launchable(p)) != TIDE_OK) return st;
+    if (p->tiles.empty()) return TIDE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    void* const slots[1] = {slot};
+    cudaError_t e;
+    if (engine == TIDE_ENGINE_CE) {
+        p->last_kernel = -1;
+        p->last_ctas = 0;
+        e = tide::ce_slot_stage(p, grads, slots, s, 0, -1, false, true);
+    } else {
+        if ((st = sync_table(p->grad_tab, grads, P, s)) != TIDE_OK) return st;
+        if ((st = sync_table(p->slot_tab, const_cast<const void* const*>(slots), 1, s)) != TIDE_OK)
+            return st;
+        p->last_kernel = K_STAGE;
+        // one source rank: one unit per tile
+        p->last_ctas = (int)std::min<int64_t>(grid_for(p, K_STAGE, max_ctas), (int64_t)p->tiles.size());
+        e = tide::launch_slot_stage(p, p->grad_tab.dev, p->slot_tab.dev, slot_numel, p->last_ctas, s, 1);
+    }
+    return e == cudaSuccess ? TIDE_OK : TIDE_ERR_CUDA;
+}
+
 extern "C" tide_status_t tide_rs_reduce_slots(const tide_plan_t* cplan, const void* const* slots,
                                               int64_t slot_numel, float* out, int64_t out_numel,
                                               int32_t scale_mode, int32_t order, int32_t max_ctas,
@@ -403,10 +450,9 @@ extern "C" tide_status_t tide_rs_reduce_slots(const tide_plan_t* cplan, const vo
     tide_plan* p = const_cast<tide_plan*>(cplan);
     tide_status_t st = check_plan(p);
     if (st != TIDE_OK) return st;
-    if ((st = all_ranks(p)) != TIDE_OK) return st;
     if ((st = check_enums(p, TIDE_ENGINE_SM, max_ctas)) != TIDE_OK) return st;
     if ((st = check_reduce_modes(scale_mode, order)) != TIDE_OK) return st;
-    const int64_t n_out = (int64_t)p->world * p->shard_numel;
+    const int64_t n_out = (p->rank >= 0 ? 1 : (int64_t)p->world) * p->shard_numel;
     std::vector<Span> spans;
     spans.reserve((size_t)p->world * (p->n_params + 1) + p->n_params + 2);
     if ((st = check_slots(p, const_cast<void* const*>(slots), slot_numel, spans)) != TIDE_OK) return st;

@@ -384,21 +384,24 @@ cudaError_t ce_ag_gather(tide_plan* p, const void* const* shards, void* const* p
 // consecutive ranks, so each (k, param) pair takes one 2-D copy plus at most
 // one 1-D copy for a partial chunk.
 cudaError_t ce_slot_stage(tide_plan* p, const void* const* grads, void* const* slots,
-                          cudaStream_t caller, int64_t j0, int64_t j1, bool record) {
+                          cudaStream_t caller, int64_t j0, int64_t j1, bool record, bool one_source) {
     const int64_t W = p->world, P = p->n_params, Ns = p->shard_numel;
+    const int64_t sources = one_source ? 1 : W;
     if (j1 < 0) j1 = P * W;
     if (j1 <= j0) return cudaSuccess;
     std::vector<const void*> key;
     if (record) {
-        key.reserve((size_t)(W * P + W));
-        for (int64_t j = 0; j < W * P; ++j) key.push_back(grads[j]);
-        for (int64_t k = 0; k < W; ++k) key.push_back(slots[k]);
+        key.reserve((size_t)(sources * P + sources + 1));
+        for (int64_t j = 0; j < sources * P; ++j) key.push_back(grads[j]);
+        for (int64_t k = 0; k < sources; ++k) key.push_back(slots[k]);
+        key.push_back(reinterpret_cast<const void*>(sources));
     }
     return run_call(p, caller, kCallStage, j0, j1, std::move(key), record, [&](CeIssuer* q) {
-        for (int64_t k = 0; k < W; ++k) {
-            auto& l = q->lists[k % kFanout];  // one source rank per stream at a time
+        for (int64_t k = 0; k < sources; ++k) {
             uint16_t* slot = static_cast<uint16_t*>(slots[k]);
             for (int64_t i = j0 / W; i <= (j1 - 1) / W; ++i) {
+                // one source rank per stream at a time; one rank's params spread over the streams
+                auto& l = q->lists[(one_source ? i : k) % kFanout];
                 const int64_t c = p->chunk[i], n = p->numel[i];
                 if (c == 0 || n == 0) continue;
                 const int64_t r0 = std::max<int64_t>(0, j0 - i * W), r1 = std::min<int64_t>(W, j1 - i * W);

@@ -94,9 +94,11 @@ cudaError_t launch_ag_place(const tide_plan* p, const uint16_t* ag, int64_t ag_n
 // Placement from W per-rank shards (d_shard_tab[r]: rank r's [Ns] shard).
 cudaError_t launch_ag_gather(const tide_plan* p, const void* const* d_shard_tab, int64_t shard_numel,
                              const void* const* d_param_tab, int grid, cudaStream_t stream);
+// Stages `sources` source ranks: W (d_grad_tab [W*P], d_slot_tab [W]) or 1 (one
+// rank's gradients, d_grad_tab [P], into the one slot d_slot_tab[0]).
 cudaError_t launch_slot_stage(const tide_plan* p, const void* const* d_grad_tab,
                               const void* const* d_slot_tab, int64_t slot_numel, int grid,
-                              cudaStream_t stream);
+                              cudaStream_t stream, int32_t sources);
 
 // Copy-engine variants (no kernels).
 cudaError_t ce_ag_place(tide_plan* p, const uint16_t* ag, void* const* params,
@@ -107,9 +109,11 @@ cudaError_t ce_ag_gather(tide_plan* p, const void* const* shards, void* const* p
 // Stages the chunks [j0, j1) (numbered i*W + r as in chunk_tile_begin; j1 < 0:
 // all) from every source rank k into slot k.  The copies are issued directly
 // (`record` = false): a recorded graph of them measured slower (Wan2.2 group:
-// 3.55 against 4.07 TB/s; within 2 % elsewhere).
+// 3.55 against 4.07 TB/s; within 2 % elsewhere).  one_source: grads holds one
+// rank's P gradients and slots one slot, which receives them.
 cudaError_t ce_slot_stage(tide_plan* p, const void* const* grads, void* const* slots,
-                          cudaStream_t stream, int64_t j0 = 0, int64_t j1 = -1, bool record = false);
+                          cudaStream_t stream, int64_t j0 = 0, int64_t j1 = -1, bool record = false,
+                          bool one_source = false);
 // Stops and frees the plan's copy-issuing threads and recorded graphs.
 void ce_release(tide_plan* p);
 

@@ -102,18 +102,50 @@ def shard_table(layout: ArenaLayout, world: int, n_procs: int, shard_base) -> li
     return out
 
 
+_MAPPED = {}   # (handle bytes, device) -> [base, users]: one mapping per peer allocation
+
+
+def open_shared(handle: bytes, device: int):
+    """tide_ipc_open, once per (allocation, device) in this process.  CUDA maps an IPC handle
+    at most once per process and device, and the caching allocator may put buffers of several
+    owners' objects (arenas of different parameter groups) in one allocation: later users of
+    the same handle get the first mapping, counted."""
+    key = (bytes(handle), int(device))
+    ent = _MAPPED.get(key)
+    if ent is not None:
+        ent[1] += 1
+        return T.TIDE_OK, ent[0]
+    st, base = T.tide_ipc_open(handle, device)
+    if st == T.TIDE_OK:
+        _MAPPED[key] = [base, 1]
+    return st, base
+
+
+def close_shared(base: int, device: int) -> int:
+    """Drop one user of a mapping made by open_shared; unmap it when none is left."""
+    for key, ent in _MAPPED.items():
+        if ent[0] == base and key[1] == device:
+            ent[1] -= 1
+            if ent[1] > 0:
+                return T.TIDE_OK
+            del _MAPPED[key]
+            break
+    return T.tide_ipc_close(base, device)
+
+
 class PeerMaps:
     """The other processes' arenas mapped into this one, on this process's device.
 
     exports[p] is process p's {name: (handle bytes, byte offset)} as tide_ipc_export gave it;
     `local` maps name -> this process's own address.  An allocation exported under several
-    names is opened once.  opener/closer default to the library's IPC calls (tests pass fakes).
+    names is opened once.  opener/closer default to open_shared/close_shared (tests pass
+    fakes).
     """
 
     def __init__(self, exports, me: int, device: int, local: dict, opener=None, closer=None):
         self.device = device
-        self._close = closer or T.tide_ipc_close
-        open_fn = opener or T.tide_ipc_open
+        self._close = closer or close_shared
+        open_fn = opener or open_shared
         self._bases = {}
         self.addr = {}
         try:

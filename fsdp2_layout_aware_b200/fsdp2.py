@@ -1,0 +1,271 @@
+"""TIDE's collectives inside FSDP2's own ``fully_shard``, one process per rank.
+
+Around its collectives stock FSDP2 runs two layout conversions (weekinpapers.com, Abstract;
+kongchang.com, "The Root of FSDP2 Communication Overhead"):
+  * all-gather: each rank copies its bf16 shard into row r of a flat [W][Ns] buffer, the
+    buffer is all-gathered, and a copy-out (``fsdp::split_with_sizes_copy``) splits it into
+    the unsharded parameters;
+  * reduce-scatter: each rank packs its bf16 gradients into a flat fp32 [W][Ns] buffer
+    (``fsdp::chunk_cat``), which is reduce-scattered.
+TIDE folds the copy-out into the all-gather's addressing and replaces the fp32 pack with
+gradients read where they are, staged bf16 into the vacated all-gather slot under Slot-Reuse
+(same Abstract; kongchang.com, "TIDE's Design Approach").  ``fully_shard_tide`` applies
+``fully_shard`` and then, for the module's parameter group:
+  * ``TideAllGather`` (``set_custom_all_gather``): the [W][Ns] buffer FSDP2 asks for is a
+    persistent bf16 arena of this rank, mapped into every other rank through CUDA IPC.
+    FSDP2's own copy-in writes this rank's row; the collective itself only waits until every
+    rank's row is in place.  FSDP2's copy-out on that arena becomes ``tide_ag_gather_place``:
+    row k read from rank k's arena and placed straight into the unsharded parameters, pad
+    rows zeroed.  No rank ever holds the gathered [W][Ns] buffer.
+  * ``TideReduceScatter`` (``set_custom_reduce_scatter``): the fp32 [W][Ns] input FSDP2 asks
+    for is one element expanded to that shape, never written.  FSDP2's pack on it becomes
+    ``tide_rs_stage_one``: this rank's bf16 gradients staged into its arena (the all-gather
+    slot, free once every rank has placed from it).  The collective is
+    ``tide_rs_reduce_slots`` with this rank's one-rank plan: its fp32 shard reduced in rank
+    order from rows r of every rank's arena, x fl32(1/W) for FSDP2's average.
+The copy-out and the pack are replaced through their dispatcher entries: on a buffer of a
+TIDE group the library call runs; on any other buffer FSDP2's own implementation does.
+
+Ranks meet only at host barriers of the process group (synchronize, then barrier), placed so
+that no rank writes its arena while another may still read it: before a placement (every
+row is in), after it (before anyone stages gradients over its row), before a reduction
+(every rank staged) and after it (before the next copy-in).  The parameter group must have
+bf16 compute parameters and fp32 reduction (the mixed-precision policy set here); every
+collective is synchronous.
+"""
+from __future__ import annotations
+
+import math
+import threading
+import warnings
+
+from . import exchange as X
+from . import tide as T
+
+_AG = {}          # data_ptr of a group's arena -> TideGroup
+_RS = {}          # data_ptr of a group's expanded reduce-scatter input -> TideGroup
+_LOCK = threading.Lock()
+_INSTALLED = False
+_LIB = None
+
+
+class TideGroup:
+    """The TIDE state of one FSDP2 parameter group on this rank.
+
+    shapes: the group's unsharded parameter shapes in FSDP2's order.  Every rank builds its
+    groups in the same order (the handle exchange is a collective).
+    """
+
+    def __init__(self, shapes, group=None, device=None, engine: int = T.TIDE_ENGINE_SM,
+                 order: int = T.TIDE_ORDER_RANK):
+        import torch
+        import torch.distributed as dist
+
+        self.group = group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        if self.world < 2:
+            raise ValueError("TIDE's collectives need at least 2 ranks")
+        self.device = torch.device("cuda", torch.cuda.current_device()) if device is None \
+            else torch.device(device)
+        self.engine, self.order = engine, order
+        W, r = self.world, self.rank
+        self.shapes = [tuple(int(d) for d in s) for s in shapes]
+        self.plan = T.Plan(self.shapes, W, device=self.device)             # placement, staging
+        self.rank_plan = T.Plan(self.shapes, W, device=self.device, rank=r)  # this rank's shard
+        Ns = self.plan.shard_numel
+        self.shard_numel = Ns
+        self.chunks = [self.plan.query(i)["chunk_numel"] for i in range(len(self.shapes))]
+        self.arena = torch.zeros(W * Ns, dtype=torch.bfloat16, device=self.device)
+        self.rs_input = torch.zeros(1, dtype=torch.float32, device=self.device)
+        torch.cuda.synchronize(self.device)
+        exports = X.all_exports(X.export({"arena": self.arena}), group)
+        self.peers = X.PeerMaps(exports, r, self.device.index, {"arena": self.arena.data_ptr()})
+        bases = self.peers.bases("arena", W)
+        # row k of rank k's arena is rank k's shard; the slots are the whole arenas
+        self.shard_table = T.PointerTable([b + 2 * k * Ns for k, b in enumerate(bases)], [Ns] * W,
+                                          keep=[self.arena])
+        self.slot_table = T.PointerTable(list(bases), [W * Ns] * W, keep=[self.arena])
+        with _LOCK:
+            _AG[self.arena.data_ptr()] = self
+            _RS[self.rs_input.data_ptr()] = self
+        self.placements = 0
+        self.reductions = 0
+
+    def meet(self) -> None:
+        import torch
+        import torch.distributed as dist
+        torch.cuda.synchronize(self.device)
+        dist.barrier(self.group)
+
+    def place(self, out) -> None:
+        """FSDP2's copy-out: every rank's row into the unsharded parameters (TIDE-AG)."""
+        if len(out) != len(self.shapes):
+            raise ValueError("copy-out outputs do not match the group's parameters")
+        for t, c in zip(out, self.chunks):
+            if t.numel() != self.world * c or not t.is_contiguous():
+                raise ValueError("copy-out output is not a parameter's padded storage")
+        self.plan.ag_gather_place(self.shard_table, T.TensorTable(list(out)), engine=self.engine)
+        self.meet()                                   # every rank has read every row
+        self.placements += 1
+
+    def stage(self, grads) -> None:
+        """FSDP2's pack: this rank's bf16 gradients into its arena (Slot-Reuse phase 1)."""
+        import torch
+        if len(grads) != len(self.shapes):
+            raise ValueError("gradients do not match the group's parameters")
+        for g, s in zip(grads, self.shapes):
+            if g.dtype != torch.bfloat16 or tuple(g.shape) != s or not g.is_contiguous():
+                raise ValueError("TIDE staging takes the parameters' contiguous bf16 gradients")
+        self.plan.rs_stage_one(T.TensorTable(list(grads)), self.arena, engine=self.engine)
+
+    def reduce(self, out, op) -> None:
+        """The reduce-scatter: this rank's fp32 shard from rows r of every arena (TIDE-RS)."""
+        import torch
+        import torch.distributed as dist
+        if out.dtype != torch.float32 or out.numel() != self.shard_numel or not out.is_contiguous():
+            raise ValueError("reduce-scatter output is not this rank's fp32 shard")
+        if op == dist.ReduceOp.AVG:
+            scale = T.TIDE_SCALE_INV_WORLD
+        elif op == dist.ReduceOp.SUM:
+            scale = T.TIDE_SCALE_NONE
+        else:
+            raise ValueError(f"reduce op {op} is not a sum or an average")
+        self.meet()                                   # every rank's gradients are staged
+        self.rank_plan.rs_reduce_slots(self.slot_table, out, scale_mode=scale, order=self.order)
+        self.meet()                                   # nobody copies in over a row still read
+        self.reductions += 1
+
+    def close(self) -> None:
+        """Unmap the peers' arenas once no rank can still read them (a collective)."""
+        if self.peers is None:
+            return
+        self.meet()
+        with _LOCK:
+            _AG.pop(self.arena.data_ptr(), None)
+            _RS.pop(self.rs_input.data_ptr(), None)
+        self.peers.close()
+        self.meet()
+        self.peers = None
+
+
+def _comm_classes():
+    from torch.distributed.fsdp._fully_shard._fsdp_api import AllGather, ReduceScatter
+
+    class TideAllGather(AllGather):
+        """FSDP2's all-gather for a TIDE group: the buffer is the group's arena; the call
+        waits for every rank's row (the placement runs in FSDP2's copy-out)."""
+
+        def __init__(self, tg: TideGroup):
+            self.tg = tg
+
+        def allocate(self, size, *, dtype, device):
+            import torch
+            if dtype != torch.bfloat16 or math.prod(int(s) for s in size) != self.tg.arena.numel():
+                raise ValueError("all-gather buffer is not the group's bf16 [W][Ns] arena")
+            return self.tg.arena
+
+        def __call__(self, output_tensor, input_tensor, group, async_op=False):
+            if output_tensor.data_ptr() != self.tg.arena.data_ptr():
+                raise ValueError("all-gather output is not the group's arena")
+            self.tg.meet()                            # every rank's row is in its arena
+            return None
+
+    class TideReduceScatter(ReduceScatter):
+        """FSDP2's reduce-scatter for a TIDE group: no fp32 input buffer; the reduction
+        reads every rank's staged arena."""
+
+        def __init__(self, tg: TideGroup):
+            self.tg = tg
+
+        def allocate(self, size, *, dtype, device):
+            import torch
+            n = math.prod(int(s) for s in size)
+            if dtype != torch.float32:
+                raise ValueError("TIDE's reduce-scatter reduces into fp32")
+            if n == self.tg.world * self.tg.shard_numel:
+                return self.tg.rs_input.expand(n)     # FSDP2's packed input: never materialized
+            if n == self.tg.shard_numel:
+                return torch.empty(n, dtype=torch.float32, device=self.tg.device)
+            raise ValueError("unexpected reduce-scatter buffer size")
+
+        def __call__(self, output_tensor, input_tensor, group, op, async_op=False):
+            if input_tensor.data_ptr() != self.tg.rs_input.data_ptr():
+                raise ValueError("reduce-scatter input is not the group's")
+            self.tg.reduce(output_tensor, op)
+            return None
+
+    return TideAllGather, TideReduceScatter
+
+
+def _install() -> None:
+    """Route FSDP2's copy-out and pack to the library for TIDE groups' buffers."""
+    global _INSTALLED, _LIB
+    if _INSTALLED:
+        return
+    import torch
+    from torch.distributed.fsdp._fully_shard import _fsdp_collectives as C
+
+    stock_split, stock_cat = C.split_with_sizes_copy, C.chunk_cat
+
+    def split_with_sizes_copy(all_gather_output, all_gather_input_split_sizes, dim=0, *, out):
+        tg = _AG.get(all_gather_output.data_ptr())
+        if tg is None:
+            return stock_split(all_gather_output, all_gather_input_split_sizes, dim, out=out)
+        if dim != 1 or list(all_gather_input_split_sizes) != tg.chunks:
+            raise ValueError("copy-out of a TIDE group with another layout")
+        tg.place(out)
+
+    def chunk_cat(tensors, dim, num_chunks, out):
+        tg = _RS.get(out.data_ptr())
+        if tg is None:
+            return stock_cat(tensors, dim, num_chunks, out)
+        if dim != 0 or num_chunks != tg.world:
+            raise ValueError("pack of a TIDE group with another layout")
+        tg.stage(tensors)
+
+    lib = torch.library.Library("fsdp", "IMPL")  # noqa: TOR901
+    with warnings.catch_warnings():
+        warnings.simplefilter("ignore")           # replacing FSDP2's CUDA kernels is the point
+        lib.impl("split_with_sizes_copy", split_with_sizes_copy, "CUDA", allow_override=True)
+        lib.impl("chunk_cat", chunk_cat, "CUDA", allow_override=True)
+    _LIB = lib
+    _INSTALLED = True
+
+
+def fully_shard_tide(module, group=None, *, reshard_after_forward=True,
+                     engine: int = T.TIDE_ENGINE_SM, order: int = T.TIDE_ORDER_RANK):
+    """``fully_shard(module)`` over `group` with bf16 compute parameters and fp32 gradient
+    reduction, its all-gather and reduce-scatter done by TIDE.  Apply it to submodules
+    first, then to the root, in the same order on every rank.  Returns the module."""
+    import torch
+    import torch.distributed as dist
+    from torch.distributed.device_mesh import DeviceMesh
+    from torch.distributed.fsdp import MixedPrecisionPolicy, fully_shard
+
+    _install()
+    pg = group if group is not None else dist.group.WORLD
+    mesh = DeviceMesh.from_group(pg, "cuda")
+    fully_shard(module, mesh=mesh, reshard_after_forward=reshard_after_forward,
+                mp_policy=MixedPrecisionPolicy(param_dtype=torch.bfloat16, reduce_dtype=torch.float32))
+    param_group = module._get_fsdp_state()._fsdp_param_group
+    if param_group is None:                       # every parameter belongs to a submodule
+        return module
+    shapes = [tuple(fp._orig_size) for fp in param_group.fsdp_params]
+    tg = TideGroup(shapes, pg, engine=engine, order=order)
+    ag_cls, rs_cls = _comm_classes()
+    module.set_custom_all_gather(ag_cls(tg))
+    module.set_custom_reduce_scatter(rs_cls(tg))
+    module._tide_group = tg
+    return module
+
+
+def tide_groups(module) -> list:
+    """The TIDE groups of `module` and its submodules, in module order."""
+    return [m._tide_group for m in module.modules() if getattr(m, "_tide_group", None) is not None]
+
+
+def close(module) -> None:
+    """Unmap every TIDE group of `module` (a collective: all ranks, same order)."""
+    for tg in tide_groups(module):
+        tg.close()

@@ -80,6 +80,7 @@ _SIGNATURES = {
     "tide_rs_reduce": (_i32, [_vp, _P(_vp), _P(_i64), _vp, _i64, _i32, _i32, _P(_vp), _i64,
                               _i32, _i32, _vp]),
     "tide_rs_stage": (_i32, [_vp, _P(_vp), _P(_i64), _P(_vp), _i64, _i32, _i32, _vp]),
+    "tide_rs_stage_one": (_i32, [_vp, _P(_vp), _P(_i64), _vp, _i64, _i32, _i32, _vp]),
     "tide_rs_reduce_slots": (_i32, [_vp, _P(_vp), _i64, _vp, _i64, _i32, _i32, _i32, _vp]),
     "tide_rs_reduce_noalloc": (_i32, [_P(tide_param_t), _i32, _i32, _P(_vp), _P(_i64), _vp, _i64,
                                       _i32, _i32, _vp]),
@@ -259,6 +260,12 @@ def tide_rs_stage(plan, grads, grad_numel, slots, slot_numel: int, engine: int, 
     slot_arr = _ptr_array(slots) if slots is not None else None
     return lib().tide_rs_stage(plan, _ptr_array(grads), _i64_array(grad_numel), slot_arr,
                                slot_numel, engine, max_ctas, stream)
+
+
+def tide_rs_stage_one(plan, grads, grad_numel, slot: int, slot_numel: int, engine: int,
+                      max_ctas: int, stream: int) -> int:
+    return lib().tide_rs_stage_one(plan, _ptr_array(grads), _i64_array(grad_numel), slot, slot_numel,
+                                   engine, max_ctas, stream)
 
 
 def tide_rs_reduce_slots(plan, slots, slot_numel: int, out: int, out_numel: int, scale_mode: int,
@@ -456,8 +463,18 @@ class Plan:
                            _stream_handle(stream))
         _check(st, "tide_rs_stage")
 
+    def rs_stage_one(self, grads, slot, engine: int = TIDE_ENGINE_SM, max_ctas: int = 0,
+                     stream=None) -> None:
+        """One rank's P gradients into its own slot (bf16 [W][Ns])."""
+        g = _table(grads)
+        st = tide_rs_stage_one(self.handle, g.ptrs, g.numels, slot.data_ptr(), slot.numel(), engine,
+                               max_ctas, _stream_handle(stream))
+        _check(st, "tide_rs_stage_one")
+
     def rs_reduce_slots(self, slots, out, scale_mode: int = TIDE_SCALE_INV_WORLD,
                         order: int = TIDE_ORDER_RANK, max_ctas: int = 0, stream=None) -> None:
+        """Every rank's shard from the W slots ([W][Ns] out); with a one-rank plan, that rank's
+        shard ([Ns] out), the slots possibly peers' memory."""
         s = _table(slots)
         st = tide_rs_reduce_slots(self.handle, s.ptrs, s.min_numel, out.data_ptr(), out.numel(),
                                   scale_mode, order, max_ctas, _stream_handle(stream))

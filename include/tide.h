@@ -1,6 +1,6 @@
 /*
  * tide.h - C ABI of libtide.so: layout-aware reduce-scatter and all-gather
- * placement for FSDP2-style per-parameter storage, on one GPU.
+ * placement for FSDP2-style per-parameter storage.
  *
  * Source of the method: "The Endgame of FSDP Communication: Layout-Aware
  * Collectives on Copy Engines, RDMA, and NVSwitch" (weekinpapers.com, Abstract)
@@ -13,7 +13,10 @@
  * fp32 shards (TIDE-RS), so neither a copy-out nor a packed fp32 staging
  * buffer exists.  This library implements the per-rank arithmetic and
  * addressing of those two collectives with the network taken out: the W
- * data-parallel ranks are W sets of buffers on the calling GPU.
+ * data-parallel ranks are W sets of buffers that the calling GPU's kernels
+ * read, its own memory or, through CUDA IPC (tide_ipc_*), other processes'
+ * buffers, with one-rank plans (tide_plan_group_rank) for a process that holds
+ * one rank.
  *
  * Layout (the pages leave it open; this is the reading every call follows):
  *   param i has shape (d0_i, ...) with inner_i = product of the trailing dims;
@@ -264,8 +267,27 @@ TIDE_API tide_status_t tide_rs_stage(const tide_plan_t* plan, const void* const*
                             int32_t engine, int32_t max_ctas, void* stream);
 
 /*
+ * Slot-Reuse phase 1 for the one rank a process holds (same passages): that
+ * rank's gradients alone are copied, still bf16, into its own slot,
+ *   slot[r*Ns + off_i + e] = g_i[r*c_i + e]  for valid positions, every r;
+ * pad positions of the slot are not written.  This is tide_rs_stage's copy for
+ * one source rank (its result does not depend on which rank that is): each
+ * process stages its own gradients, and the slots then reach the other ranks as
+ * peer memory.  grads is a host array of P device pointers (grad_numel[i] >=
+ * d0_i*inner_i), slot one bf16 buffer of slot_numel >= W*Ns elements, which
+ * must not overlap any gradient.  engine SM (one launch) or CE.  Needs an
+ * all-rank plan.
+ */
+TIDE_API tide_status_t tide_rs_stage_one(const tide_plan_t* plan, const void* const* grads,
+                                         const int64_t* grad_numel, void* slot, int64_t slot_numel,
+                                         int32_t engine, int32_t max_ctas, void* stream);
+
+/*
  * Slot-Reuse phase 2: out[r*Ns + j] = s * fl32(sum_k fp32(slot_k[r*Ns + j])) at
  * valid positions (from the plan), +0.0 at pad positions.  One kernel launch.
+ * With a one-rank plan (rank r) out is that rank's shard only, fp32 [Ns]
+ * (out_numel >= Ns): out[j] = s * fl32(sum_k fp32(slot_k[r*Ns + j])); the
+ * slots may then be peers' memory.
  */
 TIDE_API tide_status_t tide_rs_reduce_slots(const tide_plan_t* plan, const void* const* slots,
                                    int64_t slot_numel, float* out, int64_t out_numel,

@@ -341,12 +341,39 @@ def test_rank_plan_arguments():
     assert ag(plan, a) == T.TIDE_ERR_INVALID_ARG
     assert T.tide_rs_stage(plan.handle, a["grads"], a["gnum"], a["slots"], a["n_slot"], 0, 0,
                            0) == T.TIDE_ERR_INVALID_ARG
-    assert T.tide_rs_reduce_slots(plan.handle, a["slots"], a["n_slot"], a["out"], a["n_out"], 1, 0,
-                                  0, 0) == T.TIDE_ERR_INVALID_ARG
+    assert T.tide_rs_stage_one(plan.handle, a["grads"][:g.n_params], a["gnum"][:g.n_params],
+                               a["slots"][0], a["n_slot"], 0, 0, 0) == T.TIDE_ERR_INVALID_ARG
+    # the slot reduction takes it: one shard out, read from rank 2's rows of every slot
+    assert T.tide_rs_reduce_slots(plan.handle, a["slots"], a["n_slot"], a["out"], L.Ns, 1, 0,
+                                  0, 0) == T.TIDE_ERR_DEVICE
+    assert T.tide_rs_reduce_slots(plan.handle, a["slots"], a["n_slot"], a["out"], L.Ns - 1, 1, 0,
+                                  0, 0) == T.TIDE_ERR_SIZE
+    assert T.tide_rs_reduce_slots(plan.handle, a["slots"], a["n_slot"] - 1, a["out"], L.Ns, 1, 0,
+                                  0, 0) == T.TIDE_ERR_SIZE
     assert T.tide_rs_reduce_pipelined(plan.handle, a["grads"], a["gnum"], a["out"], a["n_out"], 1, 0,
                                       a["slots"], a["n_slot"], 1, 0, 0, 0) == T.TIDE_ERR_INVALID_ARG
     assert T.tide_ag_gather_place(plan.handle, a["slots"], L.Ns, a["params"], a["pnum"], 0, 0,
                                   0) == T.TIDE_ERR_INVALID_ARG
+
+
+def test_stage_one_validation(tiny_plan, args):
+    P = configs.tiny().n_params
+    grads, gnum, slot, n = args["grads"][P:2 * P], args["gnum"][P:2 * P], args["slots"][1], args["n_slot"]
+
+    def stage(g=grads, gn=gnum, sl=slot, ns=n, engine=0, cap=0):
+        return T.tide_rs_stage_one(tiny_plan.handle, g, gn, sl, ns, engine, cap, 0)
+    assert stage() == T.TIDE_ERR_DEVICE              # valid: stops at the host-only plan
+    assert stage(engine=1) == T.TIDE_ERR_DEVICE
+    assert stage(engine=2) == T.TIDE_ERR_INVALID_ARG
+    assert stage(cap=-1) == T.TIDE_ERR_INVALID_ARG
+    assert stage(g=[0] + grads[1:]) == T.TIDE_ERR_INVALID_ARG
+    assert stage(g=grads[:2] + [grads[2] + 1] + grads[3:]) == T.TIDE_ERR_ALIGNMENT
+    assert stage(gn=gnum[:4] + [gnum[4] - 1]) == T.TIDE_ERR_SIZE
+    assert stage(sl=0) == T.TIDE_ERR_INVALID_ARG
+    assert stage(sl=slot + 1) == T.TIDE_ERR_ALIGNMENT
+    assert stage(ns=n - 1) == T.TIDE_ERR_SIZE
+    assert stage(sl=grads[3]) == T.TIDE_ERR_INVALID_ARG      # the slot overlaps a gradient
+    assert stage(g=[grads[0]] * P, gn=[max(gnum)] * P) == T.TIDE_ERR_DEVICE   # grads may alias
 
 
 def test_gather_place_validation(tiny_plan, args):

@@ -1,0 +1,74 @@
+"""FSDP2's own fully_shard with TIDE's all-gather and reduce-scatter (fsdp2_layout_aware_b200.fsdp2).
+
+2 and 3 processes share this GPU, each a rank of FSDP2 (bf16 compute parameters, fp32
+reduction, fp32 master parameters, SGD) over a small network, sharded per layer and at the
+root.  FSDP2's copy-out runs as tide_ag_gather_place from every rank's arena, its fp32 pack
+as tide_rs_stage_one into the rank's own arena, its reduce-scatter as tide_rs_reduce_slots.
+Checked bit for bit against the oracle at every call of every step:
+  * each placement: the padded parameters each rank placed equal the oracle's copy-out of
+    the rank-major concatenation of the rows all ranks had copied in;
+  * each staging: the rank's arena equals the oracle's staging of the rank's gradients (at
+    valid positions; pads keep what they held);
+  * each reduction: the rank's fp32 shard equals rows r of the oracle's reduce-scatter of all
+    ranks' gradients, x fl32(1/W) (FSDP2 asks for an average).
+"""
+import json
+
+import numpy as np
+import pytest
+
+import oracle
+
+from _dist_helpers import run_procs
+
+pytestmark = pytest.mark.gpu
+
+pytest.importorskip("torch.distributed.fsdp._fully_shard._fsdp_collectives")
+
+
+def _load(tmp, name):
+    return np.load(tmp / name)
+
+
+@pytest.mark.parametrize("world,engine,order", [(2, 0, 0), (3, 0, 0), (3, 1, 1)],
+                         ids=["w2_sm_rank", "w3_sm_rank", "w3_ce_tree"])
+def test_fully_shard_with_tide_collectives_matches_the_oracle(world, engine, order, tmp_path):
+    from _fsdp2_tide_workers import fsdp2_tide_worker
+    steps, lr = 3, 0.05
+    run_procs(fsdp2_tide_worker, world,
+              lambda port: (world, port, steps, lr, str(tmp_path), engine, order))
+    shapes = [[tuple(s) for s in g] for g in json.loads((tmp_path / "shapes.json").read_text())]
+    counts = [json.loads((tmp_path / f"counts_{r}.json").read_text()) for r in range(world)]
+    assert all({k: v for k, v in c.items() if k != "losses"} ==
+               {k: v for k, v in counts[0].items() if k != "losses"} for c in counts)
+    rs_oracle = oracle.rs_reduce if order == 0 else oracle.rs_reduce_tree
+    for g, S in enumerate(shapes):
+        L = oracle.layout(world, S)
+        P = len(S)
+        n_place = counts[0][f"place_{g}"]
+        n_reduce = counts[0][f"reduce_{g}"]
+        assert n_place >= steps and n_reduce == steps and counts[0][f"stage_{g}"] == steps
+        for n in range(n_place):
+            ag = np.concatenate([_load(tmp_path, f"row_{g}_{n}_{k}.npy") for k in range(world)])
+            want = oracle.ag_copyout(world, S, ag)
+            for r in range(world):
+                for i in range(P):
+                    got = _load(tmp_path, f"placed_{g}_{n}_{r}_{i}.npy")
+                    assert np.array_equal(got, want[i]), (g, n, r, i)
+        for n in range(n_reduce):
+            grads = [[_load(tmp_path, f"grad_{g}_{n}_{k}_{i}.npy") for i in range(P)]
+                     for k in range(world)]
+            for k in range(world):
+                exp = _load(tmp_path, f"slot0_{g}_{n}_{k}.npy").copy()
+                oracle.slot_stage(world, S, grads[k], exp)
+                assert np.array_equal(_load(tmp_path, f"slot1_{g}_{n}_{k}.npy"), exp), (g, n, k)
+            ref = rs_oracle(world, S, grads, 1).reshape(world, L.Ns)
+            for r in range(world):
+                got = _load(tmp_path, f"shard_{g}_{n}_{r}.npy")
+                assert np.array_equal(got.view(np.uint32), ref[r].view(np.uint32)), (g, n, r)
+    # training moved the parameters: the last placement of each group differs from the first
+    for g, S in enumerate(shapes):
+        last = counts[0][f"place_{g}"] - 1
+        first = np.concatenate([_load(tmp_path, f"placed_{g}_0_0_{i}.npy") for i in range(len(S))])
+        final = np.concatenate([_load(tmp_path, f"placed_{g}_{last}_0_{i}.npy") for i in range(len(S))])
+        assert not np.array_equal(first, final), g

@@ -273,6 +273,45 @@ def test_slot_reuse_equals_plain_and_oracle(group, engine):
         assert np.array_equal(bits_of(slots[k]), exp)
 
 
+ONE_GROUPS = [configs.tiny(), degenerate(), mini_wan(), configs.qwen3moe(4), GROUPS[-3],
+              aligned_group(8, 62)]
+
+
+@pytest.mark.parametrize("group", ONE_GROUPS, ids=[f"{g.name}_w{g.world}" for g in ONE_GROUPS])
+@pytest.mark.parametrize("engine", [T.TIDE_ENGINE_SM, T.TIDE_ENGINE_CE])
+def test_each_rank_stages_its_own_slot_and_reduces_its_shard(group, engine):
+    """Slot-Reuse as ranks that are processes run it: rank k stages only its own gradients into
+    its own slot (tide_rs_stage_one), then rank r's one-rank plan reduces its shard from rows r
+    of all W slots (tide_rs_reduce_slots).  Slot pads start as 0xFFFF (a bf16 NaN), so a read of
+    a pad would show.  Each slot equals the oracle's staging of that rank, and each shard the
+    oracle's rows r, in rank and in tree order."""
+    W = group.world
+    grads = synth.grads_host(group, seed=61)
+    dev = grads_to_dev(group, grads)
+    plan = T.Plan(group.shapes, W)
+    L = oracle.layout(W, group.shapes)
+    slots = [torch.full((W * L.Ns,), -1, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+             for _ in range(W)]
+    for k in range(W):
+        plan.rs_stage_one(dev[k], slots[k], engine=engine)
+    torch.cuda.synchronize()
+    plan.check()
+    for k in range(W):
+        exp = np.full(W * L.Ns, 0xFFFF, dtype=np.uint16)
+        oracle.slot_stage(W, group.shapes, grads[k], exp)
+        assert np.array_equal(bits_of(slots[k]), exp), k
+    for order, ref in ((T.TIDE_ORDER_RANK, oracle.rs_reduce(W, group.shapes, grads, 1)),
+                       (T.TIDE_ORDER_TREE, oracle.rs_reduce_tree(W, group.shapes, grads, 1))):
+        ref = ref.reshape(W, L.Ns)
+        for r in range(W):
+            mine = T.Plan(group.shapes, W, rank=r)
+            out = torch.full((L.Ns,), float("nan"), device="cuda")
+            mine.rs_reduce_slots(slots, out, scale_mode=T.TIDE_SCALE_INV_WORLD, order=order)
+            torch.cuda.synchronize()
+            mine.check()
+            assert np.array_equal(f32_bits(out), ref[r].view(np.uint32)), (order, r)
+
+
 V32_GROUPS = [aligned_group(w, 40 + w) for w in (2, 5, 8, 13, 16)] + [configs.qwen3moe(4)]
 
 
