@@ -45,8 +45,8 @@ from . import tide as T
 _AG = {}          # data_ptr of a group's arena -> TideGroup
 _RS = {}          # data_ptr of a group's expanded reduce-scatter input -> TideGroup
 _LOCK = threading.Lock()
-_INSTALLED = False
-_LIB = None
+_INSTALLED = set()   # dispatch keys whose copy-out and pack are routed here
+_LIBS = []
 
 
 class TideGroup:
@@ -198,10 +198,10 @@ def _comm_classes():
     return TideAllGather, TideReduceScatter
 
 
-def _install() -> None:
-    """Route FSDP2's copy-out and pack to the library for TIDE groups' buffers."""
-    global _INSTALLED, _LIB
-    if _INSTALLED:
+def _install(dispatch_key: str = "CUDA") -> None:
+    """Route FSDP2's copy-out and pack on `dispatch_key` tensors to the registered groups
+    (_AG, _RS); every other buffer keeps FSDP2's own implementation."""
+    if dispatch_key in _INSTALLED:
         return
     import torch
     from torch.distributed.fsdp._fully_shard import _fsdp_collectives as C
@@ -226,11 +226,11 @@ def _install() -> None:
 
     lib = torch.library.Library("fsdp", "IMPL")  # noqa: TOR901
     with warnings.catch_warnings():
-        warnings.simplefilter("ignore")           # replacing FSDP2's CUDA kernels is the point
-        lib.impl("split_with_sizes_copy", split_with_sizes_copy, "CUDA", allow_override=True)
-        lib.impl("chunk_cat", chunk_cat, "CUDA", allow_override=True)
-    _LIB = lib
-    _INSTALLED = True
+        warnings.simplefilter("ignore")           # replacing FSDP2's kernels is the point
+        lib.impl("split_with_sizes_copy", split_with_sizes_copy, dispatch_key, allow_override=True)
+        lib.impl("chunk_cat", chunk_cat, dispatch_key, allow_override=True)
+    _LIBS.append(lib)                             # the registrations live as long as the library
+    _INSTALLED.add(dispatch_key)
 
 
 def fully_shard_tide(module, group=None, *, reshard_after_forward=True,

@@ -103,3 +103,120 @@ def fsdp2_tide_worker(rank, world, port, steps, lr, out_dir, engine, order):
         F.close(model)
     finally:
         dist.destroy_process_group()
+
+
+class OracleGroup:
+    """A TIDE group for FSDP2 on the CPU whose placement, staging and reduction are the
+    oracle's, with gloo collectives standing in for the peer reads: it checks FSDP2's side of
+    fsdp2_layout_aware_b200.fsdp2 (which buffers it asks for, in which order, and what lands
+    where) without a GPU."""
+
+    def __init__(self, shapes):
+        import torch
+        import torch.distributed as dist
+        from fsdp2_layout_aware_b200 import fsdp2 as F
+        from fsdp2_layout_aware_b200 import tide as T
+        self.world, self.rank = dist.get_world_size(), dist.get_rank()
+        self.shapes = [tuple(int(d) for d in s) for s in shapes]
+        plan = T.Plan(self.shapes, self.world, host_only=True)
+        self.shard_numel = plan.shard_numel
+        self.chunks = [plan.query(i)["chunk_numel"] for i in range(len(self.shapes))]
+        self.arena = torch.zeros(self.world * self.shard_numel, dtype=torch.bfloat16)
+        self.rs_input = torch.zeros(1)
+        self.device = torch.device("cpu")
+        self.calls = []
+        F._AG[self.arena.data_ptr()] = self
+        F._RS[self.rs_input.data_ptr()] = self
+
+    def meet(self):
+        import torch.distributed as dist
+        dist.barrier()
+
+    def _all(self, t):
+        import torch
+        import torch.distributed as dist
+        bufs = [torch.empty_like(t) for _ in range(self.world)]
+        dist.all_gather(bufs, t.contiguous())
+        return [b.view(torch.int16).numpy().view(np.uint16) for b in bufs]
+
+    def place(self, out):
+        import oracle
+        import torch
+        self.calls.append("place")
+        Ns, r = self.shard_numel, self.rank
+        rows = self._all(self.arena[r * Ns:(r + 1) * Ns])
+        want = oracle.ag_copyout(self.world, self.shapes, np.concatenate(rows))
+        for t, w in zip(out, want):
+            t.view(-1).view(torch.int16).copy_(torch.from_numpy(w.view(np.int16)))
+        self.meet()
+
+    def stage(self, grads):
+        import oracle
+        import torch
+        self.calls.append("stage")
+        bits = [g.detach().contiguous().view(torch.int16).numpy().reshape(-1).view(np.uint16) for g in grads]
+        slot = self.arena.view(torch.int16).numpy().view(np.uint16)   # shares the arena's memory
+        oracle.slot_stage(self.world, self.shapes, bits, slot)
+
+    def reduce(self, out, op):
+        import oracle
+        import torch
+        import torch.distributed as dist
+        self.calls.append("reduce")
+        self.meet()
+        slots = self._all(self.arena)
+        scale = 1 if op == dist.ReduceOp.AVG else 0
+        res = oracle.rs_reduce_slots(self.world, self.shapes, slots, scale)
+        Ns, r = self.shard_numel, self.rank
+        out.copy_(torch.from_numpy(res[r * Ns:(r + 1) * Ns].copy()))
+        self.meet()
+
+
+def fsdp2_oracle_worker(rank, world, port, steps, lr, out_dir):
+    """Stock FSDP2, then FSDP2 with the TIDE comms and operator routing of
+    fsdp2_layout_aware_b200.fsdp2 over OracleGroups, on the CPU; saves both runs' sharded
+    gradients of every step and final sharded parameters."""
+    import torch
+    import torch.distributed as dist
+    from torch.distributed.device_mesh import DeviceMesh
+    from torch.distributed.fsdp import MixedPrecisionPolicy, fully_shard
+    from fsdp2_layout_aware_b200 import fsdp2 as F
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
+    try:
+        mesh = DeviceMesh.from_group(dist.group.WORLD, "cpu")
+        policy = MixedPrecisionPolicy(param_dtype=torch.bfloat16, reduce_dtype=torch.float32)
+        gen = torch.Generator().manual_seed(100 + rank)
+        x, y = torch.randn(16, 40, generator=gen), torch.randn(16, 10, generator=gen)
+        calls = {}
+        for arm in ("stock", "tide"):
+            torch.manual_seed(0)
+            model = _net()
+            groups = []
+            for m in (model.l1, model.l2, model):
+                fully_shard(m, mesh=mesh, mp_policy=policy)
+                if arm == "tide":
+                    F._install("CPU")
+                    pg = m._get_fsdp_state()._fsdp_param_group
+                    tg = OracleGroup([tuple(fp._orig_size) for fp in pg.fsdp_params])
+                    ag_cls, rs_cls = F._comm_classes()
+                    m.set_custom_all_gather(ag_cls(tg))
+                    m.set_custom_reduce_scatter(rs_cls(tg))
+                    groups.append(tg)
+            opt = torch.optim.SGD(model.parameters(), lr=lr)
+            for step in range(steps):
+                ((model(x).float() - y) ** 2).mean().backward()
+                for i, p in enumerate(model.parameters()):
+                    np.save(os.path.join(out_dir, f"{arm}_grad_{step}_{rank}_{i}.npy"),
+                            p.grad.to_local().detach().numpy())
+                opt.step()
+                opt.zero_grad()
+            for i, p in enumerate(model.parameters()):
+                np.save(os.path.join(out_dir, f"{arm}_param_{rank}_{i}.npy"), p.to_local().detach().numpy())
+            calls[arm] = [tg.calls for tg in groups]
+        with open(os.path.join(out_dir, f"calls_{rank}.json"), "w") as f:
+            json.dump(calls["tide"], f)
+    finally:
+        dist.destroy_process_group()

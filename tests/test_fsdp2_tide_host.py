@@ -1,0 +1,40 @@
+"""FSDP2's side of fsdp2_layout_aware_b200.fsdp2, on the CPU.
+
+FSDP2 (fully_shard, bf16 compute, fp32 reduction, SGD) runs over 2 and 3 gloo processes
+twice: stock, and with TIDE's all-gather and reduce-scatter comms plus the copy-out and pack
+routed to TIDE groups, whose data movement is the oracle's (placement, Slot-Reuse staging,
+slot reduction x fl32(1/W)) with gloo standing in for the peer reads.  The sharded gradients
+of every step and the final parameters must be stock FSDP2's: bit for bit at W = 2 (one add,
+and 1/2 is exact), within fp32 rounding of a reordered 3-term sum at W = 3.  Every TIDE group
+must have seen each placement, staging and reduction FSDP2 should ask for.
+"""
+import json
+
+import numpy as np
+import pytest
+
+from _dist_helpers import run_procs
+
+pytest.importorskip("torch.distributed.fsdp._fully_shard._fsdp_collectives")
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_fsdp2_with_tide_comms_gives_stock_fsdp2_results(world, tmp_path):
+    from _fsdp2_tide_workers import fsdp2_oracle_worker
+    steps, lr = 3, 0.05
+    run_procs(fsdp2_oracle_worker, world, lambda port: (world, port, steps, lr, str(tmp_path)))
+    for r in range(world):
+        names = [f"grad_{s}_{r}_{i}" for s in range(steps) for i in range(5)] + \
+                [f"param_{r}_{i}" for i in range(5)]
+        for name in names:
+            a, b = np.load(tmp_path / f"stock_{name}.npy"), np.load(tmp_path / f"tide_{name}.npy")
+            assert a.shape == b.shape, name
+            if world == 2:
+                assert np.array_equal(a.view(np.uint32), b.view(np.uint32)), name
+            else:
+                np.testing.assert_allclose(b, a, rtol=1e-5, atol=1e-7, err_msg=name)
+        calls = json.loads((tmp_path / f"calls_{r}.json").read_text())
+        # groups in fully_shard order: l1, l2 (resharded after forward: placed again in
+        # backward), then the root (kept unsharded from forward to backward)
+        assert calls[0] == calls[1] == ["place", "place", "stage", "reduce"] * steps
+        assert calls[2] == ["place", "stage", "reduce"] * steps
