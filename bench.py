@@ -462,6 +462,22 @@ ROW_KINDS = {
 }
 
 
+def rs_sm_time(rs_ms: float, rs_ctas: int, variants: dict, sms: int) -> dict:
+    """SM time of the reduce-scatter's layout work, stock against TIDE: SMs held x duration,
+    the one-GPU analogue of the pages' lower RS SM time (weekinpapers.com, Abstract).  A
+    TIDE kernel holds min(CTAs, SMs) SMs for its launch, copy-engine staging holds none, and
+    torch's pack and add kernels are counted at the whole GPU."""
+    stock = sms * variants["stock_torch_pack_reduce"]["ms"]
+    tide = min(rs_ctas, sms) * rs_ms
+    slot = variants["slot_reduce"]
+    reuse = min(slot.get("ctas", sms), sms) * slot["ms"]
+    return {"unit": "SM-ms", "stock_pack_reduce": round(stock, 2), "tide_rs_reduce": round(tide, 2),
+            "tide_slot_reuse_ce": round(reuse, 2),
+            "note": "Slot-Reuse with copy-engine staging: the staging holds no SM, the reduction "
+                    "of the slots does",
+            "stock_over_tide": round(stock / tide, 2), "stock_over_slot_reuse_ce": round(stock / reuse, 2)}
+
+
 def jsonl_rows(res, group_name, world):
     """One flat row per (config, op, mode, ctas) of a bench line."""
     rows = []
@@ -1147,6 +1163,8 @@ def bench_workload(args, group, rank, world, device, dist_on):
         # the step's figures above stand even if a variant fails: record the error instead
         try:
             res["variants"] = run_variants(wl, max(3, min(K, 20)), stream, peak, flush)
+            res["rs_sm_time"] = rs_sm_time(rs_ms, rs_ctas, res["variants"],
+                                           torch.cuda.get_device_properties(device).multi_processor_count)
         except Exception as e:  # noqa: BLE001
             res["variants_error"] = f"{type(e).__name__}: {e}"
             wl.drop_slots()

@@ -105,3 +105,15 @@ def test_jsonl_rows_flatten_a_bench_line():
     assert by["slot_reuse_pipelined_seg4"]["same_bits_as_plain"] is False
     assert all(r["config"] == "llama70b" and r["world"] == 8 and r["oracle_GB/s"] == 1.9 for r in rows)
     assert all(json.loads(json.dumps(r)) == r for r in rows)
+
+
+def test_rs_sm_time_counts_sms_held_times_duration():
+    import bench
+    v = {"stock_torch_pack_reduce": {"ms": 30.0}, "slot_reduce": {"ms": 2.5, "ctas": 296}}
+    r = bench.rs_sm_time(2.4, 296, v, 148)
+    assert r["stock_pack_reduce"] == 148 * 30.0
+    assert r["tide_rs_reduce"] == round(148 * 2.4, 2)          # 296 CTAs hold the 148 SMs
+    assert r["tide_slot_reuse_ce"] == 148 * 2.5                 # the staging holds none
+    assert r["stock_over_tide"] == round(30.0 / 2.4, 2)
+    capped = bench.rs_sm_time(40.0, 4, v, 148)                 # 4 CTAs hold 4 SMs
+    assert capped["tide_rs_reduce"] == 160.0
