@@ -31,7 +31,9 @@ that no rank writes its arena while another may still read it: before a placemen
 row is in), after it (before anyone stages gradients over its row), before a reduction
 (every rank staged) and after it (before the next copy-in).  The parameter group must have
 bf16 compute parameters and fp32 reduction (the mixed-precision policy set here); every
-collective is synchronous.
+collective is synchronous.  Every parameter of a group must receive a gradient in each
+backward: FSDP2 leaves parameters without one out of its reduce-scatter, which changes the
+buffer layout, and the group's calls then refuse the buffers with an error.
 """
 from __future__ import annotations
 
