@@ -1,4 +1,5 @@
-"""GPU parity at the full model-shaped sizes, every element, in the benchmark's launch configuration.
+"""GPU parity at full size, every element, in the benchmark's launch configuration: the three
+model-shaped groups and every group of the W sweep (W = 2 ... 64, 34 GB of gradients at 64).
 
 TIDE-RS (weekinpapers.com, Abstract: per-parameter bf16 gradients reduced into
 fp32 rank-major shards) and TIDE-AG (same Abstract: the all-gather result lands
@@ -27,7 +28,8 @@ pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 SEED = 1
 
 
-@pytest.mark.parametrize("name", ["llama70b", "qwen3moe", "wan14b"])
+@pytest.mark.parametrize("name", ["llama70b", "qwen3moe", "wan14b"] +
+                         [f"sweep_w{w}" for w in configs.SWEEP_WORLDS])
 def test_every_element_rs_and_ag(name):
     group = configs.by_name(name)
     W = group.world
