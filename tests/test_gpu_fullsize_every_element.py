@@ -28,10 +28,18 @@ pytestmark = [pytest.mark.gpu, pytest.mark.slow]
 SEED = 1
 
 
-@pytest.mark.parametrize("name", ["llama70b", "qwen3moe", "wan14b"] +
-                         [f"sweep_w{w}" for w in configs.SWEEP_WORLDS])
-def test_every_element_rs_and_ag(name):
+CASES = [(n, T.TIDE_ORDER_RANK) for n in ["llama70b", "qwen3moe", "wan14b"] +
+         [f"sweep_w{w}" for w in configs.SWEEP_WORLDS]] + \
+        [(n, T.TIDE_ORDER_TREE) for n in ["llama70b", "qwen3moe", "wan14b"]]
+
+
+@pytest.mark.parametrize("name,order", CASES,
+                         ids=[f"{n}_{'tree' if o else 'rank'}" for n, o in CASES])
+def test_every_element_rs_and_ag(name, order):
+    """Rank order against the oracle's reduce-scatter; tree order (the 32-byte tree kernels
+    on these groups) against the oracle's tree sums."""
     group = configs.by_name(name)
+    rs_oracle = oracle.rs_reduce if order == T.TIDE_ORDER_RANK else oracle.rs_reduce_tree
     W = group.world
     torch.cuda.empty_cache()
     plan = T.Plan(group.shapes, W)
@@ -40,7 +48,7 @@ def test_every_element_rs_and_ag(name):
 
     grads = synth.dev_grads(group, SEED)
     out = torch.full((W * L.Ns,), float("nan"), device="cuda")
-    plan.rs_reduce(grads, out, scale_mode=T.TIDE_SCALE_INV_WORLD)     # the benchmark's call
+    plan.rs_reduce(grads, out, scale_mode=T.TIDE_SCALE_INV_WORLD, order=order)  # the bench's call
     torch.cuda.synchronize()
     plan.check()
     del grads
@@ -62,7 +70,7 @@ def test_every_element_rs_and_ag(name):
         sub = (group.shapes[i],)
         # RS: rows off_i .. off_i + c_i of every rank's shard
         g_host = [[synth.grad_host(group, SEED, k, i)] for k in range(W)]
-        want = oracle.rs_reduce(W, sub, g_host, 1).view(np.uint32)
+        want = rs_oracle(W, sub, g_host, 1).view(np.uint32)
         del g_host
         got = shards[:, L.off[i]: L.off[i] + c].contiguous().cpu().numpy().reshape(-1).view(np.uint32)
         bad = np.nonzero(got != want)[0]
