@@ -19,8 +19,8 @@
 //   - each thread owns 8 consecutive outputs per step: W independent 16-byte
 //     streaming loads (in groups of G ranks to bound registers), an fp32 sum
 //     with __fadd_rn (no contraction), the optional __fmul_rn scale, two 16-byte
-//     streaming stores; for 5 <= W <= 16 and 32-byte aligned groups, 16 outputs
-//     per step with 32-byte loads and stores instead;
+//     streaming stores; for W = 2 or W >= 5 and 32-byte aligned groups, 16
+//     outputs per step with 32-byte loads and stores instead;
 //   - tiles whose addresses are not all 16-byte aligned (possible only when
 //     the group's sizes break alignment) fall back to coalesced scalar loads;
 //   - ragged tile ends and pad rows are finished element by element.
@@ -36,13 +36,15 @@
 namespace tide {
 namespace {
 
-// The 32-byte path measured faster for 5 <= W <= 16 (70B W=8: 7.03 vs 6.89
-// TB/s; Qwen3 W=8: 7.08 vs 6.87; Wan2.2 W=16: 6.93 vs 6.90) and slower at
-// W=64 (6.90 vs 7.01), where 16-byte loads keep more ranks in flight.  At W = 2
-// it beats the 16-byte two-rank kernel by 20-27 % (67 MB to 1.1 GB groups:
-// 3.41 vs 2.73, 5.02 vs 3.95, 5.31 vs 4.45 TB/s); at W = 3 and 4 it does not
-// (5.34 vs 5.39, 6.18 vs 6.16 and 5.64 vs 5.78), so they keep 16-byte loads.
-constexpr int kV32MaxWorld = 16;
+// The 32-byte path measured faster for W >= 5 (70B W=8: 7.03 vs 6.89 TB/s;
+// Qwen3 W=8: 7.08 vs 6.87; Wan2.2 W=16: 6.93 vs 6.90; the sweep's W = 32 and 64
+// groups: 6.90 vs 6.68 and 6.85 vs 6.71; 16 x 1536x4096 at W = 24: 6.88 vs
+// 6.54; 16 x 1024x4096 at W = 128: 6.89 vs 6.65).  At W = 2 it beats the
+// 16-byte two-rank kernel by 20-27 % (67 MB to 1.1 GB groups: 3.41 vs 2.73,
+// 5.02 vs 3.95, 5.31 vs 4.45 TB/s); at W = 3 and 4 it does not (5.34 vs 5.39,
+// 6.18 vs 6.16 and 5.64 vs 5.78), so they keep 16-byte loads.  Its registers
+// do not grow with W: the ranks are loaded 8 at a time and added in order.
+constexpr int kV32MaxWorld = TIDE_MAX_WORLD;
 
 struct RsParams {
     const tide_tile_t* tiles;

@@ -379,7 +379,7 @@ TIDE_API tide_status_t tide_rs_reduce_noalloc(const tide_param_t* params, int32_
  * The reductions use kernels 4/5 (one CTA per SM, TMA loads into shared memory)
  * when the plan was built with TIDE_PLAN_TMA, every tile starts on an
  * 8-element boundary and every source and the output are 16-byte aligned.
- * Otherwise they use the 32-byte kernels (rank order 6/7 when W = 2 or 5 <= W <= 16,
+ * Otherwise they use the 32-byte kernels (rank order 6/7 when W = 2 or W >= 5,
  * tree order 11/12 when W is 2, 4, 8 or 16) if every tile starts on a 16-element
  * boundary and every source and the output are 32-byte aligned; else kernels
  * 0/3 (rank order) or 8/9 (tree order).

@@ -312,12 +312,12 @@ def test_each_rank_stages_its_own_slot_and_reduces_its_shard(group, engine):
             assert np.array_equal(f32_bits(out), ref[r].view(np.uint32)), (order, r)
 
 
-V32_GROUPS = [aligned_group(w, 40 + w) for w in (2, 5, 8, 13, 16)] + [configs.qwen3moe(4)]
+V32_GROUPS = [aligned_group(w, 40 + w) for w in (2, 5, 8, 13, 16, 24, 32, 64)] + [configs.qwen3moe(4)]
 
 
 @pytest.mark.parametrize("group", V32_GROUPS, ids=[f"{g.name}_w{g.world}" for g in V32_GROUPS])
 def test_rs_32_byte_path(group):
-    """W = 2 or 5 <= W <= 16 with 32-byte aligned tiles takes the 32-byte variant; same bits."""
+    """W = 2 or W >= 5 with 32-byte aligned tiles takes the 32-byte variant; same bits."""
     grads = synth.grads_host(group, seed=34)
     L = oracle.layout(group.world, group.shapes)
     aligned16 = all((r * c) % 16 == 0 and (r * L.Ns + o) % 16 == 0
