@@ -80,6 +80,8 @@ _SIGNATURES = {
     "tide_rs_reduce": (_i32, [_vp, _P(_vp), _P(_i64), _vp, _i64, _i32, _i32, _P(_vp), _i64,
                               _i32, _i32, _vp]),
     "tide_rs_stage": (_i32, [_vp, _P(_vp), _P(_i64), _P(_vp), _i64, _i32, _i32, _vp]),
+    "tide_flag_signal": (_i32, [_vp, ctypes.c_uint32, _vp]),
+    "tide_flag_wait": (_i32, [_P(_vp), _i32, ctypes.c_uint32, _i64, _vp, _vp]),
     "tide_rs_stage_one": (_i32, [_vp, _P(_vp), _P(_i64), _vp, _i64, _i32, _i32, _vp]),
     "tide_rs_reduce_slots": (_i32, [_vp, _P(_vp), _i64, _vp, _i64, _i32, _i32, _i32, _vp]),
     "tide_rs_reduce_noalloc": (_i32, [_P(tide_param_t), _i32, _i32, _P(_vp), _P(_i64), _vp, _i64,
@@ -260,6 +262,19 @@ def tide_rs_stage(plan, grads, grad_numel, slots, slot_numel: int, engine: int, 
     slot_arr = _ptr_array(slots) if slots is not None else None
     return lib().tide_rs_stage(plan, _ptr_array(grads), _i64_array(grad_numel), slot_arr,
                                slot_numel, engine, max_ctas, stream)
+
+
+def tide_flag_signal(flag: int, value: int, stream: int = 0) -> int:
+    """Store `value` into the device flag at `flag` after every earlier write of this device
+    (stream-ordered, release semantics at system scope)."""
+    return lib().tide_flag_signal(flag, value & 0xFFFFFFFF, stream)
+
+
+def tide_flag_wait(flags, value: int, timeout_ns: int, status: int, stream: int = 0) -> int:
+    """One kernel that polls the device flags until each reaches epoch `value` or timeout_ns
+    passes, then writes the int32 at `status`: 0, or 1 + the first late flag's index."""
+    return lib().tide_flag_wait(_ptr_array(flags), len(flags), value & 0xFFFFFFFF, timeout_ns,
+                                status, stream)
 
 
 def tide_rs_stage_one(plan, grads, grad_numel, slot: int, slot_numel: int, engine: int,

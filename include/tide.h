@@ -430,6 +430,36 @@ TIDE_API tide_status_t tide_ipc_open(const void* handle, int32_t device, void** 
 TIDE_API tide_status_t tide_ipc_close(void* base, int32_t device);
 TIDE_API tide_status_t tide_peer_access(int32_t device, int32_t peer, int32_t* can_access);
 
+/*
+ * Ordering between ranks on the device, with bounded waits (weekinpapers.com,
+ * Abstract: each rank's collectives read the other ranks' buffers in place, so
+ * a rank may read a peer's buffer only after the peer wrote it, and overwrite
+ * its own only after every peer read it).  Both calls are stream-ordered on
+ * the current device and need no plan; flags are 32-bit words in device
+ * memory, this process's own or a peer's mapped with tide_ipc_open.
+ *
+ * tide_flag_signal: one kernel thread makes every earlier write of this device
+ * visible to the whole system, then stores `value` into *flag with release
+ * semantics.  TIDE_ERR_INVALID_ARG for a NULL flag, TIDE_ERR_ALIGNMENT if it
+ * is not 4-byte aligned.
+ *
+ * tide_flag_wait: one CTA polls the n flags (flags: a host array of n device
+ * pointers, 1 <= n <= TIDE_MAX_WORLD) with acquire loads until each holds
+ * `value` or a later epoch (flag - value, as a signed 32-bit difference, >= 0),
+ * or until timeout_ns (1 ns .. 60 s) has passed; it then writes *status (a
+ * device int32): 0 if every flag got there, else 1 + the index of the first
+ * one that did not.  The wait always ends: at the time limit, and as a second
+ * bound after an iteration cap.  Work queued after it on the stream runs when
+ * it ends, whatever the status, so the caller reads *status before trusting
+ * that work.  A waiting kernel must not be the only way its flag can be set
+ * on the same GPU (no two launches that wait on one another share a GPU).
+ * TIDE_ERR_INVALID_ARG / TIDE_ERR_ALIGNMENT for bad arguments, checked before
+ * anything is enqueued.
+ */
+TIDE_API tide_status_t tide_flag_signal(void* flag, uint32_t value, void* stream);
+TIDE_API tide_status_t tide_flag_wait(const void* const* flags, int32_t n, uint32_t value,
+                                      int64_t timeout_ns, int32_t* status, void* stream);
+
 TIDE_API const char* tide_status_string(tide_status_t status);
 TIDE_API int32_t tide_abi_version(void);
 

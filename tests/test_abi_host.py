@@ -463,3 +463,18 @@ def test_ipc_calls_validate_their_arguments_on_the_host():
     assert T.tide_ipc_close(1 << 40, -1) == T.TIDE_ERR_INVALID_ARG
     assert T.tide_peer_access(3, 3) == (T.TIDE_OK, 1)        # a device always reads itself
     assert T.tide_peer_access(-1, 0)[0] == T.TIDE_ERR_INVALID_ARG
+
+
+def test_flag_calls_validate_their_arguments_on_the_host():
+    f = BASE + 4096
+    assert T.tide_flag_signal(0, 1) == T.TIDE_ERR_INVALID_ARG
+    assert T.tide_flag_signal(f + 2, 1) == T.TIDE_ERR_ALIGNMENT
+    status = BASE + 8192
+    assert T.tide_flag_wait([], 1, 1000, status) == T.TIDE_ERR_INVALID_ARG            # n = 0
+    assert T.tide_flag_wait([f] * (T.TIDE_MAX_WORLD + 1), 1, 1000, status) == T.TIDE_ERR_INVALID_ARG
+    assert T.tide_flag_wait([f], 1, 0, status) == T.TIDE_ERR_INVALID_ARG               # no time limit
+    assert T.tide_flag_wait([f], 1, 61 * 10**9, status) == T.TIDE_ERR_INVALID_ARG      # over 60 s
+    assert T.tide_flag_wait([f], 1, 1000, 0) == T.TIDE_ERR_INVALID_ARG                 # no status word
+    assert T.tide_flag_wait([f], 1, 1000, status + 1) == T.TIDE_ERR_ALIGNMENT
+    assert T.tide_flag_wait([f, 0], 1, 1000, status) == T.TIDE_ERR_INVALID_ARG
+    assert T.tide_flag_wait([f, f + 6], 1, 1000, status) == T.TIDE_ERR_ALIGNMENT
