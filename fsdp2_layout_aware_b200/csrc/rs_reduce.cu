@@ -41,9 +41,12 @@ namespace {
 // groups: 6.90 vs 6.68 and 6.85 vs 6.71; 16 x 1536x4096 at W = 24: 6.88 vs
 // 6.54; 16 x 1024x4096 at W = 128: 6.89 vs 6.65).  At W = 2 it beats the
 // 16-byte two-rank kernel by 20-27 % (67 MB to 1.1 GB groups: 3.41 vs 2.73,
-// 5.02 vs 3.95, 5.31 vs 4.45 TB/s); at W = 3 and 4 it does not (5.34 vs 5.39,
-// 6.18 vs 6.16 and 5.64 vs 5.78), so they keep 16-byte loads.  Its registers
-// do not grow with W: the ranks are loaded 8 at a time and added in order.
+// 5.02 vs 3.95, 5.31 vs 4.45 TB/s), and its two-rank form at 4 CTAs per SM
+// beats its eight-rank form by 6-24 % (the sweep's 67 MB group: 4.17 vs 3.43;
+// 134 MB: 6.24 vs 5.03; 1 GB: 5.79 vs 5.45).  At W = 3 and 4 neither form wins
+// on the large groups (1 GB: 6.12 vs 6.24 and 6.12 vs 6.39 for the four-rank
+// form), so they keep 16-byte loads.  Its registers do not grow with W: the
+// ranks are loaded 8 at a time and added in order.
 constexpr int kV32MaxWorld = TIDE_MAX_WORLD;
 
 struct RsParams {
@@ -207,8 +210,9 @@ template <bool SLOT, bool TREE>
 KernelFn pick(int world, bool v32) {
     // (in the tree order every W <= G is one group, so G < 8 kernels never merge)
     if constexpr (!TREE) {
-        // W = 2 in rank order: the 32-byte kernel (one group, two ranks loaded)
-        if (v32 && world == 2) return rs_reduce_kernel<8, 1, SLOT, false, true, 0>;
+        // W = 2 in rank order: the 32-byte kernel over one group of two ranks (64
+        // registers, 4 CTAs per SM; the group of 8 held 119 registers and 2 CTAs per SM)
+        if (v32 && world == 2) return rs_reduce_kernel<2, 1, SLOT, false, true, 0>;
     }
     // (for W <= 2 the tree is one add, the same as rank order, so the rank-order
     // kernels serve it)
