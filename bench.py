@@ -878,8 +878,11 @@ def run_interference(device, seed, quick=False):
             torch.cuda.synchronize()
             return e0.elapsed_time(e1) / n_gemm
 
+        # warm both GEMM streams: cuBLAS sets up a stream's workspace on its first GEMM, and a
+        # cold high-priority stream would inflate that point's time alone
         for _ in range(3 if quick else 5):
             gemm_alone()
+            gemm_alone(s_gemm_hi)
         g = {"gemm": f"bf16 {m}x{n}x{k} torch.matmul (cuBLAS), {n_gemm} per batch",
              "kernel": launch["kernel"], "grid": launch["grid"], "ctas": launch["ctas"],
              "single_wave": (launch["ctas"] <= sms) if launch["ctas"] else None, "points": []}
@@ -1533,8 +1536,11 @@ def run_nccl_compare(group, lay, mine, n_procs, device, grads, rs_tide, short_rs
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / n_gemm
 
+    # the first batch on each stream warms it (cuBLAS sets up a stream's workspace on its
+    # first GEMM); the second is timed
     alone = ev_ms(gemm_batch, s_gemm, 1) / n_gemm
     alone = ev_ms(gemm_batch, s_gemm, 1) / n_gemm
+    alone_hi = ev_ms(gemm_batch, s_gemm_hi, 1) / n_gemm
     alone_hi = ev_ms(gemm_batch, s_gemm_hi, 1) / n_gemm
     cover = alone * n_gemm * 2.0
 
