@@ -1366,6 +1366,29 @@ def run_exchange(args, group, proc, n_procs, device, shared_device):
         ce_ms = timed_calls(lambda: ag(T.TIDE_ENGINE_CE), max(3, min(K, 10)), stream)
         dist.barrier()
         ce_ms = max_over_ranks([ce_ms], device)[0]
+        # the reduction as the pages' two-phase pipeline: the copy engines pull this GPU's rows of
+        # every rank's gradients (peers' over NVLink) into local slots, the SMs reduce them
+        # segment by segment; compared on the device with the plain call's shards
+        pipe = {"segments": min(4, W)}
+        try:
+            rows = {k: [torch.empty(Ns, dtype=torch.bfloat16, device=device) for _ in range(W)]
+                    for k in mine}
+            cs = torch.cuda.Stream(device)
+            plain = {k: outs[k].clone() for k in mine}
+
+            def rs_pipe():
+                for k in mine:
+                    plans[k].rs_reduce_pipelined(gtab, outs[k], rows[k], pipe["segments"], cs)
+
+            pipe_ms = timed_calls(rs_pipe, max(3, min(K, 10)), stream)
+            torch.cuda.synchronize()
+            pipe["same_bits_as_plain"] = all(
+                bool(torch.equal(outs[k].view(torch.int32), plain[k].view(torch.int32))) for k in mine)
+            del rows, plain
+        except Exception as e:  # noqa: BLE001  (the step's figures stand)
+            pipe_ms, pipe["error"] = -1.0, f"{type(e).__name__}: {e}"
+        dist.barrier()
+        pipe_ms = max_over_ranks([pipe_ms], device)[0]
         k_rs, ctas_rs = plans[mine[0]].last_launch()
         nccl = None
         if not shared_device and not args.no_interference:
@@ -1430,7 +1453,11 @@ def run_exchange(args, group, proc, n_procs, device, shared_device):
                 "ag_gather_place": {"ms": round(ag_ms, 4), "alg_bytes": B["ag"],
                                     "nvlink_bytes": B["ag_nvlink"]},
                 "ag_gather_place_ce": {"ms": round(ce_ms, 4), "alg_bytes": B["ag"],
-                                       "nvlink_bytes": B["ag_nvlink"], "kernel": "copy engines"}},
+                                       "nvlink_bytes": B["ag_nvlink"], "kernel": "copy engines"},
+                "rs_reduce_pipelined_ce": {"ms": round(pipe_ms, 4), "alg_bytes": B["rs"],
+                                           "nvlink_bytes": B["rs_nvlink"],
+                                           "kernel": "copy engines pull the rows, SMs reduce them",
+                                           **pipe}},
             "gpu_launches": K * (1 + len(mine)),
             "clocks": clk.summary(),
             "e2e": e2e,

@@ -476,17 +476,27 @@ extern "C" tide_status_t tide_rs_reduce_pipelined(const tide_plan_t* cplan, cons
     tide_plan* p = const_cast<tide_plan*>(cplan);
     tide_status_t st = check_plan(p);
     if (st != TIDE_OK) return st;
-    if ((st = all_ranks(p)) != TIDE_OK) return st;
     if ((st = check_enums(p, TIDE_ENGINE_SM, max_ctas)) != TIDE_OK) return st;
     if ((st = check_reduce_modes(scale_mode, order)) != TIDE_OK) return st;
     if (n_segments < 1 || n_segments > p->world) return TIDE_ERR_INVALID_ARG;
-    const int64_t W = p->world, n_out = W * p->shard_numel;
+    // a one-rank plan (rank r) stages and reduces rank r's rows only: out is [Ns] and each
+    // slot holds one source rank's row r ([Ns]); an all-rank plan's slots are [W][Ns]
+    const bool one = p->rank >= 0;
+    const int64_t W = p->world, n_out = (one ? 1 : W) * p->shard_numel;
     std::vector<Span> spans;
     spans.reserve((size_t)p->world * (p->n_params + 1) + p->n_params + 2);
     if ((st = check_grads(p, grads, grad_numel, spans)) != TIDE_OK) return st;
     if ((st = check_buf(out, out_numel, n_out, 4)) != TIDE_OK) return st;
     add_span(spans, out, 4 * n_out, true);
-    if ((st = check_slots(p, slots, slot_numel, spans)) != TIDE_OK) return st;
+    if (!one) {
+        if ((st = check_slots(p, slots, slot_numel, spans)) != TIDE_OK) return st;
+    } else {
+        if (slots == nullptr) return TIDE_ERR_INVALID_ARG;
+        for (int64_t k = 0; k < W; ++k) {
+            if ((st = check_buf(slots[k], slot_numel, p->shard_numel, 2)) != TIDE_OK) return st;
+            add_span(spans, slots[k], 2 * p->shard_numel, true);
+        }
+    }
     if (overlaps(spans)) return TIDE_ERR_INVALID_ARG;
     if ((st = launchable(p)) != TIDE_OK) return st;
     if (p->tiles.empty()) return TIDE_OK;
@@ -510,7 +520,9 @@ extern "C" tide_status_t tide_rs_reduce_pipelined(const tide_plan_t* cplan, cons
         const int64_t j0 = bounds[seg], j1 = bounds[seg + 1];
         if (j1 == j0) continue;
         // phase 1 of these chunks on the copy engines ...
-        if (tide::ce_slot_stage(p, grads, slots, cs, j0, j1, false) != cudaSuccess) return TIDE_ERR_CUDA;
+        if ((one ? tide::ce_rank_stage(p, grads, slots, cs, j0, j1)
+                 : tide::ce_slot_stage(p, grads, slots, cs, j0, j1, false)) != cudaSuccess)
+            return TIDE_ERR_CUDA;
         cudaEvent_t done = p->seg_events[seg];
         if (cudaEventRecord(done, cs) != cudaSuccess || cudaStreamWaitEvent(s, done, 0) != cudaSuccess)
             return TIDE_ERR_CUDA;

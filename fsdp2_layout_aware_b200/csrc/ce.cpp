@@ -241,7 +241,7 @@ CeOp rows_op(void* dst, size_t dpitch, const void* src, size_t spitch, size_t wi
 // Recorded graphs kept per plan (the least recently used one is replaced).
 constexpr size_t kMaxCeGraphs = 4;
 
-enum { kCallPlace = 1, kCallGather = 2, kCallStage = 3 };
+enum { kCallPlace = 1, kCallGather = 2, kCallStage = 3, kCallRankStage = 4 };
 
 // Issue the planned lists (q->lists) as one call on `stream`: replay the graph
 // recorded for (kind, j0, j1, key) if there is one, else record it now and
@@ -413,6 +413,29 @@ cudaError_t ce_slot_stage(tide_plan* p, const void* const* grads, void* const* s
                 const int64_t rem = n - full * c;       // rank `full` holds a partial chunk
                 if (rem > 0 && full < W && full >= r0 && full < r1)
                     l.push_back(rows_op(dst + full * Ns, 0, g + full * c, 0, 2 * rem, 1));
+            }
+        }
+    });
+}
+
+// One rank's Slot-Reuse phase 1 (a one-rank plan, rank r): for the chunks
+// [j0, j1) that are rank r's (chunk i*W + r), chunk r of every source rank k's
+// gradient of param i goes to slots[k] + off_i, one 1-D copy per (k, i) with
+// data, on the fan-out stream of the source rank.  The sources may be peers'
+// memory, so the copy engines carry the transfer.
+cudaError_t ce_rank_stage(tide_plan* p, const void* const* grads, void* const* slots,
+                          cudaStream_t caller, int64_t j0, int64_t j1) {
+    const int64_t W = p->world, P = p->n_params, r = p->rank;
+    return run_call(p, caller, kCallRankStage, j0, j1, {}, false, [&](CeIssuer* q) {
+        for (int64_t i = j0 / W; i < P && i * W + r < j1; ++i) {
+            if (i * W + r < j0) continue;
+            const int64_t c = p->chunk[i];
+            const int64_t valid = std::min(c, std::max<int64_t>(0, p->numel[i] - r * c));
+            if (valid == 0) continue;
+            for (int64_t k = 0; k < W; ++k) {
+                const uint16_t* g = static_cast<const uint16_t*>(grads[k * P + i]) + r * c;
+                uint16_t* dst = static_cast<uint16_t*>(slots[k]) + p->offset[i];
+                q->lists[k % kFanout].push_back(rows_op(dst, 0, g, 0, 2 * valid, 1));
             }
         }
     });

@@ -114,6 +114,10 @@ cudaError_t ce_ag_gather(tide_plan* p, const void* const* shards, void* const* p
 cudaError_t ce_slot_stage(tide_plan* p, const void* const* grads, void* const* slots,
                           cudaStream_t stream, int64_t j0 = 0, int64_t j1 = -1, bool record = false,
                           bool one_source = false);
+// A one-rank plan's phase 1: chunk `rank` of every rank k's gradients into
+// slots[k] (that rank's row only, Ns elements), for the chunks [j0, j1).
+cudaError_t ce_rank_stage(tide_plan* p, const void* const* grads, void* const* slots,
+                          cudaStream_t stream, int64_t j0, int64_t j1);
 // Stops and frees the plan's copy-issuing threads and recorded graphs.
 void ce_release(tide_plan* p);
 

@@ -309,6 +309,12 @@ TIDE_API tide_status_t tide_rs_reduce_slots(const tide_plan_t* plan, const void*
  * work enqueued on `stream` after it sees the complete result.  `copy_stream`
  * may equal `stream` (the phases then run one after the other).  The plan
  * creates its pacing events (no device memory) on first use.
+ * With a one-rank plan (rank r) the call is that rank's share of the
+ * exchange: out is its fp32 shard [Ns] (out_numel >= Ns), and slots[k] receives
+ * rank k's row r only (slot_numel >= Ns each): chunk r of rank k's gradient of
+ * param i lands at slots[k] + off_i.  The gradients may be peers' memory, so
+ * the copy engines carry the transfer and the SMs reduce from local slots;
+ * the result equals the one-rank tide_rs_reduce (same bits).
  */
 TIDE_API tide_status_t tide_rs_reduce_pipelined(const tide_plan_t* plan, const void* const* grads,
                                                 const int64_t* grad_numel, float* out,

@@ -53,13 +53,20 @@ def exchange_worker(proc, n_procs, port, shapes, world, seed, out_dir):
             gtab = T.PointerTable(gp, gn, keep=[grads])
             stab = T.PointerTable(X.shard_table(lay, world, n_procs, peers.bases("shards", n_procs)),
                                   [Ns] * world, keep=[shards])
-            outs, trees = {}, {}
+            outs, trees, pipes = {}, {}, {}
             for k in mine:
                 plan = T.Plan(group.shapes, world, rank=k)
                 outs[k] = torch.full((Ns,), float("nan"), device="cuda")
                 plan.rs_reduce(gtab, outs[k], scale_mode=T.TIDE_SCALE_INV_WORLD)
                 trees[k] = torch.full((Ns,), float("nan"), device="cuda")
                 plan.rs_reduce(gtab, trees[k], scale_mode=T.TIDE_SCALE_NONE, order=T.TIDE_ORDER_TREE)
+                # the same shard with the copy engines pulling row k of every rank's gradients
+                # (peers' included) into local slots, reduced segment by segment on the SMs
+                rows = [torch.full((Ns,), -1, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+                        for _ in range(world)]
+                pipes[k] = torch.full((Ns,), float("nan"), device="cuda")
+                plan.rs_reduce_pipelined(gtab, pipes[k], rows, min(3, world), torch.cuda.Stream(),
+                                         scale_mode=T.TIDE_SCALE_INV_WORLD)
                 torch.cuda.synchronize()
                 plan.check()
             placed = {}
@@ -73,6 +80,7 @@ def exchange_worker(proc, n_procs, port, shapes, world, seed, out_dir):
             for k in mine:
                 np.save(os.path.join(out_dir, f"rs_{k}.npy"), outs[k].cpu().numpy())
                 np.save(os.path.join(out_dir, f"tree_{k}.npy"), trees[k].cpu().numpy())
+                np.save(os.path.join(out_dir, f"pipe_{k}.npy"), pipes[k].cpu().numpy())
             for name, params in placed.items():
                 for i, p in enumerate(params):
                     np.save(os.path.join(out_dir, f"ag_{name}_{proc}_{i}.npy"), bits_of(p))

@@ -350,8 +350,15 @@ def test_rank_plan_arguments():
                                   0, 0) == T.TIDE_ERR_SIZE
     assert T.tide_rs_reduce_slots(plan.handle, a["slots"], a["n_slot"] - 1, a["out"], L.Ns, 1, 0,
                                   0, 0) == T.TIDE_ERR_SIZE
-    assert T.tide_rs_reduce_pipelined(plan.handle, a["grads"], a["gnum"], a["out"], a["n_out"], 1, 0,
-                                      a["slots"], a["n_slot"], 1, 0, 0, 0) == T.TIDE_ERR_INVALID_ARG
+    # the pipelined Slot-Reuse takes it: one shard out, each slot one source rank's row
+    def pipe(out_n=L.Ns, slot_n=L.Ns, segs=1):
+        return T.tide_rs_reduce_pipelined(plan.handle, a["grads"], a["gnum"], a["out"], out_n, 1, 0,
+                                          a["slots"], slot_n, segs, 0, 0, 0)
+    assert pipe() == T.TIDE_ERR_DEVICE
+    assert pipe(segs=g.world) == T.TIDE_ERR_DEVICE
+    assert pipe(segs=g.world + 1) == T.TIDE_ERR_INVALID_ARG
+    assert pipe(out_n=L.Ns - 1) == T.TIDE_ERR_SIZE
+    assert pipe(slot_n=L.Ns - 1) == T.TIDE_ERR_SIZE
     assert T.tide_ag_gather_place(plan.handle, a["slots"], L.Ns, a["params"], a["pnum"], 0, 0,
                                   0) == T.TIDE_ERR_INVALID_ARG
 

@@ -54,6 +54,7 @@ def test_exchange_over_ipc_matches_oracle(world, n_procs, tmp_path):
     for k in range(world):
         assert np.array_equal(np.load(tmp_path / f"rs_{k}.npy").view(np.uint32), ref[k]), k
         assert np.array_equal(np.load(tmp_path / f"tree_{k}.npy").view(np.uint32), tree[k]), k
+        assert np.array_equal(np.load(tmp_path / f"pipe_{k}.npy").view(np.uint32), ref[k]), k
     for p in range(n_procs):
         for name in ("sm", "ce"):
             for i in range(group.n_params):

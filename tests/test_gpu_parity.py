@@ -393,6 +393,39 @@ def test_slot_reuse_pipelined(group, segments):
             assert np.array_equal(bits_of(slots[k]), exp)
 
 
+@pytest.mark.parametrize("group", PIPE_GROUPS, ids=[f"{g.name}_w{g.world}" for g in PIPE_GROUPS])
+def test_one_rank_pipelined_pulls_its_rows_on_the_copy_engines(group):
+    """A one-rank plan's pipelined Slot-Reuse: the copy engines pull row r of every rank's
+    gradients into W compact slots, the SMs reduce them segment by segment.  Each rank's shard
+    equals the oracle's rows r (rank order, and tree order against the tree oracle), and each
+    slot holds the oracle's staging of that rank restricted to row r (its pads untouched)."""
+    W = group.world
+    grads = synth.grads_host(group, seed=57)
+    L = oracle.layout(W, group.shapes)
+    refs = {T.TIDE_ORDER_RANK: oracle.rs_reduce(W, group.shapes, grads, 1).reshape(W, L.Ns),
+            T.TIDE_ORDER_TREE: oracle.rs_reduce_tree(W, group.shapes, grads, 1).reshape(W, L.Ns)}
+    staged = []
+    for k in range(W):
+        exp = np.full(W * L.Ns, 0xFFFF, dtype=np.uint16)
+        oracle.slot_stage(W, group.shapes, grads[k], exp)
+        staged.append(exp.reshape(W, L.Ns))
+    dev = grads_to_dev(group, grads)
+    cs = torch.cuda.Stream()
+    for r in range(W):
+        plan = T.Plan(group.shapes, W, rank=r)
+        for order in (T.TIDE_ORDER_RANK, T.TIDE_ORDER_TREE):
+            for n_seg in sorted({1, min(3, W), W}):
+                rows = [torch.full((L.Ns,), -1, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+                        for _ in range(W)]
+                out = torch.full((L.Ns,), float("nan"), device="cuda")
+                plan.rs_reduce_pipelined(dev, out, rows, n_seg, cs, order=order)
+                torch.cuda.synchronize()
+                plan.check()
+                assert np.array_equal(f32_bits(out), refs[order][r].view(np.uint32)), (r, order, n_seg)
+                for k in range(W):
+                    assert np.array_equal(bits_of(rows[k]), staged[k][r]), (r, k, n_seg)
+
+
 def test_slot_phases_separately():
     group = mini_wan()
     grads = synth.grads_host(group, seed=52)
