@@ -35,6 +35,7 @@ void free_device(tide_plan* p) {
     cudaFree(p->d_tiles);
     cudaFree(p->d_numel);
     cudaFree(p->d_err);
+    cudaFree(p->d_counter);
     cudaFree(p->grad_tab.dev);
     cudaFree(p->param_tab.dev);
     cudaFree(p->slot_tab.dev);
@@ -42,6 +43,7 @@ void free_device(tide_plan* p) {
     p->d_tiles = nullptr;
     p->d_numel = nullptr;
     p->d_err = nullptr;
+    p->d_counter = nullptr;
     p->grad_tab.dev = p->param_tab.dev = p->slot_tab.dev = p->shard_tab.dev = nullptr;
 }
 
@@ -62,6 +64,7 @@ tide_status_t upload(tide_plan* p) {
     if (e == cudaSuccess) e = dev_alloc(&p->d_tiles, T, &total);
     if (e == cudaSuccess) e = dev_alloc(&p->d_numel, 2 * P, &total);
     if (e == cudaSuccess) e = dev_alloc(&p->d_err, 1, &total);
+    if (e == cudaSuccess) e = dev_alloc(&p->d_counter, 2, &total);
     if (e == cudaSuccess) e = dev_alloc(&p->grad_tab.dev, W * P, &total);
     if (e == cudaSuccess) e = dev_alloc(&p->param_tab.dev, P, &total);
     if (e == cudaSuccess) e = dev_alloc(&p->slot_tab.dev, W, &total);
@@ -84,6 +87,8 @@ tide_status_t upload(tide_plan* p) {
         e = cudaMemcpy(p->d_numel, n2.data(), sizeof(int64_t) * 2 * P, cudaMemcpyHostToDevice);
     }
     if (st == TIDE_OK && e == cudaSuccess) e = cudaMemset(p->d_err, 0, sizeof(int32_t));
+    if (st == TIDE_OK && e == cudaSuccess)
+        e = cudaMemset(p->d_counter, 0, 2 * sizeof(unsigned long long));
     if (st == TIDE_OK && e == cudaSuccess)
         e = cudaDeviceGetAttribute(&p->sm_count, cudaDevAttrMultiProcessorCount, p->device);
     if (st == TIDE_OK && e != cudaSuccess) st = TIDE_ERR_CUDA;

@@ -62,6 +62,10 @@ struct RsParams {
     float scale;
     int32_t do_scale;
     int32_t* err;
+    // dynamic != 0: after its first tile (blockIdx.x) each CTA claims the next unclaimed
+    // tile from counter[0]; counter[1] counts finished CTAs.  Both are zero at launch.
+    int32_t dynamic;
+    unsigned long long* counter;
 };
 
 // V32: 32-byte loads and stores (16 outputs per thread per step); the host
@@ -96,12 +100,26 @@ rs_reduce_kernel(const RsParams a) {
     const int W = a.world;
 
     // Every thread keeps the next tile's descriptor in registers: its load is
-    // in flight while the current tile is reduced, so no tile waits on it.
+    // in flight while the current tile is reduced, so no tile waits on it.  The
+    // next tile is t + gridDim.x, or, with dynamic claiming, one claimed from
+    // the counter at the start of the current tile (the claim is in flight
+    // while the tile's sources are staged, and read after the tile's barrier).
+    __shared__ int64_t s_next[2];
+    // (claiming is compiled only into the kernels of W > 4 outside the one-group tree: those
+    // run at 3-4 CTAs per SM on 64-80 registers, which the claim's registers would push
+    // into spills; the host's flag is then ignored and they keep the fixed stride)
+    constexpr bool kClaim = G >= 8 && !(TREE && NG == -1);
+    const bool dyn = kClaim && a.dynamic;
     int64_t t = blockIdx.x;
     tide_tile_t next = t < a.n_tiles ? a.tiles[t] : tide_tile_t{};
-    for (int buf = 0; t < a.n_tiles; t += gridDim.x, buf ^= 1) {
+    for (int buf = 0; t < a.n_tiles; buf ^= 1) {
         const tide_tile_t tl = next;
-        if (t + gridDim.x < a.n_tiles) next = a.tiles[t + gridDim.x];
+        int64_t nt = t + gridDim.x;
+        if (dyn) {
+            if (tid == 0) s_next[buf] = (int64_t)gridDim.x + (int64_t)atomicAdd(a.counter, 1ull);
+        } else if (nt < a.n_tiles) {
+            next = a.tiles[nt];
+        }
 
         // Range check of the descriptor against the buffers the host validated.
         const bool param_ok = tl.param >= 0 && tl.param < a.n_params;
@@ -129,7 +147,14 @@ rs_reduce_kernel(const RsParams a) {
             misaligned |= (reinterpret_cast<uintptr_t>(dst) & 31) != 0;
         }
         const bool scalar_only = __syncthreads_or(misaligned);
-        if (!ok) continue;  // skipped after the barrier, so every tile keeps exactly one
+        if (dyn) {
+            nt = s_next[buf];
+            if (nt < a.n_tiles) next = a.tiles[nt];
+        }
+        if (!ok) {  // skipped after the barrier, so every tile keeps exactly one
+            t = nt;
+            continue;
+        }
 
         int nv;  // 8-element units covered by the vector body
         if (V32) {
@@ -201,6 +226,17 @@ rs_reduce_kernel(const RsParams a) {
         }
         // Pad positions are +0.0.
         for (int e = tl.n_valid + tid; e < tl.n_total; e += kThreads) dst[e] = 0.0f;
+        t = nt;
+    }
+    // With dynamic claiming the last CTA to finish puts both counters back to zero for the
+    // next launch on the stream (each CTA's claims precede its count, fenced).
+    if (dyn && tid == 0) {
+        __threadfence();
+        if (atomicAdd(a.counter + 1, 1ull) == (unsigned long long)gridDim.x - 1) {
+            a.counter[0] = 0;
+            a.counter[1] = 0;
+            __threadfence();
+        }
     }
 }
 
@@ -283,6 +319,14 @@ cudaError_t launch_rs_reduce(const tide_plan* p, const void* const* d_src_tab, b
     a.scale = scale;
     a.do_scale = do_scale ? 1 : 0;
     a.err = p->d_err;
+    // Claiming tiles as CTAs finish evens out CTAs that run slower than others (their end
+    // is the launch's tail): 70B W=8 7.06 -> 7.18 TB/s, Wan2.2 W=16 6.94 -> 7.17, the
+    // sweep's W = 64 group 6.86 -> 7.14.  A claim costs a global atomic per tile, hidden by
+    // a second CTA on the SM; with few tiles per CTA there is no tail to even out and the
+    // claims cost more than they save (sweep W=2: -10 %, W=8: -1 %), so launches with under
+    // 2 CTAs per SM or under 16 tiles per CTA keep the fixed stride, and so does W <= 4.
+    a.dynamic = (p->world > 4 && grid >= 2 * p->sm_count && t1 - t0 >= 16 * (int64_t)grid) ? 1 : 0;
+    a.counter = p->d_counter;
     (void)cudaGetLastError();  // drop an error left by an earlier failed runtime call
     select(p->world, slot, order, v32)<<<grid, kThreads, 0, stream>>>(a);
     return cudaGetLastError();

@@ -59,6 +59,7 @@ struct tide_plan {
     tide_tile_t* d_tiles = nullptr;
     int64_t* d_numel = nullptr;
     int32_t* d_err = nullptr;
+    unsigned long long* d_counter = nullptr;  // the reduction's tile claim counters (2 words)
     PtrTable grad_tab, param_tab, slot_tab, shard_tab;
     int64_t workspace_bytes = 0;
 

@@ -35,7 +35,8 @@
  *   - All arguments are validated on the host before anything is enqueued; on
  *     any error status nothing has been enqueued.
  *   - A plan keeps small device tables (tile list, pointer tables, an error
- *     word).  A pointer table is re-uploaded, stream-ordered, only when its
+ *     word, and two counters with which the reduction's CTAs claim tiles on long
+ *     launches; the launch's last CTA puts them back to zero).  A pointer table is re-uploaded, stream-ordered, only when its
  *     contents change.  One plan must be used from one stream at a time (or the
  *     caller orders the streams) and from one host thread at a time; different
  *     plans are independent.

@@ -673,8 +673,9 @@ def test_workspace_is_tables_only():
         g = configs.by_name(name)
         plan = T.Plan(g.shapes, g.world)
         W, P = g.world, g.n_params
-        # tiles, numel table, error word, pointer tables: grads, params, slots, shards
-        expect = plan.n_tiles * 32 + 2 * P * 8 + 4 + W * P * 8 + P * 8 + W * 8 + W * 8
+        # tiles, numel table, error word, the reduction's two tile-claim counters, pointer
+        # tables: grads, params, slots, shards
+        expect = plan.n_tiles * 32 + 2 * P * 8 + 4 + 2 * 8 + W * P * 8 + P * 8 + W * 8 + W * 8
         assert plan.workspace_bytes == expect
 
 
@@ -749,3 +750,28 @@ def test_copy_engine_calls_replay_recorded_graphs(group):
             oracle.slot_stage(W, group.shapes, grads[k], exp)
             assert np.array_equal(bits_of(slots[k]), exp)
     plan.check()
+
+
+def test_tile_claims_on_long_launches_repeat_and_mix_with_fixed_strides():
+    """Launches with 2+ CTAs per SM and 16+ tiles per CTA claim tiles from the plan's counters,
+    and the launch's last CTA puts them back to zero.  Back-to-back launches on one plan
+    (claiming, claiming, a capped fixed-stride launch, claiming, Slot-Reuse) each give the
+    oracle's bits, so no launch inherits another's claims."""
+    group = configs.Group("claims", 8, tuple((1024, 4096) for _ in range(16)))
+    grads = synth.grads_host(group, seed=63)
+    ref = oracle.rs_reduce(8, group.shapes, grads, 1).view(np.uint32)
+    plan = T.Plan(group.shapes, 8)
+    assert plan.n_tiles >= 16 * plan.launch_ctas(T.K_RS_V32, 0)
+    dev = grads_to_dev(group, grads)
+    n = 8 * plan.shard_numel
+    for cap in (0, 0, 7, 0):
+        out = torch.full((n,), float("nan"), device="cuda")
+        plan.rs_reduce(dev, out, max_ctas=cap)
+        torch.cuda.synchronize()
+        plan.check()
+        assert np.array_equal(f32_bits(out), ref), cap
+    slots = [torch.empty(n, dtype=torch.bfloat16, device="cuda") for _ in range(8)]
+    out = torch.full((n,), float("nan"), device="cuda")
+    plan.rs_reduce(dev, out, slots=slots)
+    torch.cuda.synchronize()
+    assert np.array_equal(f32_bits(out), ref)
