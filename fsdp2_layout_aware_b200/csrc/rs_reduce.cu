@@ -12,7 +12,8 @@
 // Design (HBM-bound: W*2 bytes read and 4 bytes written per output element,
 // ~(W-1)/(2W+4) flop/byte, so no tensor cores):
 //   - a persistent grid, at most max_ctas CTAs, walks the plan's tile list
-//     round-robin; a tile is a piece of one (param, rank) chunk of up to
+//     round-robin, or on long launches claims tiles from a counter as CTAs
+//     finish them; a tile is a piece of one (param, rank) chunk of up to
 //     TIDE_TILE_ELEMS elements, so tiny MoE chunks and huge dense chunks mix;
 //   - per tile the W source addresses are staged in shared memory once (one
 //     barrier per tile; the next tile's descriptor is already in registers);
