@@ -775,3 +775,14 @@ def test_tile_claims_on_long_launches_repeat_and_mix_with_fixed_strides():
     plan.rs_reduce(dev, out, slots=slots)
     torch.cuda.synchronize()
     assert np.array_equal(f32_bits(out), ref)
+    # two plans claim from their own counters: their launches may run at the same time
+    other = T.Plan(group.shapes, 8)
+    outs = [torch.full((n,), float("nan"), device="cuda") for _ in range(2)]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    torch.cuda.synchronize()
+    for _ in range(2):
+        for pl, o, st in zip((plan, other), outs, streams):
+            pl.rs_reduce(dev, o, stream=st)
+    torch.cuda.synchronize()
+    for o in outs:
+        assert np.array_equal(f32_bits(o), ref)
