@@ -148,3 +148,48 @@ def test_exchange_bytes_add_up_to_the_single_gpu_step():
         # NVLink: the share of each read held by other processes
         assert sum(b["rs_nvlink"] for b in parts) == B1["rs_read"] * (g.world - per) // g.world
         assert all(b["ag_nvlink"] == B1["ag_read"] * (g.world - per) // g.world for b in parts)
+
+
+def test_a_peer_allocation_is_mapped_once_and_unmapped_after_its_last_user(monkeypatch):
+    """CUDA maps an IPC handle at most once per process and device, and several arenas (of
+    different parameter groups) may share one allocation: open_shared hands later users the
+    first mapping and close_shared unmaps only after the last of them."""
+    calls = []
+
+    def fake_open(handle, device):
+        calls.append(("open", bytes(handle), device))
+        return T.TIDE_OK, 0x1000 * (len(calls) + 1)
+
+    def fake_close(base, device):
+        calls.append(("close", base, device))
+        return T.TIDE_OK
+
+    monkeypatch.setattr(T, "tide_ipc_open", fake_open)
+    monkeypatch.setattr(T, "tide_ipc_close", fake_close)
+    monkeypatch.setattr(X, "_MAPPED", {})
+    h1, h2 = b"a" * T.TIDE_IPC_HANDLE_BYTES, b"b" * T.TIDE_IPC_HANDLE_BYTES
+    st, b1 = X.open_shared(h1, 0)
+    st2, b1_again = X.open_shared(h1, 0)
+    st3, b2 = X.open_shared(h2, 0)
+    st4, b1_other_device = X.open_shared(h1, 1)
+    assert st == st2 == st3 == st4 == T.TIDE_OK
+    assert b1 == b1_again and len({b1, b2, b1_other_device}) == 3
+    assert [c[0] for c in calls] == ["open", "open", "open"]
+    assert X.close_shared(b1, 0) == T.TIDE_OK            # one user of h1 on device 0 remains
+    assert [c[0] for c in calls].count("close") == 0
+    assert X.close_shared(b1, 0) == T.TIDE_OK            # the last one: unmapped now
+    assert calls[-1] == ("close", b1, 0)
+    X.close_shared(b2, 0)
+    X.close_shared(b1_other_device, 1)
+    assert X._MAPPED == {}
+    # two PeerMaps over exports that share an allocation open it once between them
+    exports = [{"arena": (h1, 0)}, {"arena": (h1, 4096)}]
+    calls.clear()
+    m1 = X.PeerMaps(exports[:1] + [{"arena": (h2, 0)}], 1, 0, {"arena": 0xAAAA})
+    m2 = X.PeerMaps([{"arena": (h1, 256)}, {"arena": (h2, 0)}], 1, 0, {"arena": 0xBBBB})
+    assert [c[0] for c in calls] == ["open"]
+    assert m2.bases("arena", 2)[0] == m1.bases("arena", 2)[0] + 256
+    m1.close()
+    assert [c[0] for c in calls] == ["open"]
+    m2.close()
+    assert [c[0] for c in calls] == ["open", "close"]
