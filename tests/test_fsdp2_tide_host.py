@@ -38,3 +38,45 @@ def test_fsdp2_with_tide_comms_gives_stock_fsdp2_results(world, tmp_path):
         # backward), then the root (kept unsharded from forward to backward)
         assert calls[0] == calls[1] == ["place", "place", "stage", "reduce"] * steps
         assert calls[2] == ["place", "stage", "reduce"] * steps
+
+
+def test_tide_comms_hand_out_the_groups_buffers_and_refuse_others():
+    """The all-gather buffer FSDP2 asks for is the group's arena; the reduce-scatter's fp32
+    [W][Ns] input is one element expanded to that shape (never materialized) and its [Ns]
+    output a fresh fp32 tensor; any other request is refused."""
+    import types
+
+    import torch
+    from fsdp2_layout_aware_b200 import fsdp2 as F
+
+    W, Ns = 3, 40
+    tg = types.SimpleNamespace(world=W, shard_numel=Ns, device=torch.device("cpu"),
+                               arena=torch.zeros(W * Ns, dtype=torch.bfloat16),
+                               rs_input=torch.zeros(1), reduced=[])
+    tg.reduce = lambda out, op: tg.reduced.append((out.numel(), op))
+    tg.meet = lambda: None
+    ag_cls, rs_cls = F._comm_classes()
+    ag, rs = ag_cls(tg), rs_cls(tg)
+    buf = ag.allocate((W * Ns,), dtype=torch.bfloat16, device=tg.device)
+    assert buf.data_ptr() == tg.arena.data_ptr()
+    with pytest.raises(ValueError):
+        ag.allocate((W * Ns + 1,), dtype=torch.bfloat16, device=tg.device)
+    with pytest.raises(ValueError):
+        ag.allocate((W * Ns,), dtype=torch.float32, device=tg.device)
+    assert ag(buf, buf[:Ns], group=None) is None
+    with pytest.raises(ValueError):
+        ag(torch.zeros(W * Ns, dtype=torch.bfloat16), buf[:Ns], group=None)
+    inp = rs.allocate((W * Ns,), dtype=torch.float32, device=tg.device)
+    assert inp.shape == (W * Ns,) and inp.stride() == (0,) and inp.data_ptr() == tg.rs_input.data_ptr()
+    assert inp.view(W, -1).data_ptr() == tg.rs_input.data_ptr()     # FSDP2's pack target
+    out = rs.allocate((Ns,), dtype=torch.float32, device=tg.device)
+    assert out.shape == (Ns,) and out.dtype == torch.float32 and out.data_ptr() != inp.data_ptr()
+    with pytest.raises(ValueError):
+        rs.allocate((Ns + 1,), dtype=torch.float32, device=tg.device)
+    with pytest.raises(ValueError):
+        rs.allocate((Ns,), dtype=torch.bfloat16, device=tg.device)
+    import torch.distributed as dist
+    assert rs(out, inp, group=None, op=dist.ReduceOp.AVG) is None
+    assert tg.reduced == [(Ns, dist.ReduceOp.AVG)]
+    with pytest.raises(ValueError):
+        rs(out, torch.zeros(W * Ns), group=None, op=dist.ReduceOp.AVG)
