@@ -117,3 +117,17 @@ def test_rs_sm_time_counts_sms_held_times_duration():
     assert r["stock_over_tide"] == round(30.0 / 2.4, 2)
     capped = bench.rs_sm_time(40.0, 4, v, 148)                 # 4 CTAs hold 4 SMs
     assert capped["tide_rs_reduce"] == 160.0
+
+
+def test_traffic_record_is_current_and_close_to_the_algorithmic_bytes():
+    """profiles/ncu_traffic.txt holds one small-case capture per kernel, keyed by a digest of
+    its sources: every entry matches the sources as they are now (so the bench reports its
+    traffic), and the scaled traffic of a 70B launch is within 0.5 % of the algorithmic bytes
+    (a kernel that re-read its inputs would show up here)."""
+    import bench
+    for kernel, sources in (("rs_v32", bench.RS_SOURCES), ("rs_tree_v32", bench.RS_SOURCES),
+                            ("ag", bench.AG_SOURCES)):
+        rd, wr = (13690208256, 3422552064) if kernel.startswith("rs") else (3422552064, 3422552064)
+        traffic, note = bench.ncu_traffic(kernel, sources, rd, wr)
+        assert traffic is not None, (kernel, note)
+        assert abs(traffic / (rd + wr) - 1.0) < 0.005, (kernel, traffic)
