@@ -786,3 +786,21 @@ def test_tile_claims_on_long_launches_repeat_and_mix_with_fixed_strides():
     torch.cuda.synchronize()
     for o in outs:
         assert np.array_equal(f32_bits(o), ref)
+
+
+@pytest.mark.parametrize("world", [128, 256])
+def test_widest_groups_both_orders(world):
+    """W = 128 and 256 (the library's limit): rank order on the 32-byte kernel, tree order on
+    the run-time merge-stack kernel, both against the oracle; a ragged param and a param with
+    fewer rows than ranks included."""
+    group = configs.Group(f"wide_w{world}", world,
+                          ((world * 24, 32), (world * 3 + 5, 16), (7, 48), (world * 48,)))
+    grads = synth.grads_host(group, seed=67)
+    for order, fn, kernel in ((0, oracle.rs_reduce, T.K_RS_V32), (1, oracle.rs_reduce_tree, T.K_RS_TREE)):
+        ref = fn(world, group.shapes, grads, 1)
+        out, _, plan = run_rs(group, grads, scale=1, order=order)
+        assert plan.last_launch()[0] == kernel
+        assert np.array_equal(f32_bits(out), ref.view(np.uint32)), order
+    E, A = oracle.exact_f64(world, group.shapes, grads)
+    out, _, _ = run_rs(group, grads, scale=0, order=1)
+    assert np.all(np.abs(out.cpu().numpy().astype(np.float64) - E) <= 1e-6 * A)
