@@ -231,3 +231,47 @@ def test_device_generator_matches_host():
             h = synth.grad_host(q, 3, k, i)
             assert np.array_equal(bits_of(devq[k][i]), h)
             assert (i in zero) == (not h.any())
+
+
+def test_a_param_beyond_2_to_the_31_elements():
+    """One param of (2^21 + 3) x 1024 = 2,147,486,720 elements (more than 2^31) over W = 2: its
+    chunk offsets, the fp32 shards' indices and the placement's destination indices pass 2^31,
+    so any 32-bit element index would show.  Sampled outputs (chunk ends, the valid/pad
+    boundary, random positions, and the positions around element 2^31 of the output and of
+    the padded storage) against the oracle's answer for each position, RS and AG."""
+    group = configs.Group("beyond_2_31", 2, ((2 ** 21 + 3, 1024), (5,)))
+    rng = np.random.default_rng(11)
+    torch.cuda.empty_cache()
+    plan = T.Plan(group.shapes, group.world)
+    L = oracle.layout(group.world, group.shapes)
+    assert group.numel(0) > 2 ** 31 and 2 * L.Ns > 2 ** 31
+    grads = synth.dev_grads(group, SEED)
+    out = torch.full((2 * L.Ns,), float("nan"), device="cuda")
+    plan.rs_reduce(grads, out, scale_mode=T.TIDE_SCALE_INV_WORLD)
+    torch.cuda.synchronize()
+    plan.check()
+    check_rs(group, out, L, 1, rng, n_random=5000)
+    pos = [(int(f // L.Ns), int(f % L.Ns)) for f in range(2 ** 31 - 40, 2 ** 31 + 40)]
+    flat = torch.tensor([r * L.Ns + j for r, j in pos], dtype=torch.int64, device="cuda")
+    got = out[flat].cpu().numpy()
+    assert np.array_equal(got.view(np.uint32), expected_rs(group, L, pos, 1).view(np.uint32))
+    del grads, out
+    torch.cuda.empty_cache()
+    ag = synth.dev_ag(group, L.Ns, SEED)
+    params = [torch.full((2 * L.c[i],), 0x7777, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+              for i in range(group.n_params)]
+    plan.ag_place(ag, params)
+    torch.cuda.synchronize()
+    plan.check()
+    check_ag(group, params, L, rng, n_random=2000)
+    qs = list(range(2 ** 31 - 40, 2 ** 31 + 40))
+    got = bits_of(params[0][torch.tensor(qs, dtype=torch.int64, device="cuda")])
+    exp = np.zeros(len(qs), dtype=np.uint16)
+    for n, q in enumerate(qs):
+        st, a = oracle.ag_source(2, group.shapes, 0, q)
+        if st == 1:
+            exp[n] = synth.gather_bf16(np.array([a % L.Ns], dtype=np.int64), SEED, synth.STREAM_AG,
+                                       a // L.Ns, 0, group.param_sigma)[0]
+    assert np.array_equal(got, exp)
+    del ag, params
+    torch.cuda.empty_cache()
