@@ -628,6 +628,7 @@ def test_cuda_graph_capture_and_replay(group):
     plan.check()
 
 
+@pytest.mark.filterwarnings("ignore:Warning. Profiler clears events")
 def test_copy_engine_paths_launch_no_kernel():
     """AG placement and Slot-Reuse staging on the copy engines use no SM: the CUDA
     activity trace of those calls holds memcpy/memset records and no kernel."""
