@@ -36,7 +36,8 @@
  *     any error status nothing has been enqueued.
  *   - A plan keeps small device tables (tile list, pointer tables, an error
  *     word, and two counters with which the reduction's CTAs claim tiles on long
- *     launches; the launch's last CTA puts them back to zero).  A pointer table is re-uploaded, stream-ordered, only when its
+ *     launches; the launch's last CTA puts them back to zero, so two reductions of
+ *     one plan must never run at the same time: they would share the counters).  A pointer table is re-uploaded, stream-ordered, only when its
  *     contents change.  One plan must be used from one stream at a time (or the
  *     caller orders the streams) and from one host thread at a time; different
  *     plans are independent.
