@@ -31,9 +31,9 @@ that no rank writes its arena while another may still read it: before a placemen
 row is in), after it (before anyone stages gradients over its row), before a reduction
 (every rank staged) and after it (before the next copy-in).  The parameter group must have
 bf16 compute parameters and fp32 reduction (the mixed-precision policy set here); every
-collective is synchronous.  Every parameter of a group must receive a gradient in each
-backward: FSDP2 leaves parameters without one out of its reduce-scatter, which changes the
-buffer layout, and the group's calls then refuse the buffers with an error.
+collective is synchronous.  Parameters without a gradient (frozen ones) are left out of
+FSDP2's reduce-scatter; the layout of the ones that have one follows from their shapes in
+group order, and the group builds plans for that subset on first use.
 """
 from __future__ import annotations
 
@@ -93,6 +93,23 @@ class TideGroup:
             _RS[self.rs_input.data_ptr()] = self
         self.placements = 0
         self.reductions = 0
+        # plans for the parameters that get gradients, when some do not (frozen ones): FSDP2
+        # reduce-scatters only those, in group order, so their shapes fix the layout
+        self._sub_plans = {}
+        self.pending = None   # (one-rank plan, shard numel) of the staged reduction
+
+    def plans_for(self, shapes):
+        """(all-rank plan, one-rank plan, shard numel) for a reduction over `shapes`."""
+        shapes = tuple(tuple(int(d) for d in s) for s in shapes)
+        if list(shapes) == self.shapes:
+            return self.plan, self.rank_plan, self.shard_numel
+        ent = self._sub_plans.get(shapes)
+        if ent is None:
+            plan = T.Plan(shapes, self.world, device=self.device)
+            ent = (plan, T.Plan(shapes, self.world, device=self.device, rank=self.rank),
+                   plan.shard_numel)
+            self._sub_plans[shapes] = ent
+        return ent
 
     def meet(self) -> None:
         import torch
@@ -112,20 +129,27 @@ class TideGroup:
         self.placements += 1
 
     def stage(self, grads) -> None:
-        """FSDP2's pack: this rank's bf16 gradients into its arena (Slot-Reuse phase 1)."""
+        """FSDP2's pack: this rank's bf16 gradients into its arena (Slot-Reuse phase 1).  The
+        gradients are those of the group's parameters that got one, in group order."""
         import torch
-        if len(grads) != len(self.shapes):
+        if not 0 < len(grads) <= len(self.shapes):
             raise ValueError("gradients do not match the group's parameters")
-        for g, s in zip(grads, self.shapes):
-            if g.dtype != torch.bfloat16 or tuple(g.shape) != s or not g.is_contiguous():
+        for g in grads:
+            if g.dtype != torch.bfloat16 or not g.is_contiguous() or g.dim() == 0:
                 raise ValueError("TIDE staging takes the parameters' contiguous bf16 gradients")
-        self.plan.rs_stage_one(T.TensorTable(list(grads)), self.arena, engine=self.engine)
+        plan, rank_plan, ns = self.plans_for([tuple(g.shape) for g in grads])
+        plan.rs_stage_one(T.TensorTable(list(grads)), self.arena, engine=self.engine)
+        self.pending = (rank_plan, ns)
 
     def reduce(self, out, op) -> None:
         """The reduce-scatter: this rank's fp32 shard from rows r of every arena (TIDE-RS)."""
         import torch
         import torch.distributed as dist
-        if out.dtype != torch.float32 or out.numel() != self.shard_numel or not out.is_contiguous():
+        if self.pending is None:
+            raise ValueError("reduce-scatter without staged gradients")
+        rank_plan, ns = self.pending
+        self.pending = None
+        if out.dtype != torch.float32 or out.numel() != ns or not out.is_contiguous():
             raise ValueError("reduce-scatter output is not this rank's fp32 shard")
         if op == dist.ReduceOp.AVG:
             scale = T.TIDE_SCALE_INV_WORLD
@@ -134,7 +158,7 @@ class TideGroup:
         else:
             raise ValueError(f"reduce op {op} is not a sum or an average")
         self.meet()                                   # every rank's gradients are staged
-        self.rank_plan.rs_reduce_slots(self.slot_table, out, scale_mode=scale, order=self.order)
+        rank_plan.rs_reduce_slots(self.slot_table, out, scale_mode=scale, order=self.order)
         self.meet()                                   # nobody copies in over a row still read
         self.reductions += 1
 
@@ -181,15 +205,18 @@ def _comm_classes():
             self.tg = tg
 
         def allocate(self, size, *, dtype, device):
+            # FSDP2 asks for the packed input, packs (the staging), then asks for the output
             import torch
             n = math.prod(int(s) for s in size)
             if dtype != torch.float32:
                 raise ValueError("TIDE's reduce-scatter reduces into fp32")
-            if n == self.tg.world * self.tg.shard_numel:
+            if self.tg.pending is None:
+                if n % self.tg.world or n > self.tg.world * self.tg.shard_numel:
+                    raise ValueError("unexpected reduce-scatter input size")
                 return self.tg.rs_input.expand(n)     # FSDP2's packed input: never materialized
-            if n == self.tg.shard_numel:
-                return torch.empty(n, dtype=torch.float32, device=self.tg.device)
-            raise ValueError("unexpected reduce-scatter buffer size")
+            if n != self.tg.pending[1]:
+                raise ValueError("unexpected reduce-scatter output size")
+            return torch.empty(n, dtype=torch.float32, device=self.tg.device)
 
         def __call__(self, output_tensor, input_tensor, group, op, async_op=False):
             if input_tensor.data_ptr() != self.tg.rs_input.data_ptr():

@@ -30,7 +30,7 @@ def _net():
     return Net()
 
 
-def fsdp2_tide_worker(rank, world, port, steps, lr, out_dir, engine, order):
+def fsdp2_tide_worker(rank, world, port, steps, lr, out_dir, engine, order, frozen=False):
     import torch
     import torch.distributed as dist
     from fsdp2_layout_aware_b200 import fsdp2 as F
@@ -43,6 +43,8 @@ def fsdp2_tide_worker(rank, world, port, steps, lr, out_dir, engine, order):
         torch.cuda.set_device(0)
         torch.manual_seed(0)                      # the same initial parameters on every rank
         model = _net().cuda()
+        if frozen:
+            model.l1.bias.requires_grad_(False)      # left out of its group's reduce-scatter
         for m in (model.l1, model.l2, model):
             F.fully_shard_tide(m, engine=engine, order=order)
         groups = F.tide_groups(model)
@@ -74,6 +76,9 @@ def fsdp2_tide_worker(rank, world, port, steps, lr, out_dir, engine, order):
         def stage(tg, grads):
             g, n = tick("stage", tg)
             torch.cuda.synchronize()
+            if rank == 0:
+                with open(os.path.join(out_dir, f"staged_shapes_{g}_{n}.json"), "w") as f:
+                    json.dump([tuple(t.shape) for t in grads], f)
             for i, t in enumerate(grads):
                 save(f"grad_{g}_{n}_{rank}_{i}.npy", bits_of(t))
             save(f"slot0_{g}_{n}_{rank}.npy", bits_of(tg.arena))
@@ -125,6 +130,7 @@ class OracleGroup:
         self.rs_input = torch.zeros(1)
         self.device = torch.device("cpu")
         self.calls = []
+        self.pending = None
         F._AG[self.arena.data_ptr()] = self
         F._RS[self.rs_input.data_ptr()] = self
 
@@ -154,25 +160,30 @@ class OracleGroup:
         import oracle
         import torch
         self.calls.append("stage")
+        shapes = [tuple(g.shape) for g in grads]            # the parameters that got gradients
+        ns = oracle.layout(self.world, shapes).Ns
         bits = [g.detach().contiguous().view(torch.int16).numpy().reshape(-1).view(np.uint16) for g in grads]
         slot = self.arena.view(torch.int16).numpy().view(np.uint16)   # shares the arena's memory
-        oracle.slot_stage(self.world, self.shapes, bits, slot)
+        oracle.slot_stage(self.world, shapes, bits, slot[:self.world * ns])
+        self.pending = (shapes, ns)
 
     def reduce(self, out, op):
         import oracle
         import torch
         import torch.distributed as dist
         self.calls.append("reduce")
+        shapes, ns = self.pending
+        self.pending = None
         self.meet()
-        slots = self._all(self.arena)
+        slots = [s[:self.world * ns] for s in self._all(self.arena)]
         scale = 1 if op == dist.ReduceOp.AVG else 0
-        res = oracle.rs_reduce_slots(self.world, self.shapes, slots, scale)
-        Ns, r = self.shard_numel, self.rank
-        out.copy_(torch.from_numpy(res[r * Ns:(r + 1) * Ns].copy()))
+        res = oracle.rs_reduce_slots(self.world, shapes, slots, scale)
+        r = self.rank
+        out.copy_(torch.from_numpy(res[r * ns:(r + 1) * ns].copy()))
         self.meet()
 
 
-def fsdp2_oracle_worker(rank, world, port, steps, lr, out_dir):
+def fsdp2_oracle_worker(rank, world, port, steps, lr, out_dir, frozen=False):
     """Stock FSDP2, then FSDP2 with the TIDE comms and operator routing of
     fsdp2_layout_aware_b200.fsdp2 over OracleGroups, on the CPU; saves both runs' sharded
     gradients of every step and final sharded parameters."""
@@ -194,6 +205,8 @@ def fsdp2_oracle_worker(rank, world, port, steps, lr, out_dir):
         for arm in ("stock", "tide"):
             torch.manual_seed(0)
             model = _net()
+            if frozen:
+                model.l1.bias.requires_grad_(False)   # left out of its group's reduce-scatter
             groups = []
             for m in (model.l1, model.l2, model):
                 fully_shard(m, mesh=mesh, mp_policy=policy)
@@ -209,8 +222,9 @@ def fsdp2_oracle_worker(rank, world, port, steps, lr, out_dir):
             for step in range(steps):
                 ((model(x).float() - y) ** 2).mean().backward()
                 for i, p in enumerate(model.parameters()):
-                    np.save(os.path.join(out_dir, f"{arm}_grad_{step}_{rank}_{i}.npy"),
-                            p.grad.to_local().detach().numpy())
+                    if p.grad is not None:
+                        np.save(os.path.join(out_dir, f"{arm}_grad_{step}_{rank}_{i}.npy"),
+                                p.grad.to_local().detach().numpy())
                 opt.step()
                 opt.zero_grad()
             for i, p in enumerate(model.parameters()):

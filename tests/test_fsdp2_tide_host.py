@@ -18,13 +18,17 @@ from _dist_helpers import run_procs
 pytest.importorskip("torch.distributed.fsdp._fully_shard._fsdp_collectives")
 
 
-@pytest.mark.parametrize("world", [2, 3])
-def test_fsdp2_with_tide_comms_gives_stock_fsdp2_results(world, tmp_path):
+@pytest.mark.parametrize("world,frozen", [(2, False), (3, False), (2, True)],
+                         ids=["w2", "w3", "w2_frozen_param"])
+def test_fsdp2_with_tide_comms_gives_stock_fsdp2_results(world, frozen, tmp_path):
+    """With a frozen parameter (no gradient) its group reduce-scatters the others only."""
     from _fsdp2_tide_workers import fsdp2_oracle_worker
     steps, lr = 3, 0.05
-    run_procs(fsdp2_oracle_worker, world, lambda port: (world, port, steps, lr, str(tmp_path)))
+    run_procs(fsdp2_oracle_worker, world,
+              lambda port: (world, port, steps, lr, str(tmp_path), frozen))
+    trained = [0, 1, 3, 4] if frozen else list(range(5))      # parameters() order: scale, l1.w, l1.b, ...
     for r in range(world):
-        names = [f"grad_{s}_{r}_{i}" for s in range(steps) for i in range(5)] + \
+        names = [f"grad_{s}_{r}_{i}" for s in range(steps) for i in trained] + \
                 [f"param_{r}_{i}" for i in range(5)]
         for name in names:
             a, b = np.load(tmp_path / f"stock_{name}.npy"), np.load(tmp_path / f"tide_{name}.npy")
@@ -52,7 +56,7 @@ def test_tide_comms_hand_out_the_groups_buffers_and_refuse_others():
     W, Ns = 3, 40
     tg = types.SimpleNamespace(world=W, shard_numel=Ns, device=torch.device("cpu"),
                                arena=torch.zeros(W * Ns, dtype=torch.bfloat16),
-                               rs_input=torch.zeros(1), reduced=[])
+                               rs_input=torch.zeros(1), reduced=[], pending=None)
     tg.reduce = lambda out, op: tg.reduced.append((out.numel(), op))
     tg.meet = lambda: None
     ag_cls, rs_cls = F._comm_classes()
@@ -66,15 +70,22 @@ def test_tide_comms_hand_out_the_groups_buffers_and_refuse_others():
     assert ag(buf, buf[:Ns], group=None) is None
     with pytest.raises(ValueError):
         ag(torch.zeros(W * Ns, dtype=torch.bfloat16), buf[:Ns], group=None)
+    # before staging FSDP2 asks for the packed input: any [W][n] up to the group's
     inp = rs.allocate((W * Ns,), dtype=torch.float32, device=tg.device)
     assert inp.shape == (W * Ns,) and inp.stride() == (0,) and inp.data_ptr() == tg.rs_input.data_ptr()
     assert inp.view(W, -1).data_ptr() == tg.rs_input.data_ptr()     # FSDP2's pack target
+    assert rs.allocate((W * 8,), dtype=torch.float32, device=tg.device).shape == (W * 8,)
+    for bad in (W * Ns + W, W * 8 + 1):
+        with pytest.raises(ValueError):
+            rs.allocate((bad,), dtype=torch.float32, device=tg.device)
+    with pytest.raises(ValueError):
+        rs.allocate((W * Ns,), dtype=torch.bfloat16, device=tg.device)
+    # after staging (its shard numel known) it asks for the output
+    tg.pending = (None, Ns)
     out = rs.allocate((Ns,), dtype=torch.float32, device=tg.device)
     assert out.shape == (Ns,) and out.dtype == torch.float32 and out.data_ptr() != inp.data_ptr()
     with pytest.raises(ValueError):
         rs.allocate((Ns + 1,), dtype=torch.float32, device=tg.device)
-    with pytest.raises(ValueError):
-        rs.allocate((Ns,), dtype=torch.bfloat16, device=tg.device)
     import torch.distributed as dist
     assert rs(out, inp, group=None, op=dist.ReduceOp.AVG) is None
     assert tg.reduced == [(Ns, dist.ReduceOp.AVG)]

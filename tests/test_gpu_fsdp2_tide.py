@@ -30,13 +30,16 @@ def _load(tmp, name):
     return np.load(tmp / name)
 
 
-@pytest.mark.parametrize("world,engine,order", [(2, 0, 0), (3, 0, 0), (3, 1, 1)],
-                         ids=["w2_sm_rank", "w3_sm_rank", "w3_ce_tree"])
-def test_fully_shard_with_tide_collectives_matches_the_oracle(world, engine, order, tmp_path):
+@pytest.mark.parametrize("world,engine,order,frozen", [(2, 0, 0, False), (3, 0, 0, False),
+                                                       (3, 1, 1, False), (2, 0, 0, True)],
+                         ids=["w2_sm_rank", "w3_sm_rank", "w3_ce_tree", "w2_frozen_param"])
+def test_fully_shard_with_tide_collectives_matches_the_oracle(world, engine, order, frozen, tmp_path):
+    """(With a frozen parameter its group stages and reduces the others only, in the layout
+    their shapes give.)"""
     from _fsdp2_tide_workers import fsdp2_tide_worker
     steps, lr = 3, 0.05
     run_procs(fsdp2_tide_worker, world,
-              lambda port: (world, port, steps, lr, str(tmp_path), engine, order))
+              lambda port: (world, port, steps, lr, str(tmp_path), engine, order, frozen))
     shapes = [[tuple(s) for s in g] for g in json.loads((tmp_path / "shapes.json").read_text())]
     counts = [json.loads((tmp_path / f"counts_{r}.json").read_text()) for r in range(world)]
     assert all({k: v for k, v in c.items() if k != "losses"} ==
@@ -56,13 +59,15 @@ def test_fully_shard_with_tide_collectives_matches_the_oracle(world, engine, ord
                     got = _load(tmp_path, f"placed_{g}_{n}_{r}_{i}.npy")
                     assert np.array_equal(got, want[i]), (g, n, r, i)
         for n in range(n_reduce):
-            grads = [[_load(tmp_path, f"grad_{g}_{n}_{k}_{i}.npy") for i in range(P)]
+            Sr = [tuple(x) for x in json.loads((tmp_path / f"staged_shapes_{g}_{n}.json").read_text())]
+            Lr = oracle.layout(world, Sr)
+            grads = [[_load(tmp_path, f"grad_{g}_{n}_{k}_{i}.npy") for i in range(len(Sr))]
                      for k in range(world)]
             for k in range(world):
                 exp = _load(tmp_path, f"slot0_{g}_{n}_{k}.npy").copy()
-                oracle.slot_stage(world, S, grads[k], exp)
+                oracle.slot_stage(world, Sr, grads[k], exp[:world * Lr.Ns])
                 assert np.array_equal(_load(tmp_path, f"slot1_{g}_{n}_{k}.npy"), exp), (g, n, k)
-            ref = rs_oracle(world, S, grads, 1).reshape(world, L.Ns)
+            ref = rs_oracle(world, Sr, grads, 1).reshape(world, Lr.Ns)
             for r in range(world):
                 got = _load(tmp_path, f"shard_{g}_{n}_{r}.npy")
                 assert np.array_equal(got.view(np.uint32), ref[r].view(np.uint32)), (g, n, r)
