@@ -312,6 +312,21 @@ def make_flush(device, nbytes):
     return lambda: buf.sum()
 
 
+def same_run_copy(device, nbytes=4 * 2 ** 30, K=5):
+    """This GPU's copy bandwidth in this run: one device-to-device cudaMemcpyAsync of
+    `nbytes` (torch's copy_ between two contiguous buffers), timed with CUDA events over K
+    copies after two untimed ones.  Each copy reads and writes `nbytes`, both far larger
+    than L2, so the figure is HBM's; the kernels' fractions against it sit beside the
+    roofline's fraction of the recorded peak."""
+    import torch
+    src = torch.ones(nbytes // 2, dtype=torch.bfloat16, device=device)
+    dst = torch.empty_like(src)
+    ms = timed_calls(lambda: dst.copy_(src), K, torch.cuda.current_stream(device))
+    del src, dst
+    torch.cuda.empty_cache()
+    return ms, 2 * nbytes
+
+
 def run_variants(wl, K, stream, peak, flush):
     """The other hot-path modes on the same workload, each timed on its own.
 
@@ -1162,6 +1177,16 @@ def bench_workload(args, group, rank, world, device, dist_on):
         # what the stock path would hold instead: one full-group fp32 rank-major buffer per rank
         "stock_fp32_buffer_bytes": 4 * group.world * wl.Ns,
     }
+    if not args.profile_small:   # a capture run keeps a few hundred MB on the device
+        copy_ms, copy_bytes = same_run_copy(device)
+        copy_ms = max_over_ranks([copy_ms], device)[0]
+        copy_gbs = copy_bytes / (copy_ms * 1e-3) / 1e9
+        res["copy_same_run"] = {"what": "device-to-device cudaMemcpyAsync of 4 GiB (reads and writes "
+                                        "4 GiB), after the timed steps, 5 copies",
+                                "ms": round(copy_ms, 4), "GB/s": round(copy_gbs, 1),
+                                "rs_frac": round(rs_gbs / copy_gbs, 4),
+                                "ag_frac": round(ag_gbs / copy_gbs, 4),
+                                "step_frac": round(value / world / copy_gbs, 4)}
     if not args.no_variants:
         # the step's figures above stand even if a variant fails: record the error instead
         try:
