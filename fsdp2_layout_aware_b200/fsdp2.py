@@ -33,7 +33,10 @@ row is in), after it (before anyone stages gradients over its row), before a red
 bf16 compute parameters and fp32 reduction (the mixed-precision policy set here); every
 collective is synchronous.  Parameters without a gradient (frozen ones) are left out of
 FSDP2's reduce-scatter; the layout of the ones that have one follows from their shapes in
-group order, and the group builds plans for that subset on first use.
+group order, and the group builds plans for that subset on first use.  Gradient
+accumulation works with gradient sync on (every micro-batch reduce-scattered, FSDP2 summing
+the fp32 shards); with sync off FSDP2 accumulates fp32 unsharded gradients, which TIDE's bf16
+staging refuses.
 """
 from __future__ import annotations
 
@@ -49,6 +52,23 @@ _RS = {}          # data_ptr of a group's expanded reduce-scatter input -> TideG
 _LOCK = threading.Lock()
 _INSTALLED = set()   # dispatch keys whose copy-out and pack are routed here
 _LIBS = []
+
+
+def _check_grads(grads, n_params) -> None:
+    """Refuse what TIDE's staging cannot take: more gradients than parameters, or gradients
+    that are not contiguous bf16.  FSDP2 hands over fp32 gradients when they were accumulated
+    with gradient sync off (it keeps such gradients in the fp32 reduce dtype); TIDE's reduction
+    reads bf16 gradients, so such accumulation must reduce-scatter every micro-batch instead
+    (sync on: FSDP2 then sums the fp32 shards)."""
+    import torch
+    if not 0 < len(grads) <= n_params:
+        raise ValueError("gradients do not match the group's parameters")
+    for g in grads:
+        if g.dtype == torch.float32:
+            raise ValueError("fp32 gradients (accumulated with gradient sync off): TIDE reduces "
+                             "bf16 gradients; keep gradient sync on while accumulating")
+        if g.dtype != torch.bfloat16 or not g.is_contiguous() or g.dim() == 0:
+            raise ValueError("TIDE staging takes the parameters' contiguous bf16 gradients")
 
 
 class TideGroup:
@@ -131,12 +151,7 @@ class TideGroup:
     def stage(self, grads) -> None:
         """FSDP2's pack: this rank's bf16 gradients into its arena (Slot-Reuse phase 1).  The
         gradients are those of the group's parameters that got one, in group order."""
-        import torch
-        if not 0 < len(grads) <= len(self.shapes):
-            raise ValueError("gradients do not match the group's parameters")
-        for g in grads:
-            if g.dtype != torch.bfloat16 or not g.is_contiguous() or g.dim() == 0:
-                raise ValueError("TIDE staging takes the parameters' contiguous bf16 gradients")
+        _check_grads(grads, len(self.shapes))
         plan, rank_plan, ns = self.plans_for([tuple(g.shape) for g in grads])
         plan.rs_stage_one(T.TensorTable(list(grads)), self.arena, engine=self.engine)
         self.pending = (rank_plan, ns)
@@ -262,16 +277,22 @@ def _install(dispatch_key: str = "CUDA") -> None:
     _INSTALLED.add(dispatch_key)
 
 
-def fully_shard_tide(module, group=None, *, reshard_after_forward=True,
+def fully_shard_tide(module, group=None, *, reshard_after_forward=None,
                      engine: int = T.TIDE_ENGINE_SM, order: int = T.TIDE_ORDER_RANK):
     """``fully_shard(module)`` over `group` with bf16 compute parameters and fp32 gradient
     reduction, its all-gather and reduce-scatter done by TIDE.  Apply it to submodules
-    first, then to the root, in the same order on every rank.  Returns the module."""
+    first, then to the root, in the same order on every rank.  Returns the module.
+
+    reshard_after_forward: as FSDP2's (None: True for submodules, False for the root), except
+    that resharding to a smaller world (an int) is refused: every all-gather of a TIDE group
+    spans the whole group."""
     import torch
     import torch.distributed as dist
     from torch.distributed.device_mesh import DeviceMesh
     from torch.distributed.fsdp import MixedPrecisionPolicy, fully_shard
 
+    if not (reshard_after_forward is None or isinstance(reshard_after_forward, bool)):
+        raise ValueError("TIDE groups reshard to the whole group or not at all")
     _install()
     pg = group if group is not None else dist.group.WORLD
     mesh = DeviceMesh.from_group(pg, "cuda")

@@ -30,7 +30,40 @@ def _net():
     return Net()
 
 
-def fsdp2_tide_worker(rank, world, port, steps, lr, out_dir, engine, order, frozen=False):
+MODES = ("plain", "frozen", "accum", "no_reshard", "accum_unsynced")
+
+
+def _backward(model, x, y, mode):
+    """One step's backward on (x, y).  accum: two micro-batches, each reduce-scattered (FSDP2
+    sums the fp32 shards); accum_unsynced: the first with FSDP2's gradient sync off (its
+    unsharded gradients kept, in fp32, for the second).  Returns the last loss."""
+    if mode in ("accum", "accum_unsynced"):
+        model.set_requires_gradient_sync(mode == "accum")
+        ((model(x[:8]).float() - y[:8]) ** 2).mean().backward()
+        model.set_requires_gradient_sync(True)
+        loss = ((model(x[8:]).float() - y[8:]) ** 2).mean()
+    else:
+        loss = ((model(x).float() - y) ** 2).mean()
+    loss.backward()
+    return float(loss)
+
+
+def _train(model, opt, x, y, steps, mode):
+    losses = []
+    for _ in range(steps):
+        losses.append(_backward(model, x, y, mode))
+        opt.step()
+        opt.zero_grad()
+    return losses
+
+
+def _shard_args(mode):
+    """fully_shard keyword arguments of a test mode (FSDP2's default otherwise: resharded
+    after forward, the root excepted)."""
+    return {"reshard_after_forward": False} if mode == "no_reshard" else {}
+
+
+def fsdp2_tide_worker(rank, world, port, steps, lr, out_dir, engine, order, mode="plain"):
     import torch
     import torch.distributed as dist
     from fsdp2_layout_aware_b200 import fsdp2 as F
@@ -43,10 +76,10 @@ def fsdp2_tide_worker(rank, world, port, steps, lr, out_dir, engine, order, froz
         torch.cuda.set_device(0)
         torch.manual_seed(0)                      # the same initial parameters on every rank
         model = _net().cuda()
-        if frozen:
+        if mode == "frozen":
             model.l1.bias.requires_grad_(False)      # left out of its group's reduce-scatter
         for m in (model.l1, model.l2, model):
-            F.fully_shard_tide(m, engine=engine, order=order)
+            F.fully_shard_tide(m, engine=engine, order=order, **_shard_args(mode))
         groups = F.tide_groups(model)
         gid = {id(tg): g for g, tg in enumerate(groups)}
         if rank == 0:
@@ -96,13 +129,7 @@ def fsdp2_tide_worker(rank, world, port, steps, lr, out_dir, engine, order, froz
         gen = torch.Generator(device="cuda").manual_seed(100 + rank)
         x = torch.randn(16, 40, device="cuda", generator=gen)
         y = torch.randn(16, 10, device="cuda", generator=gen)
-        losses = []
-        for _ in range(steps):
-            loss = ((model(x).float() - y) ** 2).mean()
-            loss.backward()
-            opt.step()
-            opt.zero_grad()
-            losses.append(float(loss))
+        losses = _train(model, opt, x, y, steps, mode)
         with open(os.path.join(out_dir, f"counts_{rank}.json"), "w") as f:
             json.dump({f"{k[0]}_{k[1]}": v for k, v in count.items()} | {"losses": losses}, f)
         F.close(model)
@@ -159,6 +186,8 @@ class OracleGroup:
     def stage(self, grads):
         import oracle
         import torch
+        from fsdp2_layout_aware_b200 import fsdp2 as F
+        F._check_grads(grads, len(self.shapes))
         self.calls.append("stage")
         shapes = [tuple(g.shape) for g in grads]            # the parameters that got gradients
         ns = oracle.layout(self.world, shapes).Ns
@@ -183,7 +212,7 @@ class OracleGroup:
         self.meet()
 
 
-def fsdp2_oracle_worker(rank, world, port, steps, lr, out_dir, frozen=False):
+def fsdp2_oracle_worker(rank, world, port, steps, lr, out_dir, mode="plain"):
     """Stock FSDP2, then FSDP2 with the TIDE comms and operator routing of
     fsdp2_layout_aware_b200.fsdp2 over OracleGroups, on the CPU; saves both runs' sharded
     gradients of every step and final sharded parameters."""
@@ -205,11 +234,11 @@ def fsdp2_oracle_worker(rank, world, port, steps, lr, out_dir, frozen=False):
         for arm in ("stock", "tide"):
             torch.manual_seed(0)
             model = _net()
-            if frozen:
+            if mode == "frozen":
                 model.l1.bias.requires_grad_(False)   # left out of its group's reduce-scatter
             groups = []
             for m in (model.l1, model.l2, model):
-                fully_shard(m, mesh=mesh, mp_policy=policy)
+                fully_shard(m, mesh=mesh, mp_policy=policy, **_shard_args(mode))
                 if arm == "tide":
                     F._install("CPU")
                     pg = m._get_fsdp_state()._fsdp_param_group
@@ -219,8 +248,17 @@ def fsdp2_oracle_worker(rank, world, port, steps, lr, out_dir, frozen=False):
                     m.set_custom_reduce_scatter(rs_cls(tg))
                     groups.append(tg)
             opt = torch.optim.SGD(model.parameters(), lr=lr)
+            if arm == "tide" and mode == "accum_unsynced":
+                try:
+                    _backward(model, x, y, mode)
+                    refusal = None
+                except ValueError as e:
+                    refusal = str(e)
+                with open(os.path.join(out_dir, f"refusal_{rank}.json"), "w") as f:
+                    json.dump(refusal, f)
+                return
             for step in range(steps):
-                ((model(x).float() - y) ** 2).mean().backward()
+                _backward(model, x, y, mode)
                 for i, p in enumerate(model.parameters()):
                     if p.grad is not None:
                         np.save(os.path.join(out_dir, f"{arm}_grad_{step}_{rank}_{i}.npy"),

@@ -18,15 +18,30 @@ from _dist_helpers import run_procs
 pytest.importorskip("torch.distributed.fsdp._fully_shard._fsdp_collectives")
 
 
-@pytest.mark.parametrize("world,frozen", [(2, False), (3, False), (2, True)],
-                         ids=["w2", "w3", "w2_frozen_param"])
-def test_fsdp2_with_tide_comms_gives_stock_fsdp2_results(world, frozen, tmp_path):
-    """With a frozen parameter (no gradient) its group reduce-scatters the others only."""
+# The calls each TIDE group sees per step, in fully_shard order: l1, l2, then the root.
+# Resharded after forward, l1 and l2 are placed again in backward; the root stays unsharded
+# from forward to backward.  Accumulating over two micro-batches, each is reduce-scattered.
+# Kept unsharded after forward, every group is placed once.
+CALLS = {
+    "plain": (["place", "place", "stage", "reduce"], ["place", "stage", "reduce"]),
+    "frozen": (["place", "place", "stage", "reduce"], ["place", "stage", "reduce"]),
+    "accum": (["place", "place", "stage", "reduce"] * 2, ["place", "stage", "reduce"] * 2),
+    "no_reshard": (["place", "stage", "reduce"], ["place", "stage", "reduce"]),
+}
+
+
+@pytest.mark.parametrize("world,mode", [(2, "plain"), (3, "plain"), (2, "frozen"), (2, "accum"),
+                                        (3, "no_reshard")],
+                         ids=["w2", "w3", "w2_frozen_param", "w2_grad_accumulation",
+                              "w3_no_reshard_after_forward"])
+def test_fsdp2_with_tide_comms_gives_stock_fsdp2_results(world, mode, tmp_path):
+    """With a frozen parameter (no gradient) its group reduce-scatters the others only; with
+    gradient accumulation the reduced gradients are the sum over both micro-batches."""
     from _fsdp2_tide_workers import fsdp2_oracle_worker
     steps, lr = 3, 0.05
     run_procs(fsdp2_oracle_worker, world,
-              lambda port: (world, port, steps, lr, str(tmp_path), frozen))
-    trained = [0, 1, 3, 4] if frozen else list(range(5))      # parameters() order: scale, l1.w, l1.b, ...
+              lambda port: (world, port, steps, lr, str(tmp_path), mode))
+    trained = [0, 1, 3, 4] if mode == "frozen" else list(range(5))  # scale, l1.w, l1.b, ...
     for r in range(world):
         names = [f"grad_{s}_{r}_{i}" for s in range(steps) for i in trained] + \
                 [f"param_{r}_{i}" for i in range(5)]
@@ -38,10 +53,22 @@ def test_fsdp2_with_tide_comms_gives_stock_fsdp2_results(world, frozen, tmp_path
             else:
                 np.testing.assert_allclose(b, a, rtol=1e-5, atol=1e-7, err_msg=name)
         calls = json.loads((tmp_path / f"calls_{r}.json").read_text())
-        # groups in fully_shard order: l1, l2 (resharded after forward: placed again in
-        # backward), then the root (kept unsharded from forward to backward)
-        assert calls[0] == calls[1] == ["place", "place", "stage", "reduce"] * steps
-        assert calls[2] == ["place", "stage", "reduce"] * steps
+        inner, root = CALLS[mode]
+        assert calls[0] == calls[1] == inner * steps, calls
+        assert calls[2] == root * steps, calls
+
+
+def test_accumulation_with_gradient_sync_off_is_refused_at_the_staging(tmp_path):
+    """With gradient sync off FSDP2 keeps the micro-batch's unsharded gradients in the fp32
+    reduce dtype and hands them to the pack of the next synced backward; TIDE's staging
+    takes bf16 gradients only and says so, on every rank, before any reduction."""
+    from _fsdp2_tide_workers import fsdp2_oracle_worker
+    world = 2
+    run_procs(fsdp2_oracle_worker, world,
+              lambda port: (world, port, 1, 0.05, str(tmp_path), "accum_unsynced"))
+    for r in range(world):
+        msg = json.loads((tmp_path / f"refusal_{r}.json").read_text())
+        assert msg is not None and "fp32 gradients" in msg and "sync" in msg, msg
 
 
 def test_tide_comms_hand_out_the_groups_buffers_and_refuse_others():
@@ -91,3 +118,14 @@ def test_tide_comms_hand_out_the_groups_buffers_and_refuse_others():
     assert tg.reduced == [(Ns, dist.ReduceOp.AVG)]
     with pytest.raises(ValueError):
         rs(out, torch.zeros(W * Ns), group=None, op=dist.ReduceOp.AVG)
+
+
+def test_resharding_to_a_smaller_world_is_refused():
+    """An int reshard_after_forward would all-gather over part of the group in backward;
+    TIDE groups refuse it before touching the module."""
+    import torch
+    from fsdp2_layout_aware_b200 import fsdp2 as F
+    m = torch.nn.Linear(4, 4)
+    with pytest.raises(ValueError):
+        F.fully_shard_tide(m, reshard_after_forward=2)
+    assert not hasattr(m, "_tide_group")

@@ -30,16 +30,20 @@ def _load(tmp, name):
     return np.load(tmp / name)
 
 
-@pytest.mark.parametrize("world,engine,order,frozen", [(2, 0, 0, False), (3, 0, 0, False),
-                                                       (3, 1, 1, False), (2, 0, 0, True)],
-                         ids=["w2_sm_rank", "w3_sm_rank", "w3_ce_tree", "w2_frozen_param"])
-def test_fully_shard_with_tide_collectives_matches_the_oracle(world, engine, order, frozen, tmp_path):
+@pytest.mark.parametrize("world,engine,order,mode",
+                         [(2, 0, 0, "plain"), (3, 0, 0, "plain"), (3, 1, 1, "plain"),
+                          (2, 0, 0, "frozen"), (2, 1, 0, "accum"), (3, 0, 1, "no_reshard")],
+                         ids=["w2_sm_rank", "w3_sm_rank", "w3_ce_tree", "w2_frozen_param",
+                              "w2_ce_rank_grad_accumulation", "w3_sm_tree_no_reshard"])
+def test_fully_shard_with_tide_collectives_matches_the_oracle(world, engine, order, mode, tmp_path):
     """(With a frozen parameter its group stages and reduces the others only, in the layout
-    their shapes give.)"""
+    their shapes give; accumulating, each of a step's two micro-batches is reduced; kept
+    unsharded after forward, each group is placed once a step.)"""
     from _fsdp2_tide_workers import fsdp2_tide_worker
     steps, lr = 3, 0.05
     run_procs(fsdp2_tide_worker, world,
-              lambda port: (world, port, steps, lr, str(tmp_path), engine, order, frozen))
+              lambda port: (world, port, steps, lr, str(tmp_path), engine, order, mode))
+    per_step = 2 if mode == "accum" else 1
     shapes = [[tuple(s) for s in g] for g in json.loads((tmp_path / "shapes.json").read_text())]
     counts = [json.loads((tmp_path / f"counts_{r}.json").read_text()) for r in range(world)]
     assert all({k: v for k, v in c.items() if k != "losses"} ==
@@ -50,7 +54,8 @@ def test_fully_shard_with_tide_collectives_matches_the_oracle(world, engine, ord
         P = len(S)
         n_place = counts[0][f"place_{g}"]
         n_reduce = counts[0][f"reduce_{g}"]
-        assert n_place >= steps and n_reduce == steps and counts[0][f"stage_{g}"] == steps
+        assert n_place >= steps * per_step and n_reduce == steps * per_step
+        assert counts[0][f"stage_{g}"] == n_reduce
         for n in range(n_place):
             ag = np.concatenate([_load(tmp_path, f"row_{g}_{n}_{k}.npy") for k in range(world)])
             want = oracle.ag_copyout(world, S, ag)
