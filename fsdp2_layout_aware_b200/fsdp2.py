@@ -26,7 +26,8 @@ gradients read where they are, staged bf16 into the vacated all-gather slot unde
 The copy-out and the pack are replaced through their dispatcher entries: on a buffer of a
 TIDE group the library call runs; on any other buffer FSDP2's own implementation does.
 
-Ranks meet only at host barriers of the process group (synchronize, then barrier), placed so
+Ranks meet only at host barriers of the process group (wait for this rank's stream, then
+barrier), placed so
 that no rank writes its arena while another may still read it: before a placement (every
 row is in), after it (before anyone stages gradients over its row), before a reduction
 (every rank staged) and after it (before the next copy-in).  The parameter group must have
@@ -131,10 +132,17 @@ class TideGroup:
             self._sub_plans[shapes] = ent
         return ent
 
-    def meet(self) -> None:
+    def meet(self, device_wide: bool = False) -> None:
+        """Wait for this rank's work on the current stream (where FSDP2 issues the collective,
+        after its copy-in or pack; and where this group enqueued its placement or reduction),
+        then meet every rank.  Work that FSDP2 queued on other streams, compute among it, keeps
+        running.  device_wide: wait for every stream of the device instead."""
         import torch
         import torch.distributed as dist
-        torch.cuda.synchronize(self.device)
+        if device_wide:
+            torch.cuda.synchronize(self.device)
+        else:
+            torch.cuda.current_stream(self.device).synchronize()
         dist.barrier(self.group)
 
     def place(self, out) -> None:
@@ -181,12 +189,12 @@ class TideGroup:
         """Unmap the peers' arenas once no rank can still read them (a collective)."""
         if self.peers is None:
             return
-        self.meet()
+        self.meet(device_wide=True)
         with _LOCK:
             _AG.pop(self.arena.data_ptr(), None)
             _RS.pop(self.rs_input.data_ptr(), None)
         self.peers.close()
-        self.meet()
+        self.meet(device_wide=True)
         self.peers = None
 
 
