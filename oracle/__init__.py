@@ -56,6 +56,11 @@ def _load():
         for name in ("orc_ag_copyout", "orc_pack_f32", "orc_slot_stage"):
             getattr(lib, name).argtypes = [i64, i64, vp, vp, vp, vp]
             getattr(lib, name).restype = ctypes.c_int
+        for name in ("orc_rs_reduce_f32", "orc_rs_reduce_slots_f32"):
+            getattr(lib, name).argtypes = [i64, i64, vp, vp, vp, i32, vp]
+            getattr(lib, name).restype = ctypes.c_int
+        lib.orc_slot_stage_f32.argtypes = [i64, i64, vp, vp, vp, vp]
+        lib.orc_slot_stage_f32.restype = ctypes.c_int
         for name in ("orc_rs_reduce", "orc_rs_reduce_slots", "orc_rs_reduce_tree"):
             getattr(lib, name).argtypes = [i64, i64, vp, vp, vp, i32, vp]
             getattr(lib, name).restype = ctypes.c_int
@@ -167,6 +172,41 @@ def rs_reduce_slots(world: int, shapes, slots, scale_mode: int) -> np.ndarray:
     sl = [np.ascontiguousarray(s, dtype=np.uint16).reshape(-1) for s in slots]
     _load().orc_rs_reduce_slots(world, len(shapes), d0.ctypes.data, inner.ctypes.data, _ptrs(sl),
                                 scale_mode, out.ctypes.data)
+    return out
+
+
+def rs_reduce_f32(world: int, shapes, grads, scale_mode: int) -> np.ndarray:
+    """rs_reduce for fp32 gradients: grads[k][i] contiguous float32 arrays (or their uint32
+    bits).  Returns fp32 [W*Ns]."""
+    d0, inner = _dims(shapes)
+    P = len(shapes)
+    Ns = layout(world, shapes).Ns
+    out = np.empty(world * Ns, dtype=np.float32)
+    flat = [np.ascontiguousarray(grads[k][i]).reshape(-1).view(np.float32)
+            for k in range(world) for i in range(P)]
+    _load().orc_rs_reduce_f32(world, P, d0.ctypes.data, inner.ctypes.data, _ptrs(flat),
+                              scale_mode, out.ctypes.data)
+    return out
+
+
+def slot_stage_f32(world: int, shapes, g_rank, slot: np.ndarray) -> None:
+    """Stage one rank's fp32 grads into `slot` ([W*Ns] of 4-byte words: float32 or uint32) in
+    place, as a copy of the words; pads untouched."""
+    d0, inner = _dims(shapes)
+    g = [np.ascontiguousarray(x).reshape(-1).view(np.uint32) for x in g_rank]
+    assert slot.dtype.itemsize == 4 and slot.flags.c_contiguous
+    _load().orc_slot_stage_f32(world, len(shapes), d0.ctypes.data, inner.ctypes.data, _ptrs(g),
+                               slot.ctypes.data)
+
+
+def rs_reduce_slots_f32(world: int, shapes, slots, scale_mode: int) -> np.ndarray:
+    """Slot-Reuse phase 2 over fp32 slots ([W*Ns] each, float32 or their uint32 bits)."""
+    d0, inner = _dims(shapes)
+    Ns = layout(world, shapes).Ns
+    out = np.empty(world * Ns, dtype=np.float32)
+    sl = [np.ascontiguousarray(s).reshape(-1).view(np.float32) for s in slots]
+    _load().orc_rs_reduce_slots_f32(world, len(shapes), d0.ctypes.data, inner.ctypes.data,
+                                    _ptrs(sl), scale_mode, out.ctypes.data)
     return out
 
 

@@ -211,6 +211,92 @@ int orc_rs_reduce_slots(int64_t W, int64_t P, const int64_t* d0, const int64_t* 
 }
 
 /*
+ * fp32 gradients.  While gradient sync is off, FSDP2 keeps a parameter's
+ * gradients in its fp32 reduce dtype, and the next synced backward packs those
+ * fp32 gradients as they are: the same pack into the fp32 rank-major buffer
+ * with no conversion, then the same reduce-scatter (weekinpapers.com,
+ * Abstract: the gradients that TIDE-RS reads in place are the ones the stock
+ * path packs).  These three functions are the bf16 ones above with fp32
+ * inputs: pack, then the rank-order sum from rank 0's pack, then the optional
+ * multiply; Slot-Reuse staging as a copy of the 4-byte words, pads untouched.
+ */
+static void pack_f32_of_f32(int64_t W, int64_t P, const int64_t* d0, const int64_t* inner,
+                            const int64_t* S, const int64_t* off, int64_t Ns,
+                            const float* const* g, float* buf) {
+    for (int64_t r = 0; r < W; ++r) {
+        for (int64_t i = 0; i < P; ++i) {
+            for (int64_t s = 0; s < S[i]; ++s) {
+                int64_t row = r * S[i] + s;
+                float* dst = buf + r * Ns + off[i] + s * inner[i];
+                for (int64_t t = 0; t < inner[i]; ++t)
+                    dst[t] = row < d0[i] ? g[i][row * inner[i] + t] : 0.0f;
+            }
+        }
+    }
+}
+
+int orc_rs_reduce_f32(int64_t W, int64_t P, const int64_t* d0, const int64_t* inner,
+                      const float* const* grads, int32_t scale_mode, float* out) {
+    int64_t *S = malloc(sizeof(int64_t) * (P + 1)), *c = malloc(sizeof(int64_t) * (P + 1)),
+            *off = malloc(sizeof(int64_t) * (P + 1)), Ns = 0;
+    if (!S || !c || !off) { free(S); free(c); free(off); return -1; }
+    orc_layout(W, P, d0, inner, S, c, off, &Ns);
+    int64_t n = W * Ns;
+    float* packed = malloc(sizeof(float) * (size_t)(n > 0 ? n : 1));
+    if (!packed) { free(S); free(c); free(off); return -1; }
+    pack_f32_of_f32(W, P, d0, inner, S, off, Ns, grads, out);
+    for (int64_t k = 1; k < W; ++k) {
+        pack_f32_of_f32(W, P, d0, inner, S, off, Ns, grads + k * P, packed);
+        for (int64_t j = 0; j < n; ++j) out[j] = out[j] + packed[j];
+    }
+    if (scale_mode == 1) {
+        float sc = 1.0f / (float)W;
+        for (int64_t j = 0; j < n; ++j) out[j] = out[j] * sc;
+    }
+    free(packed); free(S); free(c); free(off);
+    return 0;
+}
+
+int orc_slot_stage_f32(int64_t W, int64_t P, const int64_t* d0, const int64_t* inner,
+                       const uint32_t* const* g, uint32_t* slot) {
+    int64_t *S = malloc(sizeof(int64_t) * (P + 1)), *c = malloc(sizeof(int64_t) * (P + 1)),
+            *off = malloc(sizeof(int64_t) * (P + 1)), Ns = 0;
+    if (!S || !c || !off) { free(S); free(c); free(off); return -1; }
+    orc_layout(W, P, d0, inner, S, c, off, &Ns);
+    for (int64_t r = 0; r < W; ++r)
+        for (int64_t i = 0; i < P; ++i)
+            for (int64_t s = 0; s < S[i]; ++s) {
+                int64_t row = r * S[i] + s;
+                if (row >= d0[i]) continue;
+                for (int64_t t = 0; t < inner[i]; ++t)
+                    slot[r * Ns + off[i] + s * inner[i] + t] = g[i][row * inner[i] + t];
+            }
+    free(S); free(c); free(off);
+    return 0;
+}
+
+int orc_rs_reduce_slots_f32(int64_t W, int64_t P, const int64_t* d0, const int64_t* inner,
+                            const float* const* slots, int32_t scale_mode, float* out) {
+    int64_t *S = malloc(sizeof(int64_t) * (P + 1)), *c = malloc(sizeof(int64_t) * (P + 1)),
+            *off = malloc(sizeof(int64_t) * (P + 1)), Ns = 0;
+    if (!S || !c || !off) { free(S); free(c); free(off); return -1; }
+    orc_layout(W, P, d0, inner, S, c, off, &Ns);
+    float sc = 1.0f / (float)W;
+    for (int64_t r = 0; r < W; ++r)
+        for (int64_t i = 0; i < P; ++i)
+            for (int64_t e = 0; e < c[i]; ++e) {
+                int64_t j = r * Ns + off[i] + e;
+                int64_t row = r * S[i] + (inner[i] ? e / inner[i] : 0);
+                if (row >= d0[i]) { out[j] = 0.0f; continue; }
+                float acc = slots[0][j];
+                for (int64_t k = 1; k < W; ++k) acc = acc + slots[k][j];
+                out[j] = scale_mode == 1 ? acc * sc : acc;
+            }
+    free(S); free(c); free(off);
+    return 0;
+}
+
+/*
  * The tree order on one position: v[0..n) are replaced, level by level, by the
  * sums of adjacent pairs (v[0]+v[1], v[2]+v[3], ...), an odd last value carried
  * unchanged, until one value is left.  fp32 adds, round-to-nearest-even.

@@ -31,6 +31,12 @@ MUTANTS = {
                             "for (int64_t j = 0; j + 1 < n; j += 2) v[m++] = v[j] + v[n - 1 - j];"),
     "tree_odd_one_dropped": ("if (n % 2 == 1) v[m++] = v[n - 1];", "if (n % 2 == 1) m += 0;"),
     "exact_magnitude_keeps_sign": ("mag += v < 0 ? -v : v;", "mag += v;"),
+    "f32_pack_reads_bf16": ("dst[t] = row < d0[i] ? g[i][row * inner[i] + t] : 0.0f;",
+                            "dst[t] = row < d0[i] ? bf16_to_f32(((const uint16_t*)g[i])[row * inner[i] + t]) : 0.0f;"),
+    "f32_slots_drop_last_rank": ("for (int64_t k = 1; k < W; ++k) acc = acc + slots[k][j];",
+                                 "for (int64_t k = 1; k < W - 1; ++k) acc = acc + slots[k][j];"),
+    "f32_scales_by_W_not_inverse": ("        float sc = 1.0f / (float)W;\n        for (int64_t j = 0; j < n; ++j) out[j] = out[j] * sc;",
+                                    "        float sc = (float)W;\n        for (int64_t j = 0; j < n; ++j) out[j] = out[j] * sc;"),
     "ranks_added_in_reverse": ("pack_f32(W, P, d0, inner, S, off, Ns, grads + k * P, packed);",
                                "pack_f32(W, P, d0, inner, S, off, Ns, grads + (W - k) * P, packed);"),
 }

@@ -463,3 +463,110 @@ def test_exact_sums_against_integer_brute_force(W):
     a_ref = torch_rank_major(W, grp.shapes, [torch.from_numpy(t) for t in mag], 0).numpy()
     assert np.array_equal(E, e_ref.astype(np.float64) * 2.0 ** -10)
     assert np.array_equal(A, a_ref.astype(np.float64) * 2.0 ** -10)
+
+
+# --------------------------------------------------------------------------- fp32 gradients
+
+
+def _f32_grads_of(grads):
+    """The fp32 values of bf16 gradients (the widening is exact)."""
+    return [[f32_of(g) for g in rk] for rk in grads]
+
+
+@pytest.mark.parametrize("grp", [configs.tiny(), mini_wan(), degenerate(), mini_sweep(64)]
+                         + [random_group(np.random.default_rng(77 + w), w, 4) for w in (1, 3, 5, 16)],
+                         ids=lambda g: f"{g.name}_w{g.world}")
+def test_f32_inputs_holding_bf16_values_give_the_bf16_results(grp):
+    """fp32 gradients whose values are bf16 values reduce to the pinned bf16 results, bit for
+    bit, directly and through fp32 slots (stale slot contents: NaN)."""
+    W = grp.world
+    L = oracle.layout(W, grp.shapes)
+    grads = synth.grads_host(grp, seed=31)
+    g32 = _f32_grads_of(grads)
+    slots = [np.full(W * L.Ns, 0xFFFFFFFF, dtype=np.uint32) for _ in range(W)]
+    for k in range(W):
+        oracle.slot_stage_f32(W, grp.shapes, g32[k], slots[k])
+    for scale in (0, 1):
+        want = oracle.rs_reduce(W, grp.shapes, grads, scale).view(np.uint32)
+        assert np.array_equal(oracle.rs_reduce_f32(W, grp.shapes, g32, scale).view(np.uint32), want)
+        assert np.array_equal(oracle.rs_reduce_slots_f32(W, grp.shapes, slots, scale).view(np.uint32),
+                              want)
+
+
+@pytest.mark.parametrize("W", [1, 2, 3, 8, 64])
+def test_f32_sums_keep_bits_below_bf16_precision(W):
+    """Multiples of 2^-20 around 1 (not bf16 values) sum exactly: int64 brute force, laid out
+    by the torch.chunk builder.  A pack or a staging that drops the low 16 bits fails."""
+    grp = configs.Group("f32ints", W, ((65, 9), (301,), (3, 3)))
+    rng = np.random.default_rng(100 + W)
+    ints = [[rng.integers(-8, 9, size=grp.numel(i)) + (2 ** 20 if k == 0 else 0)
+             for i in range(grp.n_params)] for k in range(W)]
+    g32 = [[(m.astype(np.float64) * 2.0 ** -20).astype(np.float32) for m in rk] for rk in ints]
+    assert np.array_equal(g32[0][0].astype(np.float64) * 2 ** 20, ints[0][0])   # exact inputs
+    tot = [sum(ints[k][i] for k in range(W)).astype(np.int64) for i in range(grp.n_params)]
+    ref = torch_rank_major(W, grp.shapes, [torch.from_numpy(t) for t in tot], 0).numpy()
+    ref = ref.astype(np.float64) * 2.0 ** -20
+    assert np.array_equal(oracle.rs_reduce_f32(W, grp.shapes, g32, 0).astype(np.float64), ref)
+    L = oracle.layout(W, grp.shapes)
+    slots = [np.zeros(W * L.Ns, dtype=np.float32) for _ in range(W)]
+    for k in range(W):
+        oracle.slot_stage_f32(W, grp.shapes, g32[k], slots[k])
+    assert np.array_equal(oracle.rs_reduce_slots_f32(W, grp.shapes, slots, 0).astype(np.float64), ref)
+
+
+def test_f32_rank_order_is_fixed_and_signed_zeros():
+    shapes = ((3,),)
+    def run(vals):
+        return oracle.rs_reduce_f32(3, shapes, [[np.full(3, v, dtype=np.float32)] for v in vals], 0)[0]
+    assert run([1.0, 2.0 ** -24, 2.0 ** -24]) == np.float32(1.0)
+    assert run([2.0 ** -24, 2.0 ** -24, 1.0]) == np.float32(1.0 + 2.0 ** -23)
+    W, shapes = 4, ((5, 2), (3,))
+    neg = [[np.full(10, -0.0, np.float32), np.full(3, -0.0, np.float32)] for _ in range(W)]
+    out = oracle.rs_reduce_f32(W, shapes, neg, 0).view(np.uint32)
+    mask = valid_mask(configs.Group("z", W, shapes))
+    assert np.all(out[mask] == 0x80000000) and np.all(out[~mask] == 0)
+
+
+@pytest.mark.parametrize("grp", [configs.tiny(), degenerate()], ids=lambda g: g.name)
+def test_f32_slot_stage_matches_torch_chunk(grp):
+    """Staging one rank's fp32 gradients: the torch.chunk builder's rank-major buffer at valid
+    positions, the slot's old words (NaN) at pads."""
+    W = grp.world
+    L = oracle.layout(W, grp.shapes)
+    rng = np.random.default_rng(5)
+    g = [rng.standard_normal(grp.numel(i)).astype(np.float32) for i in range(grp.n_params)]
+    slot = np.full(W * L.Ns, 0xFFFFFFFF, dtype=np.uint32)
+    oracle.slot_stage_f32(W, grp.shapes, g, slot)
+    ref = torch_rank_major(W, grp.shapes, [torch.from_numpy(x.view(np.int32)) for x in g], -1).numpy()
+    mask = valid_mask(grp)
+    assert np.array_equal(slot[mask], ref.view(np.uint32)[mask])
+    assert np.all(slot[~mask] == 0xFFFFFFFF)
+
+
+def test_f32_gloo_reduce_scatter_agrees(tmp_path):
+    """torch.distributed.reduce_scatter_tensor (gloo, 4 processes) on FSDP2-packed fp32
+    buffers of fp32 gradients: bit for bit on exact sums, within the fp32 bound otherwise."""
+    from _dist_helpers import run_gloo_reduce_scatter
+    grp = configs.tiny()
+    W = grp.world
+    rng = np.random.default_rng(6)
+    exact = [[((rng.integers(-8, 9, size=grp.numel(i)) + 2 ** 20) * 2.0 ** -20).astype(np.float32)
+              for i in range(grp.n_params)] for _ in range(W)]
+    general = [[rng.standard_normal(grp.numel(i)).astype(np.float32) * np.float32(1e-3)
+                for i in range(grp.n_params)] for _ in range(W)]
+    for grads, bitwise in ((exact, True), (general, False)):
+        packed = [torch_rank_major(W, grp.shapes, [torch.from_numpy(x) for x in grads[k]], 0.0)
+                  for k in range(W)]
+        got = np.concatenate(run_gloo_reduce_scatter([p.numpy() for p in packed], tmp_path))
+        out = oracle.rs_reduce_f32(W, grp.shapes, grads, 0)
+        if bitwise:
+            assert np.array_equal(got.view(np.uint32), out.view(np.uint32))
+        else:
+            ex = torch_rank_major(W, grp.shapes, [torch.from_numpy(sum(grads[k][i].astype(np.float64)
+                                                                      for k in range(W)))
+                                                  for i in range(grp.n_params)], 0.0).numpy()
+            mag = torch_rank_major(W, grp.shapes, [torch.from_numpy(sum(np.abs(grads[k][i]).astype(np.float64)
+                                                                       for k in range(W)))
+                                                   for i in range(grp.n_params)], 0.0).numpy()
+            bound = (W - 1) * 2.0 ** -24 * mag
+            assert np.all(np.abs(got - ex) <= bound) and np.all(np.abs(out - ex) <= bound)
