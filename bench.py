@@ -453,7 +453,29 @@ def run_variants(wl, K, stream, peak, flush):
         n = wl.group.numel(i)
         same &= bool(torch.equal(p[:n].view(torch.int16), q[:n].view(torch.int16)))
     out["stock_torch_copyout"]["same_valid_bits_as_tide"] = same
-    del pack, stock, stock_params, ref_out, ref_params
+    del pack, stock, stock_params
+    # fp32 gradients (FSDP2's, accumulated with gradient sync off) through fp32 slots: each
+    # rank's gradients widened to fp32 (exactly) and staged into its own slot, then the slots
+    # reduced in rank order, which must give the plain reduction's bits
+    f32_bytes = 4 * W * W * Ns
+    if f32_bytes <= 32 * 2 ** 30:
+        N = B["N"]
+        slots32 = [torch.empty(W * Ns, dtype=torch.float32, device=wl.out.device) for _ in range(W)]
+        for k in range(W):
+            g32 = T.TensorTable([t.float() for t in wl.grads[k]])
+            if k == 0:
+                rec("stage_one_f32", timed_calls(lambda: wl.plan.rs_stage_one_f32(g32, slots32[0]),
+                                                 K, stream, flush), 8 * N, 1, wl.plan)
+            else:
+                wl.plan.rs_stage_one_f32(g32, slots32[k])
+            del g32
+        wl.out.fill_(float("nan"))
+        rec("slot_reduce_f32", timed_calls(lambda: wl.plan.rs_reduce_slots_f32(slots32, wl.out),
+                                           K, stream, flush), 4 * W * N + 4 * W * Ns, 1, wl.plan, same_rs)
+        del slots32
+    else:
+        out["slot_reduce_f32"] = {"skipped": f"fp32 slots of {f32_bytes / 2 ** 30:.0f} GiB"}
+    del ref_out, ref_params
     wl.drop_slots()
     return out
 
@@ -472,6 +494,8 @@ ROW_KINDS = {
     "rs_reduce_one_rank": ("rs_reduce", "one rank's shard (one-rank plan), rank order"),
     "ag_gather_place_sm": ("ag_gather_place", "SM, from per-rank shards"),
     "ag_gather_place_ce": ("ag_gather_place", "copy engines, from per-rank shards"),
+    "stage_one_f32": ("slot_stage", "fp32 gradients of one rank, SM"),
+    "slot_reduce_f32": ("slot_reduce", "fp32 slots, SM, rank order"),
     "stock_torch_pack_reduce": ("stock_rs", "torch _chunk_cat pack + add"),
     "stock_torch_copyout": ("stock_ag", "torch split_with_sizes_copy"),
 }
@@ -499,6 +523,8 @@ def jsonl_rows(res, group_name, world):
     cpu = res.get("cpu_baseline") or {}
     entries = list(res.get("kernels", {}).items()) + list(res.get("variants", {}).items())
     for name, e in entries:
+        if "skipped" in e:
+            continue
         op, mode = ROW_KINDS.get(name, (name, ""))
         if name.startswith("slot_reuse_pipelined_seg"):
             op, mode = "slot_reuse", f"pipelined, {name.rsplit('seg', 1)[1]} segments"

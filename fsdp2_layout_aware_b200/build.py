@@ -20,7 +20,7 @@ LIB = os.path.join(HERE, "libtide.so")
 INCLUDE = os.path.join(ROOT, "include")
 
 SOURCES = ["plan.cpp", "api.cpp", "ce.cpp", "rs_reduce.cu", "rs_reduce_tma.cu", "ag_place.cu",
-           "rs_reduce_noalloc.cu", "ipc.cpp", "flags.cu"]
+           "rs_reduce_noalloc.cu", "ipc.cpp", "flags.cu", "f32_grads.cu"]
 HEADERS = ["tide_internal.h", "device_common.cuh", "reduce_ranks.cuh", "tma.cuh"]
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",

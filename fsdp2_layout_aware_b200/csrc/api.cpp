@@ -466,6 +466,75 @@ extern "C" tide_status_t tide_rs_reduce_slots(const tide_plan_t* cplan, const vo
                              order, max_ctas, static_cast<cudaStream_t>(stream));
 }
 
+extern "C" tide_status_t tide_rs_stage_one_f32(const tide_plan_t* cplan, const float* const* grads,
+                                               const int64_t* grad_numel, float* slot, int64_t slot_numel,
+                                               int32_t max_ctas, void* stream) {
+    ApiRange range("tide_rs_stage_one_f32");
+    tide_plan* p = const_cast<tide_plan*>(cplan);
+    tide_status_t st = check_plan(p);
+    if (st != TIDE_OK) return st;
+    if ((st = all_ranks(p)) != TIDE_OK) return st;
+    if ((st = check_enums(p, TIDE_ENGINE_SM, max_ctas)) != TIDE_OK) return st;
+    const int64_t W = p->world, P = p->n_params;
+    std::vector<Span> spans;
+    spans.reserve((size_t)P + 1);
+    if (P > 0 && (grads == nullptr || grad_numel == nullptr)) return TIDE_ERR_INVALID_ARG;
+    for (int64_t i = 0; i < P; ++i) {
+        if ((st = check_buf(grads[i], grad_numel[i], p->numel[i], 4)) != TIDE_OK) return st;
+        add_span(spans, grads[i], 4 * p->numel[i], false);
+    }
+    if ((st = check_buf(slot, slot_numel, W * p->shard_numel, 4)) != TIDE_OK) return st;
+    add_span(spans, slot, 4 * W * p->shard_numel, true);
+    if (overlaps(spans)) return TIDE_ERR_INVALID_ARG;
+    if ((st = launchable(p)) != TIDE_OK) return st;
+    if (p->tiles.empty()) return TIDE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = sync_table(p->grad_tab, reinterpret_cast<const void* const*>(grads), P, s)) != TIDE_OK)
+        return st;
+    p->last_kernel = K_STAGE_F32;
+    p->last_ctas = grid_for(p, K_STAGE_F32, max_ctas);
+    cudaError_t e = tide::launch_stage_f32(p, p->grad_tab.dev, slot, slot_numel, p->last_ctas, s);
+    return e == cudaSuccess ? TIDE_OK : TIDE_ERR_CUDA;
+}
+
+extern "C" tide_status_t tide_rs_reduce_slots_f32(const tide_plan_t* cplan, const float* const* slots,
+                                                  int64_t slot_numel, float* out, int64_t out_numel,
+                                                  int32_t scale_mode, int32_t max_ctas, void* stream) {
+    ApiRange range("tide_rs_reduce_slots_f32");
+    tide_plan* p = const_cast<tide_plan*>(cplan);
+    tide_status_t st = check_plan(p);
+    if (st != TIDE_OK) return st;
+    if ((st = check_enums(p, TIDE_ENGINE_SM, max_ctas)) != TIDE_OK) return st;
+    if ((st = check_reduce_modes(scale_mode, TIDE_ORDER_RANK)) != TIDE_OK) return st;
+    const int64_t W = p->world, need = W * p->shard_numel;
+    const int64_t n_out = (p->rank >= 0 ? 1 : W) * p->shard_numel;
+    std::vector<Span> spans;
+    spans.reserve((size_t)W + 1);
+    if (slots == nullptr) return TIDE_ERR_INVALID_ARG;
+    for (int64_t k = 0; k < W; ++k) {
+        if ((st = check_buf(slots[k], slot_numel, need, 4)) != TIDE_OK) return st;
+        add_span(spans, slots[k], 4 * need, false);
+    }
+    if ((st = check_buf(out, out_numel, n_out, 4)) != TIDE_OK) return st;
+    add_span(spans, out, 4 * n_out, true);
+    if (overlaps(spans)) return TIDE_ERR_INVALID_ARG;
+    if ((st = launchable(p)) != TIDE_OK) return st;
+    if (p->tiles.empty()) return TIDE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // a one-rank plan's tiles address its shard from 0; its rows of every slot start at rank * Ns
+    const int64_t row0 = p->rank >= 0 ? (int64_t)p->rank * p->shard_numel : 0;
+    std::vector<const void*> from((size_t)W);
+    for (int64_t k = 0; k < W; ++k) from[k] = slots[k] + row0;
+    if ((st = sync_table(p->slot_tab, from.data(), W, s)) != TIDE_OK) return st;
+    const bool v8 = p->slot_tab.aligned32 && (reinterpret_cast<uintptr_t>(out) & 31) == 0;
+    p->last_kernel = K_SLOT_RS_F32;
+    p->last_ctas = grid_for(p, K_SLOT_RS_F32, max_ctas);
+    cudaError_t e = tide::launch_reduce_slots_f32(p, p->slot_tab.dev, slot_numel - row0, out, out_numel,
+                                                  inv_world(p->world), scale_mode == TIDE_SCALE_INV_WORLD,
+                                                  v8, p->last_ctas, s);
+    return e == cudaSuccess ? TIDE_OK : TIDE_ERR_CUDA;
+}
+
 extern "C" tide_status_t tide_rs_reduce_pipelined(const tide_plan_t* cplan, const void* const* grads,
                                                   const int64_t* grad_numel, float* out,
                                                   int64_t out_numel, int32_t scale_mode,

@@ -35,9 +35,11 @@ bf16 compute parameters and fp32 reduction (the mixed-precision policy set here)
 collective is synchronous.  Parameters without a gradient (frozen ones) are left out of
 FSDP2's reduce-scatter; the layout of the ones that have one follows from their shapes in
 group order, and the group builds plans for that subset on first use.  Gradient
-accumulation works with gradient sync on (every micro-batch reduce-scattered, FSDP2 summing
-the fp32 shards); with sync off FSDP2 accumulates fp32 unsharded gradients, which TIDE's bf16
-staging refuses.
+accumulation works both ways: with gradient sync on, every micro-batch is reduce-scattered and
+FSDP2 sums the fp32 shards; with it off, FSDP2 keeps the unsharded gradients in fp32 and packs
+those at the synced backward, which become ``tide_rs_stage_one_f32`` into a fp32 slot of the
+rank (made on first use, W*Ns*4 bytes, the size of stock FSDP2's packed buffer) and
+``tide_rs_reduce_slots_f32`` (rank order).
 """
 from __future__ import annotations
 
@@ -55,21 +57,22 @@ _INSTALLED = set()   # dispatch keys whose copy-out and pack are routed here
 _LIBS = []
 
 
-def _check_grads(grads, n_params) -> None:
+def _check_grads(grads, n_params) -> bool:
     """Refuse what TIDE's staging cannot take: more gradients than parameters, or gradients
-    that are not contiguous bf16.  FSDP2 hands over fp32 gradients when they were accumulated
-    with gradient sync off (it keeps such gradients in the fp32 reduce dtype); TIDE's reduction
-    reads bf16 gradients, so such accumulation must reduce-scatter every micro-batch instead
-    (sync on: FSDP2 then sums the fp32 shards)."""
+    that are not all contiguous bf16 or all contiguous fp32.  FSDP2 hands over fp32 gradients
+    when they were accumulated with gradient sync off (it keeps those in the fp32 reduce
+    dtype).  Returns True for fp32 gradients."""
     import torch
     if not 0 < len(grads) <= n_params:
         raise ValueError("gradients do not match the group's parameters")
+    dtype = grads[0].dtype
+    if dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("TIDE staging takes bf16 or fp32 gradients")
     for g in grads:
-        if g.dtype == torch.float32:
-            raise ValueError("fp32 gradients (accumulated with gradient sync off): TIDE reduces "
-                             "bf16 gradients; keep gradient sync on while accumulating")
-        if g.dtype != torch.bfloat16 or not g.is_contiguous() or g.dim() == 0:
-            raise ValueError("TIDE staging takes the parameters' contiguous bf16 gradients")
+        if g.dtype != dtype or not g.is_contiguous() or g.dim() == 0:
+            raise ValueError("TIDE staging takes the parameters' contiguous gradients, all of "
+                             "one dtype")
+    return dtype == torch.float32
 
 
 class TideGroup:
@@ -117,7 +120,27 @@ class TideGroup:
         # plans for the parameters that get gradients, when some do not (frozen ones): FSDP2
         # reduce-scatters only those, in group order, so their shapes fix the layout
         self._sub_plans = {}
-        self.pending = None   # (one-rank plan, shard numel) of the staged reduction
+        self.pending = None   # (one-rank plan, shard numel, fp32?) of the staged reduction
+        # fp32 slots for gradients FSDP2 accumulated with sync off (made on first use)
+        self.arena32 = None
+        self.peers32 = None
+        self.slot_table32 = None
+
+    def ensure_arena32(self) -> None:
+        """This rank's fp32 [W][Ns] slot, mapped into every rank (a collective on first use:
+        every rank stages fp32 gradients at the same backward)."""
+        import torch
+        if self.arena32 is not None:
+            return
+        W, Ns = self.world, self.shard_numel
+        arena32 = torch.zeros(W * Ns, dtype=torch.float32, device=self.device)
+        torch.cuda.synchronize(self.device)
+        exports = X.all_exports(X.export({"arena32": arena32}), self.group)
+        self.peers32 = X.PeerMaps(exports, self.rank, self.device.index,
+                                  {"arena32": arena32.data_ptr()})
+        self.slot_table32 = T.PointerTable(list(self.peers32.bases("arena32", W)), [W * Ns] * W,
+                                           keep=[arena32])
+        self.arena32 = arena32
 
     def plans_for(self, shapes):
         """(all-rank plan, one-rank plan, shard numel) for a reduction over `shapes`."""
@@ -159,10 +182,14 @@ class TideGroup:
     def stage(self, grads) -> None:
         """FSDP2's pack: this rank's bf16 gradients into its arena (Slot-Reuse phase 1).  The
         gradients are those of the group's parameters that got one, in group order."""
-        _check_grads(grads, len(self.shapes))
+        f32 = _check_grads(grads, len(self.shapes))
         plan, rank_plan, ns = self.plans_for([tuple(g.shape) for g in grads])
-        plan.rs_stage_one(T.TensorTable(list(grads)), self.arena, engine=self.engine)
-        self.pending = (rank_plan, ns)
+        if f32:
+            self.ensure_arena32()
+            plan.rs_stage_one_f32(T.TensorTable(list(grads)), self.arena32)
+        else:
+            plan.rs_stage_one(T.TensorTable(list(grads)), self.arena, engine=self.engine)
+        self.pending = (rank_plan, ns, f32)
 
     def reduce(self, out, op) -> None:
         """The reduce-scatter: this rank's fp32 shard from rows r of every arena (TIDE-RS)."""
@@ -170,7 +197,7 @@ class TideGroup:
         import torch.distributed as dist
         if self.pending is None:
             raise ValueError("reduce-scatter without staged gradients")
-        rank_plan, ns = self.pending
+        rank_plan, ns, f32 = self.pending
         self.pending = None
         if out.dtype != torch.float32 or out.numel() != ns or not out.is_contiguous():
             raise ValueError("reduce-scatter output is not this rank's fp32 shard")
@@ -181,7 +208,10 @@ class TideGroup:
         else:
             raise ValueError(f"reduce op {op} is not a sum or an average")
         self.meet()                                   # every rank's gradients are staged
-        rank_plan.rs_reduce_slots(self.slot_table, out, scale_mode=scale, order=self.order)
+        if f32:
+            rank_plan.rs_reduce_slots_f32(self.slot_table32, out, scale_mode=scale)
+        else:
+            rank_plan.rs_reduce_slots(self.slot_table, out, scale_mode=scale, order=self.order)
         self.meet()                                   # nobody copies in over a row still read
         self.reductions += 1
 
@@ -194,6 +224,9 @@ class TideGroup:
             _AG.pop(self.arena.data_ptr(), None)
             _RS.pop(self.rs_input.data_ptr(), None)
         self.peers.close()
+        if self.peers32 is not None:
+            self.peers32.close()
+            self.peers32 = None
         self.meet(device_wide=True)
         self.peers = None
 

@@ -44,7 +44,8 @@ TIDE_IPC_HANDLE_BYTES = 64
 (K_RS, K_AG, K_STAGE, K_SLOT_RS, K_RS_TMA, K_SLOT_RS_TMA, K_RS_V32, K_SLOT_RS_V32, K_RS_TREE,
  K_SLOT_RS_TREE, K_AG_GATHER, K_RS_TREE_V32, K_SLOT_RS_TREE_V32) = range(13)
 KERNEL_NAMES = ("rs", "ag", "stage", "slot_rs", "rs_tma", "slot_rs_tma", "rs_v32", "slot_rs_v32",
-                "rs_tree", "slot_rs_tree", "ag_gather", "rs_tree_v32", "slot_rs_tree_v32")
+                "rs_tree", "slot_rs_tree", "ag_gather", "rs_tree_v32", "slot_rs_tree_v32",
+                "stage_f32", "slot_rs_f32")
 
 
 class tide_param_t(ctypes.Structure):
@@ -84,6 +85,8 @@ _SIGNATURES = {
     "tide_flag_wait": (_i32, [_P(_vp), _i32, ctypes.c_uint32, _i64, _vp, _vp]),
     "tide_rs_stage_one": (_i32, [_vp, _P(_vp), _P(_i64), _vp, _i64, _i32, _i32, _vp]),
     "tide_rs_reduce_slots": (_i32, [_vp, _P(_vp), _i64, _vp, _i64, _i32, _i32, _i32, _vp]),
+    "tide_rs_stage_one_f32": (_i32, [_vp, _P(_vp), _P(_i64), _vp, _i64, _i32, _vp]),
+    "tide_rs_reduce_slots_f32": (_i32, [_vp, _P(_vp), _i64, _vp, _i64, _i32, _i32, _vp]),
     "tide_rs_reduce_noalloc": (_i32, [_P(tide_param_t), _i32, _i32, _P(_vp), _P(_i64), _vp, _i64,
                                       _i32, _i32, _vp]),
     "tide_rs_reduce_pipelined": (_i32, [_vp, _P(_vp), _P(_i64), _vp, _i64, _i32, _i32, _P(_vp),
@@ -172,6 +175,16 @@ def _table(tensors) -> TensorTable:
     flat = [t for row in tensors for t in row] if tensors and isinstance(tensors[0], (list, tuple)) \
         else list(tensors)
     return TensorTable(flat)
+
+
+def _require_f32(table, *tensors) -> None:
+    """The C calls of fp32 buffers count 4-byte elements: refuse torch tensors of another
+    dtype (a PointerTable's raw addresses carry none and are taken as they are)."""
+    import torch
+    held = [] if isinstance(table, PointerTable) else list(table.tensors)
+    for t in held + list(tensors):
+        if t.dtype != torch.float32:
+            raise TypeError(f"fp32 buffer expected, got {t.dtype}")
 
 
 def _check(status: int, where: str) -> None:
@@ -288,6 +301,19 @@ def tide_rs_reduce_slots(plan, slots, slot_numel: int, out: int, out_numel: int,
     slot_arr = _ptr_array(slots) if slots is not None else None
     return lib().tide_rs_reduce_slots(plan, slot_arr, slot_numel, out, out_numel, scale_mode,
                                       order, max_ctas, stream)
+
+
+def tide_rs_stage_one_f32(plan, grads, grad_numel, slot: int, slot_numel: int, max_ctas: int,
+                          stream: int) -> int:
+    return lib().tide_rs_stage_one_f32(plan, _ptr_array(grads), _i64_array(grad_numel), slot,
+                                       slot_numel, max_ctas, stream)
+
+
+def tide_rs_reduce_slots_f32(plan, slots, slot_numel: int, out: int, out_numel: int, scale_mode: int,
+                             max_ctas: int, stream: int) -> int:
+    slot_arr = _ptr_array(slots) if slots is not None else None
+    return lib().tide_rs_reduce_slots_f32(plan, slot_arr, slot_numel, out, out_numel, scale_mode,
+                                          max_ctas, stream)
 
 
 def tide_rs_reduce_noalloc(params, world: int, grads, grad_numel, out: int, out_numel: int,
@@ -494,6 +520,23 @@ class Plan:
         st = tide_rs_reduce_slots(self.handle, s.ptrs, s.min_numel, out.data_ptr(), out.numel(),
                                   scale_mode, order, max_ctas, _stream_handle(stream))
         _check(st, "tide_rs_reduce_slots")
+
+    def rs_stage_one_f32(self, grads, slot, max_ctas: int = 0, stream=None) -> None:
+        """One rank's P fp32 gradients into its own fp32 slot ([W][Ns])."""
+        g = _table(grads)
+        _require_f32(g, slot)
+        st = tide_rs_stage_one_f32(self.handle, g.ptrs, g.numels, slot.data_ptr(), slot.numel(),
+                                   max_ctas, _stream_handle(stream))
+        _check(st, "tide_rs_stage_one_f32")
+
+    def rs_reduce_slots_f32(self, slots, out, scale_mode: int = TIDE_SCALE_INV_WORLD,
+                            max_ctas: int = 0, stream=None) -> None:
+        """rs_reduce_slots over W fp32 slots (rank order)."""
+        s = _table(slots)
+        _require_f32(s, out)
+        st = tide_rs_reduce_slots_f32(self.handle, s.ptrs, s.min_numel, out.data_ptr(), out.numel(),
+                                      scale_mode, max_ctas, _stream_handle(stream))
+        _check(st, "tide_rs_reduce_slots_f32")
 
     def rs_reduce_pipelined(self, grads, out, slots, n_segments: int, copy_stream,
                             scale_mode: int = TIDE_SCALE_INV_WORLD, order: int = TIDE_ORDER_RANK,

@@ -297,6 +297,40 @@ TIDE_API tide_status_t tide_rs_reduce_slots(const tide_plan_t* plan, const void*
                                    void* stream);
 
 /*
+ * Slot-Reuse for fp32 gradients.  While gradient sync is off, FSDP2 keeps
+ * gradients in its fp32 reduce dtype across micro-batches and packs those at the
+ * next synced backward; the layout-aware reduction applies to them unchanged
+ * (weekinpapers.com, Abstract: gradients read where they lie, reduced into fp32
+ * shards), with 4-byte slot words and no bf16 widening.  Rank order only.
+ *
+ * tide_rs_stage_one_f32: slot[r*Ns + off_i + e] = g_i[r*c_i + e] for every rank
+ * r and valid e, a copy of the 4-byte words; pad positions of the slot are not
+ * written.  grads: host array of P device pointers to fp32 gradients
+ * (grad_numel[i] >= d0_i*inner_i, 4-byte aligned); slot: one device buffer of
+ * fp32 [W][Ns] (slot_numel >= W*Ns), overlapping no gradient.  One kernel
+ * launch on the SMs.  Needs an all-rank plan (TIDE_ERR_INVALID_ARG otherwise).
+ *
+ * tide_rs_reduce_slots_f32: out[r*Ns + j] = s * fl32(sum_{k=0..W-1}
+ * slot_k[r*Ns + j]), summed in rank order from slot_0 in fp32 (round to nearest
+ * even, no fused multiply-add), s = fl32(1/W) under TIDE_SCALE_INV_WORLD; +0.0
+ * at pad positions.  slots: host array of W device pointers to fp32 [W][Ns]
+ * buffers of slot_numel >= W*Ns elements each (read only; peers' memory is
+ * accepted).  out: fp32 [W][Ns], or fp32 [Ns] with a one-rank plan (rank r),
+ * whose sums then read rows [r*Ns, (r+1)*Ns) of every slot.  out must not
+ * overlap a slot.  One kernel launch.
+ *
+ * Both: errors as tide_rs_stage_one / tide_rs_reduce_slots (TIDE_ERR_ALIGNMENT
+ * for a buffer that is not 4-byte aligned); nothing is enqueued on error; the
+ * caller owns every buffer.
+ */
+TIDE_API tide_status_t tide_rs_stage_one_f32(const tide_plan_t* plan, const float* const* grads,
+                                             const int64_t* grad_numel, float* slot, int64_t slot_numel,
+                                             int32_t max_ctas, void* stream);
+TIDE_API tide_status_t tide_rs_reduce_slots_f32(const tide_plan_t* plan, const float* const* slots,
+                                                int64_t slot_numel, float* out, int64_t out_numel,
+                                                int32_t scale_mode, int32_t max_ctas, void* stream);
+
+/*
  * Slot-Reuse with the two phases overlapped (weekinpapers.com Abstract: the
  * two-phase pipeline keeps gradient reads apart from the reduction's
  * progress, and copy engines move the gradients).  Same result as
@@ -383,7 +417,8 @@ TIDE_API tide_status_t tide_rs_reduce_noalloc(const tide_param_t* params, int32_
  * 8 = RS reduce in tree order, 9 = slot reduce in tree order,
  * 10 = AG placement from per-rank shards (tide_ag_gather_place),
  * 11 = RS reduce in tree order with 32-byte loads, 12 = slot reduce in tree
- * order with 32-byte loads.
+ * order with 32-byte loads, 13 = Slot-Reuse stage of fp32 gradients
+ * (tide_rs_stage_one_f32), 14 = slot reduce of fp32 slots (tide_rs_reduce_slots_f32).
  * The reductions use kernels 4/5 (one CTA per SM, TMA loads into shared memory)
  * when the plan was built with TIDE_PLAN_TMA, every tile starts on an
  * 8-element boundary and every source and the output are 16-byte aligned.

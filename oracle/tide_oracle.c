@@ -247,7 +247,7 @@ int orc_rs_reduce_f32(int64_t W, int64_t P, const int64_t* d0, const int64_t* in
     pack_f32_of_f32(W, P, d0, inner, S, off, Ns, grads, out);
     for (int64_t k = 1; k < W; ++k) {
         pack_f32_of_f32(W, P, d0, inner, S, off, Ns, grads + k * P, packed);
-        for (int64_t j = 0; j < n; ++j) out[j] = out[j] + packed[j];
+        for (int64_t j = 0; j < n; ++j) out[j] += packed[j];
     }
     if (scale_mode == 1) {
         float sc = 1.0f / (float)W;

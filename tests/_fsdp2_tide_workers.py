@@ -67,7 +67,7 @@ def fsdp2_tide_worker(rank, world, port, steps, lr, out_dir, engine, order, mode
     import torch
     import torch.distributed as dist
     from fsdp2_layout_aware_b200 import fsdp2 as F
-    from _gpu_helpers import bits_of
+    from _gpu_helpers import bits_of, f32_bits
 
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
@@ -109,15 +109,20 @@ def fsdp2_tide_worker(rank, world, port, steps, lr, out_dir, engine, order, mode
         def stage(tg, grads):
             g, n = tick("stage", tg)
             torch.cuda.synchronize()
+            f32 = grads[0].dtype == torch.float32    # accumulated with gradient sync off
             if rank == 0:
                 with open(os.path.join(out_dir, f"staged_shapes_{g}_{n}.json"), "w") as f:
-                    json.dump([tuple(t.shape) for t in grads], f)
+                    json.dump({"shapes": [tuple(t.shape) for t in grads], "f32": f32}, f)
+            bits = f32_bits if f32 else bits_of
             for i, t in enumerate(grads):
-                save(f"grad_{g}_{n}_{rank}_{i}.npy", bits_of(t))
-            save(f"slot0_{g}_{n}_{rank}.npy", bits_of(tg.arena))
+                save(f"grad_{g}_{n}_{rank}_{i}.npy", bits(t))
+            if f32:
+                tg.ensure_arena32()
+            arena = (lambda: tg.arena32) if f32 else (lambda: tg.arena)
+            save(f"slot0_{g}_{n}_{rank}.npy", bits(arena()))
             stage0(tg, grads)
             torch.cuda.synchronize()
-            save(f"slot1_{g}_{n}_{rank}.npy", bits_of(tg.arena))
+            save(f"slot1_{g}_{n}_{rank}.npy", bits(arena()))
 
         def reduce(tg, out, op):
             g, n = tick("reduce", tg)
@@ -158,6 +163,7 @@ class OracleGroup:
         self.device = torch.device("cpu")
         self.calls = []
         self.pending = None
+        self.arena32 = None
         F._AG[self.arena.data_ptr()] = self
         F._RS[self.rs_input.data_ptr()] = self
 
@@ -171,6 +177,13 @@ class OracleGroup:
         bufs = [torch.empty_like(t) for _ in range(self.world)]
         dist.all_gather(bufs, t.contiguous())
         return [b.view(torch.int16).numpy().view(np.uint16) for b in bufs]
+
+    def _all32(self, t):
+        import torch
+        import torch.distributed as dist
+        bufs = [torch.empty_like(t) for _ in range(self.world)]
+        dist.all_gather(bufs, t.contiguous())
+        return [b.numpy() for b in bufs]
 
     def place(self, out):
         import oracle
@@ -187,26 +200,38 @@ class OracleGroup:
         import oracle
         import torch
         from fsdp2_layout_aware_b200 import fsdp2 as F
-        F._check_grads(grads, len(self.shapes))
+        f32 = F._check_grads(grads, len(self.shapes))
         self.calls.append("stage")
         shapes = [tuple(g.shape) for g in grads]            # the parameters that got gradients
         ns = oracle.layout(self.world, shapes).Ns
-        bits = [g.detach().contiguous().view(torch.int16).numpy().reshape(-1).view(np.uint16) for g in grads]
-        slot = self.arena.view(torch.int16).numpy().view(np.uint16)   # shares the arena's memory
-        oracle.slot_stage(self.world, shapes, bits, slot[:self.world * ns])
-        self.pending = (shapes, ns)
+        if f32:                                             # accumulated with gradient sync off
+            if self.arena32 is None:
+                self.arena32 = torch.zeros(self.world * self.shard_numel)
+            words = [g.detach().contiguous().numpy().reshape(-1).view(np.uint32) for g in grads]
+            slot = self.arena32.numpy().view(np.uint32)     # shares the fp32 slot's memory
+            oracle.slot_stage_f32(self.world, shapes, words, slot[:self.world * ns])
+        else:
+            bits = [g.detach().contiguous().view(torch.int16).numpy().reshape(-1).view(np.uint16)
+                    for g in grads]
+            slot = self.arena.view(torch.int16).numpy().view(np.uint16)   # shares the arena's memory
+            oracle.slot_stage(self.world, shapes, bits, slot[:self.world * ns])
+        self.pending = (shapes, ns, f32)
 
     def reduce(self, out, op):
         import oracle
         import torch
         import torch.distributed as dist
         self.calls.append("reduce")
-        shapes, ns = self.pending
+        shapes, ns, f32 = self.pending
         self.pending = None
         self.meet()
-        slots = [s[:self.world * ns] for s in self._all(self.arena)]
         scale = 1 if op == dist.ReduceOp.AVG else 0
-        res = oracle.rs_reduce_slots(self.world, shapes, slots, scale)
+        if f32:
+            slots = [s[:self.world * ns] for s in self._all32(self.arena32)]
+            res = oracle.rs_reduce_slots_f32(self.world, shapes, slots, scale)
+        else:
+            slots = [s[:self.world * ns] for s in self._all(self.arena)]
+            res = oracle.rs_reduce_slots(self.world, shapes, slots, scale)
         r = self.rank
         out.copy_(torch.from_numpy(res[r * ns:(r + 1) * ns].copy()))
         self.meet()
@@ -248,15 +273,6 @@ def fsdp2_oracle_worker(rank, world, port, steps, lr, out_dir, mode="plain"):
                     m.set_custom_reduce_scatter(rs_cls(tg))
                     groups.append(tg)
             opt = torch.optim.SGD(model.parameters(), lr=lr)
-            if arm == "tide" and mode == "accum_unsynced":
-                try:
-                    _backward(model, x, y, mode)
-                    refusal = None
-                except ValueError as e:
-                    refusal = str(e)
-                with open(os.path.join(out_dir, f"refusal_{rank}.json"), "w") as f:
-                    json.dump(refusal, f)
-                return
             for step in range(steps):
                 _backward(model, x, y, mode)
                 for i, p in enumerate(model.parameters()):

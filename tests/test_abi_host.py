@@ -485,3 +485,79 @@ def test_flag_calls_validate_their_arguments_on_the_host():
     assert T.tide_flag_wait([f], 1, 1000, status + 1) == T.TIDE_ERR_ALIGNMENT
     assert T.tide_flag_wait([f, 0], 1, 1000, status) == T.TIDE_ERR_INVALID_ARG
     assert T.tide_flag_wait([f, f + 6], 1, 1000, status) == T.TIDE_ERR_ALIGNMENT
+
+
+def f32_args(group):
+    """Fake fp32 buffers: one rank's gradients, W fp32 slots, the fp32 output."""
+    W, P = group.world, group.n_params
+    L = oracle.layout(W, group.shapes)
+    f = Fake()
+    f.next = BASE + (1 << 41)                        # clear of the other fake buffers
+    return dict(grads=[f.buf(4 * group.numel(i)) for i in range(P)],
+                gnum=[group.numel(i) for i in range(P)],
+                slots=[f.buf(4 * W * L.Ns) for _ in range(W)], n_slot=W * L.Ns,
+                out=f.buf(4 * W * L.Ns), n_out=W * L.Ns, Ns=L.Ns)
+
+
+def test_f32_stage_validation(tiny_plan):
+    a = f32_args(configs.tiny())
+    g, gn, sl, n = a["grads"], a["gnum"], a["slots"][0], a["n_slot"]
+
+    def stage(g=g, gn=gn, sl=sl, ns=n, cap=0, plan=tiny_plan):
+        return T.tide_rs_stage_one_f32(plan.handle, g, gn, sl, ns, cap, 0)
+    assert stage() == T.TIDE_ERR_DEVICE              # valid: stops at the host-only plan
+    assert stage(cap=-1) == T.TIDE_ERR_INVALID_ARG
+    assert stage(g=[0] + g[1:]) == T.TIDE_ERR_INVALID_ARG
+    assert stage(g=g[:2] + [g[2] + 2] + g[3:]) == T.TIDE_ERR_ALIGNMENT   # 2-byte aligned is not enough
+    assert stage(gn=gn[:4] + [gn[4] - 1]) == T.TIDE_ERR_SIZE
+    assert stage(sl=0) == T.TIDE_ERR_INVALID_ARG
+    assert stage(sl=sl + 2) == T.TIDE_ERR_ALIGNMENT
+    assert stage(ns=n - 1) == T.TIDE_ERR_SIZE
+    assert stage(sl=g[3]) == T.TIDE_ERR_INVALID_ARG  # the slot overlaps a gradient
+    # a gradient's fp32 bytes end where its bf16 bytes would not: the spans are 4-byte ones
+    assert stage(sl=g[4] + 4 * (gn[4] - 1)) == T.TIDE_ERR_INVALID_ARG
+    one_rank = T.Plan(configs.tiny().shapes, 4, host_only=True, rank=1)
+    assert stage(plan=one_rank) == T.TIDE_ERR_INVALID_ARG
+
+
+def test_f32_reduce_slots_validation(tiny_plan):
+    a = f32_args(configs.tiny())
+    sl, n, out, n_out = a["slots"], a["n_slot"], a["out"], a["n_out"]
+
+    def red(sl=sl, ns=n, o=out, no=n_out, scale=1, cap=0, plan=tiny_plan):
+        return T.tide_rs_reduce_slots_f32(plan.handle, sl, ns, o, no, scale, cap, 0)
+    assert red() == T.TIDE_ERR_DEVICE
+    assert red(scale=0) == T.TIDE_ERR_DEVICE
+    assert red(scale=2) == T.TIDE_ERR_INVALID_ARG
+    assert red(cap=-3) == T.TIDE_ERR_INVALID_ARG
+    assert red(sl=None) == T.TIDE_ERR_INVALID_ARG
+    assert red(sl=[sl[0] + 2] + sl[1:]) == T.TIDE_ERR_ALIGNMENT
+    assert red(sl=sl[:3] + [0]) == T.TIDE_ERR_INVALID_ARG
+    assert red(ns=n - 1) == T.TIDE_ERR_SIZE
+    assert red(no=n_out - 1) == T.TIDE_ERR_SIZE
+    assert red(o=out + 2) == T.TIDE_ERR_ALIGNMENT
+    assert red(o=sl[2]) == T.TIDE_ERR_INVALID_ARG     # out overlaps a slot
+    assert red(sl=[sl[0]] * 4) == T.TIDE_ERR_DEVICE   # slots may alias (only read)
+    # a one-rank plan: one shard out
+    one_rank = T.Plan(configs.tiny().shapes, 4, host_only=True, rank=3)
+    assert red(plan=one_rank, no=a["Ns"]) == T.TIDE_ERR_DEVICE
+    assert red(plan=one_rank, no=a["Ns"] - 1) == T.TIDE_ERR_SIZE
+
+
+def test_f32_bindings_refuse_other_dtypes():
+    """The Plan methods of the fp32 calls refuse torch tensors that are not fp32 before any
+    call: the C calls count 4-byte elements."""
+    import torch
+    plan = T.Plan(configs.tiny().shapes, 4, host_only=True)
+    g = configs.tiny()
+    L = oracle.layout(4, g.shapes)
+    bf = [torch.zeros(g.numel(i), dtype=torch.bfloat16) for i in range(g.n_params)]
+    f32 = [torch.zeros(g.numel(i)) for i in range(g.n_params)]
+    with pytest.raises(TypeError):
+        plan.rs_stage_one_f32(bf, torch.zeros(4 * L.Ns))
+    with pytest.raises(TypeError):
+        plan.rs_stage_one_f32(f32, torch.zeros(4 * L.Ns, dtype=torch.bfloat16))
+    with pytest.raises(TypeError):
+        plan.rs_reduce_slots_f32([torch.zeros(4 * L.Ns, dtype=torch.bfloat16)] * 4, torch.zeros(4 * L.Ns))
+    with pytest.raises(TypeError):
+        plan.rs_reduce_slots_f32([torch.zeros(4 * L.Ns)] * 4, torch.zeros(4 * L.Ns, dtype=torch.float16))

@@ -27,16 +27,20 @@ CALLS = {
     "frozen": (["place", "place", "stage", "reduce"], ["place", "stage", "reduce"]),
     "accum": (["place", "place", "stage", "reduce"] * 2, ["place", "stage", "reduce"] * 2),
     "no_reshard": (["place", "stage", "reduce"], ["place", "stage", "reduce"]),
+    "accum_unsynced": (["place", "place", "place", "place", "stage", "reduce"],
+                       ["place", "place", "stage", "reduce"]),
 }
 
 
 @pytest.mark.parametrize("world,mode", [(2, "plain"), (3, "plain"), (2, "frozen"), (2, "accum"),
-                                        (3, "no_reshard")],
+                                        (3, "no_reshard"), (2, "accum_unsynced"), (3, "accum_unsynced")],
                          ids=["w2", "w3", "w2_frozen_param", "w2_grad_accumulation",
-                              "w3_no_reshard_after_forward"])
+                              "w3_no_reshard_after_forward", "w2_accumulation_sync_off",
+                              "w3_accumulation_sync_off"])
 def test_fsdp2_with_tide_comms_gives_stock_fsdp2_results(world, mode, tmp_path):
     """With a frozen parameter (no gradient) its group reduce-scatters the others only; with
-    gradient accumulation the reduced gradients are the sum over both micro-batches."""
+    gradient accumulation the reduced gradients are the sum over both micro-batches (sync off:
+    FSDP2 packs fp32 gradients, staged into the fp32 slots)."""
     from _fsdp2_tide_workers import fsdp2_oracle_worker
     steps, lr = 3, 0.05
     run_procs(fsdp2_oracle_worker, world,
@@ -58,17 +62,17 @@ def test_fsdp2_with_tide_comms_gives_stock_fsdp2_results(world, mode, tmp_path):
         assert calls[2] == root * steps, calls
 
 
-def test_accumulation_with_gradient_sync_off_is_refused_at_the_staging(tmp_path):
-    """With gradient sync off FSDP2 keeps the micro-batch's unsharded gradients in the fp32
-    reduce dtype and hands them to the pack of the next synced backward; TIDE's staging
-    takes bf16 gradients only and says so, on every rank, before any reduction."""
-    from _fsdp2_tide_workers import fsdp2_oracle_worker
-    world = 2
-    run_procs(fsdp2_oracle_worker, world,
-              lambda port: (world, port, 1, 0.05, str(tmp_path), "accum_unsynced"))
-    for r in range(world):
-        msg = json.loads((tmp_path / f"refusal_{r}.json").read_text())
-        assert msg is not None and "fp32 gradients" in msg and "sync" in msg, msg
+def test_staging_takes_bf16_or_fp32_gradients_of_one_dtype():
+    import torch
+    from fsdp2_layout_aware_b200 import fsdp2 as F
+    bf, f32 = torch.zeros(4, 3, dtype=torch.bfloat16), torch.zeros(4, 3)
+    assert F._check_grads([bf, bf], 2) is False
+    assert F._check_grads([f32], 2) is True
+    for bad, n in (([bf, f32], 2), ([torch.zeros(3, dtype=torch.float16)], 1), ([bf, bf, bf], 2),
+                   ([], 2), ([torch.zeros(4, 6, dtype=torch.bfloat16)[:, :3]], 1),
+                   ([torch.zeros((), dtype=torch.bfloat16)], 1)):
+        with pytest.raises(ValueError):
+            F._check_grads(bad, n)
 
 
 def test_tide_comms_hand_out_the_groups_buffers_and_refuse_others():

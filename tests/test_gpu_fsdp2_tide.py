@@ -32,13 +32,16 @@ def _load(tmp, name):
 
 @pytest.mark.parametrize("world,engine,order,mode",
                          [(2, 0, 0, "plain"), (3, 0, 0, "plain"), (3, 1, 1, "plain"),
-                          (2, 0, 0, "frozen"), (2, 1, 0, "accum"), (3, 0, 1, "no_reshard")],
+                          (2, 0, 0, "frozen"), (2, 1, 0, "accum"), (3, 0, 1, "no_reshard"),
+                          (3, 0, 0, "accum_unsynced")],
                          ids=["w2_sm_rank", "w3_sm_rank", "w3_ce_tree", "w2_frozen_param",
-                              "w2_ce_rank_grad_accumulation", "w3_sm_tree_no_reshard"])
+                              "w2_ce_rank_grad_accumulation", "w3_sm_tree_no_reshard",
+                              "w3_sm_rank_accumulation_sync_off"])
 def test_fully_shard_with_tide_collectives_matches_the_oracle(world, engine, order, mode, tmp_path):
     """(With a frozen parameter its group stages and reduces the others only, in the layout
     their shapes give; accumulating, each of a step's two micro-batches is reduced; kept
-    unsharded after forward, each group is placed once a step.)"""
+    unsharded after forward, each group is placed once a step; accumulating with gradient
+    sync off, FSDP2 packs fp32 gradients, staged into fp32 slots and reduced in rank order.)"""
     from _fsdp2_tide_workers import fsdp2_tide_worker
     steps, lr = 3, 0.05
     run_procs(fsdp2_tide_worker, world,
@@ -64,15 +67,18 @@ def test_fully_shard_with_tide_collectives_matches_the_oracle(world, engine, ord
                     got = _load(tmp_path, f"placed_{g}_{n}_{r}_{i}.npy")
                     assert np.array_equal(got, want[i]), (g, n, r, i)
         for n in range(n_reduce):
-            Sr = [tuple(x) for x in json.loads((tmp_path / f"staged_shapes_{g}_{n}.json").read_text())]
+            staged = json.loads((tmp_path / f"staged_shapes_{g}_{n}.json").read_text())
+            Sr, f32 = [tuple(x) for x in staged["shapes"]], staged["f32"]
+            assert f32 == (mode == "accum_unsynced")
             Lr = oracle.layout(world, Sr)
             grads = [[_load(tmp_path, f"grad_{g}_{n}_{k}_{i}.npy") for i in range(len(Sr))]
                      for k in range(world)]
             for k in range(world):
                 exp = _load(tmp_path, f"slot0_{g}_{n}_{k}.npy").copy()
-                oracle.slot_stage(world, Sr, grads[k], exp[:world * Lr.Ns])
+                (oracle.slot_stage_f32 if f32 else oracle.slot_stage)(world, Sr, grads[k],
+                                                                      exp[:world * Lr.Ns])
                 assert np.array_equal(_load(tmp_path, f"slot1_{g}_{n}_{k}.npy"), exp), (g, n, k)
-            ref = rs_oracle(world, Sr, grads, 1).reshape(world, Lr.Ns)
+            ref = (oracle.rs_reduce_f32 if f32 else rs_oracle)(world, Sr, grads, 1).reshape(world, Lr.Ns)
             for r in range(world):
                 got = _load(tmp_path, f"shard_{g}_{n}_{r}.npy")
                 assert np.array_equal(got.view(np.uint32), ref[r].view(np.uint32)), (g, n, r)
