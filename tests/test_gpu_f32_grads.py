@@ -29,7 +29,8 @@ def groups():
     return [configs.tiny(), degenerate(), mini_wan(), mini_sweep(2), mini_sweep(8),
             configs.Group("two_tiles", 4, ((4 * 2048 + 3, 9),)),
             random_group(rng, 3, 6, name="rand_w3"), random_group(rng, 5, 5, name="rand_w5"),
-            random_group(rng, 64, 4, name="rand_w64")]
+            random_group(rng, 64, 4, name="rand_w64"),
+            random_group(rng, 256, 3, max_rows=600, name="rand_w256")]
 
 
 def f32_grads(group, seed):
