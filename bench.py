@@ -464,6 +464,9 @@ def run_variants(wl, K, stream, peak, flush):
         for k in range(W):
             g32 = T.TensorTable([t.float() for t in wl.grads[k]])
             if k == 0:
+                rec("stage_one_f32_ce",
+                    timed_calls(lambda: wl.plan.rs_stage_one_f32(g32, slots32[0], engine=T.TIDE_ENGINE_CE),
+                                K, stream, flush), 8 * N, 0, wl.plan)
                 rec("stage_one_f32", timed_calls(lambda: wl.plan.rs_stage_one_f32(g32, slots32[0]),
                                                  K, stream, flush), 8 * N, 1, wl.plan)
             else:
@@ -495,6 +498,7 @@ ROW_KINDS = {
     "ag_gather_place_sm": ("ag_gather_place", "SM, from per-rank shards"),
     "ag_gather_place_ce": ("ag_gather_place", "copy engines, from per-rank shards"),
     "stage_one_f32": ("slot_stage", "fp32 gradients of one rank, SM"),
+    "stage_one_f32_ce": ("slot_stage", "fp32 gradients of one rank, copy engines"),
     "slot_reduce_f32": ("slot_reduce", "fp32 slots, SM, rank order"),
     "stock_torch_pack_reduce": ("stock_rs", "torch _chunk_cat pack + add"),
     "stock_torch_copyout": ("stock_ag", "torch split_with_sizes_copy"),

@@ -468,13 +468,13 @@ extern "C" tide_status_t tide_rs_reduce_slots(const tide_plan_t* cplan, const vo
 
 extern "C" tide_status_t tide_rs_stage_one_f32(const tide_plan_t* cplan, const float* const* grads,
                                                const int64_t* grad_numel, float* slot, int64_t slot_numel,
-                                               int32_t max_ctas, void* stream) {
+                                               int32_t engine, int32_t max_ctas, void* stream) {
     ApiRange range("tide_rs_stage_one_f32");
     tide_plan* p = const_cast<tide_plan*>(cplan);
     tide_status_t st = check_plan(p);
     if (st != TIDE_OK) return st;
     if ((st = all_ranks(p)) != TIDE_OK) return st;
-    if ((st = check_enums(p, TIDE_ENGINE_SM, max_ctas)) != TIDE_OK) return st;
+    if ((st = check_enums(p, engine, max_ctas)) != TIDE_OK) return st;
     const int64_t W = p->world, P = p->n_params;
     std::vector<Span> spans;
     spans.reserve((size_t)P + 1);
@@ -489,6 +489,14 @@ extern "C" tide_status_t tide_rs_stage_one_f32(const tide_plan_t* cplan, const f
     if ((st = launchable(p)) != TIDE_OK) return st;
     if (p->tiles.empty()) return TIDE_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (engine == TIDE_ENGINE_CE) {
+        p->last_kernel = -1;
+        p->last_ctas = 0;
+        void* const slots[1] = {slot};
+        cudaError_t e = tide::ce_slot_stage(p, reinterpret_cast<const void* const*>(grads), slots, s, 0, -1,
+                                            false, true, 4);
+        return e == cudaSuccess ? TIDE_OK : TIDE_ERR_CUDA;
+    }
     if ((st = sync_table(p->grad_tab, reinterpret_cast<const void* const*>(grads), P, s)) != TIDE_OK)
         return st;
     p->last_kernel = K_STAGE_F32;

@@ -241,7 +241,7 @@ CeOp rows_op(void* dst, size_t dpitch, const void* src, size_t spitch, size_t wi
 // Recorded graphs kept per plan (the least recently used one is replaced).
 constexpr size_t kMaxCeGraphs = 4;
 
-enum { kCallPlace = 1, kCallGather = 2, kCallStage = 3, kCallRankStage = 4 };
+enum { kCallPlace = 1, kCallGather = 2, kCallStage = 3, kCallRankStage = 4, kCallStageF32 = 5 };
 
 // Issue the planned lists (q->lists) as one call on `stream`: replay the graph
 // recorded for (kind, j0, j1, key) if there is one, else record it now and
@@ -382,10 +382,12 @@ cudaError_t ce_ag_gather(tide_plan* p, const void* const* shards, void* const* p
 // Stage the chunks [j0, j1) (chunk i*W + r: rank r's rows of param i) from
 // every source rank k into slot k.  Within one param the chunks of a range are
 // consecutive ranks, so each (k, param) pair takes one 2-D copy plus at most
-// one 1-D copy for a partial chunk.
+// one 1-D copy for a partial chunk.  esize: bytes per element (2 for bf16
+// gradients and slots, 4 for fp32).
 cudaError_t ce_slot_stage(tide_plan* p, const void* const* grads, void* const* slots,
-                          cudaStream_t caller, int64_t j0, int64_t j1, bool record, bool one_source) {
-    const int64_t W = p->world, P = p->n_params, Ns = p->shard_numel;
+                          cudaStream_t caller, int64_t j0, int64_t j1, bool record, bool one_source,
+                          int esize) {
+    const int64_t W = p->world, P = p->n_params, Ns = p->shard_numel, e = esize;
     const int64_t sources = one_source ? 1 : W;
     if (j1 < 0) j1 = P * W;
     if (j1 <= j0) return cudaSuccess;
@@ -396,23 +398,25 @@ cudaError_t ce_slot_stage(tide_plan* p, const void* const* grads, void* const* s
         for (int64_t k = 0; k < sources; ++k) key.push_back(slots[k]);
         key.push_back(reinterpret_cast<const void*>(sources));
     }
-    return run_call(p, caller, kCallStage, j0, j1, std::move(key), record, [&](CeIssuer* q) {
+    const int kind = esize == 4 ? kCallStageF32 : kCallStage;
+    return run_call(p, caller, kind, j0, j1, std::move(key), record, [&](CeIssuer* q) {
         for (int64_t k = 0; k < sources; ++k) {
-            uint16_t* slot = static_cast<uint16_t*>(slots[k]);
+            char* slot = static_cast<char*>(slots[k]);
             for (int64_t i = j0 / W; i <= (j1 - 1) / W; ++i) {
                 // one source rank per stream at a time; one rank's params spread over the streams
                 auto& l = q->lists[(one_source ? i : k) % kFanout];
                 const int64_t c = p->chunk[i], n = p->numel[i];
                 if (c == 0 || n == 0) continue;
                 const int64_t r0 = std::max<int64_t>(0, j0 - i * W), r1 = std::min<int64_t>(W, j1 - i * W);
-                const uint16_t* g = static_cast<const uint16_t*>(grads[k * P + i]);
-                uint16_t* dst = slot + p->offset[i];
+                const char* g = static_cast<const char*>(grads[k * P + i]);
+                char* dst = slot + e * p->offset[i];
                 const int64_t full = std::min(W, n / c);  // ranks [0, full) hold whole chunks
                 const int64_t fr1 = std::min(full, r1);
-                if (fr1 > r0) l.push_back(rows_op(dst + r0 * Ns, 2 * Ns, g + r0 * c, 2 * c, 2 * c, fr1 - r0));
+                if (fr1 > r0)
+                    l.push_back(rows_op(dst + e * r0 * Ns, e * Ns, g + e * r0 * c, e * c, e * c, fr1 - r0));
                 const int64_t rem = n - full * c;       // rank `full` holds a partial chunk
                 if (rem > 0 && full < W && full >= r0 && full < r1)
-                    l.push_back(rows_op(dst + full * Ns, 0, g + full * c, 0, 2 * rem, 1));
+                    l.push_back(rows_op(dst + e * full * Ns, 0, g + e * full * c, 0, e * rem, 1));
             }
         }
     });

@@ -124,10 +124,11 @@ cudaError_t ce_ag_gather(tide_plan* p, const void* const* shards, void* const* p
 // all) from every source rank k into slot k.  The copies are issued directly
 // (`record` = false): a recorded graph of them measured slower (Wan2.2 group:
 // 3.55 against 4.07 TB/s; within 2 % elsewhere).  one_source: grads holds one
-// rank's P gradients and slots one slot, which receives them.
+// rank's P gradients and slots one slot, which receives them.  esize: bytes per
+// element of the gradients and slots (2: bf16, 4: fp32).
 cudaError_t ce_slot_stage(tide_plan* p, const void* const* grads, void* const* slots,
                           cudaStream_t stream, int64_t j0 = 0, int64_t j1 = -1, bool record = false,
-                          bool one_source = false);
+                          bool one_source = false, int esize = 2);
 // A one-rank plan's phase 1: chunk `rank` of every rank k's gradients into
 // slots[k] (that rank's row only, Ns elements), for the chunks [j0, j1).
 cudaError_t ce_rank_stage(tide_plan* p, const void* const* grads, void* const* slots,

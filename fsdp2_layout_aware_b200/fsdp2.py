@@ -186,7 +186,7 @@ class TideGroup:
         plan, rank_plan, ns = self.plans_for([tuple(g.shape) for g in grads])
         if f32:
             self.ensure_arena32()
-            plan.rs_stage_one_f32(T.TensorTable(list(grads)), self.arena32)
+            plan.rs_stage_one_f32(T.TensorTable(list(grads)), self.arena32, engine=self.engine)
         else:
             plan.rs_stage_one(T.TensorTable(list(grads)), self.arena, engine=self.engine)
         self.pending = (rank_plan, ns, f32)

@@ -85,7 +85,7 @@ _SIGNATURES = {
     "tide_flag_wait": (_i32, [_P(_vp), _i32, ctypes.c_uint32, _i64, _vp, _vp]),
     "tide_rs_stage_one": (_i32, [_vp, _P(_vp), _P(_i64), _vp, _i64, _i32, _i32, _vp]),
     "tide_rs_reduce_slots": (_i32, [_vp, _P(_vp), _i64, _vp, _i64, _i32, _i32, _i32, _vp]),
-    "tide_rs_stage_one_f32": (_i32, [_vp, _P(_vp), _P(_i64), _vp, _i64, _i32, _vp]),
+    "tide_rs_stage_one_f32": (_i32, [_vp, _P(_vp), _P(_i64), _vp, _i64, _i32, _i32, _vp]),
     "tide_rs_reduce_slots_f32": (_i32, [_vp, _P(_vp), _i64, _vp, _i64, _i32, _i32, _vp]),
     "tide_rs_reduce_noalloc": (_i32, [_P(tide_param_t), _i32, _i32, _P(_vp), _P(_i64), _vp, _i64,
                                       _i32, _i32, _vp]),
@@ -303,10 +303,10 @@ def tide_rs_reduce_slots(plan, slots, slot_numel: int, out: int, out_numel: int,
                                       order, max_ctas, stream)
 
 
-def tide_rs_stage_one_f32(plan, grads, grad_numel, slot: int, slot_numel: int, max_ctas: int,
-                          stream: int) -> int:
+def tide_rs_stage_one_f32(plan, grads, grad_numel, slot: int, slot_numel: int, engine: int,
+                          max_ctas: int, stream: int) -> int:
     return lib().tide_rs_stage_one_f32(plan, _ptr_array(grads), _i64_array(grad_numel), slot,
-                                       slot_numel, max_ctas, stream)
+                                       slot_numel, engine, max_ctas, stream)
 
 
 def tide_rs_reduce_slots_f32(plan, slots, slot_numel: int, out: int, out_numel: int, scale_mode: int,
@@ -521,12 +521,13 @@ class Plan:
                                   scale_mode, order, max_ctas, _stream_handle(stream))
         _check(st, "tide_rs_reduce_slots")
 
-    def rs_stage_one_f32(self, grads, slot, max_ctas: int = 0, stream=None) -> None:
+    def rs_stage_one_f32(self, grads, slot, engine: int = TIDE_ENGINE_SM, max_ctas: int = 0,
+                         stream=None) -> None:
         """One rank's P fp32 gradients into its own fp32 slot ([W][Ns])."""
         g = _table(grads)
         _require_f32(g, slot)
         st = tide_rs_stage_one_f32(self.handle, g.ptrs, g.numels, slot.data_ptr(), slot.numel(),
-                                   max_ctas, _stream_handle(stream))
+                                   engine, max_ctas, _stream_handle(stream))
         _check(st, "tide_rs_stage_one_f32")
 
     def rs_reduce_slots_f32(self, slots, out, scale_mode: int = TIDE_SCALE_INV_WORLD,

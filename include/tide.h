@@ -307,8 +307,10 @@ TIDE_API tide_status_t tide_rs_reduce_slots(const tide_plan_t* plan, const void*
  * r and valid e, a copy of the 4-byte words; pad positions of the slot are not
  * written.  grads: host array of P device pointers to fp32 gradients
  * (grad_numel[i] >= d0_i*inner_i, 4-byte aligned); slot: one device buffer of
- * fp32 [W][Ns] (slot_numel >= W*Ns), overlapping no gradient.  One kernel
- * launch on the SMs.  Needs an all-rank plan (TIDE_ERR_INVALID_ARG otherwise).
+ * fp32 [W][Ns] (slot_numel >= W*Ns), overlapping no gradient.  engine SM (one
+ * kernel launch) or CE (per param one 2-D copy plus at most one 1-D copy on the
+ * copy engines, no kernel).  Needs an all-rank plan (TIDE_ERR_INVALID_ARG
+ * otherwise).
  *
  * tide_rs_reduce_slots_f32: out[r*Ns + j] = s * fl32(sum_{k=0..W-1}
  * slot_k[r*Ns + j]), summed in rank order from slot_0 in fp32 (round to nearest
@@ -325,7 +327,7 @@ TIDE_API tide_status_t tide_rs_reduce_slots(const tide_plan_t* plan, const void*
  */
 TIDE_API tide_status_t tide_rs_stage_one_f32(const tide_plan_t* plan, const float* const* grads,
                                              const int64_t* grad_numel, float* slot, int64_t slot_numel,
-                                             int32_t max_ctas, void* stream);
+                                             int32_t engine, int32_t max_ctas, void* stream);
 TIDE_API tide_status_t tide_rs_reduce_slots_f32(const tide_plan_t* plan, const float* const* slots,
                                                 int64_t slot_numel, float* out, int64_t out_numel,
                                                 int32_t scale_mode, int32_t max_ctas, void* stream);

@@ -503,9 +503,11 @@ def test_f32_stage_validation(tiny_plan):
     a = f32_args(configs.tiny())
     g, gn, sl, n = a["grads"], a["gnum"], a["slots"][0], a["n_slot"]
 
-    def stage(g=g, gn=gn, sl=sl, ns=n, cap=0, plan=tiny_plan):
-        return T.tide_rs_stage_one_f32(plan.handle, g, gn, sl, ns, cap, 0)
+    def stage(g=g, gn=gn, sl=sl, ns=n, cap=0, plan=tiny_plan, engine=0):
+        return T.tide_rs_stage_one_f32(plan.handle, g, gn, sl, ns, engine, cap, 0)
     assert stage() == T.TIDE_ERR_DEVICE              # valid: stops at the host-only plan
+    assert stage(engine=1) == T.TIDE_ERR_DEVICE
+    assert stage(engine=2) == T.TIDE_ERR_INVALID_ARG
     assert stage(cap=-1) == T.TIDE_ERR_INVALID_ARG
     assert stage(g=[0] + g[1:]) == T.TIDE_ERR_INVALID_ARG
     assert stage(g=g[:2] + [g[2] + 2] + g[3:]) == T.TIDE_ERR_ALIGNMENT   # 2-byte aligned is not enough

@@ -1,8 +1,8 @@
 """fp32 gradients through Slot-Reuse (tide_rs_stage_one_f32, tide_rs_reduce_slots_f32) against
 the oracle, bit for bit.
 
-Every source rank stages its fp32 gradients into its own fp32 slot (stale contents: NaN, so a
-pad that is read shows); the slots must equal the oracle's staging word for word (pads keep
+Every source rank stages its fp32 gradients into its own fp32 slot, on the SMs or on the copy
+engines (stale contents: NaN, so a pad that is read shows); the slots must equal the oracle's staging word for word (pads keep
 the NaN), and the reduction of all ranks' shards (all-rank plan) and of each rank's shard
 (one-rank plans) must equal the oracle's fp32 reduction bit for bit, with and without the
 1/W scale, on the vector path (32-byte aligned buffers), on the element path (buffers shifted
@@ -57,25 +57,26 @@ def dev_f32(arr, shift=0):
     return t.view(torch.float32)
 
 
-def stage_all(group, grads, plan, shift, cap=0):
+def stage_all(group, grads, plan, shift, cap=0, engine=T.TIDE_ENGINE_SM):
     W = group.world
     L = oracle.layout(W, group.shapes)
     slots = [dev_f32(np.full(W * L.Ns, NAN, np.uint32), shift) for _ in range(W)]
     for k in range(W):
         g = [dev_f32(grads[k][i], shift) for i in range(group.n_params)]
-        plan.rs_stage_one_f32(g, slots[k], max_ctas=cap)
+        plan.rs_stage_one_f32(g, slots[k], engine=engine, max_ctas=cap)
     torch.cuda.synchronize()
     return slots
 
 
+@pytest.mark.parametrize("engine", [T.TIDE_ENGINE_SM, T.TIDE_ENGINE_CE], ids=["sm", "ce"])
 @pytest.mark.parametrize("shift", [0, 1], ids=["aligned", "shifted"])
 @pytest.mark.parametrize("group", groups(), ids=lambda g: f"{g.name}_w{g.world}")
-def test_f32_slot_reuse_matches_the_oracle(group, shift):
+def test_f32_slot_reuse_matches_the_oracle(group, shift, engine):
     W = group.world
     L = oracle.layout(W, group.shapes)
     grads = f32_grads(group, seed=W * 100 + group.n_params)
     plan = T.Plan(group.shapes, W)
-    slots = stage_all(group, grads, plan, shift)
+    slots = stage_all(group, grads, plan, shift, engine=engine)
     for k in range(W):
         want = np.full(W * L.Ns, NAN, np.uint32)
         oracle.slot_stage_f32(W, group.shapes, grads[k], want)

@@ -33,10 +33,10 @@ def _load(tmp, name):
 @pytest.mark.parametrize("world,engine,order,mode",
                          [(2, 0, 0, "plain"), (3, 0, 0, "plain"), (3, 1, 1, "plain"),
                           (2, 0, 0, "frozen"), (2, 1, 0, "accum"), (3, 0, 1, "no_reshard"),
-                          (3, 0, 0, "accum_unsynced")],
+                          (3, 0, 0, "accum_unsynced"), (2, 1, 1, "accum_unsynced")],
                          ids=["w2_sm_rank", "w3_sm_rank", "w3_ce_tree", "w2_frozen_param",
                               "w2_ce_rank_grad_accumulation", "w3_sm_tree_no_reshard",
-                              "w3_sm_rank_accumulation_sync_off"])
+                              "w3_sm_rank_accumulation_sync_off", "w2_ce_tree_accumulation_sync_off"])
 def test_fully_shard_with_tide_collectives_matches_the_oracle(world, engine, order, mode, tmp_path):
     """(With a frozen parameter its group stages and reduces the others only, in the layout
     their shapes give; accumulating, each of a step's two micro-batches is reduced; kept
