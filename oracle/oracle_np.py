@@ -67,6 +67,29 @@ def rs_direct(world: int, shapes, grads, scale_mode: int) -> np.ndarray:
     return out
 
 
+def rs_direct_f32(world: int, shapes, grads, scale_mode: int) -> np.ndarray:
+    """rs_direct for fp32 gradients (grads[k][i]: flat float32, or their uint32 bits): the
+    same definition with the fp32 values taken as they are."""
+    S, c, off, Ns = layout(world, shapes)
+    out = np.zeros(world * Ns, dtype=np.float32)
+    inv = np.float32(1.0) / np.float32(world)
+    g = [[np.ascontiguousarray(x).reshape(-1).view(np.float32) for x in row] for row in grads]
+    for i, shp in enumerate(shapes):
+        n_i = _numel(shp)
+        for r in range(world):
+            lo = r * c[i]
+            hi = min(lo + c[i], n_i)
+            if hi <= lo:
+                continue
+            acc = g[0][i][lo:hi].copy()
+            for k in range(1, world):
+                acc = acc + g[k][i][lo:hi]
+            if scale_mode == 1:
+                acc = acc * inv
+            out[r * Ns + off[i]: r * Ns + off[i] + (hi - lo)] = acc
+    return out
+
+
 def ag_direct(world: int, shapes, ag: np.ndarray) -> list:
     """ag: uint16 [W, Ns].  Returns per-param padded storage (flat uint16, W*c_i each)."""
     S, c, off, Ns = layout(world, shapes)

@@ -570,3 +570,16 @@ def test_f32_gloo_reduce_scatter_agrees(tmp_path):
                                                    for i in range(grp.n_params)], 0.0).numpy()
             bound = (W - 1) * 2.0 ** -24 * mag
             assert np.all(np.abs(got - ex) <= bound) and np.all(np.abs(out - ex) <= bound)
+
+
+@pytest.mark.parametrize("grp", groups_for_agreement(), ids=lambda g: f"{g.name}_w{g.world}")
+def test_two_oracles_agree_on_f32_gradients(grp):
+    """The C oracle's fp32 pack-then-sum and the numpy direct-index definition, bit for bit,
+    on random fp32 gradients with a wide exponent range."""
+    rng = np.random.default_rng(grp.world * 7 + grp.n_params)
+    grads = [[(rng.standard_normal(grp.numel(i)) * np.exp2(rng.integers(-30, 10, size=grp.numel(i))))
+              .astype(np.float32) for i in range(grp.n_params)] for _ in range(grp.world)]
+    for scale in (0, 1):
+        a = oracle.rs_reduce_f32(grp.world, grp.shapes, grads, scale)
+        b = oracle_np.rs_direct_f32(grp.world, grp.shapes, grads, scale)
+        assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
