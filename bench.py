@@ -476,6 +476,12 @@ def run_variants(wl, K, stream, peak, flush):
         rec("slot_reduce_f32", timed_calls(lambda: wl.plan.rs_reduce_slots_f32(slots32, wl.out),
                                            K, stream, flush), 4 * W * N + 4 * W * Ns, 1, wl.plan, same_rs)
         del slots32
+        # ... and read in place, every rank's fp32 gradients at once (TIDE-RS itself)
+        g32_all = T.TensorTable([t.float() for row in wl.grads for t in row])
+        wl.out.fill_(float("nan"))
+        rec("rs_reduce_f32", timed_calls(lambda: wl.plan.rs_reduce_f32(g32_all, wl.out), K, stream, flush),
+            4 * W * N + 4 * W * Ns, 1, wl.plan, same_rs)
+        del g32_all
     else:
         out["slot_reduce_f32"] = {"skipped": f"fp32 slots of {f32_bytes / 2 ** 30:.0f} GiB"}
     del ref_out, ref_params
@@ -500,6 +506,7 @@ ROW_KINDS = {
     "stage_one_f32": ("slot_stage", "fp32 gradients of one rank, SM"),
     "stage_one_f32_ce": ("slot_stage", "fp32 gradients of one rank, copy engines"),
     "slot_reduce_f32": ("slot_reduce", "fp32 slots, SM, rank order"),
+    "rs_reduce_f32": ("rs_reduce", "fp32 gradients read in place, SM, rank order"),
     "stock_torch_pack_reduce": ("stock_rs", "torch _chunk_cat pack + add"),
     "stock_torch_copyout": ("stock_ag", "torch split_with_sizes_copy"),
 }

@@ -543,6 +543,42 @@ extern "C" tide_status_t tide_rs_reduce_slots_f32(const tide_plan_t* cplan, cons
     return e == cudaSuccess ? TIDE_OK : TIDE_ERR_CUDA;
 }
 
+extern "C" tide_status_t tide_rs_reduce_f32(const tide_plan_t* cplan, const float* const* grads,
+                                            const int64_t* grad_numel, float* out, int64_t out_numel,
+                                            int32_t scale_mode, int32_t max_ctas, void* stream) {
+    ApiRange range("tide_rs_reduce_f32");
+    tide_plan* p = const_cast<tide_plan*>(cplan);
+    tide_status_t st = check_plan(p);
+    if (st != TIDE_OK) return st;
+    if ((st = check_enums(p, TIDE_ENGINE_SM, max_ctas)) != TIDE_OK) return st;
+    if ((st = check_reduce_modes(scale_mode, TIDE_ORDER_RANK)) != TIDE_OK) return st;
+    const int64_t W = p->world, P = p->n_params;
+    const int64_t n_out = (p->rank >= 0 ? 1 : W) * p->shard_numel;
+    std::vector<Span> spans;
+    spans.reserve((size_t)(W * P) + 1);
+    if (W * P > 0 && (grads == nullptr || grad_numel == nullptr)) return TIDE_ERR_INVALID_ARG;
+    for (int64_t k = 0; k < W; ++k)
+        for (int64_t i = 0; i < P; ++i) {
+            const int64_t j = k * P + i;
+            if ((st = check_buf(grads[j], grad_numel[j], p->numel[i], 4)) != TIDE_OK) return st;
+            add_span(spans, grads[j], 4 * p->numel[i], false);
+        }
+    if ((st = check_buf(out, out_numel, n_out, 4)) != TIDE_OK) return st;
+    add_span(spans, out, 4 * n_out, true);
+    if (overlaps(spans)) return TIDE_ERR_INVALID_ARG;
+    if ((st = launchable(p)) != TIDE_OK) return st;
+    if (p->tiles.empty()) return TIDE_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = sync_table(p->grad_tab, reinterpret_cast<const void* const*>(grads), W * P, s)) != TIDE_OK)
+        return st;
+    const bool v8 = p->grad_tab.aligned32 && (reinterpret_cast<uintptr_t>(out) & 31) == 0;
+    p->last_kernel = K_RS_F32;
+    p->last_ctas = grid_for(p, K_RS_F32, max_ctas);
+    cudaError_t e = tide::launch_reduce_f32(p, p->grad_tab.dev, out, out_numel, inv_world(p->world),
+                                            scale_mode == TIDE_SCALE_INV_WORLD, v8, p->last_ctas, s);
+    return e == cudaSuccess ? TIDE_OK : TIDE_ERR_CUDA;
+}
+
 extern "C" tide_status_t tide_rs_reduce_pipelined(const tide_plan_t* cplan, const void* const* grads,
                                                   const int64_t* grad_numel, float* out,
                                                   int64_t out_numel, int32_t scale_mode,

@@ -11,7 +11,9 @@
 //           rank, every row of its slot; slot pads are not written);
 //   reduce: out[j] = s * fl32(sum_{k=0..W-1} slot_k[row0 + j]) from slot_0 in
 //           rank order, +0.0 at pads (row0 = rank*Ns for a one-rank plan,
-//           applied by the host to the slot pointers).
+//           applied by the host to the slot pointers);
+//   direct: out[r*Ns + off_i + e] = s * fl32(sum_k g_{k,i}[r*c_i + e]), TIDE-RS
+//           itself on fp32 gradients read where they lie (no slot).
 // Both are HBM-bound (stage: 4 + 4 bytes per element; reduce: 4W + 4).  CTAs
 // walk the plan's tiles round-robin.  Each thread keeps four 32-byte vectors in
 // flight: the staging loads four before storing them, the reduction issues one
@@ -42,6 +44,9 @@ struct ReduceF32Params {
     int64_t n_tiles;
     const void* const* slot_tab;  // [W] fp32 slots, already advanced to the plan's first row
     int64_t src_bound;            // elements readable from each of those pointers
+    const void* const* grad_tab;  // direct: [W*P] fp32 gradients, k*P + i
+    const int64_t* numel;         // direct: [P] unpadded numel
+    int32_t n_params;
     float* out;
     int64_t out_numel;
     int32_t world;
@@ -124,32 +129,49 @@ __device__ __forceinline__ void add8(float (&acc)[8], const V8& v) {
     for (int l = 0; l < 8; ++l) acc[l] = __fadd_rn(acc[l], __uint_as_float(v.w[l]));
 }
 
-__global__ void __launch_bounds__(kThreads) reduce_slots_f32_kernel(const ReduceF32Params a) {
-    __shared__ const float* s_slot[TIDE_MAX_WORLD];
+// SLOT: the sources are the W slots, read at the output position (tile dst_off).
+// Otherwise (direct): the sources are the W ranks' gradients of the tile's param,
+// read at the tile's src_off, with no staging at all; their pointers are put in
+// shared memory tile by tile.  s_src[k] + src0 is rank k's first element of the tile.
+template <bool SLOT>
+__global__ void __launch_bounds__(kThreads) reduce_f32_kernel(const ReduceF32Params a) {
+    __shared__ const float* s_src[TIDE_MAX_WORLD];
     __shared__ tide_tile_t s_tile;
     const int W = a.world;
-    for (int k = threadIdx.x; k < W; k += kThreads) s_slot[k] = static_cast<const float*>(a.slot_tab[k]);
+    if (SLOT)
+        for (int k = threadIdx.x; k < W; k += kThreads) s_src[k] = static_cast<const float*>(a.slot_tab[k]);
     for (int64_t t = blockIdx.x; t < a.n_tiles; t += gridDim.x) {
         __syncthreads();
         if (threadIdx.x == 0) s_tile = a.tiles[t];
         __syncthreads();
         const tide_tile_t tl = s_tile;
         const int64_t base = tl.dst_off;
-        const bool ok = tl.n_valid >= 0 && tl.n_valid <= tl.n_total && base >= 0 &&
-                        base + tl.n_total <= a.out_numel && base + tl.n_valid <= a.src_bound;
+        bool ok = tl.n_valid >= 0 && tl.n_valid <= tl.n_total && base >= 0 && base + tl.n_total <= a.out_numel;
+        if (SLOT)
+            ok = ok && base + tl.n_valid <= a.src_bound;
+        else
+            ok = ok && tl.param >= 0 && tl.param < a.n_params &&
+                 (tl.n_valid == 0 || (tl.src_off >= 0 && tl.src_off + tl.n_valid <= a.numel[tl.param]));
         if (!ok) {
             if (threadIdx.x == 0) atomicOr(a.err, TIDE_KCHECK_TILE);
             continue;
         }
+        const int64_t src0 = SLOT ? base : tl.src_off;
+        if (!SLOT) {
+            // (every thread has finished the previous tile: the barriers above lie between)
+            for (int k = threadIdx.x; k < W; k += kThreads)
+                s_src[k] = static_cast<const float*>(a.grad_tab[(int64_t)k * a.n_params + tl.param]);
+            __syncthreads();
+        }
         // whole 32-byte vectors of valid elements, then the element loop for the rest
-        const int64_t nv = (a.v8 && (base & 7) == 0) ? (tl.n_valid >> 3) : 0;
+        const int64_t nv = (a.v8 && ((base | src0) & 7) == 0) ? (tl.n_valid >> 3) : 0;
         for (int64_t v0 = threadIdx.x; v0 < nv; v0 += (int64_t)kThreads * kVecU) {
             float acc[kVecU][8];
 #pragma unroll
             for (int u = 0; u < kVecU; ++u) {
                 const int64_t v = v0 + (int64_t)u * kThreads;
                 if (v < nv) {
-                    const V8 x = ld_stream_v8(s_slot[0] + base + 8 * v);
+                    const V8 x = ld_stream_v8(s_src[0] + src0 + 8 * v);
 #pragma unroll
                     for (int l = 0; l < 8; ++l) acc[u][l] = __uint_as_float(x.w[l]);
                 }
@@ -159,7 +181,7 @@ __global__ void __launch_bounds__(kThreads) reduce_slots_f32_kernel(const Reduce
 #pragma unroll
                 for (int u = 0; u < kVecU; ++u) {
                     const int64_t v = v0 + (int64_t)u * kThreads;
-                    if (v < nv) x[u] = ld_stream_v8(s_slot[k] + base + 8 * v);
+                    if (v < nv) x[u] = ld_stream_v8(s_src[k] + src0 + 8 * v);
                 }
 #pragma unroll
                 for (int u = 0; u < kVecU; ++u)
@@ -180,8 +202,8 @@ __global__ void __launch_bounds__(kThreads) reduce_slots_f32_kernel(const Reduce
         for (int64_t e = 8 * nv + threadIdx.x; e < tl.n_total; e += kThreads) {
             float r = 0.0f;
             if (e < tl.n_valid) {
-                r = s_slot[0][base + e];
-                for (int k = 1; k < W; ++k) r = __fadd_rn(r, s_slot[k][base + e]);
+                r = s_src[0][src0 + e];
+                for (int k = 1; k < W; ++k) r = __fadd_rn(r, s_src[k][src0 + e]);
                 if (a.do_scale) r = __fmul_rn(r, a.scale);
             }
             a.out[base + e] = r;
@@ -198,10 +220,10 @@ int stage_f32_blocks_per_sm() {
     return n;
 }
 
-int reduce_f32_blocks_per_sm() {
+int reduce_f32_blocks_per_sm(bool slot) {
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, reduce_slots_f32_kernel, kThreads, 0) !=
-        cudaSuccess)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &n, slot ? reduce_f32_kernel<true> : reduce_f32_kernel<false>, kThreads, 0) != cudaSuccess)
         return 0;
     return n;
 }
@@ -239,8 +261,35 @@ cudaError_t launch_reduce_slots_f32(const tide_plan* p, const void* const* d_slo
     a.do_scale = do_scale ? 1 : 0;
     a.v8 = v8 ? 1 : 0;
     a.err = p->d_err;
+    a.grad_tab = nullptr;
+    a.numel = nullptr;
+    a.n_params = p->n_params;
     (void)cudaGetLastError();
-    reduce_slots_f32_kernel<<<grid, kThreads, 0, stream>>>(a);
+    reduce_f32_kernel<true><<<grid, kThreads, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_reduce_f32(const tide_plan* p, const void* const* d_grad_tab, float* out,
+                              int64_t out_numel, float scale, bool do_scale, bool v8, int grid,
+                              cudaStream_t stream) {
+    if (p->tiles.empty() || grid <= 0) return cudaSuccess;
+    ReduceF32Params a;
+    a.tiles = p->d_tiles;
+    a.n_tiles = (int64_t)p->tiles.size();
+    a.slot_tab = nullptr;
+    a.src_bound = 0;
+    a.grad_tab = d_grad_tab;
+    a.numel = p->d_numel;
+    a.n_params = p->n_params;
+    a.out = out;
+    a.out_numel = out_numel;
+    a.world = p->world;
+    a.scale = scale;
+    a.do_scale = do_scale ? 1 : 0;
+    a.v8 = v8 ? 1 : 0;
+    a.err = p->d_err;
+    (void)cudaGetLastError();
+    reduce_f32_kernel<false><<<grid, kThreads, 0, stream>>>(a);
     return cudaGetLastError();
 }
 

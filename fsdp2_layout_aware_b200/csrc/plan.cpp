@@ -110,9 +110,10 @@ tide_status_t upload(tide_plan* p) {
         p->blocks_per_sm[K_AG_GATHER] = tide::ag_blocks_per_sm(true);
         p->blocks_per_sm[K_STAGE] = tide::stage_blocks_per_sm();
         p->blocks_per_sm[K_STAGE_F32] = tide::stage_f32_blocks_per_sm();
-        p->blocks_per_sm[K_SLOT_RS_F32] = tide::reduce_f32_blocks_per_sm();
+        p->blocks_per_sm[K_SLOT_RS_F32] = tide::reduce_f32_blocks_per_sm(true);
+        p->blocks_per_sm[K_RS_F32] = tide::reduce_f32_blocks_per_sm(false);
         for (int k : {K_RS, K_AG, K_STAGE, K_SLOT_RS, K_RS_TREE, K_SLOT_RS_TREE, K_AG_GATHER, K_STAGE_F32,
-                      K_SLOT_RS_F32})
+                      K_SLOT_RS_F32, K_RS_F32})
             if (p->blocks_per_sm[k] <= 0) st = TIDE_ERR_CUDA;
         // 0 here (not enough shared memory) only disables the bulk-copy path
         p->blocks_per_sm[K_RS_TMA] = p->blocks_per_sm[K_SLOT_RS_TMA] = tide::rs_tma_blocks_per_sm(p->world);

@@ -14,7 +14,7 @@ enum : int32_t {
     K_RS = 0, K_AG = 1, K_STAGE = 2, K_SLOT_RS = 3, K_RS_TMA = 4, K_SLOT_RS_TMA = 5,
     K_RS_V32 = 6, K_SLOT_RS_V32 = 7, K_RS_TREE = 8, K_SLOT_RS_TREE = 9, K_AG_GATHER = 10,
     K_RS_TREE_V32 = 11, K_SLOT_RS_TREE_V32 = 12, K_STAGE_F32 = 13, K_SLOT_RS_F32 = 14,
-    K_COUNT = 15
+    K_RS_F32 = 15, K_COUNT = 16
 };
 
 // A device pointer table with a host mirror: re-uploaded only when it changes.
@@ -81,7 +81,7 @@ int rs_tma_blocks_per_sm(int world);  // also opts the TMA kernels in to their s
 int ag_blocks_per_sm(bool gather);
 int stage_blocks_per_sm();
 int stage_f32_blocks_per_sm();
-int reduce_f32_blocks_per_sm();
+int reduce_f32_blocks_per_sm(bool slot);
 
 // Kernel launches; return the launch's cudaError_t.
 // The RS launchers work on the plan's tiles [t0, t1) (t1 < 0: to the end).
@@ -113,6 +113,11 @@ cudaError_t launch_stage_f32(const tide_plan* p, const void* const* d_grad_tab, 
 cudaError_t launch_reduce_slots_f32(const tide_plan* p, const void* const* d_slot_tab, int64_t src_bound,
                                     float* out, int64_t out_numel, float scale, bool do_scale, bool v8,
                                     int grid, cudaStream_t stream);
+// TIDE-RS on fp32 gradients read in place (d_grad_tab [W*P], k*P + i); v8: every
+// gradient and out are 32-byte aligned.
+cudaError_t launch_reduce_f32(const tide_plan* p, const void* const* d_grad_tab, float* out,
+                              int64_t out_numel, float scale, bool do_scale, bool v8, int grid,
+                              cudaStream_t stream);
 
 // Copy-engine variants (no kernels).
 cudaError_t ce_ag_place(tide_plan* p, const uint16_t* ag, void* const* params,

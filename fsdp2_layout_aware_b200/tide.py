@@ -45,7 +45,7 @@ TIDE_IPC_HANDLE_BYTES = 64
  K_SLOT_RS_TREE, K_AG_GATHER, K_RS_TREE_V32, K_SLOT_RS_TREE_V32) = range(13)
 KERNEL_NAMES = ("rs", "ag", "stage", "slot_rs", "rs_tma", "slot_rs_tma", "rs_v32", "slot_rs_v32",
                 "rs_tree", "slot_rs_tree", "ag_gather", "rs_tree_v32", "slot_rs_tree_v32",
-                "stage_f32", "slot_rs_f32")
+                "stage_f32", "slot_rs_f32", "rs_f32")
 
 
 class tide_param_t(ctypes.Structure):
@@ -87,6 +87,7 @@ _SIGNATURES = {
     "tide_rs_reduce_slots": (_i32, [_vp, _P(_vp), _i64, _vp, _i64, _i32, _i32, _i32, _vp]),
     "tide_rs_stage_one_f32": (_i32, [_vp, _P(_vp), _P(_i64), _vp, _i64, _i32, _i32, _vp]),
     "tide_rs_reduce_slots_f32": (_i32, [_vp, _P(_vp), _i64, _vp, _i64, _i32, _i32, _vp]),
+    "tide_rs_reduce_f32": (_i32, [_vp, _P(_vp), _P(_i64), _vp, _i64, _i32, _i32, _vp]),
     "tide_rs_reduce_noalloc": (_i32, [_P(tide_param_t), _i32, _i32, _P(_vp), _P(_i64), _vp, _i64,
                                       _i32, _i32, _vp]),
     "tide_rs_reduce_pipelined": (_i32, [_vp, _P(_vp), _P(_i64), _vp, _i64, _i32, _i32, _P(_vp),
@@ -309,6 +310,12 @@ def tide_rs_stage_one_f32(plan, grads, grad_numel, slot: int, slot_numel: int, e
                                        slot_numel, engine, max_ctas, stream)
 
 
+def tide_rs_reduce_f32(plan, grads, grad_numel, out: int, out_numel: int, scale_mode: int,
+                       max_ctas: int, stream: int) -> int:
+    return lib().tide_rs_reduce_f32(plan, _ptr_array(grads), _i64_array(grad_numel), out, out_numel,
+                                    scale_mode, max_ctas, stream)
+
+
 def tide_rs_reduce_slots_f32(plan, slots, slot_numel: int, out: int, out_numel: int, scale_mode: int,
                              max_ctas: int, stream: int) -> int:
     slot_arr = _ptr_array(slots) if slots is not None else None
@@ -529,6 +536,15 @@ class Plan:
         st = tide_rs_stage_one_f32(self.handle, g.ptrs, g.numels, slot.data_ptr(), slot.numel(),
                                    engine, max_ctas, _stream_handle(stream))
         _check(st, "tide_rs_stage_one_f32")
+
+    def rs_reduce_f32(self, grads, out, scale_mode: int = TIDE_SCALE_INV_WORLD, max_ctas: int = 0,
+                      stream=None) -> None:
+        """rs_reduce for fp32 gradients (grads[k][i], or a flat k*P + i table), rank order."""
+        g = _table(grads)
+        _require_f32(g, out)
+        st = tide_rs_reduce_f32(self.handle, g.ptrs, g.numels, out.data_ptr(), out.numel(), scale_mode,
+                                max_ctas, _stream_handle(stream))
+        _check(st, "tide_rs_reduce_f32")
 
     def rs_reduce_slots_f32(self, slots, out, scale_mode: int = TIDE_SCALE_INV_WORLD,
                             max_ctas: int = 0, stream=None) -> None:

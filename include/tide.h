@@ -325,6 +325,18 @@ TIDE_API tide_status_t tide_rs_reduce_slots(const tide_plan_t* plan, const void*
  * for a buffer that is not 4-byte aligned); nothing is enqueued on error; the
  * caller owns every buffer.
  */
+/*
+ * TIDE-RS on fp32 gradients read where they lie (no slot, no packed buffer):
+ * out[r*Ns + off_i + e] = s * fl32(sum_{k=0..W-1} g_{k,i}[r*c_i + e]) in rank
+ * order from g_0 (fp32, round to nearest even), +0.0 at pad positions; with a
+ * one-rank plan (rank r) out is that rank's fp32 [Ns] shard.  grads: host array
+ * of W*P device pointers to fp32 gradients, index k*P + i (grad_numel[k*P+i] >=
+ * d0_i*inner_i; 4-byte aligned; peers' memory accepted); out must overlap no
+ * gradient.  One kernel launch.  Errors as tide_rs_reduce.
+ */
+TIDE_API tide_status_t tide_rs_reduce_f32(const tide_plan_t* plan, const float* const* grads,
+                                          const int64_t* grad_numel, float* out, int64_t out_numel,
+                                          int32_t scale_mode, int32_t max_ctas, void* stream);
 TIDE_API tide_status_t tide_rs_stage_one_f32(const tide_plan_t* plan, const float* const* grads,
                                              const int64_t* grad_numel, float* slot, int64_t slot_numel,
                                              int32_t engine, int32_t max_ctas, void* stream);
@@ -420,7 +432,8 @@ TIDE_API tide_status_t tide_rs_reduce_noalloc(const tide_param_t* params, int32_
  * 10 = AG placement from per-rank shards (tide_ag_gather_place),
  * 11 = RS reduce in tree order with 32-byte loads, 12 = slot reduce in tree
  * order with 32-byte loads, 13 = Slot-Reuse stage of fp32 gradients
- * (tide_rs_stage_one_f32), 14 = slot reduce of fp32 slots (tide_rs_reduce_slots_f32).
+ * (tide_rs_stage_one_f32), 14 = slot reduce of fp32 slots (tide_rs_reduce_slots_f32),
+ * 15 = RS reduce of fp32 gradients (tide_rs_reduce_f32).
  * The reductions use kernels 4/5 (one CTA per SM, TMA loads into shared memory)
  * when the plan was built with TIDE_PLAN_TMA, every tile starts on an
  * 8-element boundary and every source and the output are 16-byte aligned.

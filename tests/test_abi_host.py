@@ -546,6 +546,34 @@ def test_f32_reduce_slots_validation(tiny_plan):
     assert red(plan=one_rank, no=a["Ns"] - 1) == T.TIDE_ERR_SIZE
 
 
+def test_f32_direct_reduce_validation(tiny_plan):
+    g = configs.tiny()
+    W, P = g.world, g.n_params
+    L = oracle.layout(W, g.shapes)
+    f = Fake()
+    f.next = BASE + (1 << 42)
+    grads = [f.buf(4 * g.numel(i)) for _ in range(W) for i in range(P)]
+    gnum = [g.numel(i) for _ in range(W) for i in range(P)]
+    out = f.buf(4 * W * L.Ns)
+
+    def red(gr=grads, gn=gnum, o=out, no=W * L.Ns, scale=1, cap=0, plan=tiny_plan):
+        return T.tide_rs_reduce_f32(plan.handle, gr, gn, o, no, scale, cap, 0)
+    assert red() == T.TIDE_ERR_DEVICE
+    assert red(scale=0) == T.TIDE_ERR_DEVICE
+    assert red(scale=5) == T.TIDE_ERR_INVALID_ARG
+    assert red(cap=-1) == T.TIDE_ERR_INVALID_ARG
+    assert red(gr=[0] + grads[1:]) == T.TIDE_ERR_INVALID_ARG
+    assert red(gr=grads[:7] + [grads[7] + 2] + grads[8:]) == T.TIDE_ERR_ALIGNMENT
+    assert red(gn=gnum[:6] + [gnum[6] - 1] + gnum[7:]) == T.TIDE_ERR_SIZE
+    assert red(no=W * L.Ns - 1) == T.TIDE_ERR_SIZE
+    assert red(o=out + 2) == T.TIDE_ERR_ALIGNMENT
+    assert red(o=grads[9]) == T.TIDE_ERR_INVALID_ARG     # out overlaps a gradient
+    assert red(gr=[grads[0]] * (W * P), gn=[max(gnum)] * (W * P)) == T.TIDE_ERR_DEVICE  # grads may alias
+    one_rank = T.Plan(g.shapes, W, host_only=True, rank=2)
+    assert red(plan=one_rank, no=L.Ns) == T.TIDE_ERR_DEVICE
+    assert red(plan=one_rank, no=L.Ns - 1) == T.TIDE_ERR_SIZE
+
+
 def test_f32_bindings_refuse_other_dtypes():
     """The Plan methods of the fp32 calls refuse torch tensors that are not fp32 before any
     call: the C calls count 4-byte elements."""
@@ -563,3 +591,5 @@ def test_f32_bindings_refuse_other_dtypes():
         plan.rs_reduce_slots_f32([torch.zeros(4 * L.Ns, dtype=torch.bfloat16)] * 4, torch.zeros(4 * L.Ns))
     with pytest.raises(TypeError):
         plan.rs_reduce_slots_f32([torch.zeros(4 * L.Ns)] * 4, torch.zeros(4 * L.Ns, dtype=torch.float16))
+    with pytest.raises(TypeError):
+        plan.rs_reduce_f32([bf] * 4, torch.zeros(4 * L.Ns))

@@ -1,5 +1,5 @@
-"""fp32 gradients through Slot-Reuse (tide_rs_stage_one_f32, tide_rs_reduce_slots_f32) against
-the oracle, bit for bit.
+"""fp32 gradients through Slot-Reuse (tide_rs_stage_one_f32, tide_rs_reduce_slots_f32) and read
+in place (tide_rs_reduce_f32) against the oracle, bit for bit.
 
 Every source rank stages its fp32 gradients into its own fp32 slot, on the SMs or on the copy
 engines (stale contents: NaN, so a pad that is read shows); the slots must equal the oracle's staging word for word (pads keep
@@ -94,6 +94,34 @@ def test_f32_slot_reuse_matches_the_oracle(group, shift, engine):
             rp = T.Plan(group.shapes, W, rank=r)
             shard = dev_f32(np.full(L.Ns, NAN, np.uint32), shift)
             rp.rs_reduce_slots_f32(slots, shard, scale_mode=scale)
+            torch.cuda.synchronize()
+            assert np.array_equal(f32_bits(shard), want[r * L.Ns:(r + 1) * L.Ns]), (scale, r)
+            rp.check()
+    plan.check()
+
+
+@pytest.mark.parametrize("shift", [0, 1], ids=["aligned", "shifted"])
+@pytest.mark.parametrize("group", groups(), ids=lambda g: f"{g.name}_w{g.world}")
+def test_f32_direct_reduce_matches_the_oracle(group, shift):
+    """TIDE-RS on fp32 gradients read in place: all shards, and each rank's shard with a
+    one-rank plan, bit for bit against the oracle."""
+    W = group.world
+    L = oracle.layout(W, group.shapes)
+    grads = f32_grads(group, seed=W * 31 + group.n_params)
+    g = [[dev_f32(grads[k][i], shift) for i in range(group.n_params)] for k in range(W)]
+    table = T.TensorTable([t for row in g for t in row])
+    plan = T.Plan(group.shapes, W)
+    for scale in (0, 1):
+        want = oracle.rs_reduce_f32(W, group.shapes, grads, scale).view(np.uint32)
+        out = dev_f32(np.full(W * L.Ns, NAN, np.uint32), shift)
+        plan.rs_reduce_f32(table, out, scale_mode=scale)
+        torch.cuda.synchronize()
+        assert np.array_equal(f32_bits(out), want), scale
+        assert plan.last_launch()[0] == T.KERNEL_NAMES.index("rs_f32")
+        for r in sorted({0, W // 2, W - 1}):
+            rp = T.Plan(group.shapes, W, rank=r)
+            shard = dev_f32(np.full(L.Ns, NAN, np.uint32), shift)
+            rp.rs_reduce_f32(table, shard, scale_mode=scale)
             torch.cuda.synchronize()
             assert np.array_equal(f32_bits(shard), want[r * L.Ns:(r + 1) * L.Ns]), (scale, r)
             rp.check()
