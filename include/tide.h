@@ -16,7 +16,9 @@
  * data-parallel ranks are W sets of buffers that the calling GPU's kernels
  * read, its own memory or, through CUDA IPC (tide_ipc_*), other processes'
  * buffers, with one-rank plans (tide_plan_group_rank) for a process that holds
- * one rank.
+ * one rank.  Gradients FSDP2 keeps in fp32 (accumulated with gradient sync off)
+ * have calls of their own: tide_rs_reduce_f32, tide_rs_stage_one_f32 and
+ * tide_rs_reduce_slots_f32.
  *
  * Layout (the pages leave it open; this is the reading every call follows):
  *   param i has shape (d0_i, ...) with inner_i = product of the trailing dims;
