@@ -266,10 +266,10 @@ int orc_slot_stage_f32(int64_t W, int64_t P, const int64_t* d0, const int64_t* i
     for (int64_t r = 0; r < W; ++r)
         for (int64_t i = 0; i < P; ++i)
             for (int64_t s = 0; s < S[i]; ++s) {
-                int64_t row = r * S[i] + s;
-                if (row >= d0[i]) continue;
+                const int64_t src_row = r * S[i] + s;      /* row of the param, rank r's s-th */
+                if (src_row >= d0[i]) continue;            /* a pad row: the slot keeps its words */
                 for (int64_t t = 0; t < inner[i]; ++t)
-                    slot[r * Ns + off[i] + s * inner[i] + t] = g[i][row * inner[i] + t];
+                    slot[r * Ns + off[i] + s * inner[i] + t] = g[i][src_row * inner[i] + t];
             }
     free(S); free(c); free(off);
     return 0;

@@ -35,6 +35,10 @@ MUTANTS = {
                             "dst[t] = row < d0[i] ? bf16_to_f32(((const uint16_t*)g[i])[row * inner[i] + t]) : 0.0f;"),
     "f32_slots_drop_last_rank": ("for (int64_t k = 1; k < W; ++k) acc = acc + slots[k][j];",
                                  "for (int64_t k = 1; k < W - 1; ++k) acc = acc + slots[k][j];"),
+    "f32_stage_writes_pad_rows": ("if (src_row >= d0[i]) continue;",
+                                  "if (src_row >= d0[i]) { for (int64_t t = 0; t < inner[i]; ++t) "
+                                  "slot[r * Ns + off[i] + s * inner[i] + t] = 0; continue; }"),
+    "f32_stage_drops_row_stride": ("= g[i][src_row * inner[i] + t];", "= g[i][src_row + t * 0];"),
     "f32_scales_by_W_not_inverse": ("        float sc = 1.0f / (float)W;\n        for (int64_t j = 0; j < n; ++j) out[j] = out[j] * sc;",
                                     "        float sc = (float)W;\n        for (int64_t j = 0; j < n; ++j) out[j] = out[j] * sc;"),
     "ranks_added_in_reverse": ("pack_f32(W, P, d0, inner, S, off, Ns, grads + k * P, packed);",
