@@ -128,6 +128,26 @@ def test_f32_direct_reduce_matches_the_oracle(group, shift):
     plan.check()
 
 
+@pytest.mark.parametrize("gshift", range(8))
+def test_f32_staging_at_every_relative_alignment(gshift):
+    """Gradients shifted by 0..7 words against an aligned slot: the staging copy takes its
+    32-byte, 16-byte and word paths (with their heads and tails) and gives the oracle's slot."""
+    group = configs.Group("aligns", 4, ((4 * 3000 + 1, 3), (8 * 16 * 4,), (4 * 2048, 4)))
+    W = group.world
+    L = oracle.layout(W, group.shapes)
+    grads = f32_grads(group, seed=60 + gshift)
+    plan = T.Plan(group.shapes, W)
+    for engine in (T.TIDE_ENGINE_SM, T.TIDE_ENGINE_CE):
+        slot = dev_f32(np.full(W * L.Ns, NAN, np.uint32), 0)
+        g = [dev_f32(grads[1][i], gshift) for i in range(group.n_params)]
+        plan.rs_stage_one_f32(g, slot, engine=engine)
+        torch.cuda.synchronize()
+        want = np.full(W * L.Ns, NAN, np.uint32)
+        oracle.slot_stage_f32(W, group.shapes, grads[1], want)
+        assert np.array_equal(f32_bits(slot), want), engine
+    plan.check()
+
+
 @pytest.mark.parametrize("cap", [1, 7])
 def test_f32_cta_caps_give_the_same_bits(cap):
     group = mini_sweep(8)
