@@ -3,8 +3,10 @@
 Each case plants one mistake in a copy of oracle/tide_oracle.c (on the CPU,
 in a temporary directory), builds it, points the pin tests at it through
 TIDE_ORACLE_LIB and checks that at least one pin fails.  Every mutation keeps
-all memory accesses inside their buffers.
+all memory accesses inside their buffers.  The mutants' pin runs are separate
+processes, run a few at a time before the cases check their results.
 """
+import concurrent.futures
 import os
 import subprocess
 import sys
@@ -46,19 +48,41 @@ MUTANTS = {
 }
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_catch_planted_mistake(name, tmp_path):
+def _run_mutant(name, root):
+    """Build the mutant of `name` under `root` and run the pins against it; (returncode, output)."""
     old, new = MUTANTS[name]
     text = open(SRC).read()
-    assert text.count(old) == 1, f"mutation anchor for {name} not unique"
-    mutant_c = tmp_path / "mutant.c"
+    if text.count(old) != 1:
+        return None, f"mutation anchor for {name} not unique"
+    d = root / name
+    d.mkdir()
+    mutant_c = d / "mutant.c"
     mutant_c.write_text(text.replace(old, new))
-    lib = tmp_path / "libmutant.so"
+    lib = d / "libmutant.so"
     subprocess.run(["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared", "-o",
                     str(lib), str(mutant_c)], check=True)
-    env = dict(os.environ, TIDE_ORACLE_LIB=str(lib))
+    # one thread per pin process: the mutants run side by side
+    env = dict(os.environ, TIDE_ORACLE_LIB=str(lib), OMP_NUM_THREADS="1", MKL_NUM_THREADS="1",
+               OPENBLAS_NUM_THREADS="1")
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                         "-k", "not gloo", os.path.join(ROOT, "tests", "test_oracle_pins.py")],
-                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
-    assert r.returncode != 0, f"no pin caught mutant {name}:\n{r.stdout[-2000:]}"
-    assert "failed" in r.stdout or "Error" in r.stdout
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+    return r.returncode, r.stdout
+
+
+@pytest.fixture(scope="module")
+def mutant_runs(tmp_path_factory):
+    """Every mutant's pin run, several at a time (each is an independent process)."""
+    root = tmp_path_factory.mktemp("mutants")
+    names = sorted(MUTANTS)
+    workers = max(1, min(len(names), (os.cpu_count() or 2) // 2))
+    with concurrent.futures.ThreadPoolExecutor(max_workers=workers) as ex:
+        return dict(zip(names, ex.map(lambda n: _run_mutant(n, root), names)))
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_planted_mistake(name, mutant_runs):
+    rc, out = mutant_runs[name]
+    assert rc is not None, out
+    assert rc != 0, f"no pin caught mutant {name}:\n{out[-2000:]}"
+    assert "failed" in out or "Error" in out
